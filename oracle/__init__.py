@@ -1,0 +1,126 @@
+"""fp64 CPU oracle for the WKV recurrences -- TEST INFRASTRUCTURE ONLY.
+
+Only tests/, __graft_entry__.smoke() and bench.py (its CPU-baseline leg and its
+reference arm) may import this package.  The CUDA product path never imports,
+calls or links it, and nothing here imports the product package.
+
+The arithmetic lives in wkv_oracle.c (plain C, fp64, serial per unit); this
+module only marshals numpy arrays through ctypes.  Inputs are widened to
+float64 exactly (bf16 and fp32 values convert without rounding).
+
+Sources:
+  * WKV-4: "RWKV: Reinventing RNNs for the Transformer Era" (Chinese
+    translation), eq. 14 as referenced in the sections on temporal structure
+    (decay e^{-w}, bonus e^{u}) and gradient stability (single-step
+    time-dependent softmax).
+  * WKV-6: "RWKV-5/6 (Eagle and Finch)" summary, sections 4 (row-vector
+    convention), 4.1.2 (Eagle time mixing) and 4.2.2 (Finch per-token decay).
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_DP = ctypes.POINTER(ctypes.c_double)
+_I64 = ctypes.c_int64
+
+
+class Oracle:
+    """ctypes handle on one compiled copy of the oracle library."""
+
+    def __init__(self, lib_path: str):
+        self.path = lib_path
+        lib = ctypes.CDLL(lib_path)
+        lib.oracle_wkv4.argtypes = [_I64, _I64, _I64, _DP, _DP, _DP, _DP, _DP, _DP, _DP]
+        lib.oracle_wkv4.restype = None
+        lib.oracle_wkv6.argtypes = [_I64, _I64, _I64, _I64, _DP, _DP, _DP, _DP, _DP,
+                                    _DP, _DP, _DP, _DP]
+        lib.oracle_wkv6.restype = None
+        lib.oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.oracle_set_threads.restype = ctypes.c_int
+        self._lib = lib
+
+    def set_threads(self, n: int = 0) -> int:
+        """Set the OpenMP thread count (n <= 0 keeps it); returns the count in use."""
+        return int(self._lib.oracle_set_threads(int(n)))
+
+    @staticmethod
+    def _f64(x):
+        a = np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+        return a, a.ctypes.data_as(_DP)
+
+    def wkv4(self, w, u, k, v, s0=None, want_state=False):
+        """WKV-4 forward.  k, v: [B,T,C]; w, u: [C]; s0: [B,3,C] (a,b,p) or None.
+
+        Returns y [B,T,C] (float64), and also sT [B,3,C] when want_state.
+        """
+        k, kp = self._f64(k)
+        v, vp = self._f64(v)
+        w, wp = self._f64(w)
+        u, up = self._f64(u)
+        B, T, C = k.shape
+        assert v.shape == k.shape and w.shape == (C,) and u.shape == (C,)
+        y = np.empty((B, T, C), np.float64)
+        sT = np.empty((B, 3, C), np.float64) if want_state else None
+        if s0 is not None:
+            s0, s0p = self._f64(s0)
+            assert s0.shape == (B, 3, C)
+        else:
+            s0p = None
+        self._lib.oracle_wkv4(B, T, C, wp, up, kp, vp, s0p, y.ctypes.data_as(_DP),
+                              sT.ctypes.data_as(_DP) if sT is not None else None)
+        return (y, sT) if want_state else y
+
+    def wkv6(self, r, k, v, w, u, s0=None):
+        """WKV-6 forward.  r,k,v,w: [B,T,H,N]; u: [H,N]; s0: [B,H,N,N] or None.
+
+        Returns (y [B,T,H,N], sT [B,H,N,N]) in float64.
+        """
+        r, rp = self._f64(r)
+        k, kp = self._f64(k)
+        v, vp = self._f64(v)
+        w, wp = self._f64(w)
+        u, up = self._f64(u)
+        B, T, H, N = r.shape
+        for x in (k, v, w):
+            assert x.shape == (B, T, H, N)
+        assert u.shape == (H, N)
+        if s0 is not None:
+            s0, s0p = self._f64(s0)
+            assert s0.shape == (B, H, N, N)
+        else:
+            s0p = None
+        y = np.empty((B, T, H, N), np.float64)
+        sT = np.empty((B, H, N, N), np.float64)
+        work = np.empty((B, H, N, N), np.float64)
+        self._lib.oracle_wkv6(B, T, H, N, rp, kp, vp, wp, up, s0p, y.ctypes.data_as(_DP),
+                              sT.ctypes.data_as(_DP), work.ctypes.data_as(_DP))
+        return y, sT
+
+
+_DEFAULT = None
+
+
+def get() -> Oracle:
+    """The oracle built from oracle/wkv_oracle.c (compiled on first use if needed)."""
+    global _DEFAULT
+    if _DEFAULT is None:
+        if not _build.up_to_date():
+            _build.build()
+        _DEFAULT = Oracle(_build.LIB)
+    return _DEFAULT
+
+
+def wkv4(w, u, k, v, s0=None, want_state=False):
+    return get().wkv4(w, u, k, v, s0=s0, want_state=want_state)
+
+
+def wkv6(r, k, v, w, u, s0=None):
+    return get().wkv6(r, k, v, w, u, s0=s0)
+
+
+def set_threads(n: int = 0) -> int:
+    return get().set_threads(n)

@@ -1,0 +1,179 @@
+/*
+ * wkv_oracle.c -- plain fp64 CPU oracle for the two WKV recurrences.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Only tests/, __graft_entry__.smoke() and bench.py's
+ * CPU-baseline / reference arm may load or run this library.  The CUDA library
+ * (wkv_recurrence_02_b200) never calls it, links it or includes anything from it;
+ * the two share no code, header, table or constant.
+ *
+ * Every input is fp64 (bf16 / fp32 values the GPU sees are widened exactly by the
+ * caller), every operation is fp64, and each recurrence is walked serially in the
+ * order the pages state it.  OpenMP is used only across independent units
+ * ((b,c) for WKV-4, (b,h) for WKV-6); it never reorders work inside a unit.
+ *
+ * Sources (page title, section):
+ *  [R4]  "RWKV: Reinventing RNNs for the Transformer Era" (Chinese translation),
+ *        section "利用时间结构进行时序数据处理" (exploiting temporal structure): the time
+ *        decay e^{-w} and the bonus e^{u} of eq. 14; section "梯度稳定性和层堆叠"
+ *        (gradient stability): the attention-like score is updated by a single-step
+ *        "time-dependent softmax", which is what makes the running-max form below
+ *        the method's own evaluation order.  Eq. 14 itself is missing from the page;
+ *        its content (the weighted average written out in wkv4_step below) is the
+ *        RWKV-4 WKV definition the page refers to.
+ *  [E4]  "RWKV-5/6 (Eagle and Finch)" summary, section 4: vectors are row vectors of
+ *        size D/h and matrices act on the right.
+ *  [E412] same page, section 4.1.2 (Eagle time mixing): the state s is a sum of
+ *        k^T v; each channel of s is decayed by the matching channel of w at every
+ *        step; the learned gain u multiplies the current token's k^T v, which is
+ *        added to the state; the receptance r multiplies that sum like a query.
+ *        w = exp(-exp(omega)) lies in (0,1).
+ *  [F422] same page, section 4.2.2 (Finch time mixing): w_t varies per token.
+ */
+#include <math.h>
+#include <stddef.h>
+#include <stdint.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+int oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0) omp_set_num_threads(n);
+    return omp_get_max_threads();
+#else
+    (void)n;
+    return 1;
+#endif
+}
+
+/*
+ * WKV-4, one channel of one sequence, [R4].
+ *
+ * Definition (per channel, decay rate w, bonus u, keys k_i, values v_i):
+ *   wkv_t = ( sum_{i<t} e^{-(t-1-i) w + k_i} v_i + e^{u + k_t} v_t )
+ *         / ( sum_{i<t} e^{-(t-1-i) w + k_i}     + e^{u + k_t}     )
+ *
+ * The past sums are carried as (a, b, p) with numerator = a e^p and
+ * denominator = b e^p.  Each step rescales to the larger exponent (the
+ * "time-dependent softmax" single-step update), so no exponential overflows.
+ * After token t the state holds sum_{i<=t} e^{-(t-i) w + k_i} (v_i | 1).
+ * An empty state is a = b = 0, p = -inf.
+ */
+static void wkv4_channel(int64_t T, int64_t stride, double w, double u,
+                         const double *k, const double *v, double *y,
+                         double *a_io, double *b_io, double *p_io)
+{
+    double a = *a_io, b = *b_io, p = *p_io;
+    for (int64_t t = 0; t < T; ++t) {
+        const double kt = k[t * stride];
+        const double vt = v[t * stride];
+
+        /* output: past state (not yet decayed for this step) plus the bonus term */
+        double q = p > u + kt ? p : u + kt;
+        double e_past = exp(p - q);        /* weight of the carried sums      */
+        double e_now = exp(u + kt - q);    /* weight e^{u+k_t} of the current */
+        y[t * stride] = (e_past * a + e_now * vt) / (e_past * b + e_now);
+
+        /* state update: decay the past by e^{-w}, add e^{k_t} (v_t | 1) */
+        double q2 = p - w > kt ? p - w : kt;
+        double e_decay = exp(p - w - q2);
+        double e_key = exp(kt - q2);
+        a = e_decay * a + e_key * vt;
+        b = e_decay * b + e_key;
+        p = q2;
+    }
+    *a_io = a;
+    *b_io = b;
+    *p_io = p;
+}
+
+/*
+ * k, v, y: [B, T, C] (channel innermost); w, u: [C].
+ * s0, sT: [B, 3, C] = (a, b, p) per channel, or NULL (s0 NULL = empty state;
+ * sT NULL = not written).  sT may equal s0.
+ */
+void oracle_wkv4(int64_t B, int64_t T, int64_t C,
+                 const double *w, const double *u,
+                 const double *k, const double *v,
+                 const double *s0, double *y, double *sT)
+{
+    int64_t units = B * C;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < units; ++n) {
+        int64_t bi = n / C, c = n % C;
+        double a = 0.0, b = 0.0, p = -INFINITY;
+        if (s0) {
+            a = s0[(bi * 3 + 0) * C + c];
+            b = s0[(bi * 3 + 1) * C + c];
+            p = s0[(bi * 3 + 2) * C + c];
+        }
+        const int64_t base = bi * T * C + c;
+        wkv4_channel(T, C, w[c], u[c], k + base, v + base, y + base, &a, &b, &p);
+        if (sT) {
+            sT[(bi * 3 + 0) * C + c] = a;
+            sT[(bi * 3 + 1) * C + c] = b;
+            sT[(bi * 3 + 2) * C + c] = p;
+        }
+    }
+}
+
+/*
+ * WKV-6 (Eagle / Finch), one head of one sequence, [E4] [E412] [F422].
+ *
+ * S is N x N; row i = key channel (decayed by w_i), column j = value channel.
+ * For each token t, in this order:
+ *   o_t[j] = sum_i r_t[i] * ( S[i][j] + u[i] k_t[i] v_t[j] )
+ *   S[i][j] = w_t[i] S[i][j] + k_t[i] v_t[j]
+ * so the output reads the state before this token's decay, and the newest
+ * past key reaches the query undecayed.
+ */
+static void wkv6_head(int64_t T, int64_t N, int64_t stride,
+                      const double *r, const double *k, const double *v,
+                      const double *w, const double *u,
+                      double *S, double *y)
+{
+    for (int64_t t = 0; t < T; ++t) {
+        const double *rt = r + t * stride;
+        const double *kt = k + t * stride;
+        const double *vt = v + t * stride;
+        const double *wt = w + t * stride;
+        double *yt = y + t * stride;
+        for (int64_t j = 0; j < N; ++j) {
+            double o = 0.0;
+            for (int64_t i = 0; i < N; ++i)
+                o += rt[i] * (S[i * N + j] + u[i] * kt[i] * vt[j]);
+            yt[j] = o;
+        }
+        for (int64_t i = 0; i < N; ++i)
+            for (int64_t j = 0; j < N; ++j)
+                S[i * N + j] = wt[i] * S[i * N + j] + kt[i] * vt[j];
+    }
+}
+
+/*
+ * r, k, v, w, y: [B, T, H, N] (channel innermost); u: [H, N].
+ * s0, sT: [B, H, N, N] (row = key channel), or NULL (s0 NULL = zero state;
+ * sT NULL = not written).  sT may equal s0.  work: B*H*N*N doubles of scratch
+ * owned by the caller (the oracle allocates nothing).
+ */
+void oracle_wkv6(int64_t B, int64_t T, int64_t H, int64_t N,
+                 const double *r, const double *k, const double *v,
+                 const double *w, const double *u,
+                 const double *s0, double *y, double *sT, double *work)
+{
+    int64_t units = B * H;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < units; ++n) {
+        int64_t bi = n / H, h = n % H;
+        double *S = work + n * N * N;
+        for (int64_t e = 0; e < N * N; ++e)
+            S[e] = s0 ? s0[n * N * N + e] : 0.0;
+        const int64_t base = (bi * T * H + h) * N;
+        wkv6_head(T, N, H * N, r + base, k + base, v + base, w + base,
+                  u + h * N, S, y + base);
+        if (sT)
+            for (int64_t e = 0; e < N * N; ++e)
+                sT[n * N * N + e] = S[e];
+    }
+}

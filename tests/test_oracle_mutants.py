@@ -1,0 +1,51 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins catch each one.
+
+The mutants are built from the committed oracle source with one textual change
+each, compiled into a temporary directory; the committed oracle is untouched.
+"""
+import os
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+import pins
+
+# (name, exact text in wkv_oracle.c, replacement)
+MUTANTS = [
+    ("wkv6_drop_bonus", "u[i] * kt[i] * vt[j]", "0.0 * kt[i] * vt[j]"),
+    ("wkv6_transposed_state", "(S[i * N + j] + u[i]", "(S[j * N + i] + u[i]"),
+    ("wkv6_decay_wrong_axis", "wt[i] * S[i * N + j] + kt[i] * vt[j]",
+     "wt[j] * S[i * N + j] + kt[i] * vt[j]"),
+    ("wkv6_decay_before_output", "o += rt[i] * (S[i * N + j]", "o += rt[i] * (wt[i] * S[i * N + j]"),
+    ("wkv6_ignore_s0", "S[e] = s0 ? s0[n * N * N + e] : 0.0;", "S[e] = 0.0;"),
+    ("wkv6_wrong_head_u", "u + h * N, S, y + base", "u, S, y + base"),
+    ("wkv6_kv_swapped_in_update", "+ kt[i] * vt[j];", "+ kt[j] * vt[i];"),
+    ("wkv4_decay_sign", "double q2 = p - w > kt ? p - w : kt;\n        double e_decay = exp(p - w - q2);",
+     "double q2 = p + w > kt ? p + w : kt;\n        double e_decay = exp(p + w - q2);"),
+    ("wkv4_drop_bonus", "double e_now = exp(u + kt - q);", "double e_now = exp(kt - q);"),
+    ("wkv4_bonus_in_state", "double e_key = exp(kt - q2);", "double e_key = exp(u + kt - q2);"),
+    ("wkv4_output_after_decay", "double e_past = exp(p - q);", "double e_past = exp(p - w - q);"),
+    ("wkv4_ignore_s0_max", "p = s0[(bi * 3 + 2) * C + c];", "p = 0.0;"),
+    ("wkv4_denominator_uses_v", "(e_past * b + e_now)", "(e_past * b + e_now * vt)"),
+]
+
+
+@pytest.fixture(scope="module")
+def source():
+    with open(obuild.SRC) as f:
+        return f.read()
+
+
+def test_committed_oracle_passes_all_pins():
+    assert pins.failing_pins(oracle.get()) == []
+
+
+@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
+def test_mutant_is_caught(tmp_path, source, name, old, new):
+    assert source.count(old) == 1, f"mutation anchor for {name} not unique/present"
+    src = tmp_path / f"{name}.c"
+    src.write_text(source.replace(old, new))
+    lib = obuild.build(str(src), str(tmp_path / f"lib_{name}.so"))
+    bad = pins.failing_pins(oracle.Oracle(lib))
+    assert bad, f"no pin caught the planted mistake {name}"
