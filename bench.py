@@ -1,0 +1,476 @@
+"""Throughput of the WKV hot path on B200: WKV tokens/s and fraction of the HBM roofline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step is one pass of the whole hot path over synthetic inputs resident in HBM:
+  * WKV-4, 169M-model shape: B=8, T=1024, C=768, bf16 k/v, 12 layers (each layer its
+    own k/v buffers and independently seeded w/u), fp32 accumulation;
+  * WKV-6, Finch-1.6B shape: B=8, T=4096, H=32, N=64 bf16, random fp32 initial state;
+  * WKV-6, 7B-scale long context: B=1, T=16384 as 4 chained calls of 4096 (sT -> s0), H=64;
+  * WKV-6 decode: one T=1 step at B=256, H=64 with a random fp32 state, updated in place.
+The metric counts B*T tokens of every call (each WKV-4 layer call counts its own B*T).
+Inputs per step (~2.4 GB) exceed the 126 MB L2, so no L2 flush is needed between steps.
+
+Under torchrun each rank runs the same step on its own GPU (the path shards over
+independent sequences/heads with no exchange step: weak scaling, no collective on the
+data path); `value` is the tokens of all ranks over the max-over-ranks device time.
+
+--impl reference times the fp64 CPU oracle (the only other implementation this method
+has here) on a bounded sample of the same workload, on the host's cores.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, HERE)
+
+METRIC = "WKV tokens/sec (B·T/s) and % of roofline at 1 B200, WKV-4 and WKV-6 prefill"
+UNIT = "tokens/s"
+WORKLOAD = ("wkv4 169M shape B8 T1024 C768 x12 layers + wkv6 Finch-1.6B B8 T4096 H32 prefill "
+            "+ wkv6 7B long context B1 T16384 H64 (4x4096 chained) + wkv6 7B decode T1 B256 H64")
+TOKENS_WKV4 = 12 * 8 * 1024
+TOKENS_FINCH = 8 * 4096
+TOKENS_LONG = 1 * 16384
+TOKENS_DECODE = 256
+STEP_TOKENS = TOKENS_WKV4 + TOKENS_FINCH + TOKENS_LONG + TOKENS_DECODE
+N_HEAD = 64
+
+
+def wkv4_bytes(B, T, C):
+    return 3 * B * T * C * 2 + 2 * C * 4
+
+
+def wkv6_bytes(B, T, H, s0=True, sT=True, esz=2):
+    n = B * T * H * N_HEAD
+    st = B * H * N_HEAD * N_HEAD * 4
+    return 5 * n * esz + (st if s0 else 0) + (st if sT else 0) + H * N_HEAD * 4
+
+
+# algorithmic bytes per launch, per kernel family
+BYTES = {
+    "wkv4_scan": wkv4_bytes(8, 1024, 768),
+    "wkv6_chunked_finch": wkv6_bytes(8, 4096, 32),
+    "wkv6_chunked_long_first": wkv6_bytes(1, 4096, 64, s0=False),
+    "wkv6_chunked_long": wkv6_bytes(1, 4096, 64),
+    "wkv6_decode": wkv6_bytes(256, 1, 64),
+}
+
+
+def load_peaks():
+    p = os.path.join(HERE, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason sampling in the background (read-only)."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "50"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        threading.Thread(target=self._read, daemon=True).start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [r for (t, r) in self.rows if t0 - 0.1 <= t <= t1 + 0.1] or [r for _, r in self.rows]
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+class Workload:
+    """Device-resident inputs/outputs of one step, plus pinned host copies for e2e."""
+
+    def __init__(self, torch, inputs, device):
+        t = torch
+        self.t = t
+        dev = device
+        kv = inputs.wkv4_kv(8, 1024, 768, 0, "bf16")
+        self.w4 = []
+        for layer in range(12):
+            w, u = inputs.wkv4_wu(768, layer + 1)
+            self.w4.append({"w": w.to(dev), "u": u.to(dev), "k": kv[0].to(dev).clone(),
+                            "v": kv[1].to(dev).clone(),
+                            "y": t.empty(8, 1024, 768, dtype=t.bfloat16, device=dev)})
+        self.h_kv = (kv[0].pin_memory(), kv[1].pin_memory())
+        x = inputs.wkv6_inputs(8, 4096, 32, 64, "bf16", seed=0, s0_std=0.1)
+        self.h_finch = {k: v.pin_memory() for k, v in x.items()}
+        self.finch = {k: v.to(dev) for k, v in x.items()}
+        self.finch["y"] = t.empty_like(self.finch["r"])
+        self.finch["sT"] = t.empty_like(self.finch["s0"])
+        x = inputs.wkv6_inputs(1, 16384, 64, 64, "bf16", seed=0)
+        self.h_long = {k: (v.pin_memory() if v is not None else None) for k, v in x.items()}
+        self.long = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
+        self.long["y"] = t.empty_like(self.long["r"])
+        self.long["s"] = [t.empty(1, 64, 64, 64, device=dev) for _ in range(2)]
+        x = inputs.wkv6_inputs(256, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
+        self.h_dec = {k: v.pin_memory() for k, v in x.items()}
+        self.dec = {k: v.to(dev) for k, v in x.items()}
+        self.dec["y"] = t.empty_like(self.dec["r"])
+
+    def step(self, ops, rec=None):
+        """One pass of the hot path; rec(name, fn) wraps each launch for timing."""
+        run = rec or (lambda name, fn: fn())
+        for L in self.w4:
+            run("wkv4_scan", lambda L=L: ops.wkv4_forward(L["w"], L["u"], L["k"], L["v"], y=L["y"]))
+        f = self.finch
+        run("wkv6_chunked_finch", lambda: ops.wkv6_forward(
+            f["r"], f["k"], f["v"], f["w"], f["u"], s0=f["s0"], y=f["y"], sT=f["sT"]))
+        g = self.long
+        for c in range(4):
+            sl = slice(c * 4096, (c + 1) * 4096)
+            s_in = None if c == 0 else g["s"][(c - 1) % 2]
+            s_out = g["s"][c % 2]
+            name = "wkv6_chunked_long_first" if c == 0 else "wkv6_chunked_long"
+            run(name, lambda sl=sl, s_in=s_in, s_out=s_out: ops.wkv6_forward(
+                g["r"][:, sl], g["k"][:, sl], g["v"][:, sl], g["w"][:, sl], g["u"], s0=s_in,
+                y=g["y"][:, sl], sT=s_out))
+        d = self.dec
+        run("wkv6_decode", lambda: ops.wkv6_forward(d["r"], d["k"], d["v"], d["w"], d["u"],
+                                                    s0=d["s0"], y=d["y"], sT=d["s0"]))
+
+    launches_per_step = 12 + 1 + 4 + 1
+
+
+def run_ours(args, rank, world, dist):
+    import torch
+    from wkv_recurrence_02_b200 import inputs, ops
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    ops.load()
+    wl = Workload(torch, inputs, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # warm-up
+    for _ in range(args.warmup):
+        wl.step(ops)
+    barrier()
+
+    # timed: whole steps, plus per-launch events for the per-kernel roofline
+    events = []
+
+    def rec(name, fn):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        events.append((name, a, b))
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    t_wall0 = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        wl.step(ops, rec)
+    e1.record(stream)
+    barrier()
+    t_wall1 = time.time()
+    sampler.stop()
+    ms = e0.elapsed_time(e1)
+    per = {}
+    for name, a, b in events:
+        per.setdefault(name, []).append(a.elapsed_time(b))
+
+    # end to end through the public API with host buffers: H2D of every input, D2H of results
+    e2e_ms, h2d, d2h = run_e2e(torch, ops, wl, stream, dev, max(3, min(args.steps, 10)), barrier)
+
+    ms_t = torch.tensor([ms, e2e_ms], device=dev)
+    if dist is not None:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max, e2e_max = ms_t.tolist()
+    status = ops.device_status()
+    if rank != 0:
+        return None
+
+    hbm, peak_kind = load_peaks()
+    fam = {}
+    for name, ts in per.items():
+        kern = "wkv6_chunked" if name.startswith("wkv6_chunked") else name
+        f = fam.setdefault(kern, {"ms": 0.0, "bytes": 0.0, "launches": 0})
+        f["ms"] += sum(ts)
+        f["bytes"] += BYTES[name] * len(ts)
+        f["launches"] += len(ts)
+    total_kernel_ms = sum(f["ms"] for f in fam.values())
+    dom = max(fam, key=lambda k: fam[k]["ms"])
+    d = fam[dom]
+    achieved = d["bytes"] / (d["ms"] * 1e-3) / 1e9
+    parts = {}
+    for name, ts in sorted(per.items()):
+        avg = sum(ts) / len(ts)
+        gbs = BYTES[name] / (avg * 1e-3) / 1e9
+        parts[name] = {"avg_us": round(avg * 1e3, 2), "launches": len(ts),
+                       "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+    for k, f in fam.items():
+        parts.setdefault("share", {})[k] = round(f["ms"] / total_kernel_ms, 4)
+    traffic = load_traffic(dom)
+    cpu = cpu_baseline(args.cpu_sample_scale) if (world == 1 and not args.skip_cpu) else None
+    line = {
+        "metric": METRIC, "value": world * STEP_TOKENS * args.steps / (ms_max * 1e-3),
+        "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch CPU generator)",
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
+                   "l2": "inputs larger than L2 (~2.4 GB per step per GPU); no flush",
+                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
+        "roofline": {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 4), "traffic": traffic},
+        "parts": parts,
+        "cpu_baseline": cpu,
+        "e2e": {"value": world * STEP_TOKENS / (e2e_max * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": Workload.launches_per_step * args.steps,
+        "clocks": sampler.summary(t_wall0, t_wall1),
+        "device_status": status,
+    }
+    return line
+
+
+def run_e2e(torch, ops, wl, stream, dev, steps, barrier):
+    """Same step through the public API with inputs/outputs in pinned host memory."""
+    h_y4 = [torch.empty(8, 1024, 768, dtype=torch.bfloat16).pin_memory() for _ in range(12)]
+    h_yf = torch.empty_like(wl.h_finch["r"]).pin_memory()
+    h_sf = torch.empty_like(wl.h_finch["s0"]).pin_memory()
+    h_yl = torch.empty_like(wl.h_long["r"]).pin_memory()
+    h_sl = torch.empty(1, 64, 64, 64).pin_memory()
+    h_yd = torch.empty_like(wl.h_dec["r"]).pin_memory()
+    h_sd = torch.empty_like(wl.h_dec["s0"]).pin_memory()
+    h2d = d2h = 0
+
+    def one():
+        nonlocal h2d, d2h
+        h2d = d2h = 0
+
+        def up(dst, src):
+            nonlocal h2d
+            dst.copy_(src, non_blocking=True)
+            h2d += src.numel() * src.element_size()
+
+        def down(dst, src):
+            nonlocal d2h
+            dst.copy_(src, non_blocking=True)
+            d2h += src.numel() * src.element_size()
+
+        for i, L in enumerate(wl.w4):
+            up(L["k"], wl.h_kv[0])
+            up(L["v"], wl.h_kv[1])
+            ops.wkv4_forward(L["w"], L["u"], L["k"], L["v"], y=L["y"])
+            down(h_y4[i], L["y"])
+        f, hf = wl.finch, wl.h_finch
+        for n in ("r", "k", "v", "w", "s0"):
+            up(f[n], hf[n])
+        ops.wkv6_forward(f["r"], f["k"], f["v"], f["w"], f["u"], s0=f["s0"], y=f["y"], sT=f["sT"])
+        down(h_yf, f["y"])
+        down(h_sf, f["sT"])
+        g, hg = wl.long, wl.h_long
+        for n in ("r", "k", "v", "w"):
+            up(g[n], hg[n])
+        for c in range(4):
+            sl = slice(c * 4096, (c + 1) * 4096)
+            ops.wkv6_forward(g["r"][:, sl], g["k"][:, sl], g["v"][:, sl], g["w"][:, sl], g["u"],
+                             s0=None if c == 0 else g["s"][(c - 1) % 2], y=g["y"][:, sl],
+                             sT=g["s"][c % 2])
+        down(h_yl, g["y"])
+        down(h_sl, g["s"][1])
+        d, hd = wl.dec, wl.h_dec
+        for n in ("r", "k", "v", "w", "s0"):
+            up(d[n], hd[n])
+        ops.wkv6_forward(d["r"], d["k"], d["v"], d["w"], d["u"], s0=d["s0"], y=d["y"], sT=d["s0"])
+        down(h_yd, d["y"])
+        down(h_sd, d["s0"])
+
+    one()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        one()
+    e1.record(stream)
+    barrier()
+    return e0.elapsed_time(e1) / steps, h2d, d2h
+
+
+def load_traffic(kernel):
+    """DRAM bytes per launch of `kernel` from the committed ncu summary, if present."""
+    p = os.path.join(HERE, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    return d.get(kernel)
+
+
+# --------------------------------------------------------------------------- CPU oracle
+
+def oracle_sample(scale=1.0):
+    """Time the fp64 oracle on a bounded sample of each part of the step.
+
+    Returns (seconds for the full step extrapolated by tokens, threads, description).
+    """
+    import numpy as np
+    import oracle
+    from wkv_recurrence_02_b200 import inputs
+
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    f64 = lambda t: t.float().double().numpy()  # noqa: E731
+    total = 0.0
+    desc = []
+    # WKV-4: layer 0 on B=1 of 8 (1024 tokens x 768 channels)
+    b4 = max(1, int(round(1 * scale)))
+    kv = inputs.wkv4_kv(b4, 1024, 768, 0, "bf16")
+    w, u = inputs.wkv4_wu(768, 1)
+    a = [f64(w), f64(u), f64(kv[0]), f64(kv[1])]
+    t0 = time.perf_counter()
+    oracle.wkv4(*a)
+    dt = time.perf_counter() - t0
+    total += dt * TOKENS_WKV4 / (b4 * 1024)
+    desc.append(f"wkv4 B{b4} T1024 C768 x1 layer")
+    # WKV-6 prefill: H heads of a T=4096 sequence, scaled to Finch (H=32, B=8) and 7B (H=64, B=1)
+    hs = max(1, int(round(4 * scale)))
+    x = inputs.wkv6_inputs(1, 4096, hs, 64, "bf16", seed=0, s0_std=0.1)
+    a = [f64(x[n]) for n in ("r", "k", "v", "w")]
+    t0 = time.perf_counter()
+    oracle.wkv6(*a, f64(x["u"]), s0=np.asarray(x["s0"].double().numpy()))
+    dt = time.perf_counter() - t0
+    per_head_token = dt / (hs * 4096)
+    total += per_head_token * (TOKENS_FINCH * 32 + TOKENS_LONG * 64)
+    desc.append(f"wkv6 B1 T4096 H{hs}")
+    # decode: B rows of a T=1 step
+    bd = max(1, int(round(32 * scale)))
+    x = inputs.wkv6_inputs(bd, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
+    t0 = time.perf_counter()
+    oracle.wkv6(*[f64(x[n]) for n in ("r", "k", "v", "w")], f64(x["u"]), s0=x["s0"].double().numpy())
+    dt = time.perf_counter() - t0
+    total += dt * TOKENS_DECODE / bd
+    desc.append(f"wkv6 decode B{bd} H64")
+    return total, threads, "; ".join(desc) + "; extrapolated to one step by tokens (x heads)"
+
+
+def cpu_baseline(scale):
+    step_s, threads, desc = oracle_sample(scale)
+    return {"value": STEP_TOKENS / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": desc}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(args.cpu_sample_scale * 0.25)
+    times = []
+    threads, desc = None, None
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        s, threads, desc = oracle_sample(args.cpu_sample_scale * 0.25)
+        times.append(s)
+    wall = time.perf_counter() - t0
+    step_s = sum(times) / len(times)
+    value = STEP_TOKENS / step_s
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "impl": "reference",
+        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
+                   "sampled_wall_s": round(wall, 2)},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample-scale", type=float, default=1.0)
+    ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as tdist
+        torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist = tdist
+    try:
+        line = run_ours(args, rank, world, dist)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if dist is not None:
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

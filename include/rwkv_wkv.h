@@ -1,0 +1,154 @@
+/*
+ * rwkv_wkv.h -- C ABI of libwkv.so: the WKV time-mixing recurrences of RWKV-4 and
+ * Eagle/Finch (RWKV-5/6) on NVIDIA B200 (sm_100a).
+ *
+ * Sources (page title, section):
+ *  [R4]   "RWKV: Reinventing RNNs for the Transformer Era" (Chinese translation):
+ *         section "类 Transformer 的并行化" (time-parallel mode: the WKV update is a
+ *         serial scan of cost O(BTd)); section "梯度稳定性和层堆叠" (single-step
+ *         time-dependent softmax); section "利用时间结构进行时序数据处理" (time decay
+ *         e^{-w} and bonus e^{u} of eq. 14); section "类 RNN 的序列解码" (RNN-mode
+ *         decoding with constant memory per token).
+ *  [E412] "RWKV-5/6 (Eagle and Finch)", section 4.1.2 (Eagle time mixing): matrix-valued
+ *         state s = sum of k^T v, decayed per key channel by w, gain u on the current
+ *         token, receptance as a query; w = exp(-exp(omega)) in (0,1).  Section 4 fixes
+ *         row vectors with matrices acting on the right.
+ *  [F422] same page, section 4.2.2 (Finch time mixing): w_t varies per token and channel.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller, dense and row-major
+ *    with the channel index innermost.  The library never allocates, frees or retains
+ *    them; it reads inputs and writes outputs asynchronously on the calling thread's
+ *    stream (rwkv_set_stream) and returns before the GPU has finished.
+ *  - bf16 tensors are passed as uint16_t bit patterns (IEEE bfloat16, round-to-nearest-
+ *    even on output).  Accumulation is fp32 throughout.
+ *  - Every tensor pointer must be 16-byte aligned (RWKV_ERR_ALIGN otherwise).
+ *  - Sizes are int64_t and must be >= 0 (RWKV_ERR_SHAPE otherwise).  A call with no
+ *    output element to produce returns RWKV_OK without launching; for T == 0 the final
+ *    state is still written (a copy of s0, or the empty state).
+ *  - A pointer may be NULL only where stated, or when the tensor it names is empty.
+ *  - Outputs must not overlap any input (RWKV_ERR_ALIAS), except that a state output
+ *    may be the very same pointer as the state input (in-place state update).
+ *  - Return value: RWKV_OK (0) or a negative rwkv_status.  Argument errors are found
+ *    on the host before any CUDA call.  RWKV_ERR_CUDA means a launch or CUDA runtime
+ *    call failed; rwkv_last_error() has the text.  Faults inside a kernel that the
+ *    kernel itself detects (e.g. a bounded wait that ran out) are reported through the
+ *    device status word, read with rwkv_get_device_status().
+ *  - The library allocates no device memory of its own: its one status word is a
+ *    statically allocated __device__ variable.
+ */
+#ifndef RWKV_WKV_H
+#define RWKV_WKV_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RWKV_ABI_VERSION 1
+
+typedef enum rwkv_status {
+    RWKV_OK = 0,
+    RWKV_ERR_NULL = -1,        /* a required pointer is NULL                          */
+    RWKV_ERR_SHAPE = -2,       /* a negative size, or a size product overflows        */
+    RWKV_ERR_UNSUPPORTED = -3, /* e.g. WKV-6 head size N != 64                        */
+    RWKV_ERR_ALIAS = -4,       /* an output overlaps an input                         */
+    RWKV_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed         */
+    RWKV_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (device status)  */
+    RWKV_ERR_ALIGN = -7,       /* a tensor pointer is not 16-byte aligned             */
+    RWKV_ERR_ARG = -8          /* another invalid argument (e.g. unknown option)      */
+} rwkv_status;
+
+/* ------------------------------------------------------------------ RWKV-4 WKV [R4]
+ * Per batch row b and channel c, with keys k_t, values v_t:
+ *   y_t = ( sum_{i<t} e^{-(t-1-i) w_c + k_i} v_i + e^{u_c + k_t} v_t )
+ *       / ( sum_{i<t} e^{-(t-1-i) w_c + k_i}     + e^{u_c + k_t}     )
+ * evaluated in the running-maximum (time-dependent softmax) form, so k may be large.
+ *   w, u : [C] fp32.  w is the positive decay RATE (per-step factor e^{-w}); the
+ *          library does not exponentiate a learned parameter for you.
+ *   k, v : [B, T, C];  y : [B, T, C] (same dtype as k).
+ */
+int rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C,
+                      const float *w, const float *u,
+                      const float *k, const float *v, float *y);
+int rwkv_wkv4_forward_bf16(int64_t B, int64_t T, int64_t C,
+                           const float *w, const float *u,
+                           const uint16_t *k, const uint16_t *v, uint16_t *y);
+
+/* RWKV-4 WKV with state carry, so a sequence can be split across calls exactly
+ * ([R4] RNN-mode decoding).  State layout s0/sT: [B, 3, C] fp32 = (a, b, p) per
+ * channel, meaning numerator = a e^p and denominator = b e^p of the decayed past sums
+ * after the last token processed.  An empty state has a = b = 0 (p is then ignored;
+ * the library writes p = -1e30 for it).  s0 NULL = empty state; sT NULL = not written;
+ * sT may equal s0.  The (a, b, p) triple is not unique: compare states through
+ * a e^{p-P}, b e^{p-P} at a common P. */
+int rwkv_wkv4_forward_state(int64_t B, int64_t T, int64_t C,
+                            const float *w, const float *u,
+                            const float *k, const float *v,
+                            const float *s0, float *y, float *sT);
+int rwkv_wkv4_forward_state_bf16(int64_t B, int64_t T, int64_t C,
+                                 const float *w, const float *u,
+                                 const uint16_t *k, const uint16_t *v,
+                                 const float *s0, uint16_t *y, float *sT);
+
+/* ------------------------------------------------------- Eagle/Finch WKV-6 [E412][F422]
+ * Per batch row b and head h, state S (N x N, row i = key channel, column j = value
+ * channel), for t = 0..T-1:
+ *   y_t[j] = sum_i r_t[i] ( S[i][j] + u[i] k_t[i] v_t[j] )
+ *   S[i][j] <- w_t[i] S[i][j] + k_t[i] v_t[j]
+ * with S = s0 before the first token and sT = S after the last.
+ *   r, k, v, w, y : [B, T, H, N]; w_t in (0, 1] (Eagle: constant over t; Finch: per
+ *                   token).  w outside (0, 1] is outside the contract: results are then
+ *                   unspecified but the call never faults.
+ *   u             : [H, N] fp32.
+ *   s0, sT        : [B, H, N, N] fp32.  s0 NULL = zero state; sT NULL = not written;
+ *                   sT may equal s0 (in-place).
+ *   N must be 64 (RWKV_ERR_UNSUPPORTED otherwise).
+ * fp32 inputs run a serial fp32 kernel (SIMT).  bf16 inputs with T > 1 run the chunked
+ * tensor-core kernel (64-token chunks, bf16 operands, fp32 accumulation, state in fp32);
+ * T == 1 runs the bandwidth-bound decode kernel.
+ */
+int rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N,
+                      const float *r, const float *k, const float *v, const float *w,
+                      const float *u, const float *s0, float *y, float *sT);
+int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
+                           const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                           const uint16_t *w, const float *u, const float *s0,
+                           uint16_t *y, float *sT);
+
+/* Kernel choice for WKV-6 on the calling thread: RWKV_WKV6_AUTO (default, as above),
+ * RWKV_WKV6_SERIAL (always the serial kernel), RWKV_WKV6_CHUNKED (the chunked kernel
+ * for bf16 whatever T; ignored for fp32).  Returns RWKV_OK or RWKV_ERR_ARG. */
+#define RWKV_WKV6_AUTO 0
+#define RWKV_WKV6_SERIAL 1
+#define RWKV_WKV6_CHUNKED 2
+int rwkv_set_wkv6_algo(int algo);
+int rwkv_get_wkv6_algo(void);
+
+/* ------------------------------------------------------------------ runtime plumbing */
+/* Stream used by launches from the calling thread (a cudaStream_t; NULL = legacy
+ * default stream).  Thread-local; the caller keeps the stream alive. */
+void rwkv_set_stream(void *cuda_stream);
+void *rwkv_get_stream(void);
+
+/* Synchronises the calling thread's stream, then returns and clears the device status
+ * word of the current device: RWKV_OK, or the first error a kernel recorded since the
+ * last call (e.g. RWKV_ERR_TIMEOUT).  Returns RWKV_ERR_CUDA if the synchronisation
+ * itself fails. */
+int rwkv_get_device_status(void);
+
+/* Static description of a status code. */
+const char *rwkv_status_string(int status);
+
+/* Thread-local text of the last failing call's error ("" if none). */
+const char *rwkv_last_error(void);
+
+/* RWKV_ABI_VERSION of the loaded library. */
+int rwkv_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RWKV_WKV_H */

@@ -1,0 +1,112 @@
+"""The C ABI without a GPU: the library loads, exports every declared symbol, and
+rejects bad arguments on the host before touching CUDA.
+
+Pointers passed here are fake addresses that the library must never dereference:
+every call either fails validation or has nothing to compute.
+"""
+import ctypes
+
+import pytest
+import torch
+
+from wkv_recurrence_02_b200 import build, ops
+
+FAKE = 0x7F0000000000  # 16-byte aligned, never dereferenced
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return ops.load()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = ops.declared_functions()
+    assert len(names) >= 14
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_and_strings(lib):
+    assert lib.rwkv_abi_version() == 1
+    for code, name in ops.STATUS_NAMES.items():
+        assert lib.rwkv_status_string(code)
+    assert lib.rwkv_status_string(12345) == b"unknown status"
+
+
+def _p(off=0):
+    return ctypes.c_void_p(FAKE + off)
+
+
+def test_wkv4_validation(lib):
+    f, fb = lib.rwkv_wkv4_forward, lib.rwkv_wkv4_forward_bf16
+    assert f(-1, 4, 4, _p(), _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(4 << 20)) == -2
+    assert f(1, 4, 4, None, _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(4 << 20)) == -1
+    assert f(1, 4, 4, _p(), _p(1 << 20), None, _p(3 << 20), _p(4 << 20)) == -1
+    assert f(1, 4, 4, _p(4), _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(4 << 20)) == -7
+    # y overlapping k
+    assert fb(1, 4, 4, _p(), _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(2 << 20)) == -4
+    # nothing to compute: OK without CUDA
+    assert f(0, 4, 4, None, None, None, None, None) == 0
+    assert f(3, 0, 4, None, None, None, None, None) == 0
+    assert f(3, 7, 0, None, None, None, None, None) == 0
+    # size product overflow
+    assert f(1 << 40, 1 << 40, 4, _p(), _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(4 << 20)) == -2
+
+
+def test_wkv4_state_validation(lib):
+    f = lib.rwkv_wkv4_forward_state
+    args = [_p(), _p(1 << 20), _p(2 << 20), _p(3 << 20)]
+    # sT partially overlapping s0
+    assert f(2, 4, 8, *args, _p(5 << 20), _p(6 << 20), _p((5 << 20) + 16)) == -4
+    # sT overlapping k
+    assert f(2, 4, 8, *args, _p(5 << 20), _p(6 << 20), _p(2 << 20)) == -4
+    # y overlapping s0
+    assert f(2, 4, 8, *args, _p(5 << 20), _p(5 << 20), _p(7 << 20)) == -4
+
+
+def test_wkv6_validation(lib):
+    f = lib.rwkv_wkv6_forward_bf16
+    base = [_p(i << 24) for i in range(8)]
+    assert f(1, 4, 2, 32, *base) == -3            # N != 64
+    assert f(1, 4, 2, -64, *base) == -2
+    assert f(1, 4, 2, 64, None, *base[1:]) == -1  # r null
+    bad = list(base)
+    bad[2] = _p((2 << 24) + 8)
+    assert f(1, 4, 2, 64, *bad) == -7             # misaligned v
+    alias = list(base)
+    alias[6] = base[0]                            # y == r
+    assert f(1, 4, 2, 64, *alias) == -4
+    part = list(base)
+    part[7] = _p((5 << 24) + 64)                  # sT inside s0, not equal
+    assert f(1, 4, 2, 64, *part) == -4
+    assert f(0, 4, 2, 64, *([None] * 8)) == 0     # empty: OK without CUDA
+    assert f(2, 4, 0, 64, *([None] * 8)) == 0
+
+
+def test_algo_selection(lib):
+    assert lib.rwkv_set_wkv6_algo(7) == -8
+    for a in (1, 2, 0):
+        assert lib.rwkv_set_wkv6_algo(a) == 0
+        assert lib.rwkv_get_wkv6_algo() == a
+
+
+def test_stream_is_thread_local_setting(lib):
+    lib.rwkv_set_stream(ctypes.c_void_p(0x1234))
+    assert lib.rwkv_get_stream() == 0x1234
+    lib.rwkv_set_stream(None)
+    assert not lib.rwkv_get_stream()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="only meaningful without a GPU")
+def test_valid_call_without_gpu_fails_cleanly(lib):
+    """With no CUDA device a valid call must return RWKV_ERR_CUDA, not crash or fall back."""
+    rc = lib.rwkv_wkv4_forward(1, 4, 16, _p(), _p(1 << 20), _p(2 << 20), _p(3 << 20), _p(4 << 20))
+    assert rc == -5
+    assert lib.rwkv_last_error()
+
+
+def test_binding_refuses_cpu_tensors(lib):
+    k = torch.zeros(1, 4, 16)
+    with pytest.raises(TypeError):
+        ops.wkv4_forward(torch.zeros(16), torch.zeros(16), k, k)

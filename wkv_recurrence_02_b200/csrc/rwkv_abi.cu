@@ -1,0 +1,270 @@
+// rwkv_abi.cu -- the extern "C" boundary of libwkv.so (declared in include/rwkv_wkv.h).
+//
+// Host-side argument validation (before any CUDA call), kernel selection, the
+// thread-local stream and the device status word.  Every step of the recurrences
+// runs in the CUDA kernels of the other files; there is no CPU fallback.
+#include "rwkv_wkv.h"
+#include "wkv_internal.cuh"
+
+#include <mutex>
+#include <stdio.h>
+#include <string.h>
+
+namespace {
+
+thread_local cudaStream_t tl_stream = nullptr;
+thread_local int tl_wkv6_algo = RWKV_WKV6_AUTO;
+thread_local char tl_err[256] = "";
+
+// The library's only device memory: one status word per device, allocated statically.
+__device__ int g_device_status = 0;
+
+constexpr int kMaxDevices = 64;
+std::mutex g_status_mu;
+int *g_status_ptr[kMaxDevices] = {nullptr};
+
+int fail(int code, const char *fmt, const char *detail = "")
+{
+    snprintf(tl_err, sizeof(tl_err), fmt, detail);
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char *where)
+{
+    snprintf(tl_err, sizeof(tl_err), "%s: %s", where, cudaGetErrorString(e));
+    return RWKV_ERR_CUDA;
+}
+
+// Device address of the status word on the current device (looked up once per device).
+int status_word(int **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (dev < 0 || dev >= kMaxDevices) return fail(RWKV_ERR_CUDA, "device index out of range%s");
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_device_status);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(status)");
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    *out = g_status_ptr[dev];
+    return RWKV_OK;
+}
+
+// ---- validation helpers -----------------------------------------------------------
+
+bool mul_ok(int64_t a, int64_t b, int64_t *out)
+{
+    if (a < 0 || b < 0) return false;
+    if (a != 0 && b > INT64_MAX / 4 / a) return false;  // keep byte counts representable
+    *out = a * b;
+    return true;
+}
+
+struct Span {
+    const void *p;
+    int64_t bytes;
+};
+
+bool overlap(Span a, Span b)
+{
+    if (!a.p || !b.p || a.bytes <= 0 || b.bytes <= 0) return false;
+    uintptr_t a0 = (uintptr_t)a.p, a1 = a0 + (uintptr_t)a.bytes;
+    uintptr_t b0 = (uintptr_t)b.p, b1 = b0 + (uintptr_t)b.bytes;
+    return a0 < b1 && b0 < a1;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+// ---- WKV-4 -------------------------------------------------------------------------
+
+int wkv4_entry(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+               const void *k, const void *v, const float *s0, void *y, float *sT,
+               bool bf16, bool with_state)
+{
+    tl_err[0] = 0;
+    if (B < 0 || T < 0 || C < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
+    int64_t BT, n, ns;
+    if (!mul_ok(B, T, &BT) || !mul_ok(BT, C, &n) || !mul_ok(B * 3, C, &ns))
+        return fail(RWKV_ERR_SHAPE, "size product overflows%s");
+    const int64_t esz = bf16 ? 2 : 4;
+    const bool want_state = with_state && sT != nullptr;
+    if (n == 0 && !(want_state && ns > 0)) return RWKV_OK;
+    if (n > 0 && (!k || !v || !y)) return fail(RWKV_ERR_NULL, "k, v and y must be non-null%s");
+    if (C > 0 && B > 0 && (!w || !u)) return fail(RWKV_ERR_NULL, "w and u must be non-null%s");
+    const void *ptrs[] = {w, u, k, v, y, s0, sT};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(RWKV_ERR_ALIGN, "tensor pointers must be 16-byte aligned%s");
+    Span sy{y, n * esz}, sk{k, n * esz}, sv{v, n * esz}, sw{w, C * 4}, su{u, C * 4};
+    Span ss0{s0, with_state ? ns * 4 : 0}, ssT{sT, with_state ? ns * 4 : 0};
+    if (overlap(sy, sk) || overlap(sy, sv) || overlap(sy, sw) || overlap(sy, su) ||
+        overlap(sy, ss0) || overlap(sy, ssT))
+        return fail(RWKV_ERR_ALIAS, "y overlaps another tensor%s");
+    if (with_state && sT) {
+        if (overlap(ssT, sk) || overlap(ssT, sv) || overlap(ssT, sw) || overlap(ssT, su))
+            return fail(RWKV_ERR_ALIAS, "sT overlaps an input%s");
+        if (s0 && s0 != sT && overlap(ssT, ss0))
+            return fail(RWKV_ERR_ALIAS, "sT partially overlaps s0%s");
+    }
+    int *status = nullptr;
+    int rc = status_word(&status);
+    if (rc) return rc;
+    wkv::Wkv4Args a{B, T, C, w, u, k, v, with_state ? s0 : nullptr, y,
+                    with_state ? sT : nullptr, bf16, status};
+    cudaError_t e = wkv::wkv4_launch(a, tl_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wkv4 launch");
+    return RWKV_OK;
+}
+
+// ---- WKV-6 -------------------------------------------------------------------------
+
+int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
+               const void *v, const void *w, const float *u, const float *s0, void *y,
+               float *sT, bool bf16)
+{
+    tl_err[0] = 0;
+    if (B < 0 || T < 0 || H < 0 || N < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
+    int64_t BT, BTH, n, BH, ns;
+    if (!mul_ok(B, T, &BT) || !mul_ok(BT, H, &BTH) || !mul_ok(BTH, N, &n) ||
+        !mul_ok(B, H, &BH) || !mul_ok(BH, N * N, &ns))
+        return fail(RWKV_ERR_SHAPE, "size product overflows%s");
+    if (n == 0 && !(sT && ns > 0)) return RWKV_OK;
+    if (N != 64) return fail(RWKV_ERR_UNSUPPORTED, "head size N must be 64%s");
+    const int64_t esz = bf16 ? 2 : 4;
+    if (n > 0 && (!r || !k || !v || !w || !y))
+        return fail(RWKV_ERR_NULL, "r, k, v, w and y must be non-null%s");
+    if (BH > 0 && !u) return fail(RWKV_ERR_NULL, "u must be non-null%s");
+    const void *ptrs[] = {r, k, v, w, u, s0, y, sT};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(RWKV_ERR_ALIGN, "tensor pointers must be 16-byte aligned%s");
+    Span sy{y, n * esz}, sr{r, n * esz}, sk{k, n * esz}, sv{v, n * esz}, sw{w, n * esz};
+    Span su{u, H * N * 4}, ss0{s0, ns * 4}, ssT{sT, ns * 4};
+    const Span ins[] = {sr, sk, sv, sw, su};
+    for (const Span &s : ins)
+        if (overlap(sy, s)) return fail(RWKV_ERR_ALIAS, "y overlaps an input%s");
+    if (overlap(sy, ss0) || overlap(sy, ssT)) return fail(RWKV_ERR_ALIAS, "y overlaps a state%s");
+    if (sT) {
+        for (const Span &s : ins)
+            if (overlap(ssT, s)) return fail(RWKV_ERR_ALIAS, "sT overlaps an input%s");
+        if (s0 && s0 != sT && overlap(ssT, ss0))
+            return fail(RWKV_ERR_ALIAS, "sT partially overlaps s0%s");
+    }
+    int *status = nullptr;
+    int rc = status_word(&status);
+    if (rc) return rc;
+    if (T == 0) {  // nothing to scan: sT = s0, or the zero state
+        if (!sT || sT == s0) return RWKV_OK;
+        cudaError_t e = s0 ? cudaMemcpyAsync(sT, s0, ns * 4, cudaMemcpyDeviceToDevice, tl_stream)
+                           : cudaMemsetAsync(sT, 0, ns * 4, tl_stream);
+        return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "T=0 state copy");
+    }
+    wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, bf16, status};
+    cudaError_t e;
+    int algo = tl_wkv6_algo;
+    if (algo == RWKV_WKV6_SERIAL || !bf16)
+        e = (T == 1 && algo != RWKV_WKV6_SERIAL) ? wkv::wkv6_decode_launch(a, tl_stream)
+                                                 : wkv::wkv6_serial_launch(a, tl_stream);
+    else if (algo == RWKV_WKV6_CHUNKED || T > 1)
+        e = wkv::wkv6_chunked_launch(a, tl_stream);
+    else
+        e = wkv::wkv6_decode_launch(a, tl_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wkv6 launch");
+    return RWKV_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int rwkv_wkv4_forward(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                      const float *k, const float *v, float *y)
+{
+    return wkv4_entry(B, T, C, w, u, k, v, nullptr, y, nullptr, false, false);
+}
+
+int rwkv_wkv4_forward_bf16(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                           const uint16_t *k, const uint16_t *v, uint16_t *y)
+{
+    return wkv4_entry(B, T, C, w, u, k, v, nullptr, y, nullptr, true, false);
+}
+
+int rwkv_wkv4_forward_state(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
+                            const float *k, const float *v, const float *s0, float *y,
+                            float *sT)
+{
+    return wkv4_entry(B, T, C, w, u, k, v, s0, y, sT, false, true);
+}
+
+int rwkv_wkv4_forward_state_bf16(int64_t B, int64_t T, int64_t C, const float *w,
+                                 const float *u, const uint16_t *k, const uint16_t *v,
+                                 const float *s0, uint16_t *y, float *sT)
+{
+    return wkv4_entry(B, T, C, w, u, k, v, s0, y, sT, true, true);
+}
+
+int rwkv_wkv6_forward(int64_t B, int64_t T, int64_t H, int64_t N, const float *r,
+                      const float *k, const float *v, const float *w, const float *u,
+                      const float *s0, float *y, float *sT)
+{
+    return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, false);
+}
+
+int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,
+                           const uint16_t *k, const uint16_t *v, const uint16_t *w,
+                           const float *u, const float *s0, uint16_t *y, float *sT)
+{
+    return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, true);
+}
+
+int rwkv_set_wkv6_algo(int algo)
+{
+    if (algo != RWKV_WKV6_AUTO && algo != RWKV_WKV6_SERIAL && algo != RWKV_WKV6_CHUNKED)
+        return RWKV_ERR_ARG;
+    tl_wkv6_algo = algo;
+    return RWKV_OK;
+}
+
+int rwkv_get_wkv6_algo(void) { return tl_wkv6_algo; }
+
+void rwkv_set_stream(void *cuda_stream) { tl_stream = static_cast<cudaStream_t>(cuda_stream); }
+
+void *rwkv_get_stream(void) { return tl_stream; }
+
+int rwkv_get_device_status(void)
+{
+    int *p = nullptr;
+    int rc = status_word(&p);
+    if (rc) return rc;
+    cudaError_t e = cudaStreamSynchronize(tl_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+    int value = 0, zero = 0;
+    e = cudaMemcpy(&value, p, sizeof(int), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return cuda_fail(e, "status read");
+    e = cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+    return value;
+}
+
+const char *rwkv_status_string(int status)
+{
+    switch (status) {
+    case RWKV_OK: return "ok";
+    case RWKV_ERR_NULL: return "required pointer is null";
+    case RWKV_ERR_SHAPE: return "invalid size";
+    case RWKV_ERR_UNSUPPORTED: return "unsupported configuration";
+    case RWKV_ERR_ALIAS: return "output overlaps an input";
+    case RWKV_ERR_CUDA: return "CUDA error";
+    case RWKV_ERR_TIMEOUT: return "device-side wait timed out";
+    case RWKV_ERR_ALIGN: return "pointer not 16-byte aligned";
+    case RWKV_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+    }
+}
+
+const char *rwkv_last_error(void) { return tl_err; }
+
+int rwkv_abi_version(void) { return RWKV_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,48 @@
+// Internal declarations shared by the ABI layer and the kernel files of libwkv.so.
+// Nothing here is part of the public ABI (include/rwkv_wkv.h is).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace wkv {
+
+// Status codes written by kernels into the device status word (same values as rwkv_status).
+constexpr int kStatusTimeout = -6;
+
+// Record the first device-side error; later errors keep the first one.
+__device__ __forceinline__ void record_status(int *status, int code)
+{
+    if (status) atomicCAS(status, 0, code);
+}
+
+struct Wkv4Args {
+    int64_t B, T, C;
+    const float *w, *u;     // [C]
+    const void *k, *v;      // [B,T,C] fp32 or bf16
+    const float *s0;        // [B,3,C] or null
+    void *y;                // [B,T,C]
+    float *sT;              // [B,3,C] or null
+    bool bf16;
+    int *status;
+};
+
+struct Wkv6Args {
+    int64_t B, T, H, N;
+    const void *r, *k, *v, *w;  // [B,T,H,N] fp32 or bf16
+    const float *u;             // [H,N]
+    const float *s0;            // [B,H,N,N] or null
+    void *y;                    // [B,T,H,N]
+    float *sT;                  // [B,H,N,N] or null
+    bool bf16;
+    int *status;
+};
+
+// Each launcher returns the cudaError_t of its launch(es).
+cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s);
+cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s);
+cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s);
+cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s);
+
+}  // namespace wkv

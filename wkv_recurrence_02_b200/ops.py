@@ -1,0 +1,182 @@
+"""Thin ctypes binding of libwkv.so (include/rwkv_wkv.h) for torch CUDA tensors.
+
+Argument marshalling only: every step of the recurrences runs in the library's CUDA
+kernels.  There is no CPU fallback -- if the library is not built, or a tensor is
+not on a CUDA device, the call raises.
+
+Functions mirror the C entry points:
+  wkv4_forward(w, u, k, v, s0=None, want_state=False)   -> y            | (y, sT)
+  wkv6_forward(r, k, v, w, u, s0=None, want_state=True) -> (y, sT)      | y
+The calls are asynchronous on torch's current CUDA stream.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwkv.so")
+HEADER = os.path.join(os.path.dirname(_HERE), "include", "rwkv_wkv.h")
+
+RWKV_OK = 0
+STATUS_NAMES = {0: "RWKV_OK", -1: "RWKV_ERR_NULL", -2: "RWKV_ERR_SHAPE", -3: "RWKV_ERR_UNSUPPORTED",
+                -4: "RWKV_ERR_ALIAS", -5: "RWKV_ERR_CUDA", -6: "RWKV_ERR_TIMEOUT",
+                -7: "RWKV_ERR_ALIGN", -8: "RWKV_ERR_ARG"}
+ALGOS = {"auto": 0, "serial": 1, "chunked": 2}
+
+_i64 = ctypes.c_int64
+_vp = ctypes.c_void_p
+_lib = None
+
+
+class WkvError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"{STATUS_NAMES.get(code, code)}: {msg}")
+        self.code = code
+
+
+def declared_functions(header: str = HEADER):
+    """Names of the functions include/rwkv_wkv.h declares."""
+    with open(header) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(rwkv_[a-z0-9_]+)\s*\(", text)))
+
+
+def load(path: str = LIB_PATH):
+    """Load libwkv.so (once) and declare its signatures.  Raises if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is not built: run `python -m wkv_recurrence_02_b200.build`")
+    lib = ctypes.CDLL(path)
+    wkv4 = [_i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp]
+    wkv4s = [_i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    wkv6 = [_i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]
+    for name, args in [("rwkv_wkv4_forward", wkv4), ("rwkv_wkv4_forward_bf16", wkv4),
+                       ("rwkv_wkv4_forward_state", wkv4s), ("rwkv_wkv4_forward_state_bf16", wkv4s),
+                       ("rwkv_wkv6_forward", wkv6), ("rwkv_wkv6_forward_bf16", wkv6)]:
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = ctypes.c_int
+    lib.rwkv_set_stream.argtypes = [_vp]
+    lib.rwkv_set_stream.restype = None
+    lib.rwkv_get_stream.argtypes = []
+    lib.rwkv_get_stream.restype = _vp
+    lib.rwkv_set_wkv6_algo.argtypes = [ctypes.c_int]
+    lib.rwkv_set_wkv6_algo.restype = ctypes.c_int
+    lib.rwkv_get_wkv6_algo.argtypes = []
+    lib.rwkv_get_wkv6_algo.restype = ctypes.c_int
+    lib.rwkv_get_device_status.argtypes = []
+    lib.rwkv_get_device_status.restype = ctypes.c_int
+    lib.rwkv_status_string.argtypes = [ctypes.c_int]
+    lib.rwkv_status_string.restype = ctypes.c_char_p
+    lib.rwkv_last_error.argtypes = []
+    lib.rwkv_last_error.restype = ctypes.c_char_p
+    lib.rwkv_abi_version.argtypes = []
+    lib.rwkv_abi_version.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(rc):
+    if rc != RWKV_OK:
+        lib = load()
+        raise WkvError(rc, (lib.rwkv_last_error() or b"").decode() or
+                       lib.rwkv_status_string(rc).decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _cuda(t, name, dtype=None, shape=None):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    return t
+
+
+def _use_current_stream(lib, device):
+    lib.rwkv_set_stream(ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream))
+
+
+def wkv4_forward(w, u, k, v, s0=None, want_state=False, y=None, sT=None):
+    """RWKV-4 WKV.  k, v: [B,T,C] fp32|bf16; w, u: [C] fp32; s0: [B,3,C] fp32 or None."""
+    lib = load()
+    _cuda(k, "k")
+    B, T, C = k.shape
+    dt = k.dtype
+    if dt not in (torch.float32, torch.bfloat16):
+        raise TypeError("k must be float32 or bfloat16")
+    _cuda(v, "v", dt, (B, T, C))
+    _cuda(w, "w", torch.float32, (C,))
+    _cuda(u, "u", torch.float32, (C,))
+    _cuda(s0, "s0", torch.float32, (B, 3, C))
+    if y is None:
+        y = torch.empty_like(k)
+    _cuda(y, "y", dt, (B, T, C))
+    stateful = want_state or s0 is not None or sT is not None
+    if stateful and sT is None and want_state:
+        sT = torch.empty(B, 3, C, device=k.device, dtype=torch.float32)
+    _cuda(sT, "sT", torch.float32, (B, 3, C))
+    _use_current_stream(lib, k.device)
+    bf = dt == torch.bfloat16
+    if stateful:
+        fn = lib.rwkv_wkv4_forward_state_bf16 if bf else lib.rwkv_wkv4_forward_state
+        _check(fn(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(s0), _ptr(y), _ptr(sT)))
+    else:
+        fn = lib.rwkv_wkv4_forward_bf16 if bf else lib.rwkv_wkv4_forward
+        _check(fn(B, T, C, _ptr(w), _ptr(u), _ptr(k), _ptr(v), _ptr(y)))
+    return (y, sT) if want_state else y
+
+
+def wkv6_forward(r, k, v, w, u, s0=None, want_state=True, y=None, sT=None, algo=None):
+    """Eagle/Finch WKV-6.  r,k,v,w: [B,T,H,N] fp32|bf16; u: [H,N] fp32; s0: [B,H,N,N] fp32.
+
+    algo: None (library default), "auto", "serial" or "chunked" (this call only).
+    """
+    lib = load()
+    _cuda(r, "r")
+    B, T, H, N = r.shape
+    dt = r.dtype
+    if dt not in (torch.float32, torch.bfloat16):
+        raise TypeError("r must be float32 or bfloat16")
+    for name, t in (("k", k), ("v", v), ("w", w)):
+        _cuda(t, name, dt, (B, T, H, N))
+    _cuda(u, "u", torch.float32, (H, N))
+    _cuda(s0, "s0", torch.float32, (B, H, N, N))
+    if y is None:
+        y = torch.empty_like(r)
+    _cuda(y, "y", dt, (B, T, H, N))
+    if sT is None and want_state:
+        sT = torch.empty(B, H, N, N, device=r.device, dtype=torch.float32)
+    _cuda(sT, "sT", torch.float32, (B, H, N, N))
+    _use_current_stream(lib, r.device)
+    fn = lib.rwkv_wkv6_forward_bf16 if dt == torch.bfloat16 else lib.rwkv_wkv6_forward
+    prev = None
+    if algo is not None:
+        prev = lib.rwkv_get_wkv6_algo()
+        _check(lib.rwkv_set_wkv6_algo(ALGOS[algo]))
+    try:
+        _check(fn(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(y),
+                  _ptr(sT)))
+    finally:
+        if prev is not None:
+            lib.rwkv_set_wkv6_algo(prev)
+    return (y, sT) if want_state else y
+
+
+def device_status() -> int:
+    """Synchronise the current stream and return/clear the device status word."""
+    lib = load()
+    _use_current_stream(lib, torch.cuda.current_device())
+    return int(lib.rwkv_get_device_status())
