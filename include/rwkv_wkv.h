@@ -126,6 +126,13 @@ int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
 int rwkv_set_wkv6_algo(int algo);
 int rwkv_get_wkv6_algo(void);
 
+/* Test hook for the failure path (process-wide).  While enabled, every chunked WKV-6
+ * launch first waits on a barrier that nothing signals, with a short bound; the wait
+ * runs out, the kernel records RWKV_ERR_TIMEOUT in the device status word, releases its
+ * resources and returns without computing (outputs are then unspecified).  No fault or
+ * hang is involved.  Returns the previous setting. */
+int rwkv_debug_inject_timeout(int enable);
+
 /* ------------------------------------------------------------------ runtime plumbing */
 /* Stream used by launches from the calling thread (a cudaStream_t; NULL = legacy
  * default stream).  Thread-local; the caller keeps the stream alive. */

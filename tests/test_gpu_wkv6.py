@@ -127,3 +127,21 @@ def test_wkv6_deterministic():
     b = _gpu(x, s0=x["s0"])
     torch.cuda.synchronize()
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_wkv6_chunked_timeout_is_reported_and_context_survives():
+    """A bounded device wait that runs out (injected on the host side: a barrier nothing
+    signals) must come back as RWKV_ERR_TIMEOUT through the status word, and the next
+    call on the same context must be correct."""
+    lib = ops.load()
+    x = _inputs(1, 200, 2, "bf16", 15, s0_std=0.1)
+    assert ops.device_status() == 0
+    prev = lib.rwkv_debug_inject_timeout(1)
+    try:
+        _gpu(x, s0=x["s0"], algo="chunked")
+        st = ops.device_status()
+    finally:
+        lib.rwkv_debug_inject_timeout(prev)
+    assert st == -6, st
+    _check(x, s0=x["s0"], algo="chunked")
+    assert ops.device_status() == 0

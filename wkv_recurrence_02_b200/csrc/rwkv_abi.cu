@@ -228,6 +228,13 @@ int rwkv_set_wkv6_algo(int algo)
 
 int rwkv_get_wkv6_algo(void) { return tl_wkv6_algo; }
 
+int rwkv_debug_inject_timeout(int enable)
+{
+    int prev = wkv::g_chunked_inject_timeout;
+    wkv::g_chunked_inject_timeout = enable ? 1 : 0;
+    return prev;
+}
+
 void rwkv_set_stream(void *cuda_stream) { tl_stream = static_cast<cudaStream_t>(cuda_stream); }
 
 void *rwkv_get_stream(void) { return tl_stream; }

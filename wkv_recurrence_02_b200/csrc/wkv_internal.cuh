@@ -45,4 +45,8 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s);
 
+// Test hook: when nonzero, chunked launches first wait on a barrier that is never
+// signalled (short bound) so the timeout path runs; set via rwkv_debug_inject_timeout.
+extern int g_chunked_inject_timeout;
+
 }  // namespace wkv

@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH):
     lib.rwkv_set_wkv6_algo.restype = ctypes.c_int
     lib.rwkv_get_wkv6_algo.argtypes = []
     lib.rwkv_get_wkv6_algo.restype = ctypes.c_int
+    lib.rwkv_debug_inject_timeout.argtypes = [ctypes.c_int]
+    lib.rwkv_debug_inject_timeout.restype = ctypes.c_int
     lib.rwkv_get_device_status.argtypes = []
     lib.rwkv_get_device_status.restype = ctypes.c_int
     lib.rwkv_status_string.argtypes = [ctypes.c_int]
