@@ -121,6 +121,17 @@ def test_wkv6_extreme_decays(algo):
     _check(x, s0=x["s0"], algo=algo)
 
 
+@pytest.mark.parametrize("wval", [0.1, 0.3])
+def test_wkv6_fast_decay_channels(wval):
+    """Channels whose decay product over a 64-token chunk drops below 2^-100 (w = 0.1) take
+    the sub-block path; w = 0.3 stays on the chunk-end path.  Both must match the oracle."""
+    x = _inputs(2, 300, 2, "bf16", 16, s0_std=0.1)
+    w = x["w"].float()
+    w[..., 24:40] = wval
+    x["w"] = w.to(torch.bfloat16)
+    _check(x, s0=x["s0"], algo="chunked")
+
+
 def test_wkv6_deterministic():
     x = _inputs(2, 1000, 4, "bf16", 14, s0_std=0.1)
     a = _gpu(x, s0=x["s0"])

@@ -9,17 +9,28 @@
 // Per (batch row, channel) the past sums are carried as (a, b, p): numerator a 2^p and
 // denominator b 2^p, with p kept in log2 units so every exponential is one ex2.  The
 // per-step update is associative once a block of n steps is summarised by its local
-// state and its total decay n*w, so T is cut into 32 segments per tile:
-//   pass 1  each lane scans its own segment from the empty state;
-//   scan    a 5-step warp shuffle scan combines segment summaries across lanes,
-//           and the carry from earlier tiles (or s0) is folded in;
-//   pass 2  each lane re-walks its segment from its exact incoming state, producing y.
+// state and its total decay n*w, so T is cut into tiles of 32 segments of L tokens:
+//   pass 1  each lane summarises its own segment from the empty state, with the
+//           segment's last key as reference: the last token's weight is exactly 1, so
+//           the denominator never underflows, and every other weight is a single ex2
+//           (the decay a plain multiply).  If a weight overflows (keys more than 2^127
+//           apart) the lane redoes its segment with the running-maximum step.  The
+//           segment's largest and smallest key are noted on the way;
+//   scan    a 5-step warp shuffle scan combines segment summaries across lanes, and the
+//           carry from earlier tiles (or s0) is folded in;
+//   pass 2  each lane re-walks its segment from its exact incoming state.  When every
+//           term lies within 2^60 of the segment's largest exponent (the normal case)
+//           the walk uses that fixed reference: one ex2 per key weight and one
+//           reciprocal per output; otherwise it repeats the running-maximum step, which
+//           is exact for any inputs.
+// Both channels of a lane are carried in 64-bit register pairs and advanced with packed
+// f32x2 arithmetic.
 //
 // Layout: one CTA = one batch row x 16 channels; warp = channel pair (2 channels per
-// lane), lane = segment.  k and v of a tile (32*L tokens x 16 channels) are staged in
-// shared memory as 2-channel words in a [pair][segment][L+1] layout: the +1 pad makes
-// lane-strided reads conflict-free, and row-contiguous fills stay coalesced from HBM.
-// y overwrites k's words in place and is written back with the same coalesced pattern.
+// lane), lane = segment.  k and v tiles (32 x L tokens x 16 channels) are copied with
+// cp.async straight into a [pair][segment][L+1] layout (the +1 pad and a 4-word skew per
+// pair make both the row-contiguous fill and the lane-strided reads conflict-free).
+// y overwrites k's words in place and is written back with row-contiguous stores.
 #include "wkv_internal.cuh"
 
 namespace wkv {
@@ -32,12 +43,69 @@ constexpr int kThreads = kPairs * 32;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kPEmpty = -1e30f;  // exponent of an empty state (finite: empty+empty stays 0)
+constexpr float kFrame = 60.f;     // fixed-reference pass 2: allowed spread in log2 units
 
 __device__ __forceinline__ float ex2(float x)
 {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+__device__ __forceinline__ float rcp(float x)
+{
+    float y;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// Two fp32 channels in one 64-bit register pair (low half = first channel).
+struct P2 {
+    unsigned long long r;
+};
+
+__device__ __forceinline__ P2 pk(float lo, float hi)
+{
+    P2 p;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p.r) : "f"(lo), "f"(hi));
+    return p;
+}
+__device__ __forceinline__ float lo(P2 p)
+{
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p.r));
+    return a;
+}
+__device__ __forceinline__ float hi(P2 p)
+{
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p.r));
+    return b;
+}
+__device__ __forceinline__ P2 fma2(P2 a, P2 b, P2 c)
+{
+    P2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.r) : "l"(a.r), "l"(b.r), "l"(c.r));
+    return d;
+}
+__device__ __forceinline__ P2 mul2(P2 a, P2 b)
+{
+    P2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+__device__ __forceinline__ P2 add2(P2 a, P2 b)
+{
+    P2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+__device__ __forceinline__ P2 ex2_2(P2 x) { return pk(ex2(lo(x)), ex2(hi(x))); }
+__device__ __forceinline__ P2 rcp2(P2 x) { return pk(rcp(lo(x)), rcp(hi(x))); }
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
 struct St {
@@ -94,11 +162,19 @@ __device__ __forceinline__ St shfl_idx(St s, int lane)
 template <typename T> struct Word;
 template <> struct Word<float> {
     using type = float2;
+    __device__ static P2 unpack(float2 x) { return pk(x.x, x.y); }
     __device__ static float2 to_f2(float2 x) { return x; }
     __device__ static float2 from_f2(float2 x) { return x; }
 };
 template <> struct Word<__nv_bfloat16> {
     using type = __nv_bfloat162;
+    __device__ static P2 unpack(__nv_bfloat162 x)
+    {
+        const uint32_t w = *reinterpret_cast<uint32_t *>(&x);
+        P2 p;
+        asm("mov.b64 %0, {%1, %2};" : "=l"(p.r) : "r"(w << 16), "r"(w & 0xFFFF0000u));
+        return p;
+    }
     __device__ static float2 to_f2(__nv_bfloat162 x) { return __bfloat1622float2(x); }
     __device__ static __nv_bfloat162 from_f2(float2 x) { return __float22bfloat162_rn(x); }
 };
@@ -113,68 +189,99 @@ template <> struct Elem<__nv_bfloat16> {
     __device__ static void put(__nv_bfloat16 *p, float x) { *p = __float2bfloat16_rn(x); }
 };
 
-// Moves one tile between global [rows x 16 channels] and the staged word layout.
-// TO_SMEM: global -> smem; otherwise smem -> global.  16-byte vectors when the whole
-// channel block is in range and C keeps rows 16-byte aligned; element-wise otherwise.
-template <typename T, int L, bool TO_SMEM>
-__device__ __forceinline__ void move_tile(typename Word<T>::type *sw, T *g, int64_t row0,
-                                          int nt, int64_t C, int c0, bool vec)
+// word index of (pair, segment, j) in one tile buffer
+template <int L> __device__ __forceinline__ int widx(int pr, int seg, int j)
+{
+    return pr * (kSegs * (L + 1) + 4) + seg * (L + 1) + j;
+}
+template <int L> constexpr int tile_words() { return kPairs * (kSegs * (L + 1) + 4); }
+
+// Copies one tile (rows row0 .. row0+nt-1, channels c0..c0+15) of k and v into their
+// buffers: thread t always moves pair t % 8 of rows t/8 + 32 i, so every address steps by
+// a constant.  Word-granular cp.async when C is even; element loads otherwise.
+template <typename T, int L>
+__device__ __forceinline__ void fetch_tile(typename Word<T>::type *bk, typename Word<T>::type *bv,
+                                           const T *k, const T *v, int64_t row0, int nt, int64_t C, int c0)
 {
     using W = typename Word<T>::type;
-    constexpr int kWordsPerVec = 16 / sizeof(W);     // 4 (bf16x2) or 2 (float2)
-    constexpr int kVecPerRow = kPairs / kWordsPerVec; // 2 or 4
-    if (vec) {
+    constexpr int kRowsPerPass = kThreads / kPairs;  // 32
+    const int pr = threadIdx.x % kPairs, r0 = threadIdx.x / kPairs;
+    const int c = c0 + 2 * pr;
+    const int64_t g0 = (row0 + r0) * C + c;
+    const int64_t gstep = kRowsPerPass * C;
+    if ((C % 2) == 0 && c + 1 < C) {
+        const uint32_t sk = smem_u32(bk), sv = smem_u32(bv);
+#pragma unroll 4
+        for (int i = 0; i < L; ++i) {
+            const int r = r0 + kRowsPerPass * i;
+            if (r < nt) {
+                const uint32_t off = static_cast<uint32_t>(widx<L>(pr, r / L, r % L) * sizeof(W));
+                asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(sk + off), "l"(k + g0 + i * gstep),
+                             "n"(sizeof(W)));
+                asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(sv + off), "l"(v + g0 + i * gstep),
+                             "n"(sizeof(W)));
+            }
+        }
+    } else {
+        for (int i = 0; i < L; ++i) {
+            const int r = r0 + kRowsPerPass * i;
+            if (r < nt) {
+                const int64_t g = g0 + i * gstep;
+                float2 fk, fv;
+                fk.x = c < C ? Elem<T>::get(k + g) : 0.f;
+                fk.y = c + 1 < C ? Elem<T>::get(k + g + 1) : 0.f;
+                fv.x = c < C ? Elem<T>::get(v + g) : 0.f;
+                fv.y = c + 1 < C ? Elem<T>::get(v + g + 1) : 0.f;
+                bk[widx<L>(pr, r / L, r % L)] = Word<T>::from_f2(fk);
+                bv[widx<L>(pr, r / L, r % L)] = Word<T>::from_f2(fv);
+            }
+        }
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+// Writes y (held in the k buffer) of one tile back to global memory.
+template <typename T, int L>
+__device__ __forceinline__ void store_tile(const typename Word<T>::type *by, T *y, int64_t row0, int nt,
+                                           int64_t C, int c0)
+{
+    using W = typename Word<T>::type;
+    constexpr int kWordsPerVec = 16 / sizeof(W);      // 4 (bf16x2) or 2 (float2)
+    constexpr int kVecPerRow = kPairs / kWordsPerVec;  // 2 or 4
+    if (c0 + kCh <= C && C % 8 == 0) {
         for (int idx = threadIdx.x; idx < nt * kVecPerRow; idx += kThreads) {
-            const int r = idx / kVecPerRow, q = idx % kVecPerRow;
-            const int seg = r / L, j = r % L;
-            T *gp = g + (row0 + r) * C + c0 + q * kWordsPerVec * 2;
+            const int r = idx / kVecPerRow, qv = idx % kVecPerRow;
             union {
                 uint4 u;
                 W w[kWordsPerVec];
             } buf;
-            if (TO_SMEM) {
-                buf.u = __ldg(reinterpret_cast<const uint4 *>(gp));
 #pragma unroll
-                for (int m = 0; m < kWordsPerVec; ++m)
-                    sw[((q * kWordsPerVec + m) * kSegs + seg) * (L + 1) + j] = buf.w[m];
-            } else {
-#pragma unroll
-                for (int m = 0; m < kWordsPerVec; ++m)
-                    buf.w[m] = sw[((q * kWordsPerVec + m) * kSegs + seg) * (L + 1) + j];
-                *reinterpret_cast<uint4 *>(gp) = buf.u;
-            }
+            for (int m = 0; m < kWordsPerVec; ++m) buf.w[m] = by[widx<L>(qv * kWordsPerVec + m, r / L, r % L)];
+            *reinterpret_cast<uint4 *>(y + (row0 + r) * C + c0 + qv * kWordsPerVec * 2) = buf.u;
         }
     } else {
         for (int idx = threadIdx.x; idx < nt * kPairs; idx += kThreads) {
             const int r = idx / kPairs, pr = idx % kPairs;
-            const int seg = r / L, j = r % L;
             const int c = c0 + 2 * pr;
-            T *gp = g + (row0 + r) * C + c;
-            W &word = sw[(pr * kSegs + seg) * (L + 1) + j];
-            if (TO_SMEM) {
-                float2 f;
-                f.x = c < C ? Elem<T>::get(gp) : 0.f;
-                f.y = c + 1 < C ? Elem<T>::get(gp + 1) : 0.f;
-                word = Word<T>::from_f2(f);
-            } else {
-                float2 f = Word<T>::to_f2(word);
-                if (c < C) Elem<T>::put(gp, f.x);
-                if (c + 1 < C) Elem<T>::put(gp + 1, f.y);
-            }
+            const float2 f = Word<T>::to_f2(by[widx<L>(pr, r / L, r % L)]);
+            T *gp = y + (row0 + r) * C + c;
+            if (c < C) Elem<T>::put(gp, f.x);
+            if (c + 1 < C) Elem<T>::put(gp + 1, f.y);
         }
     }
 }
 
 template <typename T, int L>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, 3)
 wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ w,
                  const float *__restrict__ u, const T *__restrict__ k, const T *__restrict__ v,
                  const float *s0, T *__restrict__ y, float *sT)
 {
     using W = typename Word<T>::type;
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    W *sk = reinterpret_cast<W *>(smem_raw);
-    W *sv = sk + kPairs * kSegs * (L + 1);
+    W *bk = reinterpret_cast<W *>(smem_raw);  // [k, v][tile words]
+    W *bv = bk + tile_words<L>();
+    constexpr int TILE = kSegs * L;
 
     const int64_t cblocks = (C + kCh - 1) / kCh;
     const int64_t b = blockIdx.x / cblocks;
@@ -182,10 +289,12 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
     const int pr = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ca = c0 + 2 * pr, cb = ca + 1;
     const bool va = ca < C, vb = cb < C;
-    const bool vec = (c0 + kCh <= C) && (C % 8 == 0);
 
     const float w2a = va ? w[ca] * kLog2e : 0.f, w2b = vb ? w[cb] * kLog2e : 0.f;
     const float u2a = va ? u[ca] * kLog2e : 0.f, u2b = vb ? u[cb] * kLog2e : 0.f;
+    const P2 dd = pk(ex2(-w2a), ex2(-w2b));   // per-step decay factors
+    const P2 ub = pk(ex2(u2a), ex2(u2b));     // bonus factors
+    const P2 l2e = pk(kLog2e, kLog2e);
 
     const St empty{0.f, 0.f, kPEmpty};
     St carry_a = empty, carry_b = empty;
@@ -200,25 +309,54 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
     const T *kb = k + b * T_len * C;
     const T *vbp = v + b * T_len * C;
     T *yb = y + b * T_len * C;
-    const W *mk = sk + (pr * kSegs + lane) * (L + 1);
-    const W *mv = sv + (pr * kSegs + lane) * (L + 1);
-    W *my = sk + (pr * kSegs + lane) * (L + 1);
+    const W *mk = bk + widx<L>(pr, lane, 0);
+    const W *mv = bv + widx<L>(pr, lane, 0);
+    W *my = bk + widx<L>(pr, lane, 0);
 
-    for (int64_t t0 = 0; t0 < T_len; t0 += kSegs * L) {
+    for (int64_t t0 = 0; t0 < T_len; t0 += TILE) {
         const int64_t rem = T_len - t0;
-        const int nt = rem < kSegs * L ? static_cast<int>(rem) : kSegs * L;
-        move_tile<T, L, true>(sk, const_cast<T *>(kb), t0, nt, C, c0, vec);
-        move_tile<T, L, true>(sv, const_cast<T *>(vbp), t0, nt, C, c0, vec);
+        const int nt = rem < TILE ? static_cast<int>(rem) : TILE;
+        fetch_tile<T, L>(bk, bv, kb, vbp, t0, nt, C, c0);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
-
-        // pass 1: local summary of this lane's segment
         const int nv = max(0, min(L, nt - lane * L));
+
+        // pass 1: local summary against the segment's last key; key range
         St la = empty, lb = empty;
-        for (int j = 0; j < nv; ++j) {
-            const float2 kk = Word<T>::to_f2(mk[j]);
-            const float2 vv = Word<T>::to_f2(mv[j]);
-            update(la, kk.x * kLog2e, vv.x, w2a);
-            update(lb, kk.y * kLog2e, vv.y, w2b);
+        float kmaxa = -3.4e38f, kmaxb = -3.4e38f, kmina = 3.4e38f, kminb = 3.4e38f;
+        if (nv > 0) {
+            const float2 kl = Word<T>::to_f2(mk[nv - 1]);
+            const P2 nF = pk(-kl.x * kLog2e, -kl.y * kLog2e);
+            P2 A = pk(0.f, 0.f), Bs = A;
+            float kxa = -3.4e38f, kxb = -3.4e38f, kna = 3.4e38f, knb = 3.4e38f;
+#pragma unroll 4
+            for (int j = 0; j < nv; ++j) {
+                const P2 kk = Word<T>::unpack(mk[j]);
+                const P2 vv = Word<T>::unpack(mv[j]);
+                kxa = fmaxf(kxa, lo(kk));
+                kxb = fmaxf(kxb, hi(kk));
+                kna = fminf(kna, lo(kk));
+                knb = fminf(knb, hi(kk));
+                const P2 E = ex2_2(fma2(kk, l2e, nF));
+                A = fma2(dd, A, mul2(E, vv));
+                Bs = fma2(dd, Bs, E);
+            }
+            kmaxa = kxa * kLog2e;
+            kmaxb = kxb * kLog2e;
+            kmina = kna * kLog2e;
+            kminb = knb * kLog2e;
+            const float Ba = lo(Bs), Bb = hi(Bs);
+            if (w2a >= 0.f && w2b >= 0.f && Ba <= 3.0e38f && Bb <= 3.0e38f) {
+                la = {lo(A), Ba, -lo(nF)};
+                lb = {hi(A), Bb, -hi(nF)};
+            } else {
+                for (int j = 0; j < nv; ++j) {
+                    const float2 kk = Word<T>::to_f2(mk[j]);
+                    const float2 vv = Word<T>::to_f2(mv[j]);
+                    update(la, kk.x * kLog2e, vv.x, w2a);
+                    update(lb, kk.y * kLog2e, vv.y, w2b);
+                }
+            }
         }
 
         // inclusive scan over lanes (segment order) with segment lengths
@@ -249,20 +387,42 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
         carry_b = combine(carry_b, tb, n_tot * w2b);
 
         // pass 2: outputs from the exact incoming state; y replaces k in place
-        for (int j = 0; j < nv; ++j) {
-            const float2 kk = Word<T>::to_f2(mk[j]);
-            const float2 vv = Word<T>::to_f2(mv[j]);
-            const float k2a = kk.x * kLog2e, k2b = kk.y * kLog2e;
-            float2 o;
-            o.x = output(pa, k2a, vv.x, u2a);
-            o.y = output(pb, k2b, vv.y, u2b);
-            update(pa, k2a, vv.x, w2a);
-            update(pb, k2b, vv.y, w2b);
-            my[j] = Word<T>::from_f2(o);
+        const float Fa = fmaxf(pa.p, kmaxa + fmaxf(u2a, 0.f));
+        const float Fb = fmaxf(pb.p, kmaxb + fmaxf(u2b, 0.f));
+        const bool fixed = w2a >= 0.f && w2b >= 0.f && fabsf(u2a) <= kFrame && fabsf(u2b) <= kFrame &&
+                           Fa - (u2a + kmina) <= kFrame && Fb - (u2b + kminb) <= kFrame;
+        if (fixed) {
+            // every weight is 2^{x - F} <= 1 and the bonus term keeps the denominator >= 2^-60
+            const float sa = ex2(pa.p - Fa), sb = ex2(pb.p - Fb);
+            const P2 nF = pk(-Fa, -Fb);
+            P2 A = pk(pa.a * sa, pb.a * sb), Bs = pk(pa.b * sa, pb.b * sb);
+#pragma unroll 4
+            for (int j = 0; j < nv; ++j) {
+                const P2 kk = Word<T>::unpack(mk[j]);
+                const P2 vv = Word<T>::unpack(mv[j]);
+                const P2 E = ex2_2(fma2(kk, l2e, nF));
+                const P2 bE = mul2(ub, E);
+                const P2 o = mul2(fma2(bE, vv, A), rcp2(add2(Bs, bE)));
+                A = fma2(dd, A, mul2(E, vv));
+                Bs = fma2(dd, Bs, E);
+                my[j] = Word<T>::from_f2(make_float2(lo(o), hi(o)));
+            }
+        } else {
+            for (int j = 0; j < nv; ++j) {
+                const float2 kk = Word<T>::to_f2(mk[j]);
+                const float2 vv = Word<T>::to_f2(mv[j]);
+                const float k2a = kk.x * kLog2e, k2b = kk.y * kLog2e;
+                float2 o;
+                o.x = output(pa, k2a, vv.x, u2a);
+                o.y = output(pb, k2b, vv.y, u2b);
+                update(pa, k2a, vv.x, w2a);
+                update(pb, k2b, vv.y, w2b);
+                my[j] = Word<T>::from_f2(o);
+            }
         }
         __syncthreads();
-        move_tile<T, L, false>(sk, yb, t0, nt, C, c0, vec);
-        __syncthreads();
+        store_tile<T, L>(bk, yb, t0, nt, C, c0);
+        __syncthreads();  // the buffers are refilled by the next tile
     }
 
     if (sT && lane == 0) {
@@ -286,10 +446,12 @@ template <typename T, int L>
 cudaError_t launch_L(const Wkv4Args &a, cudaStream_t s)
 {
     using W = typename Word<T>::type;
-    const size_t smem = 2ull * kPairs * kSegs * (L + 1) * sizeof(W);
+    const size_t smem = 2ull * tile_words<L>() * sizeof(W);
     auto kern = wkv4_scan_kernel<T, L>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     const int64_t blocks = a.B * ((a.C + kCh - 1) / kCh);
     if (blocks == 0) return cudaSuccess;
@@ -299,6 +461,8 @@ cudaError_t launch_L(const Wkv4Args &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+// Segment length: the smallest power of two giving 32 segments that cover T, capped so a
+// tile (k and v) keeps 3 CTAs per SM within shared memory.
 template <typename T, int LMAX>
 cudaError_t launch_T(const Wkv4Args &a, cudaStream_t s)
 {

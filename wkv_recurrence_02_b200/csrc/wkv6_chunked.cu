@@ -48,23 +48,24 @@ constexpr int kC = 64;                 // tokens per chunk
 constexpr int kN = 64;                 // head size
 constexpr int kThreads = 256;
 constexpr int kTile = kC * kN * 2;     // bytes of one bf16 64x64 tile
-constexpr int kStages = 2;
+constexpr int kStages = 3;
 constexpr int kStageBytes = 4 * kTile; // r, k, v, w
-constexpr float kHazard = 8.673617379884035e-19f;  // 2^-60
+constexpr float kHazard = 8.673617379884035e-19f;  // 2^-60: sub-block factor guard
+constexpr float kFastMin = 7.888609052210118e-31f; // 2^-100: chunk-end reference guard
 
 // shared memory map (offsets from a 1024-byte aligned base)
 constexpr int OFF_STAGE = 0;                          // stage s: R | K | V | W
 constexpr int SLOT_R = 0, SLOT_K = kTile, SLOT_V = 2 * kTile, SLOT_W = 3 * kTile;
-constexpr int OFF_KB = kStages * kStageBytes;         // Kb tile
-constexpr int OFF_QI = OFF_KB + kTile;                // Qi tile
-constexpr int OFF_QO = OFF_QI + kTile;                // Qo_0 at +0, Qo_1 at +4096, Qo_2 at +8192
-constexpr int OFF_SMALL = OFF_QO + 2 * kTile;         // fp32 scratch below
-constexpr int OFF_H = OFF_SMALL;                      // [4][2][64] half-block totals
-constexpr int OFF_D = OFF_H + 4 * 2 * 64 * 4;         // [64] chunk decay
-constexpr int OFF_UB = OFF_D + 64 * 4;                // [64] bonus diagonal
-constexpr int OFF_DD = OFF_UB + 64 * 4;               // [4][16][16] exact diagonal blocks
+// A chunk on the sub-block path borrows the stage two chunks ahead as scratch:
+constexpr int SCR_KB = 0, SCR_QI = kTile, SCR_QO = 2 * kTile;  // Qo_b at SCR_QO + 4096 b
+constexpr int OFF_SB = kStages * kStageBytes;         // bf16 (D S_prev) operand, chunk-end path
+constexpr int OFF_SMALL = OFF_SB + kTile;             // fp32 bookkeeping below
+constexpr int OFF_H = OFF_SMALL;                      // [4][64] 16-token sub-block products
+constexpr int OFF_D = OFF_H + 4 * 64 * 4;             // [stage][64] chunk decay
+constexpr int OFF_UB = OFF_D + kStages * 64 * 4;      // [stage][64] bonus diagonal
+constexpr int OFF_DD = OFF_UB + kStages * 64 * 4;     // [4][16][16] exact diagonal blocks
 constexpr int OFF_BAR = OFF_DD + 4 * 16 * 16 * 4;     // mbarriers (8 bytes each)
-constexpr int OFF_MISC = OFF_BAR + 8 * 8;             // tmem base, flags
+constexpr int OFF_MISC = OFF_BAR + 16 * 8;            // tmem base, flags
 constexpr int kSmemBytes = OFF_MISC + 64 + 1024;      // + alignment slack
 
 // TMEM columns (fp32 accumulators, M = 64 layout: row m -> lane (m % 16) + 32 (m / 16))
@@ -133,12 +134,49 @@ __device__ __forceinline__ bool bar_try(uint32_t bar, uint32_t phase)
     return ok != 0;
 }
 
-// Bounded wait; returns false if the limit ran out.
+// One try_wait that may suspend the thread (no issue slots used) for up to ~20 us.
+__device__ __forceinline__ bool bar_try_sleep(uint32_t bar, uint32_t phase)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, P;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(phase), "r"(20000u)
+                 : "memory");
+    return ok != 0;
+}
+
+// Bounded wait; returns false if the limit (number of try_waits) ran out.
 __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t phase, uint32_t limit)
+{
+    for (uint32_t it = 0; it < limit; ++it)
+        if (bar_try_sleep(bar, phase)) return true;
+    return false;
+}
+
+// Bounded wait without suspending (lowest wake-up latency; used by the one issuing thread).
+__device__ __forceinline__ bool bar_wait_spin(uint32_t bar, uint32_t phase, uint32_t limit)
 {
     for (uint32_t it = 0; it < limit; ++it)
         if (bar_try(bar, phase)) return true;
     return false;
+}
+
+__device__ __forceinline__ void bar_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Named barrier over `count` threads with an OR vote.
+__device__ __forceinline__ int named_sync_or(int id, int count, int pred)
+{
+    int out;
+    asm volatile("{\n\t.reg .pred P, Q;\n\tsetp.ne.s32 P, %1, 0;\n\t"
+                 "barrier.red.or.pred Q, %2, %3, P;\n\tselp.s32 %0, 1, 0, Q;\n\t}"
+                 : "=r"(out)
+                 : "r"(pred), "r"(id), "r"(count)
+                 : "memory");
+    return out;
 }
 
 __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1,
@@ -156,32 +194,42 @@ __device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes)
                  : "memory");
 }
 
-// 16 TMEM lanes x 32 columns split in two halves: threads 0-15 get columns [c, c+16),
-// threads 16-31 get [c+16, c+32), each thread one lane.
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+// 16 TMEM lanes x 64 columns: threads 0-15 get columns [c, c+32), threads 16-31 get
+// [c+32, c+64), each thread one lane.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
 {
-    uint32_t r[16];
-    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x16.b32 "
-                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16], 16;"
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.16x32bx2.x32.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32], 32;"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
                    "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]),
-                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                   "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]),
+                   "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+                   "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]),
+                   "=r"(r[30]), "=r"(r[31])
                  : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 #pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
 {
-    asm volatile("tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, "
-                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+    asm volatile("tcgen05.st.sync.aligned.16x32bx2.x32.b32 [%0], 32, "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+                 "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
                  "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
                  "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
                  "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
                  "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
                  "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-                 "r"(__float_as_uint(v[15]))
+                 "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])), "r"(__float_as_uint(v[17])),
+                 "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])), "r"(__float_as_uint(v[20])),
+                 "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])), "r"(__float_as_uint(v[23])),
+                 "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
+                 "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
+                 "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
                  : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
@@ -237,6 +285,76 @@ struct ChunkedParams {
     int inject_timeout;
 };
 
+// TMA of chunk c (r, k, v, w tiles of one head) into its stage, one thread.
+__device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full0, const CUtensorMap *mr,
+                                            const CUtensorMap *mk, const CUtensorMap *mv,
+                                            const CUtensorMap *mw, int c, int h, int b)
+{
+    const int s = c % kStages;
+    const uint32_t dst = smem_u32(sm + OFF_STAGE + s * kStageBytes);
+    const uint32_t bar = bar_full0 + 8 * s;
+    bar_expect_tx(bar, kStageBytes);
+    const int t0 = c * kC;
+    tma_load_4d(dst + SLOT_R, mr, 0, h, t0, b, bar);
+    tma_load_4d(dst + SLOT_K, mk, 0, h, t0, b, bar);
+    tma_load_4d(dst + SLOT_V, mv, 0, h, t0, b, bar);
+    tma_load_4d(dst + SLOT_W, mw, 0, h, t0, b, bar);
+}
+
+// Sum over the 32 lanes of a warp of 16 per-lane partials (one per token m = 0..15).
+// Returns the total for token (lane >> 1) & 15 (valid in every lane).
+__device__ __forceinline__ float warp_sum16(const float (&part)[16], int lane)
+{
+    float v8[8], v4[4], v2[2];
+    const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        v8[i] = (b16 ? part[8 + i] : part[i]) + __shfl_xor_sync(0xffffffffu, b16 ? part[i] : part[8 + i], 16);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        v4[i] = (b8 ? v8[4 + i] : v8[i]) + __shfl_xor_sync(0xffffffffu, b8 ? v8[i] : v8[4 + i], 8);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        v2[i] = (b4 ? v4[2 + i] : v4[i]) + __shfl_xor_sync(0xffffffffu, b4 ? v4[i] : v4[2 + i], 4);
+    float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
+}
+
+// Chunk-end path operand tiles from one 16-token sub-block: Qx -> R slot, Kh -> K slot;
+// returns the bonus partials.  FULL: all 16 tokens valid (no bound checks).
+template <bool FULL>
+__device__ __forceinline__ void prep_fast(unsigned char *st, int a, int cp, int tv, const uint32_t (&wr)[16],
+                                          float2 after, float2 u2, float (&part)[16])
+{
+    float2 run = after;  // product of w over the tokens after the current one, to the chunk end
+#pragma unroll
+    for (int m = 15; m >= 0; --m) {
+        const int t = 16 * a + m;
+        const uint32_t off = swz(t, 4 * cp);
+        float2 rr = make_float2(0.f, 0.f), kk = rr;
+        if (FULL || t < tv) {
+            rr = ld_bf2(st + SLOT_R, off);
+            kk = ld_bf2(st + SLOT_K, off);
+        }
+        const float2 w = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m]));
+        const float2 sin = mul2(run, w);
+        st_bf2(st + SLOT_R, off, make_float2(rr.x * rcp_approx(sin.x), rr.y * rcp_approx(sin.y)));
+        st_bf2(st + SLOT_K, off, mul2(kk, run));
+        part[m] = fmaf(rr.x * u2.x, kk.x, rr.y * u2.y * kk.y);
+        run = sin;
+    }
+}
+
+// Warp roles (256 threads):
+//   warps 0-3  prep group: warp a builds the operand rows of 16-token sub-block a, running
+//              up to two chunks ahead of the TMEM group;
+//   warps 4-7  TMEM group: warp 4+q serves TMEM lanes of rows 16q..16q+15 (two 32-column
+//              halves per warp); it writes y of chunk c-1 and builds P and the state operand
+//              of chunk c in one pass; thread 128 issues every MMA and every later TMA copy.
+// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue),
+// scores done / chunk done (tcgen05.commit).  Per-chunk bookkeeping (bonus diagonal, decay,
+// path flags) lives beside the chunk's stage.
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
@@ -245,17 +363,19 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *Hs = reinterpret_cast<float *>(sm + OFF_H);
-    float *Dv = reinterpret_cast<float *>(sm + OFF_D);
-    float *UB = reinterpret_cast<float *>(sm + OFF_UB);
+    float *Hs = reinterpret_cast<float *>(sm + OFF_H);   // [4 sub-blocks][64 channels]
+    float *Dv = reinterpret_cast<float *>(sm + OFF_D);   // [stage][64]
+    float *UB = reinterpret_cast<float *>(sm + OFF_UB);  // [stage][64]
     float *DD = reinterpret_cast<float *>(sm + OFF_DD);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC);
-    // bars: 0,1 = stage full; 2 = scores done; 3 = chunk MMAs done; 4 = never arrived (test hook)
-    const uint32_t bar_full0 = smem_u32(&bars[0]);
-    const uint32_t bar_A = smem_u32(&bars[2]);
-    const uint32_t bar_O = smem_u32(&bars[3]);
-    const uint32_t bar_never = smem_u32(&bars[4]);
+    // misc: [0] TMEM base, [1] abort, [2+s] sub-block path, [5+s] exact diagonal (s = stage),
+    //       [8] chunks whose TMA has been issued
+    const uint32_t bar_full0 = smem_u32(&bars[0]);   // + 8 * stage
+    const uint32_t bar_prep0 = smem_u32(&bars[3]);   // + 8 * stage
+    const uint32_t bar_A = smem_u32(&bars[6]);
+    const uint32_t bar_O = smem_u32(&bars[7]);
+    const uint32_t bar_never = smem_u32(&bars[8]);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t bh = blockIdx.x;
@@ -263,13 +383,18 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     const int64_t T = p.T;
     const int nchunks = static_cast<int>((T + kC - 1) / kC);
     const uint32_t limit = p.spin_limit;
+    const uint32_t spin_limit = p.spin_limit * 64u;
 
     if (tid == 0) {
-        for (int s = 0; s < kStages; ++s) bar_init(bar_full0 + 8 * s, 1);
+        for (int s = 0; s < kStages; ++s) {
+            bar_init(bar_full0 + 8 * s, 1);
+            bar_init(bar_prep0 + 8 * s, 128);
+        }
         bar_init(bar_A, 1);
         bar_init(bar_O, 1);
         bar_init(bar_never, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        misc[1] = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -282,329 +407,377 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     fence_after();
     const uint32_t tbase = misc[0];
 
-    // TMA issue for one chunk into its stage (thread 0 only)
-    auto issue = [&](int c) {
-        const int s = c % kStages;
-        const uint32_t dst = smem_u32(sm + OFF_STAGE + s * kStageBytes);
-        const uint32_t bar = bar_full0 + 8 * s;
-        bar_expect_tx(bar, kStageBytes);
-        const int t0 = c * kC;
-        tma_load_4d(dst + SLOT_R, &map_r, 0, static_cast<int>(h), t0, static_cast<int>(b), bar);
-        tma_load_4d(dst + SLOT_K, &map_k, 0, static_cast<int>(h), t0, static_cast<int>(b), bar);
-        tma_load_4d(dst + SLOT_V, &map_v, 0, static_cast<int>(h), t0, static_cast<int>(b), bar);
-        tma_load_4d(dst + SLOT_W, &map_w, 0, static_cast<int>(h), t0, static_cast<int>(b), bar);
-    };
-    int issued = 0;  // chunks issued so far (thread 0)
     if (tid == 0) {
-        for (; issued < kStages && issued < nchunks; ++issued) issue(issued);
+        int n0 = 0;
+        for (; n0 < kStages - 1 && n0 < nchunks; ++n0)
+            issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, n0, static_cast<int>(h), static_cast<int>(b));
+        misc[8] = n0;
     }
-
-    // warp roles for the TMEM passes: lane quadrant q (rows 16q..16q+15), column half ch
-    const int q = warp & 3, ch = warp >> 2, hi = lane >> 4, lr = lane & 15;
-    const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * q) << 16);
-    const int row = 16 * q + lr;          // TMEM row served by this thread
-    const int col0 = 32 * ch + 16 * hi;   // first of its 16 columns
-
-    // initial state into TMEM
-    {
-        float v[16];
-        if (p.s0) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + col0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float4 x = src[i];
-                v[4 * i] = x.x;
-                v[4 * i + 1] = x.y;
-                v[4 * i + 2] = x.z;
-                v[4 * i + 3] = x.w;
-            }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = 0.f;
-        }
-        tmem_st16(tlane + COL_S + 32 * ch, v);
-    }
-
-    // prep roles: sub-block a, half hf, channel pair cp
-    const int pa = warp >> 1, phf = warp & 1, cp = lane;
-    const float2 u2 = *reinterpret_cast<const float2 *>(p.u + h * kN + 2 * cp);
 
     int abort = 0;
     if (p.inject_timeout && tid == 0) abort = !bar_wait(bar_never, 0, limit);
-    fence_before();
     abort = __syncthreads_or(abort);
-    fence_after();
-    if (abort) record_status(p.status, kStatusTimeout);
+    if (abort) misc[1] = 1;
 
-    int c = 0;
-    for (; c < nchunks && !abort; ++c) {
-        const int s = c % kStages;
-        unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
-        const int t0 = c * kC;
-        const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
-        int ok = bar_wait(bar_full0 + 8 * s, (c / kStages) & 1, limit);
-
-        // ---- prep step 1: running products within this thread's 8-token half block
-        float2 rr[8], kk[8], ww[8], pre[8], suf[8];
-        const int tb0 = 16 * pa + 8 * phf;
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int t = tb0 + m;
-            const uint32_t off = swz(t, 4 * cp);
-            if (t < tv) {
-                rr[m] = ld_bf2(st + SLOT_R, off);
-                kk[m] = ld_bf2(st + SLOT_K, off);
-                ww[m] = ld_bf2(st + SLOT_W, off);
-            } else {
-                rr[m] = make_float2(0.f, 0.f);
-                kk[m] = make_float2(0.f, 0.f);
-                ww[m] = make_float2(1.f, 1.f);
+    if (warp < 4) {
+        // =============================== prep group ===============================
+        const int a = warp, cp = lane;
+        const float2 u2 = *reinterpret_cast<const float2 *>(p.u + h * kN + 2 * cp);
+        for (int c = 0; c < nchunks && !abort; ++c) {
+            const int s = c % kStages;
+            unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
+            int ok = bar_wait(bar_full0 + 8 * s, (c / kStages) & 1, limit);
+            if (named_sync_or(1, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
             }
-        }
-        float2 run = make_float2(1.f, 1.f);
+            // w of this sub-block (raw bf16 pairs; 1.0 past the end) and its product
+            uint32_t wr[16];
+            float2 G = make_float2(1.f, 1.f);
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            pre[m] = run;
-            run = mul2(run, ww[m]);
-        }
-        const float2 Hhalf = run;
-        run = make_float2(1.f, 1.f);
-#pragma unroll
-        for (int m = 7; m >= 0; --m) {
-            suf[m] = run;
-            run = mul2(run, ww[m]);
-        }
-        // bonus diagonal sum_c r u k per token (reduce over the warp's 64 channels)
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            float part = rr[m].x * u2.x * kk[m].x + rr[m].y * u2.y * kk[m].y;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-            if (lane == m) UB[tb0 + m] = part;
-        }
-        *reinterpret_cast<float2 *>(Hs + (pa * 2 + phf) * 64 + 2 * cp) = Hhalf;
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
-
-        // ---- sub-block totals, hazard check
-        float2 G[4];
-#pragma unroll
-        for (int be = 0; be < 4; ++be)
-            G[be] = mul2(*reinterpret_cast<const float2 *>(Hs + (be * 2 + 0) * 64 + 2 * cp),
-                         *reinterpret_cast<const float2 *>(Hs + (be * 2 + 1) * 64 + 2 * cp));
-        int hazard_local = 0;
-#pragma unroll
-        for (int be = 0; be < 4; ++be) hazard_local |= (G[be].x < kHazard) | (G[be].y < kHazard);
-        const int hazard = __syncthreads_or(hazard_local);
-
-        if (hazard) {
-            // exact diagonal blocks from running products (inputs are still intact here)
-            for (int item = tid; item < 4 * 120; item += kThreads) {
-                const int ab = item / 120;
-                int pr = item % 120, tt = 1;
-                while (pr >= tt) {
-                    pr -= tt;
-                    ++tt;
-                }
-                const int ii = pr;  // 0 <= ii < tt < 16
-                const int t = 16 * ab + tt, i = 16 * ab + ii;
-                float acc = 0.f;
-                if (t < tv) {
-                    for (int cc = 0; cc < kN; cc += 2) {
-                        const float2 rt = ld_bf2(st + SLOT_R, swz(t, 2 * cc));
-                        const float2 ki = ld_bf2(st + SLOT_K, swz(i, 2 * cc));
-                        float2 f = make_float2(1.f, 1.f);
-                        for (int j = i + 1; j < t; ++j) f = mul2(f, ld_bf2(st + SLOT_W, swz(j, 2 * cc)));
-                        acc += rt.x * ki.x * f.x + rt.y * ki.y * f.y;
-                    }
-                }
-                DD[(ab * 16 + tt) * 16 + ii] = acc;
+            for (int m = 0; m < 16; ++m) {
+                const int t = 16 * a + m;
+                wr[m] = t < tv ? *reinterpret_cast<const uint32_t *>(st + SLOT_W + swz(t, 4 * cp)) : 0x3F803F80u;
+                G = mul2(G, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
             }
-            __syncthreads();
-        }
-
-        // ---- prep step 2: operand tiles (Qd -> R slot, Kd -> K slot, Kh -> W slot in place)
-        {
+            *reinterpret_cast<float2 *>(Hs + a * 64 + 2 * cp) = G;
+            named_sync_or(1, 128, 0);
+            float2 Gs[4];
+#pragma unroll
+            for (int be = 0; be < 4; ++be) Gs[be] = *reinterpret_cast<const float2 *>(Hs + be * 64 + 2 * cp);
             const float2 one = make_float2(1.f, 1.f);
-            const float2 Hb0 = *reinterpret_cast<const float2 *>(Hs + (pa * 2 + 0) * 64 + 2 * cp);
-            const float2 Hb1 = *reinterpret_cast<const float2 *>(Hs + (pa * 2 + 1) * 64 + 2 * cp);
-            const float2 lead = phf ? Hb0 : one;
-            const float2 trail = phf ? one : Hb1;
-            float2 before = one, after = one;
+            float2 D = one, before = one, after = one, cab1 = one, cab2 = one;
 #pragma unroll
             for (int be = 0; be < 4; ++be) {
-                if (be < pa) before = mul2(before, G[be]);
-                if (be > pa) after = mul2(after, G[be]);
+                D = mul2(D, Gs[be]);
+                if (be < a) before = mul2(before, Gs[be]);
+                if (be > a) after = mul2(after, Gs[be]);
+                if (be == a - 1) cab1 = Gs[be];                               // C_{a,a-2}
+                if (be == a - 1 || be == a - 2) cab2 = mul2(cab2, Gs[be]);    // C_{a,a-3}
             }
-            // C_{a,b} = prod_{beta=b+1}^{a-1} G_beta for b = a-1, a-2, a-3
-            float2 cab[3];
-            cab[0] = one;                          // b = a-1
-            cab[1] = pa >= 2 ? G[pa - 1] : one;    // b = a-2
-            cab[2] = pa >= 3 ? mul2(G[pa - 2], G[pa - 1]) : one;  // b = a-3
-            unsigned char *qo = sm + OFF_QO;
+            // single chunk-end reference unless a chunk decay product is below 2^-100
+            const int safe = named_sync_or(1, 128, (D.x < kFastMin) | (D.y < kFastMin));
+            int hazard = 0;
+            float part[16];
+            if (!safe) {
+                if (tv == kC) prep_fast<true>(st, a, cp, tv, wr, after, u2, part);
+                else prep_fast<false>(st, a, cp, tv, wr, after, u2, part);
+            } else {
+                // sub-block path; scratch = the stage two chunks ahead, free once chunk c-1 is done
+                unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
+                if (c > 0) ok = bar_wait(bar_O, (c - 1) & 1, limit);
+                int hz = 0;
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int t = tb0 + m;
-                const uint32_t off = swz(t, 4 * cp);
-                const float2 pex = mul2(lead, pre[m]);
-                const float2 pin = mul2(pex, ww[m]);
-                const float2 sex = mul2(suf[m], trail);
-                const float2 qd = mul2(rr[m], pex);
-                float2 kd;
-                kd.x = pin.x >= kHazard ? kk[m].x * rcp_approx(pin.x) : 0.f;
-                kd.y = pin.y >= kHazard ? kk[m].y * rcp_approx(pin.y) : 0.f;
-                const float2 kb = mul2(kk[m], sex);
-                st_bf2(st + SLOT_R, off, qd);
-                st_bf2(st + SLOT_K, off, kd);
-                st_bf2(sm + OFF_KB, off, kb);
-                st_bf2(sm + OFF_QI, off, mul2(qd, before));
-                st_bf2(st + SLOT_W, off, mul2(kb, after));
-#pragma unroll
-                for (int d = 1; d <= 3; ++d) {
-                    if (d <= pa) {
-                        const int bq = pa - d;  // key sub-block served by Qo_bq
-                        st_bf2(qo + 4096 * bq, off, mul2(qd, cab[d - 1]));
+                for (int be = 0; be < 4; ++be) hz |= (Gs[be].x < kHazard) | (Gs[be].y < kHazard);
+                const int vote = named_sync_or(1, 128, hz);
+                if (named_sync_or(1, 128, !ok)) {
+                    abort = 1;
+                    misc[1] = 1;
+                    break;
+                }
+                hazard = vote;
+                if (hazard) {
+                    // exact diagonal blocks from running products (inputs still intact here)
+                    for (int item = tid; item < 4 * 120; item += 128) {
+                        const int ab = item / 120;
+                        int pr = item % 120, tt = 1;
+                        while (pr >= tt) {
+                            pr -= tt;
+                            ++tt;
+                        }
+                        const int ii = pr;  // 0 <= ii < tt < 16
+                        const int t = 16 * ab + tt, i = 16 * ab + ii;
+                        float acc = 0.f;
+                        if (t < tv) {
+                            for (int cc = 0; cc < kN; cc += 2) {
+                                const float2 rt = ld_bf2(st + SLOT_R, swz(t, 2 * cc));
+                                const float2 ki = ld_bf2(st + SLOT_K, swz(i, 2 * cc));
+                                float2 f = one;
+                                for (int j = i + 1; j < t; ++j) f = mul2(f, ld_bf2(st + SLOT_W, swz(j, 2 * cc)));
+                                acc += rt.x * ki.x * f.x + rt.y * ki.y * f.y;
+                            }
+                        }
+                        DD[(ab * 16 + tt) * 16 + ii] = acc;
                     }
+                    named_sync_or(1, 128, 0);
+                }
+                float2 suf[16];
+                float2 run = one;
+#pragma unroll
+                for (int m = 15; m >= 0; --m) {
+                    suf[m] = run;
+                    run = mul2(run, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+                }
+                float2 pex = one;
+#pragma unroll
+                for (int m = 0; m < 16; ++m) {
+                    const int t = 16 * a + m;
+                    const uint32_t off = swz(t, 4 * cp);
+                    float2 rr = make_float2(0.f, 0.f), kk = rr;
+                    if (t < tv) {
+                        rr = ld_bf2(st + SLOT_R, off);
+                        kk = ld_bf2(st + SLOT_K, off);
+                    }
+                    const float2 pin = mul2(pex, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+                    const float2 qd = mul2(rr, pex);
+                    float2 kd;
+                    kd.x = pin.x >= kHazard ? kk.x * rcp_approx(pin.x) : 0.f;
+                    kd.y = pin.y >= kHazard ? kk.y * rcp_approx(pin.y) : 0.f;
+                    const float2 kbv = mul2(kk, suf[m]);
+                    st_bf2(st + SLOT_R, off, qd);
+                    st_bf2(st + SLOT_K, off, kd);
+                    st_bf2(scr + SCR_KB, off, kbv);
+                    st_bf2(scr + SCR_QI, off, mul2(qd, before));
+                    st_bf2(st + SLOT_W, off, mul2(kbv, after));
+                    if (a >= 1) st_bf2(scr + SCR_QO + 4096 * (a - 1), off, qd);              // Qo_{a-1}
+                    if (a >= 2) st_bf2(scr + SCR_QO + 4096 * (a - 2), off, mul2(qd, cab1));  // Qo_{a-2}
+                    if (a >= 3) st_bf2(scr + SCR_QO + 4096 * (a - 3), off, mul2(qd, cab2));  // Qo_{a-3}
+                    part[m] = fmaf(rr.x * u2.x, kk.x, rr.y * u2.y * kk.y);
+                    pex = pin;
                 }
             }
-            if (warp == 0) {
-                float2 D = one;
-#pragma unroll
-                for (int be = 0; be < 4; ++be) D = mul2(D, G[be]);
-                *reinterpret_cast<float2 *>(Dv + 2 * cp) = D;
+            const float tot = warp_sum16(part, lane);
+            if ((lane & 1) == 0) UB[s * 64 + 16 * a + ((lane >> 1) & 15)] = tot;
+            if (warp == 0) *reinterpret_cast<float2 *>(Dv + s * 64 + 2 * cp) = D;
+            if (tid == 0) {
+                misc[2 + s] = safe;
+                misc[5 + s] = hazard;
             }
+            fence_async_smem();
+            bar_arrive(bar_prep0 + 8 * s);
         }
-        fence_async_smem();
-        fence_before();
-        __syncthreads();
-        fence_after();
+    } else {
+        // =============================== TMEM group ===============================
+        const int q = warp - 4, hi = lane >> 4, lr = lane & 15;
+        const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        const int row = 16 * q + lr;   // TMEM row of this thread
+        const int colh = 32 * hi;      // its 32 columns start here
+        const bool issuer = tid == 128;
+        int issued = misc[8];
 
-        // ---- scores: diagonal (N=64) and off-diagonal (3 x N=16) MMAs
-        if (tid == 0) {
+        // scores of chunk c into TMEM (issuer only)
+        auto issue_scores = [&](int c) -> int {
+            const int s = c % kStages;
+            if (!bar_wait_spin(bar_prep0 + 8 * s, (c / kStages) & 1, spin_limit)) return 0;
+            fence_after();
+            unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
             const uint32_t aR = smem_u32(st + SLOT_R), aK = smem_u32(st + SLOT_K);
-            const uint32_t aKB = smem_u32(sm + OFF_KB), aQO = smem_u32(sm + OFF_QO);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
                 mma(tbase + COL_AD, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
+            if (misc[2 + s]) {
+                unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
+                const uint32_t aKB = smem_u32(scr + SCR_KB), aQO = smem_u32(scr + SCR_QO);
 #pragma unroll
-            for (int bq = 0; bq < 3; ++bq)
+                for (int bq = 0; bq < 3; ++bq)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma(tbase + COL_AO + 16 * bq, desc_k(aQO + 4096 * bq + 32 * ks),
+                            desc_k(aKB + 2048 * bq + 32 * ks), idesc(16, 0, 0), ks > 0);
+            }
+            mma_commit(bar_A);
+            return 1;
+        };
+
+        int ok = 1;
+        if (issuer && !abort) ok = issue_scores(0);
+        {   // initial state into TMEM
+            float v[32];
+            if (p.s0) {
+                const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    float4 x = src[i];
+                    v[4 * i] = x.x;
+                    v[4 * i + 1] = x.y;
+                    v[4 * i + 2] = x.z;
+                    v[4 * i + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            }
+            tmem_st32(tlane + COL_S, v);
+        }
+
+        for (int c = 0; c < nchunks && !abort; ++c) {
+            const int s = c % kStages;
+            unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
+            const int64_t t0 = static_cast<int64_t>(c) * kC;
+
+            // scores of c and all MMAs of c-1 complete
+            if (issuer && ok) {
+                ok = bar_wait_spin(bar_A, c & 1, spin_limit);
+                if (ok && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
+            }
+            if (named_sync_or(2, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
+            }
+            bar_try(bar_A, c & 1);
+            bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);
+            if (c > 0) bar_try(bar_O, (c - 1) & 1);
+            fence_after();
+            const int safe = misc[2 + s], hazard = misc[5 + s];
+
+            // TMA for later chunks: a stage is free once its previous chunk is done, unless a
+            // sub-block-path chunk still uses it as scratch
+            if (issuer) {
+                while (issued < nchunks && issued <= c + kStages - 1) {
+                    const int user = issued - 2;  // chunk that would use this stage as scratch
+                    if (user >= c && misc[2 + user % kStages]) break;
+                    issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, static_cast<int>(h),
+                                static_cast<int>(b));
+                    ++issued;
+                }
+                misc[8] = issued;
+            }
+
+            // ---- y of chunk c-1, and P of chunk c (causal scores, bonus diagonal, bf16)
+            {
+                float va[32];
+                tmem_ld32(tlane + COL_AD, va);
+                if (c > 0) {
+                    float ov[32];
+                    tmem_ld32(tlane + COL_O, ov);
+                    const int64_t tp = t0 - kC + row;
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + tp) * p.H + h) * kN + colh);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 x;
+                        x.x = pack_bf16(ov[8 * v4 + 0], ov[8 * v4 + 1]);
+                        x.y = pack_bf16(ov[8 * v4 + 2], ov[8 * v4 + 3]);
+                        x.z = pack_bf16(ov[8 * v4 + 4], ov[8 * v4 + 5]);
+                        x.w = pack_bf16(ov[8 * v4 + 6], ov[8 * v4 + 7]);
+                        dst[v4] = x;
+                    }
+                }
+                if (safe) {
+                    float vo[32];
+                    tmem_ld32(tlane + COL_AO, vo);
+#pragma unroll
+                    for (int n = 0; n < 32; ++n) {
+                        const int kbi = (colh + n) >> 4;
+                        if (kbi < q) va[n] = vo[n];
+                        else if (kbi == q && hazard) va[n] = DD[(q * 16 + lr) * 16 + ((colh + n) & 15)];
+                    }
+                }
+                const float ub = UB[s * 64 + row];
+#pragma unroll
+                for (int n = 0; n < 32; ++n) {
+                    const int i = colh + n;
+                    va[n] = i < row ? va[n] : (i == row ? ub : 0.f);
+                }
+                unsigned char *pt = st + (safe ? SLOT_K : SLOT_W);
+                st_row16_bf16(pt, row, 2 * colh, *reinterpret_cast<float(*)[16]>(&va[0]));
+                st_row16_bf16(pt, row, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&va[16]));
+            }
+            // ---- state: S *= D in TMEM; operand = bf16(D S_prev) (chunk-end path) or bf16(S_prev)
+            {
+                float sv[32];
+                tmem_ld32(tlane + COL_S, sv);
+                const float d = Dv[s * 64 + row];
+                if (safe) {
+                    st_row16_bf16(st + SLOT_R, row, 2 * colh, *reinterpret_cast<float(*)[16]>(&sv[0]));
+                    st_row16_bf16(st + SLOT_R, row, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&sv[16]));
+                }
+#pragma unroll
+                for (int n = 0; n < 32; ++n) sv[n] *= d;
+                if (!safe) {
+                    st_row16_bf16(sm + OFF_SB, row, 2 * colh, *reinterpret_cast<float(*)[16]>(&sv[0]));
+                    st_row16_bf16(sm + OFF_SB, row, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&sv[16]));
+                }
+                tmem_st32(tlane + COL_S, sv);
+            }
+            fence_async_smem();
+            fence_before();
+            named_sync_or(2, 128, 0);
+            fence_after();
+
+            if (issuer) {
+                // ---- O = P V + Q S_op ; S += Kh^T V
+                const uint32_t aV = smem_u32(st + SLOT_V);
+                uint32_t aP, aQ, aSop, aKh;
+                if (!safe) {
+                    aP = smem_u32(st + SLOT_W);
+                    aQ = smem_u32(st + SLOT_R);     // Qx
+                    aSop = smem_u32(sm + OFF_SB);   // bf16(D S_prev)
+                    aKh = smem_u32(st + SLOT_K);    // Kh, read MN-major as K^T
+                } else {
+                    unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
+                    aP = smem_u32(st + SLOT_K);
+                    aQ = smem_u32(scr + SCR_QI);    // Qi
+                    aSop = smem_u32(st + SLOT_R);   // bf16(S_prev)
+                    aKh = smem_u32(st + SLOT_W);
+                }
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma(tbase + COL_AO + 16 * bq, desc_k(aQO + 4096 * bq + 32 * ks),
-                        desc_k(aKB + 2048 * bq + 32 * ks), idesc(16, 0, 0), ks > 0);
-            mma_commit(bar_A);
-        }
-        ok = bar_wait(bar_A, c & 1, limit);
-        fence_after();
-
-        // ---- mask pass: P (bf16, causal, bonus diagonal) -> K slot
-        {
-            float vd[16], vo[16], pv[16];
-            tmem_ld16(tlane + COL_AD + 32 * ch, vd);
-            tmem_ld16(tlane + COL_AO + 32 * ch, vo);
-            const int kb = 2 * ch + hi;  // key sub-block of this thread's 16 columns
+                    mma(tbase + COL_O, desc_k(aP + 32 * ks), desc_mn(aV + 2048 * ks), idesc(64, 0, 1), ks > 0);
 #pragma unroll
-            for (int n = 0; n < 16; ++n) {
-                float val = 0.f;
-                if (kb < q) {
-                    val = vo[n];
-                } else if (kb == q) {
-                    if (n < lr) val = hazard ? DD[(q * 16 + lr) * 16 + n] : vd[n];
-                    else if (n == lr) val = UB[row];
+                for (int ks = 0; ks < 4; ++ks)
+                    mma(tbase + COL_O, desc_k(aQ + 32 * ks), desc_mn(aSop + 2048 * ks), idesc(64, 0, 1), 1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma(tbase + COL_S, desc_mn(aKh + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), 1);
+                mma_commit(bar_O);
+                // scores of the next chunk queue behind them
+                if (c + 1 < nchunks) ok = issue_scores(c + 1);
+            }
+        }
+        // ---- y of the last chunk
+        if (!abort) {
+            if (issuer) ok = bar_wait_spin(bar_O, (nchunks - 1) & 1, spin_limit);
+            if (named_sync_or(2, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+            } else {
+                bar_try(bar_O, (nchunks - 1) & 1);
+                fence_after();
+                float ov[32];
+                tmem_ld32(tlane + COL_O, ov);
+                const int64_t t0 = static_cast<int64_t>(nchunks - 1) * kC;
+                const int tv = static_cast<int>(T - t0);
+                if (row < tv) {
+                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + t0 + row) * p.H + h) * kN + colh);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        uint4 x;
+                        x.x = pack_bf16(ov[8 * v4 + 0], ov[8 * v4 + 1]);
+                        x.y = pack_bf16(ov[8 * v4 + 2], ov[8 * v4 + 3]);
+                        x.z = pack_bf16(ov[8 * v4 + 4], ov[8 * v4 + 5]);
+                        x.w = pack_bf16(ov[8 * v4 + 6], ov[8 * v4 + 7]);
+                        dst[v4] = x;
+                    }
                 }
-                pv[n] = val;
-            }
-            st_row16_bf16(st + SLOT_K, row, 32 * kb, pv);
-        }
-
-        // ---- state pass: S_prev -> bf16 operand (R slot), S *= D in TMEM
-        {
-            float sv[16];
-            tmem_ld16(tlane + COL_S + 32 * ch, sv);
-            st_row16_bf16(st + SLOT_R, row, 2 * col0, sv);
-            const float d = Dv[row];
+                if (p.sT) {
+                    float sv[32];
+                    tmem_ld32(tlane + COL_S, sv);
+                    float4 *sd = reinterpret_cast<float4 *>(p.sT + (bh * kN + row) * kN + colh);
 #pragma unroll
-            for (int n = 0; n < 16; ++n) sv[n] *= d;
-            tmem_st16(tlane + COL_S + 32 * ch, sv);
-        }
-        fence_async_smem();
-        fence_before();
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
-        fence_after();
-
-        // ---- O = P V + Qi S_prev ; S += Kh^T V
-        if (tid == 0) {
-            const uint32_t aP = smem_u32(st + SLOT_K), aV = smem_u32(st + SLOT_V);
-            const uint32_t aSb = smem_u32(st + SLOT_R), aKh = smem_u32(st + SLOT_W);
-            const uint32_t aQI = smem_u32(sm + OFF_QI);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma(tbase + COL_O, desc_k(aP + 32 * ks), desc_mn(aV + 2048 * ks), idesc(64, 0, 1), ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma(tbase + COL_O, desc_k(aQI + 32 * ks), desc_mn(aSb + 2048 * ks), idesc(64, 0, 1), 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma(tbase + COL_S, desc_mn(aKh + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), 1);
-            mma_commit(bar_O);
-        }
-        ok = bar_wait(bar_O, c & 1, limit);
-        fence_after();
-
-        // stage is free: prefetch the chunk that reuses it
-        if (tid == 0 && ok && issued < nchunks) {
-            issue(issued);
-            ++issued;
-        }
-
-        // ---- epilogue: O -> y (bf16)
-        {
-            float ov[16];
-            tmem_ld16(tlane + COL_O + 32 * ch, ov);
-            if (row < tv) {
-                uint4 a, bb;
-                a.x = pack_bf16(ov[0], ov[1]);
-                a.y = pack_bf16(ov[2], ov[3]);
-                a.z = pack_bf16(ov[4], ov[5]);
-                a.w = pack_bf16(ov[6], ov[7]);
-                bb.x = pack_bf16(ov[8], ov[9]);
-                bb.y = pack_bf16(ov[10], ov[11]);
-                bb.z = pack_bf16(ov[12], ov[13]);
-                bb.w = pack_bf16(ov[14], ov[15]);
-                uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + t0 + row) * p.H + h) * kN + col0);
-                dst[0] = a;
-                dst[1] = bb;
+                    for (int i = 0; i < 8; ++i)
+                        sd[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+                }
             }
         }
-        fence_before();
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
-        fence_after();
     }
 
-    // ---- final state
-    if (abort) record_status(p.status, kStatusTimeout);
-    if (!abort) {
-        if (p.sT) {
-            float sv[16];
-            tmem_ld16(tlane + COL_S + 32 * ch, sv);
-            float4 *dst = reinterpret_cast<float4 *>(p.sT + (bh * kN + row) * kN + col0);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+    // ---- drain after an abort, then release tensor memory
+    fence_before();
+    abort = __syncthreads_or(abort | misc[1]);
+    fence_after();
+    if (abort) {
+        record_status(p.status, kStatusTimeout);
+        if (tid == 128) {  // wait (bounded) for this CTA's own copies and MMAs
+            const int n = misc[8];
+            for (int cc = n - kStages < 0 ? 0 : n - kStages; cc < n; ++cc)
+                bar_wait(bar_full0 + 8 * (cc % kStages), (cc / kStages) & 1, limit);
+            mma_commit(bar_never);
+            bar_wait(bar_never, 0, limit);
         }
-    } else if (tid == 0) {
-        // abort: wait (bounded) for this CTA's own copies and MMAs before releasing memory
-        for (int cc = c; cc < issued; ++cc) bar_wait(bar_full0 + 8 * (cc % kStages), (cc / kStages) & 1, limit);
-        mma_commit(bar_never);
-        bar_wait(bar_never, 0, limit);
     }
     fence_before();
     __syncthreads();
@@ -663,8 +836,10 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          kSmemBytes);
     if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
-                      g_chunked_inject_timeout ? 20000u : (1u << 20), g_chunked_inject_timeout};
+                      g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout};
     wkv6_chunked_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, s>>>(mr, mk, mv, mw, prm);
     return cudaGetLastError();
 }
