@@ -34,8 +34,9 @@
  *    call failed; rwkv_last_error() has the text.  Faults inside a kernel that the
  *    kernel itself detects (e.g. a bounded wait that ran out) are reported through the
  *    device status word, read with rwkv_get_device_status().
- *  - The library allocates no device memory of its own: its one status word is a
- *    statically allocated __device__ variable.
+ *  - The library keeps no device memory of its own beyond its status word (a statically
+ *    allocated __device__ variable).  The only per-call allocation is the stream-ordered
+ *    scratch of a split chunked WKV-6 call (see rwkv_set_wkv6_segments).
  */
 #ifndef RWKV_WKV_H
 #define RWKV_WKV_H
@@ -125,6 +126,19 @@ int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
 #define RWKV_WKV6_CHUNKED 2
 int rwkv_set_wkv6_algo(int algo);
 int rwkv_get_wkv6_algo(void);
+
+/* Sequence split of the chunked WKV-6 kernel on the calling thread.  Each (b, h) sequence
+ * is walked by one CTA; when there are fewer sequences than two per SM the library cuts
+ * every sequence into G segments (of at least four 64-token chunks) that run side by
+ * side: a first state-only pass gives each segment's local end state and decay product,
+ * and each segment then starts from its exact incoming state.  The result equals the
+ * unsplit evaluation up to fp32 rounding order.  The split needs B*H*(G-1)*(N*N+N)*4 bytes
+ * of scratch, taken stream-ordered from the device's current memory pool
+ * (cudaMallocAsync / cudaFreeAsync on the calling thread's stream) within the call.
+ *   segments = 0 (default): choose G;  1: never split;  n >= 2: split into at most n.
+ * Returns RWKV_OK or RWKV_ERR_ARG. */
+int rwkv_set_wkv6_segments(int segments);
+int rwkv_get_wkv6_segments(void);
 
 /* Test hook for the failure path (process-wide).  While enabled, every chunked WKV-6
  * launch first waits on a barrier that nothing signals, with a short bound; the wait

@@ -132,6 +132,29 @@ def test_wkv6_fast_decay_channels(wval):
     _check(x, s0=x["s0"], algo="chunked")
 
 
+@pytest.mark.parametrize("segments", [1, 2, 3, 5])
+def test_wkv6_sequence_split(segments):
+    """The chunked kernel cut into segments (state-only pass, then every segment from its
+    exact incoming state) matches the oracle, with a ragged last chunk and random s0."""
+    x = _inputs(2, 1000, 2, "bf16", 17, s0_std=0.1)
+    y, sT = _gpu(x, s0=x["s0"], algo="chunked", segments=segments)
+    torch.cuda.synchronize()
+    ry, rs = _ref(x, x["s0"])
+    assert rel_inf(f64(y), ry) <= 2e-2 and rel_inf(f64(sT), rs) <= 2e-2
+
+
+def test_wkv6_sequence_split_with_subblock_chunks():
+    """Segments whose chunks take the sub-block path (fast-decaying channels)."""
+    x = _inputs(1, 900, 2, "bf16", 18, s0_std=0.1)
+    w = x["w"].float()
+    w[..., 24:40] = 0.1
+    x["w"] = w.to(torch.bfloat16)
+    y, sT = _gpu(x, s0=x["s0"], algo="chunked", segments=4)
+    torch.cuda.synchronize()
+    ry, rs = _ref(x, x["s0"])
+    assert rel_inf(f64(y), ry) <= 2e-2 and rel_inf(f64(sT), rs) <= 2e-2
+
+
 def test_wkv6_deterministic():
     x = _inputs(2, 1000, 4, "bf16", 14, s0_std=0.1)
     a = _gpu(x, s0=x["s0"])

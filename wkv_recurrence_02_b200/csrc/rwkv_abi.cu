@@ -14,6 +14,7 @@ namespace {
 
 thread_local cudaStream_t tl_stream = nullptr;
 thread_local int tl_wkv6_algo = RWKV_WKV6_AUTO;
+thread_local int tl_wkv6_segments = 0;
 thread_local char tl_err[256] = "";
 
 // The library's only device memory: one status word per device, allocated statically.
@@ -160,7 +161,7 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
                            : cudaMemsetAsync(sT, 0, ns * 4, tl_stream);
         return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "T=0 state copy");
     }
-    wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, bf16, status};
+    wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, bf16, status, tl_wkv6_segments};
     cudaError_t e;
     int algo = tl_wkv6_algo;
     if (algo == RWKV_WKV6_SERIAL || !bf16)
@@ -227,6 +228,15 @@ int rwkv_set_wkv6_algo(int algo)
 }
 
 int rwkv_get_wkv6_algo(void) { return tl_wkv6_algo; }
+
+int rwkv_set_wkv6_segments(int segments)
+{
+    if (segments < 0) return RWKV_ERR_ARG;
+    tl_wkv6_segments = segments;
+    return RWKV_OK;
+}
+
+int rwkv_get_wkv6_segments(void) { return tl_wkv6_segments; }
 
 int rwkv_debug_inject_timeout(int enable)
 {

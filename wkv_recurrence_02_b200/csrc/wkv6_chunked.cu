@@ -39,6 +39,7 @@
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <algorithm>
 #include <mutex>
 
 namespace wkv {
@@ -283,19 +284,25 @@ struct ChunkedParams {
     int *status;
     uint32_t spin_limit;
     int inject_timeout;
+    // sequence split: CTA (bh, g) covers chunks [g * seg_chunks, (g + 1) * seg_chunks)
+    int seg_chunks;        // chunks per segment (>= number of chunks when not split)
+    int state_only;        // 1: only the segment's local end state (from zero) and decay
+    float *seg;            // [B*H][segments-1][N*N + N]: local end state, then decay product
+    int nseg;              // segments per sequence
 };
+constexpr int kSegStride = kN * kN + kN;
 
 // TMA of chunk c (r, k, v, w tiles of one head) into its stage, one thread.
 __device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full0, const CUtensorMap *mr,
                                             const CUtensorMap *mk, const CUtensorMap *mv,
-                                            const CUtensorMap *mw, int c, int h, int b)
+                                            const CUtensorMap *mw, int c, int cabs, int h, int b, bool with_r)
 {
-    const int s = c % kStages;
+    const int s = c % kStages;  // c counts chunks within this CTA's segment
     const uint32_t dst = smem_u32(sm + OFF_STAGE + s * kStageBytes);
     const uint32_t bar = bar_full0 + 8 * s;
-    bar_expect_tx(bar, kStageBytes);
-    const int t0 = c * kC;
-    tma_load_4d(dst + SLOT_R, mr, 0, h, t0, b, bar);
+    bar_expect_tx(bar, with_r ? kStageBytes : kStageBytes - kTile);
+    const int t0 = cabs * kC;
+    if (with_r) tma_load_4d(dst + SLOT_R, mr, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_K, mk, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_V, mv, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_W, mw, 0, h, t0, b, bar);
@@ -381,7 +388,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     const int64_t bh = blockIdx.x;
     const int64_t b = bh / p.H, h = bh % p.H;
     const int64_t T = p.T;
-    const int nchunks = static_cast<int>((T + kC - 1) / kC);
+    const int nchunks_all = static_cast<int>((T + kC - 1) / kC);
+    const int g = blockIdx.y;                      // segment of the sequence
+    const int cb = g * p.seg_chunks;               // its first chunk
+    const int nchunks = min(p.seg_chunks, nchunks_all - cb);  // chunks in this segment
+    const bool so = p.state_only != 0;
     const uint32_t limit = p.spin_limit;
     const uint32_t spin_limit = p.spin_limit * 64u;
 
@@ -410,7 +421,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     if (tid == 0) {
         int n0 = 0;
         for (; n0 < kStages - 1 && n0 < nchunks; ++n0)
-            issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, n0, static_cast<int>(h), static_cast<int>(b));
+            issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, n0, cb + n0, static_cast<int>(h),
+                        static_cast<int>(b), !so);
         misc[8] = n0;
     }
 
@@ -426,7 +438,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         for (int c = 0; c < nchunks && !abort; ++c) {
             const int s = c % kStages;
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
             const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
             int ok = bar_wait(bar_full0 + 8 * s, (c / kStages) & 1, limit);
             if (named_sync_or(1, 128, !ok || misc[1])) {
@@ -459,10 +471,22 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 if (be == a - 1 || be == a - 2) cab2 = mul2(cab2, Gs[be]);    // C_{a,a-3}
             }
             // single chunk-end reference unless a chunk decay product is below 2^-100
-            const int safe = named_sync_or(1, 128, (D.x < kFastMin) | (D.y < kFastMin));
+            const int safe = so ? 0 : named_sync_or(1, 128, (D.x < kFastMin) | (D.y < kFastMin));
             int hazard = 0;
             float part[16];
-            if (!safe) {
+            if (so) {
+                // local end state only: Kh[i] = k_i prod_{j>i} w_j (every factor <= 1)
+                float2 run = after;
+#pragma unroll
+                for (int m = 15; m >= 0; --m) {
+                    const int t = 16 * a + m;
+                    const uint32_t off = swz(t, 4 * cp);
+                    const float2 kk = t < tv ? ld_bf2(st + SLOT_K, off) : make_float2(0.f, 0.f);
+                    st_bf2(st + SLOT_K, off, mul2(kk, run));
+                    run = mul2(run, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+                    part[m] = 0.f;
+                }
+            } else if (!safe) {
                 if (tv == kC) prep_fast<true>(st, a, cp, tv, wr, after, u2, part);
                 else prep_fast<false>(st, a, cp, tv, wr, after, u2, part);
             } else {
@@ -583,10 +607,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         };
 
         int ok = 1;
-        if (issuer && !abort) ok = issue_scores(0);
-        {   // initial state into TMEM
+        if (issuer && !abort && !so) ok = issue_scores(0);
+        {   // initial state into TMEM: s0 advanced over the earlier segments (zero for a
+            // state-only pass, which wants the segment's local contribution)
             float v[32];
-            if (p.s0) {
+            if (p.s0 && !so) {
                 const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -600,13 +625,94 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
+            if (!so) {
+                for (int gp = 0; gp < g; ++gp) {  // S <- diag(D_g') S + S_g'
+                    const float *sg = p.seg + (bh * (p.nseg - 1) + gp) * kSegStride;
+                    const float d = sg[kN * kN + row];
+                    const float4 *src = reinterpret_cast<const float4 *>(sg + row * kN + colh);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const float4 x = src[i];
+                        v[4 * i] = fmaf(d, v[4 * i], x.x);
+                        v[4 * i + 1] = fmaf(d, v[4 * i + 1], x.y);
+                        v[4 * i + 2] = fmaf(d, v[4 * i + 2], x.z);
+                        v[4 * i + 3] = fmaf(d, v[4 * i + 3], x.w);
+                    }
+                }
+            }
             tmem_st32(tlane + COL_S, v);
         }
+
+        if (so) {
+            // ---- state-only pass: S = diag(D) S + Kh^T V per chunk; then S and prod(D) out
+            float dprod = 1.f;
+            for (int c = 0; c < nchunks && !abort; ++c) {
+                const int s = c % kStages;
+                unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
+                if (issuer && ok) {
+                    ok = bar_wait_spin(bar_prep0 + 8 * s, (c / kStages) & 1, spin_limit);
+                    if (ok && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
+                }
+                if (named_sync_or(2, 128, !ok || misc[1])) {
+                    abort = 1;
+                    misc[1] = 1;
+                    break;
+                }
+                bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);
+                if (c > 0) bar_try(bar_O, (c - 1) & 1);
+                fence_after();
+                if (issuer) {
+                    while (issued < nchunks && issued <= c + kStages - 1) {
+                        issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
+                                    static_cast<int>(h), static_cast<int>(b), false);
+                        ++issued;
+                    }
+                    misc[8] = issued;
+                }
+                {
+                    float sv[32];
+                    tmem_ld32(tlane + COL_S, sv);
+                    const float d = Dv[s * 64 + row];
+                    dprod *= d;
+#pragma unroll
+                    for (int n = 0; n < 32; ++n) sv[n] *= d;
+                    tmem_st32(tlane + COL_S, sv);
+                }
+                fence_before();
+                named_sync_or(2, 128, 0);
+                fence_after();
+                if (issuer) {
+                    const uint32_t aV = smem_u32(st + SLOT_V), aKh = smem_u32(st + SLOT_K);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma(tbase + COL_S, desc_mn(aKh + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), 1);
+                    mma_commit(bar_O);
+                }
+            }
+            if (!abort) {
+                if (issuer) ok = bar_wait_spin(bar_O, (nchunks - 1) & 1, spin_limit);
+                if (named_sync_or(2, 128, !ok || misc[1])) {
+                    abort = 1;
+                    misc[1] = 1;
+                } else {
+                    bar_try(bar_O, (nchunks - 1) & 1);
+                    fence_after();
+                    float sv[32];
+                    tmem_ld32(tlane + COL_S, sv);
+                    float *sg = p.seg + (bh * (p.nseg - 1) + g) * kSegStride;
+                    float4 *dst = reinterpret_cast<float4 *>(sg + row * kN + colh);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        dst[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+                    if (hi == 0) sg[kN * kN + row] = dprod;
+                }
+            }
+        } else {
 
         for (int c = 0; c < nchunks && !abort; ++c) {
             const int s = c % kStages;
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
-            const int64_t t0 = static_cast<int64_t>(c) * kC;
+            const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
 
             // scores of c and all MMAs of c-1 complete
             if (issuer && ok) {
@@ -630,8 +736,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 while (issued < nchunks && issued <= c + kStages - 1) {
                     const int user = issued - 2;  // chunk that would use this stage as scratch
                     if (user >= c && misc[2 + user % kStages]) break;
-                    issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, static_cast<int>(h),
-                                static_cast<int>(b));
+                    issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
+                                static_cast<int>(h), static_cast<int>(b), true);
                     ++issued;
                 }
                 misc[8] = issued;
@@ -739,8 +845,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 fence_after();
                 float ov[32];
                 tmem_ld32(tlane + COL_O, ov);
-                const int64_t t0 = static_cast<int64_t>(nchunks - 1) * kC;
-                const int tv = static_cast<int>(T - t0);
+                const int64_t t0 = static_cast<int64_t>(cb + nchunks - 1) * kC;
+                const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
                 if (row < tv) {
                     uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + t0 + row) * p.H + h) * kN + colh);
 #pragma unroll
@@ -753,7 +859,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                         dst[v4] = x;
                     }
                 }
-                if (p.sT) {
+                if (p.sT && g == p.nseg - 1) {
                     float sv[32];
                     tmem_ld32(tlane + COL_S, sv);
                     float4 *sd = reinterpret_cast<float4 *>(p.sT + (bh * kN + row) * kN + colh);
@@ -763,6 +869,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 }
             }
         }
+        }  // full pass
     }
 
     // ---- drain after an abort, then release tensor memory
@@ -822,13 +929,40 @@ bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t 
 
 int g_chunked_inject_timeout = 0;  // test hook: set through rwkv_debug_inject_timeout
 
+namespace {
+int sm_count()
+{
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+}  // namespace
+
 cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
 {
     if (!a.bf16) return wkv6_serial_launch(a, s);
-    const int64_t blocks = a.B * a.H;
-    if (blocks == 0) return cudaSuccess;
-    if (blocks > 0x7fffffffLL || a.T > 0x7fffffffLL - kC || a.B > 0x7fffffffLL || a.H > 0x7fffffffLL)
+    const int64_t bh = a.B * a.H;
+    if (bh == 0) return cudaSuccess;
+    if (bh > 0x7fffffffLL || a.T > 0x7fffffffLL - kC || a.B > 0x7fffffffLL || a.H > 0x7fffffffLL)
         return cudaErrorInvalidConfiguration;
+    const int64_t nchunks = (a.T + kC - 1) / kC;
+
+    // Sequence split: with fewer (b, h) sequences than two per SM, cut each sequence into
+    // segments of >= 4 chunks that run side by side; a state-only pass first gives every
+    // segment its exact incoming state.
+    int64_t G = 1;
+    if (a.segments == 0) {
+        const int64_t slots = 2LL * sm_count();
+        if (bh < slots) G = std::min<int64_t>(slots / bh, nchunks / 4);
+    } else {
+        G = std::min<int64_t>(a.segments, nchunks);
+    }
+    G = std::max<int64_t>(G, 1);
+    const int64_t seg_chunks = (nchunks + G - 1) / G;
+    G = (nchunks + seg_chunks - 1) / seg_chunks;
+    if (G > 65535) return cudaErrorInvalidConfiguration;
+
     CUtensorMap mr, mk, mv, mw;
     if (!make_map(&mr, a.r, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H))
@@ -838,10 +972,33 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     if (e != cudaSuccess) return e;
     e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
+
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
-                      g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout};
-    wkv6_chunked_kernel<<<static_cast<unsigned>(blocks), kThreads, kSmemBytes, s>>>(mr, mk, mv, mw, prm);
-    return cudaGetLastError();
+                      g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
+                      static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G)};
+    float *seg = nullptr;
+    if (G > 1) {
+        e = cudaMallocAsync(reinterpret_cast<void **>(&seg),
+                            static_cast<size_t>(bh) * (G - 1) * kSegStride * sizeof(float), s);
+        if (e != cudaSuccess) return e;
+        ChunkedParams pa = prm;
+        pa.state_only = 1;
+        pa.seg = seg;
+        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes,
+                              s>>>(mr, mk, mv, mw, pa);
+        e = cudaGetLastError();
+        prm.seg = seg;
+    }
+    if (e == cudaSuccess) {
+        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes,
+                              s>>>(mr, mk, mv, mw, prm);
+        e = cudaGetLastError();
+    }
+    if (seg) {
+        const cudaError_t f = cudaFreeAsync(seg, s);
+        if (e == cudaSuccess) e = f;
+    }
+    return e;
 }
 
 }  // namespace wkv

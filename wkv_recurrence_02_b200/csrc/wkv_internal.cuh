@@ -37,6 +37,7 @@ struct Wkv6Args {
     float *sT;                  // [B,H,N,N] or null
     bool bf16;
     int *status;
+    int segments;               // chunked kernel: 0 = choose the sequence split, n = at most n
 };
 
 // Each launcher returns the cudaError_t of its launch(es).

@@ -68,6 +68,10 @@ def load(path: str = LIB_PATH):
     lib.rwkv_set_wkv6_algo.restype = ctypes.c_int
     lib.rwkv_get_wkv6_algo.argtypes = []
     lib.rwkv_get_wkv6_algo.restype = ctypes.c_int
+    lib.rwkv_set_wkv6_segments.argtypes = [ctypes.c_int]
+    lib.rwkv_set_wkv6_segments.restype = ctypes.c_int
+    lib.rwkv_get_wkv6_segments.argtypes = []
+    lib.rwkv_get_wkv6_segments.restype = ctypes.c_int
     lib.rwkv_debug_inject_timeout.argtypes = [ctypes.c_int]
     lib.rwkv_debug_inject_timeout.restype = ctypes.c_int
     lib.rwkv_get_device_status.argtypes = []
@@ -141,10 +145,12 @@ def wkv4_forward(w, u, k, v, s0=None, want_state=False, y=None, sT=None):
     return (y, sT) if want_state else y
 
 
-def wkv6_forward(r, k, v, w, u, s0=None, want_state=True, y=None, sT=None, algo=None):
+def wkv6_forward(r, k, v, w, u, s0=None, want_state=True, y=None, sT=None, algo=None,
+                 segments=None):
     """Eagle/Finch WKV-6.  r,k,v,w: [B,T,H,N] fp32|bf16; u: [H,N] fp32; s0: [B,H,N,N] fp32.
 
     algo: None (library default), "auto", "serial" or "chunked" (this call only).
+    segments: None (library default), 0 (auto), 1 (no sequence split) or n (at most n).
     """
     lib = load()
     _cuda(r, "r")
@@ -164,16 +170,21 @@ def wkv6_forward(r, k, v, w, u, s0=None, want_state=True, y=None, sT=None, algo=
     _cuda(sT, "sT", torch.float32, (B, H, N, N))
     _use_current_stream(lib, r.device)
     fn = lib.rwkv_wkv6_forward_bf16 if dt == torch.bfloat16 else lib.rwkv_wkv6_forward
-    prev = None
+    prev = prev_seg = None
     if algo is not None:
         prev = lib.rwkv_get_wkv6_algo()
         _check(lib.rwkv_set_wkv6_algo(ALGOS[algo]))
+    if segments is not None:
+        prev_seg = lib.rwkv_get_wkv6_segments()
+        _check(lib.rwkv_set_wkv6_segments(int(segments)))
     try:
         _check(fn(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(y),
                   _ptr(sT)))
     finally:
         if prev is not None:
             lib.rwkv_set_wkv6_algo(prev)
+        if prev_seg is not None:
+            lib.rwkv_set_wkv6_segments(prev_seg)
     return (y, sT) if want_state else y
 
 
