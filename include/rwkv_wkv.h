@@ -140,6 +140,32 @@ int rwkv_get_wkv6_algo(void);
 int rwkv_set_wkv6_segments(int segments);
 int rwkv_get_wkv6_segments(void);
 
+/* Allocation-free variant of rwkv_wkv6_forward_bf16 (the paper has no counterpart: it is
+ * a service of this library).  Some callers may not allocate device memory at all -- a
+ * serving process that has handed its whole HBM budget to its own pool, code that must
+ * not touch the allocator while other work is in flight, or a runtime that forbids
+ * allocation outside its own set-up phase.  For them this call runs the chunked kernel with
+ * the same sequence split as the default entry point, but keeps the split's scratch in a
+ * fixed array inside the library (RWKV_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU
+ * that loads the library until the process exits) and never allocates or frees memory.
+ *   segments: 0 = choose the split as rwkv_wkv6_forward_bf16 does, capped to what the
+ *             array holds; n >= 1 = split into at most n segments.  A split needing more
+ *             than RWKV_NOALLOC_SCRATCH_BYTES (B*H*(segments-1)*(N*N+N)*4 bytes) is
+ *             rejected with RWKV_ERR_SHAPE before any launch; rwkv_last_error() says why.
+ * Arguments, layouts and the result are otherwise those of rwkv_wkv6_forward_bf16 (always
+ * the chunked kernel, whatever T).
+ *   - The first call on each device looks up the array's device address (a CUDA runtime
+ *     query, no allocation); make that first call before capturing a stream into a graph.
+ *   - Every call shares the one array and it keeps what the last call left; the kernels
+ *     write every scratch entry before reading it, so nothing has to be cleared.  Calls
+ *     whose GPU work overlaps (different streams, or host threads without ordering) race
+ *     on the array: order them on one stream. */
+#define RWKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+int rwkv_wkv6_forward_bf16_noalloc(int64_t B, int64_t T, int64_t H, int64_t N,
+                                   const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                                   const uint16_t *w, const float *u, const float *s0,
+                                   uint16_t *y, float *sT, int segments);
+
 /* Test hook for the failure path (process-wide).  While enabled, every chunked WKV-6
  * launch first waits on a barrier that nothing signals, with a short bound; the wait
  * runs out, the kernel records RWKV_ERR_TIMEOUT in the device status word, releases its

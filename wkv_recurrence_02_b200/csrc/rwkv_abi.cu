@@ -175,6 +175,62 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
     return RWKV_OK;
 }
 
+// Allocation-free WKV-6 (bf16): same validation as wkv6_entry, chunked kernel only, the
+// split's scratch in the library's fixed device array.
+int wkv6_noalloc_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
+                       const void *v, const void *w, const float *u, const float *s0, void *y,
+                       float *sT, int segments)
+{
+    tl_err[0] = 0;
+    if (segments < 0) return fail(RWKV_ERR_ARG, "segments must be >= 0%s");
+    if (B < 0 || T < 0 || H < 0 || N < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
+    int64_t BT, BTH, n, BH, ns;
+    if (!mul_ok(B, T, &BT) || !mul_ok(BT, H, &BTH) || !mul_ok(BTH, N, &n) ||
+        !mul_ok(B, H, &BH) || !mul_ok(BH, N * N, &ns))
+        return fail(RWKV_ERR_SHAPE, "size product overflows%s");
+    if (n == 0 && !(sT && ns > 0)) return RWKV_OK;
+    if (N != 64) return fail(RWKV_ERR_UNSUPPORTED, "head size N must be 64%s");
+    if (n > 0 && (!r || !k || !v || !w || !y))
+        return fail(RWKV_ERR_NULL, "r, k, v, w and y must be non-null%s");
+    if (BH > 0 && !u) return fail(RWKV_ERR_NULL, "u must be non-null%s");
+    const void *ptrs[] = {r, k, v, w, u, s0, y, sT};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(RWKV_ERR_ALIGN, "tensor pointers must be 16-byte aligned%s");
+    Span sy{y, n * 2}, sr{r, n * 2}, sk{k, n * 2}, sv{v, n * 2}, sw{w, n * 2};
+    Span su{u, H * N * 4}, ss0{s0, ns * 4}, ssT{sT, ns * 4};
+    const Span ins[] = {sr, sk, sv, sw, su};
+    for (const Span &s : ins)
+        if (overlap(sy, s)) return fail(RWKV_ERR_ALIAS, "y overlaps an input%s");
+    if (overlap(sy, ss0) || overlap(sy, ssT)) return fail(RWKV_ERR_ALIAS, "y overlaps a state%s");
+    if (sT) {
+        for (const Span &s : ins)
+            if (overlap(ssT, s)) return fail(RWKV_ERR_ALIAS, "sT overlaps an input%s");
+        if (s0 && s0 != sT && overlap(ssT, ss0))
+            return fail(RWKV_ERR_ALIAS, "sT partially overlaps s0%s");
+    }
+    int *status = nullptr;
+    int rc = status_word(&status);
+    if (rc) return rc;
+    if (T == 0) {
+        if (!sT || sT == s0) return RWKV_OK;
+        cudaError_t e = s0 ? cudaMemcpyAsync(sT, s0, ns * 4, cudaMemcpyDeviceToDevice, tl_stream)
+                           : cudaMemsetAsync(sT, 0, ns * 4, tl_stream);
+        return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "T=0 state copy");
+    }
+    wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, true, status, segments};
+    size_t need = 0;
+    cudaError_t e = wkv::wkv6_chunked_launch_noalloc(a, segments, &need, tl_stream);
+    if (e == cudaErrorInvalidValue && need > wkv::kNoAllocScratchBytes) {
+        snprintf(tl_err, sizeof(tl_err),
+                 "the requested sequence split needs %zu bytes of scratch; the fixed no-allocation "
+                 "buffer holds %zu (use fewer segments)",
+                 need, wkv::kNoAllocScratchBytes);
+        return RWKV_ERR_SHAPE;
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "wkv6 no-allocation launch");
+    return RWKV_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -217,6 +273,14 @@ int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uin
                            const float *u, const float *s0, uint16_t *y, float *sT)
 {
     return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, true);
+}
+
+int rwkv_wkv6_forward_bf16_noalloc(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,
+                                   const uint16_t *k, const uint16_t *v, const uint16_t *w,
+                                   const float *u, const float *s0, uint16_t *y, float *sT,
+                                   int segments)
+{
+    return wkv6_noalloc_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, segments);
 }
 
 int rwkv_set_wkv6_algo(int algo)

@@ -1002,3 +1002,95 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
 }
 
 }  // namespace wkv
+
+// ------------------------------------------------------------------ fixed-scratch variant
+// rwkv_wkv6_forward_bf16_noalloc keeps the sequence-split scratch in this fixed array
+// instead of allocating it, for callers that may not allocate device memory at all.  Every
+// GPU that loads the library holds the array until the process exits.  The kernels reach
+// it through the address passed in their parameters.
+namespace wkv {
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+namespace {
+std::mutex g_noalloc_mu;
+float *g_noalloc_addr[64] = {nullptr};
+
+// In host code g_noalloc_scratch only names a host-side stand-in; its device address is
+// looked up once per device, with that device current.
+cudaError_t noalloc_scratch_address(float **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_addr[dev]) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_noalloc_addr[dev] = static_cast<float *>(p);
+    }
+    *out = g_noalloc_addr[dev];
+    return cudaSuccess;
+}
+}  // namespace
+
+cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t *scratch_needed,
+                                        cudaStream_t s)
+{
+    *scratch_needed = 0;
+    const int64_t bh = a.B * a.H;
+    if (bh == 0) return cudaSuccess;
+    if (bh > 0x7fffffffLL || a.T > 0x7fffffffLL - kC || a.B > 0x7fffffffLL || a.H > 0x7fffffffLL)
+        return cudaErrorInvalidConfiguration;
+    const int64_t nchunks = (a.T + kC - 1) / kC;
+    const int64_t per_segment = static_cast<int64_t>(kSegStride) * sizeof(float) * bh;
+    int64_t G = 1;
+    if (segments == 0) {  // as the allocating entry point, capped to what the array holds
+        const int64_t slots = 2LL * sm_count();
+        if (bh < slots) G = std::min<int64_t>(slots / bh, nchunks / 4);
+        G = std::min<int64_t>(G, static_cast<int64_t>(kNoAllocScratchBytes) / per_segment + 1);
+    } else {
+        G = std::min<int64_t>(segments, nchunks);
+    }
+    G = std::max<int64_t>(G, 1);
+    const int64_t seg_chunks = (nchunks + G - 1) / G;
+    G = (nchunks + seg_chunks - 1) / seg_chunks;
+    if (G > 65535) return cudaErrorInvalidConfiguration;
+    *scratch_needed = static_cast<size_t>((G - 1) * per_segment);
+    if (*scratch_needed > kNoAllocScratchBytes) return cudaErrorInvalidValue;
+
+    float *seg = nullptr;
+    if (G > 1) {
+        cudaError_t e = noalloc_scratch_address(&seg);
+        if (e != cudaSuccess) return e;
+    }
+    CUtensorMap mr, mk, mv, mw;
+    if (!make_map(&mr, a.r, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
+                      g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
+                      static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G)};
+    if (G > 1) {
+        // the state-only pass writes every scratch entry the full pass reads: nothing in the
+        // array has to start at zero, and what an earlier call left there is never read
+        ChunkedParams pa = prm;
+        pa.state_only = 1;
+        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes,
+                              s>>>(mr, mk, mv, mw, pa);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(
+        mr, mk, mv, mw, prm);
+    return cudaGetLastError();
+}
+
+}  // namespace wkv

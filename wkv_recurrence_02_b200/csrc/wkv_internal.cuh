@@ -46,6 +46,13 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s);
 
+// The chunked kernel with its sequence-split scratch in a fixed device array (no
+// allocation).  Returns cudaErrorInvalidValue with *scratch_needed > capacity when the
+// requested split does not fit.
+constexpr size_t kNoAllocScratchBytes = 4u << 20;
+cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t *scratch_needed,
+                                        cudaStream_t s);
+
 // Test hook: when nonzero, chunked launches first wait on a barrier that is never
 // signalled (short bound) so the timeout path runs; set via rwkv_debug_inject_timeout.
 extern int g_chunked_inject_timeout;

@@ -68,6 +68,8 @@ def load(path: str = LIB_PATH):
     lib.rwkv_set_wkv6_algo.restype = ctypes.c_int
     lib.rwkv_get_wkv6_algo.argtypes = []
     lib.rwkv_get_wkv6_algo.restype = ctypes.c_int
+    lib.rwkv_wkv6_forward_bf16_noalloc.argtypes = wkv6 + [ctypes.c_int]
+    lib.rwkv_wkv6_forward_bf16_noalloc.restype = ctypes.c_int
     lib.rwkv_set_wkv6_segments.argtypes = [ctypes.c_int]
     lib.rwkv_set_wkv6_segments.restype = ctypes.c_int
     lib.rwkv_get_wkv6_segments.argtypes = []
