@@ -72,14 +72,14 @@ __device__ __forceinline__ P2 pk(float lo, float hi)
 }
 __device__ __forceinline__ float lo(P2 p)
 {
-    float a, b;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p.r));
+    float a;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {%0, t}, %1;\n\t}" : "=f"(a) : "l"(p.r));
     return a;
 }
 __device__ __forceinline__ float hi(P2 p)
 {
-    float a, b;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(p.r));
+    float b;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {t, %0}, %1;\n\t}" : "=f"(b) : "l"(p.r));
     return b;
 }
 __device__ __forceinline__ P2 fma2(P2 a, P2 b, P2 c)
@@ -194,7 +194,7 @@ template <int L> __device__ __forceinline__ int widx(int pr, int seg, int j)
 {
     return pr * (kSegs * (L + 1) + 4) + seg * (L + 1) + j;
 }
-template <int L> constexpr int tile_words() { return kPairs * (kSegs * (L + 1) + 4); }
+template <int L> __host__ __device__ constexpr int tile_words() { return kPairs * (kSegs * (L + 1) + 4); }
 
 // Copies one tile (rows row0 .. row0+nt-1, channels c0..c0+15) of k and v into their
 // buffers: thread t always moves pair t % 8 of rows t/8 + 32 i, so every address steps by

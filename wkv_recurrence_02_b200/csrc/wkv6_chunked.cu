@@ -440,12 +440,14 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
             const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
             const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
-            int ok = bar_wait(bar_full0 + 8 * s, (c / kStages) & 1, limit);
+            // one thread waits for the stage; the others park on the group barrier
+            int ok = tid == 0 ? bar_wait_spin(bar_full0 + 8 * s, (c / kStages) & 1, spin_limit) : 1;
             if (named_sync_or(1, 128, !ok || misc[1])) {
                 abort = 1;
                 misc[1] = 1;
                 break;
             }
+            bar_try(bar_full0 + 8 * s, (c / kStages) & 1);
             // w of this sub-block (raw bf16 pairs; 1.0 past the end) and its product
             uint32_t wr[16];
             float2 G = make_float2(1.f, 1.f);
