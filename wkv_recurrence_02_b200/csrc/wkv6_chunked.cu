@@ -48,6 +48,7 @@ namespace {
 constexpr int kC = 64;                 // tokens per chunk
 constexpr int kN = 64;                 // head size
 constexpr int kThreads = 256;
+constexpr int kPrepThreads = 128;
 constexpr int kTile = kC * kN * 2;     // bytes of one bf16 64x64 tile
 constexpr int kStages = 3;
 constexpr int kStageBytes = 4 * kTile; // r, k, v, w
@@ -358,10 +359,13 @@ __device__ __forceinline__ void prep_fast(unsigned char *st, int a, int cp, int 
 //              up to two chunks ahead of the TMEM group;
 //   warps 4-7  TMEM group: warp 4+q serves TMEM lanes of rows 16q..16q+15 (two 32-column
 //              halves per warp); it writes y of chunk c-1 and builds P and the state operand
-//              of chunk c in one pass; thread 128 issues every MMA and every later TMA copy.
-// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue),
-// scores done / chunk done (tcgen05.commit).  Per-chunk bookkeeping (bonus diagonal, decay,
-// path flags) lives beside the chunk's stage.
+//              of chunk c in one pass.  In the full pass one elected thread of warp 4 issues
+//              the O products, of warp 5 the state update, of warp 6 the next chunk's scores
+//              (an MMA issue holds its thread for tens of cycles, so three issuers run side
+//              by side), and of warp 7 the TMA copies of later chunks.
+// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue), scores
+// done, O done, state done and stage empty (tcgen05.commit).  Per-chunk bookkeeping (bonus
+// diagonal, decay, path flags) lives beside the chunk's stage.
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
@@ -383,6 +387,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     const uint32_t bar_A = smem_u32(&bars[6]);
     const uint32_t bar_O = smem_u32(&bars[7]);
     const uint32_t bar_never = smem_u32(&bars[8]);
+    const uint32_t bar_S = smem_u32(&bars[9]);
+    const uint32_t bar_empty0 = smem_u32(&bars[10]);  // + 8 * stage: the chunk's MMAs are done
+    const uint32_t bar_drain = smem_u32(&bars[13]);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t bh = blockIdx.x;
@@ -400,7 +407,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         for (int s = 0; s < kStages; ++s) {
             bar_init(bar_full0 + 8 * s, 1);
             bar_init(bar_prep0 + 8 * s, 128);
+            bar_init(bar_empty0 + 8 * s, 2);  // O issuer and S issuer each commit
         }
+        bar_init(bar_S, 1);
+        bar_init(bar_drain, 3);
         bar_init(bar_A, 1);
         bar_init(bar_O, 1);
         bar_init(bar_never, 1);
@@ -494,7 +504,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             } else {
                 // sub-block path; scratch = the stage two chunks ahead, free once chunk c-1 is done
                 unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
-                if (c > 0) ok = bar_wait(bar_O, (c - 1) & 1, limit);
+                // chunk c-1's stage, its ((c-1)/3)-th use
+                if (c > 0 && tid == 0)
+                    ok = bar_wait_spin(bar_empty0 + 8 * ((c + 2) % kStages), ((c - 1) / kStages) & 1, spin_limit);
                 int hz = 0;
 #pragma unroll
                 for (int be = 0; be < 4; ++be) hz |= (Gs[be].x < kHazard) | (Gs[be].y < kHazard);
@@ -504,6 +516,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     misc[1] = 1;
                     break;
                 }
+                if (c > 0) bar_try(bar_empty0 + 8 * ((c + 2) % kStages), ((c - 1) / kStages) & 1);
                 hazard = vote;
                 if (hazard) {
                     // exact diagonal blocks from running products (inputs still intact here)
@@ -581,7 +594,12 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         const uint32_t tlane = tbase + (static_cast<uint32_t>(32 * q) << 16);
         const int row = 16 * q + lr;   // TMEM row of this thread
         const int colh = 32 * hi;      // its 32 columns start here
-        const bool issuer = tid == 128;
+        // one elected thread per warp: 4 issues the O products, 5 the state update, 6 the
+        // scores of the next chunk (MMA issue blocks the issuing thread, so three issuers run
+        // side by side), 7 the TMA copies
+        const bool issuer = tid == kPrepThreads;
+        const bool iss_o = issuer, iss_s = tid == kPrepThreads + 32, iss_a = tid == kPrepThreads + 64;
+        const bool iss_t = tid == kPrepThreads + 96;
         int issued = misc[8];
 
         // scores of chunk c into TMEM (issuer only)
@@ -609,7 +627,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         };
 
         int ok = 1;
-        if (issuer && !abort && !so) ok = issue_scores(0);
+        if (iss_a && !abort && !so) ok = issue_scores(0);
         {   // initial state into TMEM: s0 advanced over the earlier segments (zero for a
             // state-only pass, which wants the segment's local contribution)
             float v[32];
@@ -716,10 +734,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
             const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
 
-            // scores of c and all MMAs of c-1 complete
-            if (issuer && ok) {
-                ok = bar_wait_spin(bar_A, c & 1, spin_limit);
-                if (ok && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
+            // scores of c and all MMAs of c-1 complete (three waiters side by side)
+            if (ok) {
+                if (iss_a) ok = bar_wait_spin(bar_A, c & 1, spin_limit);
+                else if (iss_o && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
+                else if (iss_s && c > 0) ok = bar_wait_spin(bar_S, (c - 1) & 1, spin_limit);
             }
             if (named_sync_or(2, 128, !ok || misc[1])) {
                 abort = 1;
@@ -728,13 +747,16 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             }
             bar_try(bar_A, c & 1);
             bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);
-            if (c > 0) bar_try(bar_O, (c - 1) & 1);
+            if (c > 0) {
+                bar_try(bar_O, (c - 1) & 1);
+                bar_try(bar_S, (c - 1) & 1);
+            }
             fence_after();
             const int safe = misc[2 + s], hazard = misc[5 + s];
 
             // TMA for later chunks: a stage is free once its previous chunk is done, unless a
             // sub-block-path chunk still uses it as scratch
-            if (issuer) {
+            if (iss_t) {
                 while (issued < nchunks && issued <= c + kStages - 1) {
                     const int user = issued - 2;  // chunk that would use this stage as scratch
                     if (user >= c && misc[2 + user % kStages]) break;
@@ -747,8 +769,6 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 
             // ---- y of chunk c-1, and P of chunk c (causal scores, bonus diagonal, bf16)
             {
-                float va[32];
-                tmem_ld32(tlane + COL_AD, va);
                 if (c > 0) {
                     float ov[32];
                     tmem_ld32(tlane + COL_O, ov);
@@ -764,6 +784,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                         dst[v4] = x;
                     }
                 }
+                float va[32];
+                tmem_ld32(tlane + COL_AD, va);
                 if (safe) {
                     float vo[32];
                     tmem_ld32(tlane + COL_AO, vo);
@@ -806,21 +828,19 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             named_sync_or(2, 128, 0);
             fence_after();
 
-            if (issuer) {
-                // ---- O = P V + Q S_op ; S += Kh^T V
-                const uint32_t aV = smem_u32(st + SLOT_V);
-                uint32_t aP, aQ, aSop, aKh;
+            const uint32_t aV = smem_u32(st + SLOT_V);
+            if (iss_o) {
+                // ---- O = P V + Q S_op
+                uint32_t aP, aQ, aSop;
                 if (!safe) {
                     aP = smem_u32(st + SLOT_W);
                     aQ = smem_u32(st + SLOT_R);     // Qx
                     aSop = smem_u32(sm + OFF_SB);   // bf16(D S_prev)
-                    aKh = smem_u32(st + SLOT_K);    // Kh, read MN-major as K^T
                 } else {
                     unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
                     aP = smem_u32(st + SLOT_K);
                     aQ = smem_u32(scr + SCR_QI);    // Qi
                     aSop = smem_u32(st + SLOT_R);   // bf16(S_prev)
-                    aKh = smem_u32(st + SLOT_W);
                 }
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
@@ -828,22 +848,30 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma(tbase + COL_O, desc_k(aQ + 32 * ks), desc_mn(aSop + 2048 * ks), idesc(64, 0, 1), 1);
+                mma_commit(bar_O);
+                mma_commit(bar_empty0 + 8 * s);
+            } else if (iss_s) {
+                // ---- S += Kh^T V  (Kh read MN-major as its transpose)
+                const uint32_t aKh = smem_u32(st + (safe ? SLOT_W : SLOT_K));
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma(tbase + COL_S, desc_mn(aKh + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), 1);
-                mma_commit(bar_O);
-                // scores of the next chunk queue behind them
-                if (c + 1 < nchunks) ok = issue_scores(c + 1);
+                mma_commit(bar_S);
+                mma_commit(bar_empty0 + 8 * s);
+            } else if (iss_a && c + 1 < nchunks) {
+                ok = issue_scores(c + 1);  // scores of the next chunk
             }
         }
-        // ---- y of the last chunk
+        // ---- y of the last chunk, and the final state
         if (!abort) {
-            if (issuer) ok = bar_wait_spin(bar_O, (nchunks - 1) & 1, spin_limit);
+            if (iss_o) ok = bar_wait_spin(bar_O, (nchunks - 1) & 1, spin_limit);
+            else if (iss_s) ok = bar_wait_spin(bar_S, (nchunks - 1) & 1, spin_limit);
             if (named_sync_or(2, 128, !ok || misc[1])) {
                 abort = 1;
                 misc[1] = 1;
             } else {
                 bar_try(bar_O, (nchunks - 1) & 1);
+                bar_try(bar_S, (nchunks - 1) & 1);
                 fence_after();
                 float ov[32];
                 tmem_ld32(tlane + COL_O, ov);
@@ -880,12 +908,12 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     fence_after();
     if (abort) {
         record_status(p.status, kStatusTimeout);
-        if (tid == 128) {  // wait (bounded) for this CTA's own copies and MMAs
+        if (tid == kPrepThreads || tid == kPrepThreads + 32 || tid == kPrepThreads + 64) mma_commit(bar_drain);
+        if (tid == kPrepThreads) {
             const int n = misc[8];
             for (int cc = n - kStages < 0 ? 0 : n - kStages; cc < n; ++cc)
                 bar_wait(bar_full0 + 8 * (cc % kStages), (cc / kStages) & 1, limit);
-            mma_commit(bar_never);
-            bar_wait(bar_never, 0, limit);
+            bar_wait(bar_drain, 0, limit);
         }
     }
     fence_before();
@@ -939,6 +967,60 @@ int sm_count()
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
     return n;
 }
+
+// Kernel attributes (shared memory size, carveout), set once per device.
+cudaError_t configure_kernel()
+{
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+}
+
+// Stream-ordered pool for the sequence-split scratch, one per device, owned by the library.
+// It keeps up to kPoolKeepBytes reserved across synchronisations, so a call does not map
+// fresh memory each time (the process-wide default pool hands freed memory back to the
+// system at every synchronisation unless its release threshold is raised, and changing
+// that pool's attributes would affect every other user of it).
+constexpr uint64_t kPoolKeepBytes = 64ull << 20;
+
+cudaError_t scratch_pool(cudaMemPool_t *out)
+{
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        e = cudaMemPoolCreate(&pool, &props);
+        if (e != cudaSuccess) return e;
+        uint64_t keep = kPoolKeepBytes;
+        e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep);
+        if (e != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
+        }
+        pools[dev] = pool;
+    }
+    *out = pools[dev];
+    return cudaSuccess;
+}
 }  // namespace
 
 cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
@@ -969,10 +1051,7 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     if (!make_map(&mr, a.r, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaError_t e = configure_kernel();
     if (e != cudaSuccess) return e;
 
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
@@ -980,8 +1059,11 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
                       static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G)};
     float *seg = nullptr;
     if (G > 1) {
-        e = cudaMallocAsync(reinterpret_cast<void **>(&seg),
-                            static_cast<size_t>(bh) * (G - 1) * kSegStride * sizeof(float), s);
+        cudaMemPool_t pool = nullptr;
+        e = scratch_pool(&pool);
+        if (e != cudaSuccess) return e;
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&seg),
+                                    static_cast<size_t>(bh) * (G - 1) * kSegStride * sizeof(float), pool, s);
         if (e != cudaSuccess) return e;
         ChunkedParams pa = prm;
         pa.state_only = 1;
@@ -1072,10 +1154,7 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     if (!make_map(&mr, a.r, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
         !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    cudaError_t e = configure_kernel();
     if (e != cudaSuccess) return e;
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
