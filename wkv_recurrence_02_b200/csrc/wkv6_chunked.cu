@@ -277,6 +277,110 @@ __device__ __forceinline__ void st_row16_bf16(unsigned char *tile, int row, int 
     *reinterpret_cast<uint4 *>(tile + swz(row, colbyte + 16)) = b;
 }
 
+// ------------------------------------------------------------- packed fp32 pairs (f32x2)
+// Two fp32 lanes in one 64-bit register; Blackwell executes mul/fma on both in one
+// instruction.
+struct P2 {
+    unsigned long long r;
+};
+
+__device__ __forceinline__ P2 pk(float lo, float hi)
+{
+    P2 p;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(p.r) : "f"(lo), "f"(hi));
+    return p;
+}
+__device__ __forceinline__ float lo(P2 p)
+{
+    float a;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {%0, t}, %1;\n\t}" : "=f"(a) : "l"(p.r));
+    return a;
+}
+__device__ __forceinline__ float hi(P2 p)
+{
+    float b;
+    asm("{\n\t.reg .f32 t;\n\tmov.b64 {t, %0}, %1;\n\t}" : "=f"(b) : "l"(p.r));
+    return b;
+}
+__device__ __forceinline__ P2 mul2(P2 a, P2 b)
+{
+    P2 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
+__device__ __forceinline__ P2 fma2(P2 a, P2 b, P2 c)
+{
+    P2 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.r) : "l"(a.r), "l"(b.r), "l"(c.r));
+    return d;
+}
+__device__ __forceinline__ P2 one2() { return pk(1.f, 1.f); }
+__device__ __forceinline__ P2 zero2() { return pk(0.f, 0.f); }
+
+// bf16 pair (low half = first channel) -> exact fp32 pair
+__device__ __forceinline__ P2 unpack2(uint32_t x)
+{
+    P2 p;
+    asm("{\n\t.reg .b32 l, h;\n\tshl.b32 l, %1, 16;\n\tand.b32 h, %1, 0xFFFF0000;\n\tmov.b64 %0, {l, h};\n\t}"
+        : "=l"(p.r)
+        : "r"(x));
+    return p;
+}
+// fp32 pair -> bf16 pair, round to nearest even
+__device__ __forceinline__ uint32_t pack2(P2 p)
+{
+    uint32_t d;
+    asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.bf16x2.f32 %0, h, l;\n\t}" : "=r"(d) : "l"(p.r));
+    return d;
+}
+__device__ __forceinline__ P2 rcp2(P2 x) { return pk(rcp_approx(lo(x)), rcp_approx(hi(x))); }
+__device__ __forceinline__ P2 shfl_xor2(P2 x, int m)
+{
+    P2 y;
+    y.r = __shfl_xor_sync(0xffffffffu, x.r, m);
+    return y;
+}
+__device__ __forceinline__ P2 ld_p2(const float *p)
+{
+    const float2 f = *reinterpret_cast<const float2 *>(p);
+    return pk(f.x, f.y);
+}
+__device__ __forceinline__ void st_p2(float *p, P2 x) { *reinterpret_cast<float2 *>(p) = make_float2(lo(x), hi(x)); }
+
+// four channels of one token row: two packed pairs
+struct Q4 {
+    P2 a, b;  // channels (0, 1) and (2, 3)
+};
+__device__ __forceinline__ Q4 mul4(Q4 x, Q4 y) { return {mul2(x.a, y.a), mul2(x.b, y.b)}; }
+__device__ __forceinline__ Q4 one4() { return {one2(), one2()}; }
+__device__ __forceinline__ Q4 unpack4(uint2 x) { return {unpack2(x.x), unpack2(x.y)}; }
+__device__ __forceinline__ uint2 pack4(Q4 x) { return make_uint2(pack2(x.a), pack2(x.b)); }
+__device__ __forceinline__ Q4 shfl_xor4(Q4 x, int m) { return {shfl_xor2(x.a, m), shfl_xor2(x.b, m)}; }
+__device__ __forceinline__ Q4 ld_q4(const float *p) { return {ld_p2(p), ld_p2(p + 2)}; }
+__device__ __forceinline__ void st_q4(float *p, Q4 x)
+{
+    *reinterpret_cast<float4 *>(p) = make_float4(lo(x.a), hi(x.a), lo(x.b), hi(x.b));
+}
+__device__ __forceinline__ uint2 ld_u2(const unsigned char *tile, uint32_t off)
+{
+    return *reinterpret_cast<const uint2 *>(tile + off);
+}
+__device__ __forceinline__ void st_u2(unsigned char *tile, uint32_t off, uint2 x)
+{
+    *reinterpret_cast<uint2 *>(tile + off) = x;
+}
+// true if any of the four channels is below lim
+__device__ __forceinline__ bool any_below(Q4 x, float lim)
+{
+    return (lo(x.a) < lim) | (hi(x.a) < lim) | (lo(x.b) < lim) | (hi(x.b) < lim);
+}
+// sum over the four channels of r * u * k
+__device__ __forceinline__ float bonus4(Q4 r, Q4 u, Q4 k)
+{
+    const P2 acc = fma2(mul2(r.b, u.b), k.b, mul2(mul2(r.a, u.a), k.a));
+    return lo(acc) + hi(acc);
+}
+
 struct ChunkedParams {
     int64_t T, H;
     const float *u, *s0;
@@ -309,18 +413,15 @@ __device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full
     tma_load_4d(dst + SLOT_W, mw, 0, h, t0, b, bar);
 }
 
-// Sum over the 32 lanes of a warp of 16 per-lane partials (one per token m = 0..15).
-// Returns the total for token (lane >> 1) & 15 (valid in every lane).
-__device__ __forceinline__ float warp_sum16(const float (&part)[16], int lane)
+// Sum over the 16 lanes of a half-warp of 8 per-lane partials (one per token m = 0..7).
+// Returns the total for token (lane >> 1) & 7 (valid in every lane).
+__device__ __forceinline__ float half_sum8(const float (&part)[8], int lane)
 {
-    float v8[8], v4[4], v2[2];
-    const bool b16 = lane & 16, b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        v8[i] = (b16 ? part[8 + i] : part[i]) + __shfl_xor_sync(0xffffffffu, b16 ? part[i] : part[8 + i], 16);
+    float v4[4], v2[2];
+    const bool b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
 #pragma unroll
     for (int i = 0; i < 4; ++i)
-        v4[i] = (b8 ? v8[4 + i] : v8[i]) + __shfl_xor_sync(0xffffffffu, b8 ? v8[i] : v8[4 + i], 8);
+        v4[i] = (b8 ? part[4 + i] : part[i]) + __shfl_xor_sync(0xffffffffu, b8 ? part[i] : part[4 + i], 8);
 #pragma unroll
     for (int i = 0; i < 2; ++i)
         v2[i] = (b4 ? v4[2 + i] : v4[i]) + __shfl_xor_sync(0xffffffffu, b4 ? v4[i] : v4[2 + i], 4);
@@ -329,27 +430,27 @@ __device__ __forceinline__ float warp_sum16(const float (&part)[16], int lane)
     return v;
 }
 
-// Chunk-end path operand tiles from one 16-token sub-block: Qx -> R slot, Kh -> K slot;
-// returns the bonus partials.  FULL: all 16 tokens valid (no bound checks).
+// Chunk-end path operand rows of one 8-token half sub-block, four channels per thread:
+// Qx -> R slot, Kh -> K slot, and the bonus partials.  FULL: all 8 tokens valid.
 template <bool FULL>
-__device__ __forceinline__ void prep_fast(unsigned char *st, int a, int cp, int tv, const uint32_t (&wr)[16],
-                                          float2 after, float2 u2, float (&part)[16])
+__device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t cbyte, int tv, const Q4 (&w)[8],
+                                          Q4 after, Q4 u, float (&part)[8])
 {
-    float2 run = after;  // product of w over the tokens after the current one, to the chunk end
+    Q4 run = after;  // product of w over the tokens after the current one, to the chunk end
 #pragma unroll
-    for (int m = 15; m >= 0; --m) {
-        const int t = 16 * a + m;
-        const uint32_t off = swz(t, 4 * cp);
-        float2 rr = make_float2(0.f, 0.f), kk = rr;
+    for (int m = 7; m >= 0; --m) {
+        const int t = t0h + m;
+        const uint32_t off = swz(t, cbyte);
+        uint2 rr = make_uint2(0u, 0u), kk = rr;
         if (FULL || t < tv) {
-            rr = ld_bf2(st + SLOT_R, off);
-            kk = ld_bf2(st + SLOT_K, off);
+            rr = ld_u2(st + SLOT_R, off);
+            kk = ld_u2(st + SLOT_K, off);
         }
-        const float2 w = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m]));
-        const float2 sin = mul2(run, w);
-        st_bf2(st + SLOT_R, off, make_float2(rr.x * rcp_approx(sin.x), rr.y * rcp_approx(sin.y)));
-        st_bf2(st + SLOT_K, off, mul2(kk, run));
-        part[m] = fmaf(rr.x * u2.x, kk.x, rr.y * u2.y * kk.y);
+        const Q4 r = unpack4(rr), k = unpack4(kk);
+        const Q4 sin = mul4(run, w[m]);
+        st_u2(st + SLOT_R, off, pack4({mul2(r.a, rcp2(sin.a)), mul2(r.b, rcp2(sin.b))}));
+        st_u2(st + SLOT_K, off, pack4(mul4(k, run)));
+        part[m] = bonus4(r, u, k);
         run = sin;
     }
 }
@@ -443,8 +544,12 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 
     if (warp < 4) {
         // =============================== prep group ===============================
-        const int a = warp, cp = lane;
-        const float2 u2 = *reinterpret_cast<const float2 *>(p.u + h * kN + 2 * cp);
+        // warp a: 16-token sub-block a; lane: half hf (tokens 16a + 8hf .. +7) and channel
+        // quad cq (channels 4cq .. 4cq+3)
+        const int a = warp, hf = lane >> 4, cq = lane & 15;
+        const int t0h = 16 * a + 8 * hf;
+        const uint32_t cbyte = 8 * cq;
+        const Q4 u4 = ld_q4(p.u + h * kN + 4 * cq);
         for (int c = 0; c < nchunks && !abort; ++c) {
             const int s = c % kStages;
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
@@ -458,49 +563,53 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 break;
             }
             bar_try(bar_full0 + 8 * s, (c / kStages) & 1);
-            // w of this sub-block (raw bf16 pairs; 1.0 past the end) and its product
-            uint32_t wr[16];
-            float2 G = make_float2(1.f, 1.f);
+            // w of this half (1.0 past the end) and its product; the other half's product
+            Q4 w[8];
+            Q4 Gh = one4();
 #pragma unroll
-            for (int m = 0; m < 16; ++m) {
-                const int t = 16 * a + m;
-                wr[m] = t < tv ? *reinterpret_cast<const uint32_t *>(st + SLOT_W + swz(t, 4 * cp)) : 0x3F803F80u;
-                G = mul2(G, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+            for (int m = 0; m < 8; ++m) {
+                const int t = t0h + m;
+                w[m] = t < tv ? unpack4(ld_u2(st + SLOT_W, swz(t, cbyte))) : one4();
+                Gh = mul4(Gh, w[m]);
             }
-            *reinterpret_cast<float2 *>(Hs + a * 64 + 2 * cp) = G;
+            const Q4 Go = shfl_xor4(Gh, 16);
+            if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
             named_sync_or(1, 128, 0);
-            float2 Gs[4];
+            Q4 Gs[4];
 #pragma unroll
-            for (int be = 0; be < 4; ++be) Gs[be] = *reinterpret_cast<const float2 *>(Hs + be * 64 + 2 * cp);
-            const float2 one = make_float2(1.f, 1.f);
-            float2 D = one, before = one, after = one, cab1 = one, cab2 = one;
+            for (int be = 0; be < 4; ++be) Gs[be] = ld_q4(Hs + be * 64 + 4 * cq);
+            Q4 D = one4(), before = one4(), aft = one4(), cab1 = one4(), cab2 = one4();
 #pragma unroll
             for (int be = 0; be < 4; ++be) {
-                D = mul2(D, Gs[be]);
-                if (be < a) before = mul2(before, Gs[be]);
-                if (be > a) after = mul2(after, Gs[be]);
+                D = mul4(D, Gs[be]);
+                if (be < a) before = mul4(before, Gs[be]);
+                if (be > a) aft = mul4(aft, Gs[be]);
                 if (be == a - 1) cab1 = Gs[be];                               // C_{a,a-2}
-                if (be == a - 1 || be == a - 2) cab2 = mul2(cab2, Gs[be]);    // C_{a,a-3}
+                if (be == a - 1 || be == a - 2) cab2 = mul4(cab2, Gs[be]);    // C_{a,a-3}
             }
+            // products over the tokens after this half (to the chunk end), from the
+            // sub-block start to this half, and from this half's end to the sub-block end
+            const Q4 after = hf ? aft : mul4(aft, Go);
+            const Q4 lead = hf ? Go : one4(), trail = hf ? one4() : Go;
             // single chunk-end reference unless a chunk decay product is below 2^-100
-            const int safe = so ? 0 : named_sync_or(1, 128, (D.x < kFastMin) | (D.y < kFastMin));
+            const int safe = so ? 0 : named_sync_or(1, 128, any_below(D, kFastMin));
             int hazard = 0;
-            float part[16];
+            float part[8];
             if (so) {
                 // local end state only: Kh[i] = k_i prod_{j>i} w_j (every factor <= 1)
-                float2 run = after;
+                Q4 run = after;
 #pragma unroll
-                for (int m = 15; m >= 0; --m) {
-                    const int t = 16 * a + m;
-                    const uint32_t off = swz(t, 4 * cp);
-                    const float2 kk = t < tv ? ld_bf2(st + SLOT_K, off) : make_float2(0.f, 0.f);
-                    st_bf2(st + SLOT_K, off, mul2(kk, run));
-                    run = mul2(run, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+                for (int m = 7; m >= 0; --m) {
+                    const int t = t0h + m;
+                    const uint32_t off = swz(t, cbyte);
+                    const uint2 kk = t < tv ? ld_u2(st + SLOT_K, off) : make_uint2(0u, 0u);
+                    st_u2(st + SLOT_K, off, pack4(mul4(unpack4(kk), run)));
+                    run = mul4(run, w[m]);
                     part[m] = 0.f;
                 }
             } else if (!safe) {
-                if (tv == kC) prep_fast<true>(st, a, cp, tv, wr, after, u2, part);
-                else prep_fast<false>(st, a, cp, tv, wr, after, u2, part);
+                if (tv == kC) prep_fast<true>(st, t0h, cbyte, tv, w, after, u4, part);
+                else prep_fast<false>(st, t0h, cbyte, tv, w, after, u4, part);
             } else {
                 // sub-block path; scratch = the stage two chunks ahead, free once chunk c-1 is done
                 unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
@@ -509,7 +618,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     ok = bar_wait_spin(bar_empty0 + 8 * ((c + 2) % kStages), ((c - 1) / kStages) & 1, spin_limit);
                 int hz = 0;
 #pragma unroll
-                for (int be = 0; be < 4; ++be) hz |= (Gs[be].x < kHazard) | (Gs[be].y < kHazard);
+                for (int be = 0; be < 4; ++be) hz |= any_below(Gs[be], kHazard);
                 const int vote = named_sync_or(1, 128, hz);
                 if (named_sync_or(1, 128, !ok)) {
                     abort = 1;
@@ -520,6 +629,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 hazard = vote;
                 if (hazard) {
                     // exact diagonal blocks from running products (inputs still intact here)
+                    const float2 one = make_float2(1.f, 1.f);
                     for (int item = tid; item < 4 * 120; item += 128) {
                         const int ab = item / 120;
                         int pr = item % 120, tt = 1;
@@ -543,44 +653,48 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     }
                     named_sync_or(1, 128, 0);
                 }
-                float2 suf[16];
-                float2 run = one;
+                // suf[m]: product of w from token m+1 of this half to the sub-block end
+                Q4 suf[8];
+                Q4 run = trail;
 #pragma unroll
-                for (int m = 15; m >= 0; --m) {
+                for (int m = 7; m >= 0; --m) {
                     suf[m] = run;
-                    run = mul2(run, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
+                    run = mul4(run, w[m]);
                 }
-                float2 pex = one;
+                Q4 pex = lead;  // product of w from the sub-block start to the token before t
 #pragma unroll
-                for (int m = 0; m < 16; ++m) {
-                    const int t = 16 * a + m;
-                    const uint32_t off = swz(t, 4 * cp);
-                    float2 rr = make_float2(0.f, 0.f), kk = rr;
+                for (int m = 0; m < 8; ++m) {
+                    const int t = t0h + m;
+                    const uint32_t off = swz(t, cbyte);
+                    uint2 rr = make_uint2(0u, 0u), kk = rr;
                     if (t < tv) {
-                        rr = ld_bf2(st + SLOT_R, off);
-                        kk = ld_bf2(st + SLOT_K, off);
+                        rr = ld_u2(st + SLOT_R, off);
+                        kk = ld_u2(st + SLOT_K, off);
                     }
-                    const float2 pin = mul2(pex, __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&wr[m])));
-                    const float2 qd = mul2(rr, pex);
-                    float2 kd;
-                    kd.x = pin.x >= kHazard ? kk.x * rcp_approx(pin.x) : 0.f;
-                    kd.y = pin.y >= kHazard ? kk.y * rcp_approx(pin.y) : 0.f;
-                    const float2 kbv = mul2(kk, suf[m]);
-                    st_bf2(st + SLOT_R, off, qd);
-                    st_bf2(st + SLOT_K, off, kd);
-                    st_bf2(scr + SCR_KB, off, kbv);
-                    st_bf2(scr + SCR_QI, off, mul2(qd, before));
-                    st_bf2(st + SLOT_W, off, mul2(kbv, after));
-                    if (a >= 1) st_bf2(scr + SCR_QO + 4096 * (a - 1), off, qd);              // Qo_{a-1}
-                    if (a >= 2) st_bf2(scr + SCR_QO + 4096 * (a - 2), off, mul2(qd, cab1));  // Qo_{a-2}
-                    if (a >= 3) st_bf2(scr + SCR_QO + 4096 * (a - 3), off, mul2(qd, cab2));  // Qo_{a-3}
-                    part[m] = fmaf(rr.x * u2.x, kk.x, rr.y * u2.y * kk.y);
+                    const Q4 r = unpack4(rr), k = unpack4(kk);
+                    const Q4 pin = mul4(pex, w[m]);
+                    const Q4 qd = mul4(r, pex);
+                    const Q4 kinv = {rcp2(pin.a), rcp2(pin.b)};
+                    Q4 kd = mul4(k, kinv);
+                    // Kd is dropped where the in-block product underflows the guard
+                    kd.a = pk(lo(pin.a) >= kHazard ? lo(kd.a) : 0.f, hi(pin.a) >= kHazard ? hi(kd.a) : 0.f);
+                    kd.b = pk(lo(pin.b) >= kHazard ? lo(kd.b) : 0.f, hi(pin.b) >= kHazard ? hi(kd.b) : 0.f);
+                    const Q4 kbv = mul4(k, suf[m]);
+                    st_u2(st + SLOT_R, off, pack4(qd));
+                    st_u2(st + SLOT_K, off, pack4(kd));
+                    st_u2(scr + SCR_KB, off, pack4(kbv));
+                    st_u2(scr + SCR_QI, off, pack4(mul4(qd, before)));
+                    st_u2(st + SLOT_W, off, pack4(mul4(kbv, aft)));
+                    if (a >= 1) st_u2(scr + SCR_QO + 4096 * (a - 1), off, pack4(qd));              // Qo_{a-1}
+                    if (a >= 2) st_u2(scr + SCR_QO + 4096 * (a - 2), off, pack4(mul4(qd, cab1)));  // Qo_{a-2}
+                    if (a >= 3) st_u2(scr + SCR_QO + 4096 * (a - 3), off, pack4(mul4(qd, cab2)));  // Qo_{a-3}
+                    part[m] = bonus4(r, u4, k);
                     pex = pin;
                 }
             }
-            const float tot = warp_sum16(part, lane);
-            if ((lane & 1) == 0) UB[s * 64 + 16 * a + ((lane >> 1) & 15)] = tot;
-            if (warp == 0) *reinterpret_cast<float2 *>(Dv + s * 64 + 2 * cp) = D;
+            const float tot = half_sum8(part, lane);
+            if ((lane & 1) == 0) UB[s * 64 + t0h + ((lane >> 1) & 7)] = tot;
+            if (warp == 0 && hf == 0) st_q4(Dv + s * 64 + 4 * cq, D);
             if (tid == 0) {
                 misc[2 + s] = safe;
                 misc[5 + s] = hazard;
@@ -796,15 +910,28 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                         else if (kbi == q && hazard) va[n] = DD[(q * 16 + lr) * 16 + ((colh + n) & 15)];
                     }
                 }
-                const float ub = UB[s * 64 + row];
-#pragma unroll
-                for (int n = 0; n < 32; ++n) {
-                    const int i = colh + n;
-                    va[n] = i < row ? va[n] : (i == row ? ub : 0.f);
-                }
+                // causal mask per 16-column block kb of this row: kb < q kept, kb == q the
+                // diagonal block (columns before the row kept, the diagonal itself is the bonus
+                // term, written last), kb > q zero
                 unsigned char *pt = st + (safe ? SLOT_K : SLOT_W);
-                st_row16_bf16(pt, row, 2 * colh, *reinterpret_cast<float(*)[16]>(&va[0]));
-                st_row16_bf16(pt, row, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&va[16]));
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int kb = 2 * hi + j;
+                    float(&vb)[16] = *reinterpret_cast<float(*)[16]>(&va[16 * j]);
+                    if (kb > q) {
+                        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+                        *reinterpret_cast<uint4 *>(pt + swz(row, 32 * kb)) = z;
+                        *reinterpret_cast<uint4 *>(pt + swz(row, 32 * kb + 16)) = z;
+                    } else {
+                        if (kb == q) {
+#pragma unroll
+                            for (int n = 0; n < 16; ++n) vb[n] = n < lr ? vb[n] : 0.f;
+                        }
+                        st_row16_bf16(pt, row, 32 * kb, vb);
+                    }
+                }
+                if (hi == (q >> 1))  // the thread that holds the diagonal block
+                    *reinterpret_cast<__nv_bfloat16 *>(pt + swz(row, 2 * row)) = __float2bfloat16_rn(UB[s * 64 + row]);
             }
             // ---- state: S *= D in TMEM; operand = bf16(D S_prev) (chunk-end path) or bf16(S_prev)
             {

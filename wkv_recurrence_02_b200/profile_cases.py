@@ -1,0 +1,73 @@
+"""Run single WKV launches on fixed synthetic shapes, for profilers (ncu) to capture.
+
+    python -m wkv_recurrence_02_b200.profile_cases [--case NAME ...] [--reps N]
+
+Every case first makes one untimed call (so a profiler can skip it with ``-s``), then
+``--reps`` calls of the same launch.  Cases:
+
+  wkv4          RWKV-4 scan, B16 T2048 C768 bf16 (150 MB of inputs, larger than L2)
+  finch         WKV-6 chunked prefill, B8 T1024 H32 N64 bf16 with s0 (256 CTAs, 16 chunks
+                each: the Finch-1.6B prefill shape at a quarter of its length)
+  long          WKV-6 chunked prefill with sequence split, B1 T4096 H64 (state-only pass
+                then full pass)
+  decode        WKV-6 T=1 decode, B256 H64 with the state updated in place (268 MB of state)
+
+Inputs come from the seeded generators in ``inputs``; nothing here checks results.
+"""
+import argparse
+
+import torch
+
+from . import inputs, ops
+
+CASES = ("wkv4", "finch", "long", "decode")
+
+
+def _wkv4(reps):
+    x = inputs.wkv4_inputs(16, 2048, 768, "bf16", seed=0, wu_seed=1)
+    a = [x[n].cuda() for n in ("w", "u", "k", "v")]
+    y = torch.empty_like(a[2])
+    for _ in range(1 + reps):
+        ops.wkv4_forward(*a, y=y)
+
+
+def _wkv6(B, T, H, reps, s0_std=0.1):
+    x = inputs.wkv6_inputs(B, T, H, 64, "bf16", seed=0, s0_std=s0_std)
+    a = [x[n].cuda() for n in ("r", "k", "v", "w", "u")]
+    s0 = x["s0"].cuda()
+    y = torch.empty_like(a[0])
+    sT = s0 if T == 1 else torch.empty_like(s0)
+    for _ in range(1 + reps):
+        ops.wkv6_forward(*a, s0=s0, y=y, sT=sT)
+
+
+def run(case, reps=1):
+    if case == "wkv4":
+        _wkv4(reps)
+    elif case == "finch":
+        _wkv6(8, 1024, 32, reps)
+    elif case == "long":
+        _wkv6(1, 4096, 64, reps)
+    elif case == "decode":
+        _wkv6(256, 1, 64, reps)
+    else:
+        raise ValueError(f"unknown case {case!r}; choose from {CASES}")
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--case", action="append", choices=CASES,
+                    help="case to run (repeatable; default: all, in the order listed)")
+    ap.add_argument("--reps", type=int, default=1)
+    args = ap.parse_args()
+    for case in args.case or CASES:
+        run(case, args.reps)
+    torch.cuda.synchronize()
+    status = ops.device_status()
+    print("device status", status)
+    if status != 0:
+        raise SystemExit(1)
+
+
+if __name__ == "__main__":
+    main()
