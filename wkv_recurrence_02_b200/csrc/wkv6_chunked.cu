@@ -575,17 +575,15 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             const Q4 Go = shfl_xor4(Gh, 16);
             if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
             named_sync_or(1, 128, 0);
-            Q4 Gs[4];
-#pragma unroll
-            for (int be = 0; be < 4; ++be) Gs[be] = ld_q4(Hs + be * 64 + 4 * cq);
-            Q4 D = one4(), before = one4(), aft = one4(), cab1 = one4(), cab2 = one4();
+            // sub-block products from shared memory (read by index there: a register array
+            // indexed by the warp's sub-block would be placed in local memory)
+            Q4 D = one4(), before = one4(), aft = one4();
 #pragma unroll
             for (int be = 0; be < 4; ++be) {
-                D = mul4(D, Gs[be]);
-                if (be < a) before = mul4(before, Gs[be]);
-                if (be > a) aft = mul4(aft, Gs[be]);
-                if (be == a - 1) cab1 = Gs[be];                               // C_{a,a-2}
-                if (be == a - 1 || be == a - 2) cab2 = mul4(cab2, Gs[be]);    // C_{a,a-3}
+                const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
+                D = mul4(D, g);
+                before = be < a ? mul4(before, g) : before;
+                aft = be > a ? mul4(aft, g) : aft;
             }
             // products over the tokens after this half (to the chunk end), from the
             // sub-block start to this half, and from this half's end to the sub-block end
@@ -618,7 +616,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     ok = bar_wait_spin(bar_empty0 + 8 * ((c + 2) % kStages), ((c - 1) / kStages) & 1, spin_limit);
                 int hz = 0;
 #pragma unroll
-                for (int be = 0; be < 4; ++be) hz |= any_below(Gs[be], kHazard);
+                for (int be = 0; be < 4; ++be) hz |= any_below(ld_q4(Hs + be * 64 + 4 * cq), kHazard);
+                // C_{a,a-2}: product of sub-block a-1; C_{a,a-3}: of sub-blocks a-2 and a-1
+                const Q4 cab1 = a >= 1 ? ld_q4(Hs + (a - 1) * 64 + 4 * cq) : one4();
+                const Q4 cab2 = a >= 2 ? mul4(cab1, ld_q4(Hs + (a - 2) * 64 + 4 * cq)) : cab1;
                 const int vote = named_sync_or(1, 128, hz);
                 if (named_sync_or(1, 128, !ok)) {
                     abort = 1;
