@@ -114,3 +114,42 @@ def test_wkv4_deterministic():
     b = ops.wkv4_forward(*args)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+# Shapes the TMA-fed kernel takes (row pitch a multiple of 16 bytes, the segment length L
+# dividing T, T/L >= 32): several tiles, a last tile with one segment, both element types.
+@pytest.mark.parametrize("B,T,C", [(2, 2048, 64), (1, 1056, 32), (2, 4096, 16), (3, 64, 40), (1, 1024, 8)])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_wkv4_tma_shapes(B, T, C, dtype):
+    err, dt = _run(B, T, C, dtype, seed=B * 7 + T + C)
+    assert err <= TOL[dt], err
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_wkv4_tma_large_keys_take_the_exact_paths(dtype):
+    """k ~ N(60, 4) at T = 1024: the fixed-frame and last-key shortcuts give way to the
+    running-maximum steps for some segments."""
+    x = inputs.wkv4_inputs(2, 1024, 48, dtype, seed=11)
+    g = torch.Generator().manual_seed(12)
+    k = (x["k"].float() * 4.0 + 60.0 + 30.0 * torch.randn(2, 1024, 1, generator=g)).to(x["k"].dtype)
+    y = ops.wkv4_forward(dev(x["w"]), dev(x["u"]), dev(k), dev(x["v"]))
+    torch.cuda.synchronize()
+    ref = oracle.wkv4(f64(x["w"]), f64(x["u"]), f64(k), f64(x["v"]))
+    assert rel_inf(f64(y), ref) <= TOL[y.dtype]
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_wkv4_tma_state_chaining(dtype):
+    """Two TMA-path calls of 1024 tokens with the state carried equal one call of 2048."""
+    B, T, C = 2, 2048, 32
+    x = inputs.wkv4_inputs(B, T, C, dtype, seed=13)
+    w, u, k, v = dev(x["w"]), dev(x["u"]), dev(x["k"]), dev(x["v"])
+    y1, s1 = ops.wkv4_forward(w, u, k[:, :1024].contiguous(), v[:, :1024].contiguous(), want_state=True)
+    y2, s2 = ops.wkv4_forward(w, u, k[:, 1024:].contiguous(), v[:, 1024:].contiguous(), s0=s1,
+                              want_state=True)
+    torch.cuda.synchronize()
+    ref_y, ref_s = oracle.wkv4(f64(x["w"]), f64(x["u"]), f64(x["k"]), f64(x["v"]), want_state=True)
+    assert rel_inf(f64(torch.cat([y1, y2], 1)), ref_y) <= TOL[k.dtype]
+    ga, gb = wkv4_state_views(f64(s2))
+    ra, rb = wkv4_state_views(ref_s)
+    assert rel_inf(ga, ra) <= 1e-4 and np.max(np.abs(gb - rb)) <= 1e-3

@@ -15,7 +15,9 @@
 //           the denominator never underflows, and every other weight is a single ex2
 //           (the decay a plain multiply).  If a weight overflows (keys more than 2^127
 //           apart) the lane redoes its segment with the running-maximum step.  The
-//           segment's largest and smallest key are noted on the way;
+//           segment's largest and smallest key are noted on the way, and the summary is
+//           renormalised (the denominator's binary exponent moved into the reference) so
+//           that the scan compares states by their true magnitude;
 //   scan    a 5-step warp shuffle scan combines segment summaries across lanes, and the
 //           carry from earlier tiles (or s0) is folded in;
 //   pass 2  each lane re-walks its segment from its exact incoming state.  When every
@@ -32,6 +34,8 @@
 // pair make both the row-contiguous fill and the lane-strided reads conflict-free).
 // y overwrites k's words in place and is written back with row-contiguous stores.
 #include "wkv_internal.cuh"
+
+#include <mutex>
 
 namespace wkv {
 namespace {
@@ -111,6 +115,18 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p)
 struct St {
     float a, b, p;
 };
+
+// (a, b, p) with b's binary exponent moved into p, so that 1 <= b < 4.  A summary taken
+// against a reference below its largest term can have b up to 2^127; combining it with a
+// later state by the larger exponent p would then flush its (still significant) weight to
+// zero, so pass-1 summaries are brought to this form first.  Requires b >= 1.
+__device__ __forceinline__ St normalized(float a, float b, float p)
+{
+    int e = ((__float_as_int(b) >> 23) & 0xff) - 127;
+    e = e < 126 ? e : 126;
+    const float s = __int_as_float((127 - e) << 23);  // 2^-e, exact
+    return {a * s, b * s, p + static_cast<float>(e)};
+}
 
 // State `e` (earlier), followed by a block whose local state is `l` and whose total
 // log2-decay is nw (= its length times w in log2 units).
@@ -346,9 +362,11 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
             kmina = kna * kLog2e;
             kminb = knb * kLog2e;
             const float Ba = lo(Bs), Bb = hi(Bs);
-            if (w2a >= 0.f && w2b >= 0.f && Ba <= 3.0e38f && Bb <= 3.0e38f) {
-                la = {lo(A), Ba, -lo(nF)};
-                lb = {hi(A), Bb, -hi(nF)};
+            // the sums must be finite (a weight above 2^127, or a product with v, overflows)
+            if (w2a >= 0.f && w2b >= 0.f && Ba <= 3.0e38f && Bb <= 3.0e38f && fabsf(lo(A)) <= 3.0e38f &&
+                fabsf(hi(A)) <= 3.0e38f) {
+                la = normalized(lo(A), Ba, -lo(nF));
+                lb = normalized(hi(A), Bb, -hi(nF));
             } else {
                 for (int j = 0; j < nv; ++j) {
                     const float2 kk = Word<T>::to_f2(mk[j]);
@@ -442,6 +460,488 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
     }
 }
 
+// ===================================================================== TMA-fed variant
+// Used when a 16-channel block of k, v, y can be addressed by the tensor-memory
+// accelerator (row pitch C * element size a multiple of 16 bytes, 16-byte aligned bases).
+// Same algorithm and segment structure as above, different data movement:
+//   * one CTA = one batch row x 16 channels; warp h = one 16-byte unit of channels
+//     (8 bf16 or 4 fp32, carried as f32x2 pairs), lane = segment;
+//   * the tile is held token-index-major: block i (128-byte aligned, as tensor copies
+//     require) holds row i of all 32 segments, 16 channels each, and arrives as one TMA
+//     box over a 4-D view (channel, i, segment, batch) of [B, T, C] -- exact when L
+//     divides T, which the launcher requires;
+//   * y replaces k in place and leaves as one TMA store per block (clipped at the last
+//     segment and at C).
+
+template <typename T> struct Unit;
+template <> struct Unit<__nv_bfloat16> {
+    static constexpr int NC = 8;  // channels per 16-byte unit
+    __device__ static void unpack(uint4 u, P2 (&x)[4])
+    {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            asm("mov.b64 %0, {%1, %2};" : "=l"(x[q].r) : "r"(w[q] << 16), "r"(w[q] & 0xFFFF0000u));
+    }
+    __device__ static uint4 pack(const P2 (&x)[4])
+    {
+        uint32_t w[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.bf16x2.f32 %0, h, l;\n\t}"
+                : "=r"(w[q])
+                : "l"(x[q].r));
+        return make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    __device__ static float get(const unsigned char *unit, int n)
+    {
+        return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(unit)[n]);
+    }
+    __device__ static void put(unsigned char *unit, int n, float x)
+    {
+        reinterpret_cast<__nv_bfloat16 *>(unit)[n] = __float2bfloat16_rn(x);
+    }
+    static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+};
+template <> struct Unit<float> {
+    static constexpr int NC = 4;
+    __device__ static void unpack(uint4 u, P2 (&x)[2])
+    {
+        x[0] = pk(__uint_as_float(u.x), __uint_as_float(u.y));
+        x[1] = pk(__uint_as_float(u.z), __uint_as_float(u.w));
+    }
+    __device__ static uint4 pack(const P2 (&x)[2])
+    {
+        return make_uint4(__float_as_uint(lo(x[0])), __float_as_uint(hi(x[0])), __float_as_uint(lo(x[1])),
+                          __float_as_uint(hi(x[1])));
+    }
+    __device__ static float get(const unsigned char *unit, int n) { return reinterpret_cast<const float *>(unit)[n]; }
+    __device__ static void put(unsigned char *unit, int n, float x) { reinterpret_cast<float *>(unit)[n] = x; }
+    static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+};
+
+// running min / max of the keys of one unit (bf16: two channels per instruction)
+template <typename T> struct KeyRange;
+template <> struct KeyRange<__nv_bfloat16> {
+    __nv_bfloat162 mx[4], mn[4];
+    __device__ void init()
+    {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            mx[q] = __floats2bfloat162_rn(-3.0e38f, -3.0e38f);
+            mn[q] = __floats2bfloat162_rn(3.0e38f, 3.0e38f);
+        }
+    }
+    __device__ void add(uint4 u)
+    {
+        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&w[q]);
+            mx[q] = __hmax2(mx[q], x);
+            mn[q] = __hmin2(mn[q], x);
+        }
+    }
+    __device__ float max(int n) const
+    {
+        return n & 1 ? __high2float(mx[n >> 1]) : __low2float(mx[n >> 1]);
+    }
+    __device__ float min(int n) const
+    {
+        return n & 1 ? __high2float(mn[n >> 1]) : __low2float(mn[n >> 1]);
+    }
+};
+template <> struct KeyRange<float> {
+    float mx[4], mn[4];
+    __device__ void init()
+    {
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            mx[n] = -3.4e38f;
+            mn[n] = 3.4e38f;
+        }
+    }
+    __device__ void add(uint4 u)
+    {
+        const float x[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w)};
+#pragma unroll
+        for (int n = 0; n < 4; ++n) {
+            mx[n] = fmaxf(mx[n], x[n]);
+            mn[n] = fminf(mn[n], x[n]);
+        }
+    }
+    __device__ float max(int n) const { return mx[n]; }
+    __device__ float min(int n) const { return mn[n]; }
+};
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ bool mbar_try(uint32_t bar, uint32_t phase)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred P;\n\tmbarrier.try_wait.parity.shared::cta.b64 P, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, P;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(phase)
+                 : "memory");
+    return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t phase, uint32_t limit)
+{
+    for (uint32_t it = 0; it < limit; ++it)
+        if (mbar_try(bar, phase)) return true;
+    return false;
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map, int c0, int c1, int c2,
+                                            int c3, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
+                 "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3, uint32_t src)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+struct TmaParams {
+    int64_t T, C;
+    const float *w, *u, *s0;
+    float *sT;
+    int *status;
+    uint32_t spin_limit;
+};
+
+template <typename T, int L>
+__global__ void __launch_bounds__(32 * (kCh / Unit<T>::NC), 3)
+wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
+                const __grid_constant__ CUtensorMap map_y, const TmaParams p)
+{
+    constexpr int NC = Unit<T>::NC;              // channels per lane
+    constexpr int NP = NC / 2;                   // f32x2 pairs per lane
+    constexpr int RB = kCh * sizeof(T);          // bytes of one token row (16 channels)
+    constexpr int BLK = kSegs * RB;              // bytes of block i: row i of every segment
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sk = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                                          ~static_cast<uintptr_t>(127));
+    unsigned char *sv = sk + L * BLK;
+    const uint32_t bar = smem_u32(sv + L * BLK);
+
+    const int64_t C = p.C, T_len = p.T;
+    const int64_t cblocks = (C + kCh - 1) / kCh;
+    const int b = static_cast<int>(blockIdx.x / cblocks);
+    const int c0 = static_cast<int>((blockIdx.x % cblocks) * kCh);
+    const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int cb = c0 + NC * h;  // first channel of this lane
+
+    const St empty{0.f, 0.f, kPEmpty};
+    float w2[NC], u2[NC];
+    P2 dd[NP], ub[NP];
+    St carry[NC];
+#pragma unroll
+    for (int n = 0; n < NC; ++n) {
+        const int c = cb + n;
+        const bool ok = c < C;
+        w2[n] = ok ? p.w[c] * kLog2e : 0.f;
+        u2[n] = ok ? p.u[c] * kLog2e : 0.f;
+        carry[n] = empty;
+        if (p.s0 && ok) {
+            const float *sp = p.s0 + static_cast<int64_t>(b) * 3 * C;
+            if (sp[C + c] != 0.f) carry[n] = {sp[c], sp[C + c], fmaxf(sp[2 * C + c] * kLog2e, kPEmpty)};
+        }
+    }
+#pragma unroll
+    for (int q = 0; q < NP; ++q) {
+        dd[q] = pk(ex2(-w2[2 * q]), ex2(-w2[2 * q + 1]));  // per-step decay factors
+        ub[q] = pk(ex2(u2[2 * q]), ex2(u2[2 * q + 1]));    // bonus factors
+    }
+    const P2 l2e = pk(kLog2e, kLog2e), nl2e = pk(-kLog2e, -kLog2e);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+
+    // this lane's unit in row 0 of its segment; row i is BLK bytes further
+    unsigned char *uk = sk + lane * RB + 16 * h;
+    const unsigned char *uv = sv + lane * RB + 16 * h;
+    const int nsegs = static_cast<int>(T_len / L);  // L divides T
+    int abort = 0, tile = 0;
+    for (int seg0 = 0; seg0 < nsegs; seg0 += kSegs, ++tile) {
+        if (h == 0) {  // warp 0: lane i brings block i of k and v
+            if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
+            __syncwarp();
+            if (lane < L) {
+                tma_load_4d(smem_u32(sk + lane * BLK), &map_k, c0, lane, seg0, b, bar);
+                tma_load_4d(smem_u32(sv + lane * BLK), &map_v, c0, lane, seg0, b, bar);
+            }
+        }
+        abort = __syncthreads_or(!mbar_wait(bar, tile & 1, p.spin_limit));
+        if (abort) break;
+        const int nv = seg0 + lane < nsegs ? L : 0;
+
+        // pass 1: local summaries against the segment's last key; key range
+        St la[NC];
+        KeyRange<T> kr;
+        kr.init();
+#pragma unroll
+        for (int n = 0; n < NC; ++n) la[n] = empty;
+        if (nv > 0) {
+            P2 nF[NP], A[NP], Bs[NP];
+            {
+                P2 kl[NP];
+                Unit<T>::unpack(*reinterpret_cast<const uint4 *>(uk + (nv - 1) * BLK), kl);
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    nF[q] = mul2(kl[q], nl2e);
+                    A[q] = pk(0.f, 0.f);
+                    Bs[q] = A[q];
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                if (i < nv) {
+                    const uint4 ku = *reinterpret_cast<const uint4 *>(uk + i * BLK);
+                    const uint4 vu = *reinterpret_cast<const uint4 *>(uv + i * BLK);
+                    kr.add(ku);
+                    P2 kk[NP], vv[NP];
+                    Unit<T>::unpack(ku, kk);
+                    Unit<T>::unpack(vu, vv);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
+                        A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
+                        Bs[q] = fma2(dd[q], Bs[q], E);
+                    }
+                }
+            }
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                const P2 a2 = A[n >> 1], b2 = Bs[n >> 1], f2 = nF[n >> 1];
+                const float an = n & 1 ? hi(a2) : lo(a2), bn = n & 1 ? hi(b2) : lo(b2);
+                const float fn = n & 1 ? hi(f2) : lo(f2);
+                if (w2[n] >= 0.f && bn <= 3.0e38f && fabsf(an) <= 3.0e38f) {
+                    la[n] = normalized(an, bn, -fn);
+                } else {  // a weight overflowed (or negative decay): running-maximum steps
+                    St s = empty;
+                    for (int i = 0; i < nv; ++i)
+                        update(s, Unit<T>::get(uk + i * BLK, n) * kLog2e, Unit<T>::get(uv + i * BLK, n), w2[n]);
+                    la[n] = s;
+                }
+            }
+        }
+
+        // inclusive scan over lanes (segment order) with segment lengths, then the
+        // exclusive prefix with the carry from earlier tiles folded in
+        float n_inc = static_cast<float>(nv);
+#pragma unroll
+        for (int off = 1; off < kSegs; off <<= 1) {
+            const float on = __shfl_up_sync(0xffffffffu, n_inc, off);
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                const St o = shfl_up(la[n], off);
+                if (lane >= off) la[n] = combine(o, la[n], n_inc * w2[n]);
+            }
+            if (lane >= off) n_inc += on;
+        }
+        float n_exc = __shfl_up_sync(0xffffffffu, n_inc, 1);
+        if (lane == 0) n_exc = 0.f;
+        const float n_tot = __shfl_sync(0xffffffffu, n_inc, kSegs - 1);
+        St pa[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            St e = shfl_up(la[n], 1);
+            if (lane == 0) e = empty;
+            pa[n] = combine(carry[n], e, n_exc * w2[n]);
+            carry[n] = combine(carry[n], shfl_idx(la[n], kSegs - 1), n_tot * w2[n]);
+        }
+
+        // pass 2: outputs from the exact incoming state; y replaces k in place
+        bool fixed = true;
+        float F[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            F[n] = fmaxf(pa[n].p, kr.max(n) * kLog2e + fmaxf(u2[n], 0.f));
+            fixed = fixed && w2[n] >= 0.f && fabsf(u2[n]) <= kFrame &&
+                    F[n] - (u2[n] + kr.min(n) * kLog2e) <= kFrame;
+        }
+        if (fixed) {
+            // every weight is 2^{x - F} <= 1 and the bonus term keeps the denominator >= 2^-60
+            P2 A[NP], Bs[NP], nF[NP];
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float s_lo = ex2(pa[2 * q].p - F[2 * q]), s_hi = ex2(pa[2 * q + 1].p - F[2 * q + 1]);
+                A[q] = pk(pa[2 * q].a * s_lo, pa[2 * q + 1].a * s_hi);
+                Bs[q] = pk(pa[2 * q].b * s_lo, pa[2 * q + 1].b * s_hi);
+                nF[q] = pk(-F[2 * q], -F[2 * q + 1]);
+            }
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                if (i < nv) {
+                    unsigned char *ui = uk + i * BLK;
+                    const uint4 ku = *reinterpret_cast<const uint4 *>(ui);
+                    const uint4 vu = *reinterpret_cast<const uint4 *>(uv + i * BLK);
+                    P2 kk[NP], vv[NP], o[NP];
+                    Unit<T>::unpack(ku, kk);
+                    Unit<T>::unpack(vu, vv);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
+                        const P2 bE = mul2(ub[q], E);
+                        o[q] = mul2(fma2(bE, vv[q], A[q]), rcp2(add2(Bs[q], bE)));
+                        A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
+                        Bs[q] = fma2(dd[q], Bs[q], E);
+                    }
+                    *reinterpret_cast<uint4 *>(ui) = Unit<T>::pack(o);
+                }
+            }
+        } else {
+            // running-maximum steps, exact for any inputs; channel by channel (y_n replaces
+            // k_n only after k_n has been read)
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                St s = pa[n];
+                for (int i = 0; i < nv; ++i) {
+                    const float k2 = Unit<T>::get(uk + i * BLK, n) * kLog2e, vx = Unit<T>::get(uv + i * BLK, n);
+                    const float o = output(s, k2, vx, u2[n]);
+                    update(s, k2, vx, w2[n]);
+                    Unit<T>::put(uk + i * BLK, n, o);
+                }
+            }
+        }
+
+        // y of this tile: one TMA store per segment (clipped at T and C)
+        fence_async_smem();
+        __syncthreads();
+        if (h == 0 && lane < L) {
+            tma_store_4d(&map_y, c0, lane, seg0, b, smem_u32(sk + lane * BLK));
+            bulk_wait_read();  // the block is refilled by the next tile
+        }
+        __syncthreads();
+    }
+    if (h == 0) bulk_wait_all();
+    if (abort) {
+        record_status(p.status, kStatusTimeout);
+        if (threadIdx.x == 0) mbar_wait(bar, tile & 1, p.spin_limit);  // bounded: let copies land
+        return;
+    }
+
+    if (p.sT && lane == 0) {
+        float *sp = p.sT + static_cast<int64_t>(b) * 3 * C;
+#pragma unroll
+        for (int n = 0; n < NC; ++n) {
+            const int c = cb + n;
+            if (c < C) {
+                const bool e = carry[n].b == 0.f;
+                sp[c] = carry[n].a;
+                sp[C + c] = carry[n].b;
+                sp[2 * C + c] = e ? kPEmpty : carry[n].p * kLn2;
+            }
+        }
+    }
+}
+
+template <typename T, int L>
+cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
+{
+    constexpr int NC = Unit<T>::NC;
+    constexpr int RB = kCh * sizeof(T);
+    constexpr int BLK = kSegs * RB;
+    constexpr int kThr = 32 * (kCh / NC);
+    const size_t smem = 2ull * L * BLK + 128 + 16;  // k and v blocks, alignment slack, mbarrier
+    auto enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    // 4-D view (channel, token within segment, segment, batch row) of [B, T, C]; L divides T
+    const cuuint64_t dims[4] = {static_cast<cuuint64_t>(a.C), static_cast<cuuint64_t>(L),
+                                static_cast<cuuint64_t>(a.T / L), static_cast<cuuint64_t>(a.B)};
+    const cuuint64_t strides[3] = {static_cast<cuuint64_t>(a.C * sizeof(T)),
+                                   static_cast<cuuint64_t>(L * a.C * sizeof(T)),
+                                   static_cast<cuuint64_t>(a.T * a.C * sizeof(T))};
+    const cuuint32_t box[4] = {static_cast<cuuint32_t>(kCh), 1, static_cast<cuuint32_t>(kSegs), 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUtensorMap mk, mv, my;
+    const void *ptrs[3] = {a.k, a.v, a.y};
+    CUtensorMap *maps[3] = {&mk, &mv, &my};
+    for (int i = 0; i < 3; ++i)
+        if (enc(maps[i], Unit<T>::kMapType, 4, const_cast<void *>(ptrs[i]), dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    auto kern = wkv4_tma_kernel<T, L>;
+    {
+        // shared-memory attributes, once per device and instantiation
+        static std::mutex mu;
+        static bool done[64] = {};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e != cudaSuccess) return e;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            if (e != cudaSuccess) return e;
+            done[dev] = true;
+        }
+    }
+    const int64_t blocks = a.B * ((a.C + kCh - 1) / kCh);
+    const TmaParams prm{a.T, a.C, a.w, a.u, a.s0, a.sT, a.status, 1u << 22};
+    kern<<<static_cast<unsigned>(blocks), kThr, smem, s>>>(mk, mv, my, prm);
+    return cudaGetLastError();
+}
+
+// Segment length: the smallest power of two giving 32 segments that cover T, capped at
+// LMAX (a tile of k and v then takes 64 KB, three CTAs per SM).
+int pick_L(int64_t T, int LMAX)
+{
+    const int64_t per_seg = (T + kSegs - 1) / kSegs;
+    int L = 1;
+    while (L < per_seg && L < LMAX) L *= 2;
+    return L;
+}
+
+template <typename T>
+cudaError_t launch_tma_T(const Wkv4Args &a, int L, cudaStream_t s)
+{
+    switch (L) {
+    case 1: return launch_tma_L<T, 1>(a, s);
+    case 2: return launch_tma_L<T, 2>(a, s);
+    case 4: return launch_tma_L<T, 4>(a, s);
+    case 8: return launch_tma_L<T, 8>(a, s);
+    case 16: return launch_tma_L<T, 16>(a, s);
+    default: break;
+    }
+    if constexpr (sizeof(T) == 2) return launch_tma_L<T, 32>(a, s);
+    return cudaErrorInvalidValue;
+}
+
+// True when TMA can address the 16-channel blocks: row pitch a multiple of 16 bytes,
+// 16-byte aligned bases, coordinates within int32.
+bool tma_usable(const Wkv4Args &a)
+{
+    const int64_t es = a.bf16 ? 2 : 4;
+    auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+    return a.T > 0 && a.B > 0 && a.C > 0 && (a.C * es) % 16 == 0 && al16(a.k) && al16(a.v) && al16(a.y) &&
+           a.T < (int64_t(1) << 31) - 64 && a.B < (int64_t(1) << 31) && a.C < (int64_t(1) << 31) &&
+           tensor_map_encoder() != nullptr;
+}
+
 template <typename T, int L>
 cudaError_t launch_L(const Wkv4Args &a, cudaStream_t s)
 {
@@ -480,6 +980,12 @@ cudaError_t launch_T(const Wkv4Args &a, cudaStream_t s)
 cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s)
 {
     if (a.B * ((a.C + kCh - 1) / kCh) > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (tma_usable(a)) {
+        const int L = pick_L(a.T, a.bf16 ? 32 : 16);
+        // the 4-D view needs L to divide T; a box spans 32 segments, so T/L >= 32
+        if (a.T % L == 0 && a.T / L >= kSegs)
+            return a.bf16 ? launch_tma_T<__nv_bfloat16>(a, L, s) : launch_tma_T<float>(a, L, s);
+    }
     return a.bf16 ? launch_T<__nv_bfloat16, 32>(a, s) : launch_T<float, 16>(a, s);
 }
 

@@ -1052,24 +1052,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 }
 
 // ---------------------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 get_encoder()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-        cudaDriverEntryPointQueryResult q;
-        void *ptr = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    });
-    return fn;
-}
 
 // [B, T, H, N] bf16, box = 64 channels x 1 head x 64 tokens x 1 batch row
 bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t H)
 {
-    auto enc = get_encoder();
+    auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(kN), static_cast<cuuint64_t>(H),
                           static_cast<cuuint64_t>(T), static_cast<cuuint64_t>(B)};
@@ -1084,6 +1071,21 @@ bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t 
 }
 
 }  // namespace
+
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link-time driver dependency)
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        cudaDriverEntryPointQueryResult q;
+        void *ptr = nullptr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    });
+    return fn;
+}
 
 int g_chunked_inject_timeout = 0;  // test hook: set through rwkv_debug_inject_timeout
 

@@ -2,6 +2,8 @@
 // Nothing here is part of the public ABI (include/rwkv_wkv.h is).
 #pragma once
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 #include <stdint.h>
@@ -39,6 +41,9 @@ struct Wkv6Args {
     int *status;
     int segments;               // chunked kernel: 0 = choose the sequence split, n = at most n
 };
+
+// cuTensorMapEncodeTiled from the driver (null if unavailable).
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 
 // Each launcher returns the cudaError_t of its launch(es).
 cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s);
