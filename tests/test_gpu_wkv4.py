@@ -116,19 +116,19 @@ def test_wkv4_deterministic():
     assert torch.equal(a, b)
 
 
-# Shapes the TMA-fed kernel takes (row pitch a multiple of 16 bytes, the segment length L
-# dividing T, T/L >= 32): several tiles, a last tile with one segment, both element types.
+# Several tiles (the carry between them), a last tile holding one segment, 16-byte rows.
 @pytest.mark.parametrize("B,T,C", [(2, 2048, 64), (1, 1056, 32), (2, 4096, 16), (3, 64, 40), (1, 1024, 8)])
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_wkv4_tma_shapes(B, T, C, dtype):
+def test_wkv4_tile_shapes(B, T, C, dtype):
     err, dt = _run(B, T, C, dtype, seed=B * 7 + T + C)
     assert err <= TOL[dt], err
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_wkv4_tma_large_keys_take_the_exact_paths(dtype):
-    """k ~ N(60, 4) at T = 1024: the fixed-frame and last-key shortcuts give way to the
-    running-maximum steps for some segments."""
+def test_wkv4_spread_keys_take_the_exact_paths(dtype):
+    """Keys shifted per token by N(60, 30^2): the fixed-frame and last-key shortcuts give way
+    to the running-maximum steps for most segments, and pass-1 summaries whose denominator
+    reaches 2^100 and more must still combine by their true magnitude."""
     x = inputs.wkv4_inputs(2, 1024, 48, dtype, seed=11)
     g = torch.Generator().manual_seed(12)
     k = (x["k"].float() * 4.0 + 60.0 + 30.0 * torch.randn(2, 1024, 1, generator=g)).to(x["k"].dtype)
@@ -139,8 +139,8 @@ def test_wkv4_tma_large_keys_take_the_exact_paths(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-def test_wkv4_tma_state_chaining(dtype):
-    """Two TMA-path calls of 1024 tokens with the state carried equal one call of 2048."""
+def test_wkv4_state_chaining_full_tiles(dtype):
+    """Two calls of 1024 tokens (whole tiles) with the state carried equal one call of 2048."""
     B, T, C = 2, 2048, 32
     x = inputs.wkv4_inputs(B, T, C, dtype, seed=13)
     w, u, k, v = dev(x["w"]), dev(x["u"]), dev(x["k"]), dev(x["v"])

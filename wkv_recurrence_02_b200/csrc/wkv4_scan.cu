@@ -133,9 +133,11 @@ __device__ __forceinline__ St normalized(float a, float b, float p)
 __device__ __forceinline__ St combine(St e, St l, float nw)
 {
     const float pe = e.p - nw;
-    const float q = fmaxf(pe, l.p);
-    const float fe = ex2(pe - q), fl = ex2(l.p - q);
-    return {fmaf(e.a, fe, l.a * fl), fmaf(e.b, fe, l.b * fl), q};
+    const float d = pe - l.p;
+    const float x = ex2(-fabsf(d));  // the smaller side's factor; the larger side's is 1
+    const bool early = d >= 0.f;
+    const float fe = early ? 1.f : x, fl = early ? x : 1.f;
+    return {fmaf(e.a, fe, l.a * fl), fmaf(e.b, fe, l.b * fl), early ? pe : l.p};
 }
 
 // One token into the state: decay the past by 2^{-w2}, add 2^{k2} (v | 1).
@@ -471,7 +473,9 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
 //     box over a 4-D view (channel, i, segment, batch) of [B, T, C] -- exact when L
 //     divides T, which the launcher requires;
 //   * y replaces k in place and leaves as one TMA store per block (clipped at the last
-//     segment and at C).
+//     segment and at C);
+//   * two tile buffers: tile tau+1 is loaded while tile tau is scanned, and tile tau's
+//     store drains while tile tau+1 is scanned.
 
 template <typename T> struct Unit;
 template <> struct Unit<__nv_bfloat16> {
@@ -626,7 +630,7 @@ struct TmaParams {
     uint32_t spin_limit;
 };
 
-template <typename T, int L>
+template <typename T, int L, int NB>
 __global__ void __launch_bounds__(32 * (kCh / Unit<T>::NC), 3)
 wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                 const __grid_constant__ CUtensorMap map_y, const TmaParams p)
@@ -635,11 +639,12 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     constexpr int NP = NC / 2;                   // f32x2 pairs per lane
     constexpr int RB = kCh * sizeof(T);          // bytes of one token row (16 channels)
     constexpr int BLK = kSegs * RB;              // bytes of block i: row i of every segment
+    // NB buffers (tile tau in buffer tau % NB), each k blocks then v blocks; NB mbarriers.
+    // With one buffer the launcher guarantees a single tile.
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sk = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                                          ~static_cast<uintptr_t>(127));
-    unsigned char *sv = sk + L * BLK;
-    const uint32_t bar = smem_u32(sv + L * BLK);
+    unsigned char *sbase = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                                             ~static_cast<uintptr_t>(127));
+    const uint32_t bar0 = smem_u32(sbase + NB * 2 * L * BLK);  // + 8 * buffer
 
     const int64_t C = p.C, T_len = p.T;
     const int64_t cblocks = (C + kCh - 1) / kCh;
@@ -672,27 +677,41 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const P2 l2e = pk(kLog2e, kLog2e), nl2e = pk(-kLog2e, -kLog2e);
 
     if (threadIdx.x == 0) {
-        mbar_init(bar, 1);
+        for (int i = 0; i < NB; ++i) mbar_init(bar0 + 8 * i, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncthreads();
 
-    // this lane's unit in row 0 of its segment; row i is BLK bytes further
-    unsigned char *uk = sk + lane * RB + 16 * h;
-    const unsigned char *uv = sv + lane * RB + 16 * h;
     const int nsegs = static_cast<int>(T_len / L);  // L divides T
-    int abort = 0, tile = 0;
-    for (int seg0 = 0; seg0 < nsegs; seg0 += kSegs, ++tile) {
-        if (h == 0) {  // warp 0: lane i brings block i of k and v
-            if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
-            __syncwarp();
-            if (lane < L) {
-                tma_load_4d(smem_u32(sk + lane * BLK), &map_k, c0, lane, seg0, b, bar);
-                tma_load_4d(smem_u32(sv + lane * BLK), &map_v, c0, lane, seg0, b, bar);
-            }
+    const int ntiles = (nsegs + kSegs - 1) / kSegs;
+    // warp 0: lane i brings block i of k and v of tile tl into its buffer
+    auto issue = [&](int tl) {
+        unsigned char *bk = sbase + (tl % NB) * 2 * L * BLK;
+        const uint32_t bar = bar0 + 8 * (tl % NB);
+        if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
+        __syncwarp();
+        if (lane < L) {
+            tma_load_4d(smem_u32(bk + lane * BLK), &map_k, c0, lane, kSegs * tl, b, bar);
+            tma_load_4d(smem_u32(bk + L * BLK + lane * BLK), &map_v, c0, lane, kSegs * tl, b, bar);
         }
-        abort = __syncthreads_or(!mbar_wait(bar, tile & 1, p.spin_limit));
+    };
+    if (h == 0 && ntiles > 0) issue(0);
+    int abort = 0, tile = 0, issued = ntiles > 0 ? 1 : 0;
+    for (; tile < ntiles; ++tile) {
+        const int seg0 = kSegs * tile;
+        if (NB > 1 && tile + 1 < ntiles && h == 0) {
+            // the next tile goes to the other buffer, whose last tile's store must have read it
+            if (lane < L) bulk_wait_read();
+            issue(tile + 1);
+            ++issued;
+        }
+        unsigned char *sk = sbase + (tile % NB) * 2 * L * BLK;
+        const unsigned char *sv = sk + L * BLK;
+        abort = __syncthreads_or(!mbar_wait(bar0 + 8 * (tile % NB), (tile / NB) & 1, p.spin_limit));
         if (abort) break;
+        // this lane's unit in row 0 of its segment; row i is BLK bytes further
+        unsigned char *uk = sk + lane * RB + 16 * h;
+        const unsigned char *uv = sv + lane * RB + 16 * h;
         const int nv = seg0 + lane < nsegs ? L : 0;
 
         // pass 1: local summaries against the segment's last key; key range
@@ -828,16 +847,14 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         // y of this tile: one TMA store per segment (clipped at T and C)
         fence_async_smem();
         __syncthreads();
-        if (h == 0 && lane < L) {
-            tma_store_4d(&map_y, c0, lane, seg0, b, smem_u32(sk + lane * BLK));
-            bulk_wait_read();  // the block is refilled by the next tile
-        }
-        __syncthreads();
+        if (h == 0 && lane < L) tma_store_4d(&map_y, c0, lane, seg0, b, smem_u32(sk + lane * BLK));
     }
     if (h == 0) bulk_wait_all();
     if (abort) {
         record_status(p.status, kStatusTimeout);
-        if (threadIdx.x == 0) mbar_wait(bar, tile & 1, p.spin_limit);  // bounded: let copies land
+        if (threadIdx.x == 0)  // bounded: let the copies in flight land before the CTA exits
+            for (int t = tile; t < issued; ++t) mbar_wait(bar0 + 8 * (t % NB), (t / NB) & 1, p.spin_limit);
+        __syncthreads();
         return;
     }
 
@@ -856,14 +873,14 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     }
 }
 
-template <typename T, int L>
+template <typename T, int L, int NB>
 cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
 {
     constexpr int NC = Unit<T>::NC;
     constexpr int RB = kCh * sizeof(T);
     constexpr int BLK = kSegs * RB;
     constexpr int kThr = 32 * (kCh / NC);
-    const size_t smem = 2ull * L * BLK + 128 + 16;  // k and v blocks, alignment slack, mbarrier
+    const size_t smem = NB * 2ull * L * BLK + 128 + 16;  // buffers of k and v blocks, slack, mbarriers
     auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     // 4-D view (channel, token within segment, segment, batch row) of [B, T, C]; L divides T
@@ -882,7 +899,7 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
-    auto kern = wkv4_tma_kernel<T, L>;
+    auto kern = wkv4_tma_kernel<T, L, NB>;
     {
         // shared-memory attributes, once per device and instantiation
         static std::mutex mu;
@@ -906,8 +923,7 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
-// Segment length: the smallest power of two giving 32 segments that cover T, capped at
-// LMAX (a tile of k and v then takes 64 KB, three CTAs per SM).
+// Segment length: the smallest power of two giving 32 segments that cover T, capped at LMAX.
 int pick_L(int64_t T, int LMAX)
 {
     const int64_t per_seg = (T + kSegs - 1) / kSegs;
@@ -916,18 +932,29 @@ int pick_L(int64_t T, int LMAX)
     return L;
 }
 
+// One tile (T <= 32 L): one buffer of up to 64 KB.  Several tiles: two buffers of up to
+// 32 KB each (half the segment length), so tile tau+1 loads while tile tau is scanned.
+// Both keep three CTAs per SM.
 template <typename T>
-cudaError_t launch_tma_T(const Wkv4Args &a, int L, cudaStream_t s)
+cudaError_t launch_tma_T(const Wkv4Args &a, int L, int NB, cudaStream_t s)
 {
-    switch (L) {
-    case 1: return launch_tma_L<T, 1>(a, s);
-    case 2: return launch_tma_L<T, 2>(a, s);
-    case 4: return launch_tma_L<T, 4>(a, s);
-    case 8: return launch_tma_L<T, 8>(a, s);
-    case 16: return launch_tma_L<T, 16>(a, s);
-    default: break;
+    if (NB == 1) {
+        switch (L) {
+        case 1: return launch_tma_L<T, 1, 1>(a, s);
+        case 2: return launch_tma_L<T, 2, 1>(a, s);
+        case 4: return launch_tma_L<T, 4, 1>(a, s);
+        case 8: return launch_tma_L<T, 8, 1>(a, s);
+        case 16: return launch_tma_L<T, 16, 1>(a, s);
+        default: break;
+        }
+        if constexpr (sizeof(T) == 2)
+            if (L == 32) return launch_tma_L<T, 32, 1>(a, s);
+        return cudaErrorInvalidValue;
     }
-    if constexpr (sizeof(T) == 2) return launch_tma_L<T, 32>(a, s);
+    if constexpr (sizeof(T) == 2)
+        if (L == 16) return launch_tma_L<T, 16, 2>(a, s);
+    if constexpr (sizeof(T) == 4)
+        if (L == 8) return launch_tma_L<T, 8, 2>(a, s);
     return cudaErrorInvalidValue;
 }
 
@@ -981,10 +1008,15 @@ cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s)
 {
     if (a.B * ((a.C + kCh - 1) / kCh) > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (tma_usable(a)) {
-        const int L = pick_L(a.T, a.bf16 ? 32 : 16);
+        const int lmax = a.bf16 ? 32 : 16;
+        int L = pick_L(a.T, lmax), NB = 1;
+        if (a.T > static_cast<int64_t>(kSegs) * L) {  // several tiles: two half-size buffers
+            L = pick_L(a.T, lmax / 2);
+            NB = 2;
+        }
         // the 4-D view needs L to divide T; a box spans 32 segments, so T/L >= 32
         if (a.T % L == 0 && a.T / L >= kSegs)
-            return a.bf16 ? launch_tma_T<__nv_bfloat16>(a, L, s) : launch_tma_T<float>(a, L, s);
+            return a.bf16 ? launch_tma_T<__nv_bfloat16>(a, L, NB, s) : launch_tma_T<float>(a, L, NB, s);
     }
     return a.bf16 ? launch_T<__nv_bfloat16, 32>(a, s) : launch_T<float, 16>(a, s);
 }

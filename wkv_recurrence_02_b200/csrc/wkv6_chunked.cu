@@ -254,10 +254,6 @@ __device__ __forceinline__ float2 ld_bf2(const unsigned char *tile, uint32_t off
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + off));
 }
 
-__device__ __forceinline__ void st_bf2(unsigned char *tile, uint32_t off, float2 x)
-{
-    *reinterpret_cast<uint32_t *>(tile + off) = pack_bf16(x.x, x.y);
-}
 
 __device__ __forceinline__ float2 mul2(float2 a, float2 b) { return make_float2(a.x * b.x, a.y * b.y); }
 
@@ -315,7 +311,6 @@ __device__ __forceinline__ P2 fma2(P2 a, P2 b, P2 c)
     return d;
 }
 __device__ __forceinline__ P2 one2() { return pk(1.f, 1.f); }
-__device__ __forceinline__ P2 zero2() { return pk(0.f, 0.f); }
 
 // bf16 pair (low half = first channel) -> exact fp32 pair
 __device__ __forceinline__ P2 unpack2(uint32_t x)
@@ -345,7 +340,6 @@ __device__ __forceinline__ P2 ld_p2(const float *p)
     const float2 f = *reinterpret_cast<const float2 *>(p);
     return pk(f.x, f.y);
 }
-__device__ __forceinline__ void st_p2(float *p, P2 x) { *reinterpret_cast<float2 *>(p) = make_float2(lo(x), hi(x)); }
 
 // four channels of one token row: two packed pairs
 struct Q4 {
