@@ -5,7 +5,7 @@
 Every case first makes one untimed call (so a profiler can skip it with ``-s``), then
 ``--reps`` calls of the same launch.  Cases:
 
-  wkv4          RWKV-4 scan, B16 T2048 C768 bf16 (150 MB of inputs, larger than L2)
+  wkv4          RWKV-4 scan, B8 T1024 C768 bf16: one layer of the 169M model's shape
   finch         WKV-6 chunked prefill, B8 T1024 H32 N64 bf16 with s0 (256 CTAs, 16 chunks
                 each: the Finch-1.6B prefill shape at a quarter of its length)
   long          WKV-6 chunked prefill with sequence split, B1 T4096 H64 (state-only pass
@@ -24,7 +24,7 @@ CASES = ("wkv4", "finch", "long", "decode")
 
 
 def _wkv4(reps):
-    x = inputs.wkv4_inputs(16, 2048, 768, "bf16", seed=0, wu_seed=1)
+    x = inputs.wkv4_inputs(8, 1024, 768, "bf16", seed=0, wu_seed=1)
     a = [x[n].cuda() for n in ("w", "u", "k", "v")]
     y = torch.empty_like(a[2])
     for _ in range(1 + reps):
