@@ -583,8 +583,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             // sub-block start to this half, and from this half's end to the sub-block end
             const Q4 after = hf ? aft : mul4(aft, Go);
             const Q4 lead = hf ? Go : one4(), trail = hf ? one4() : Go;
-            // single chunk-end reference unless a chunk decay product is below 2^-100
-            const int safe = so ? 0 : named_sync_or(1, 128, any_below(D, kFastMin));
+            // single chunk-end reference unless a chunk decay product is below 2^-100.  Every
+            // warp's 32 lanes cover all 16 channel quads, so a warp vote is the chunk's vote
+            // (the same in all four warps): no group barrier.
+            const int safe = so ? 0 : __any_sync(0xffffffffu, any_below(D, kFastMin));
             int hazard = 0;
             float part[8];
             if (so) {
@@ -614,7 +616,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 // C_{a,a-2}: product of sub-block a-1; C_{a,a-3}: of sub-blocks a-2 and a-1
                 const Q4 cab1 = a >= 1 ? ld_q4(Hs + (a - 1) * 64 + 4 * cq) : one4();
                 const Q4 cab2 = a >= 2 ? mul4(cab1, ld_q4(Hs + (a - 2) * 64 + 4 * cq)) : cab1;
-                const int vote = named_sync_or(1, 128, hz);
+                const int vote = __any_sync(0xffffffffu, hz);  // all channels, as above
                 if (named_sync_or(1, 128, !ok)) {
                     abort = 1;
                     misc[1] = 1;
