@@ -174,6 +174,24 @@ class Workload:
     launches_per_step = 12 + 1 + 4 + 1
 
 
+def max_over_ranks(values, dist, device=None):
+    """Each value's maximum over all ranks (the job's time is its slowest rank's); the
+    identity with one process.  Works with any process-group backend: CPU tensors for gloo,
+    device tensors for nccl."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_tokens_per_s(world, tokens_per_step_per_rank, steps, ms_max):
+    """Whole-job throughput: every rank runs the same fixed work per step (weak scaling),
+    so the job processes world x tokens per step in the slowest rank's time."""
+    return world * tokens_per_step_per_rank * steps / (ms_max * 1e-3)
+
+
 def run_ours(args, rank, world, dist):
     import torch
     from wkv_recurrence_02_b200 import inputs, ops
@@ -228,10 +246,7 @@ def run_ours(args, rank, world, dist):
     # end to end through the public API with host buffers: H2D of every input, D2H of results
     e2e_ms, h2d, d2h = run_e2e(torch, ops, wl, stream, dev, max(3, min(args.steps, 10)), barrier)
 
-    ms_t = torch.tensor([ms, e2e_ms], device=dev)
-    if dist is not None:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max, e2e_max = ms_t.tolist()
+    ms_max, e2e_max = max_over_ranks([ms, e2e_ms], dist, device=dev)
     status = ops.device_status()
     if rank != 0:
         return None
@@ -263,7 +278,7 @@ def run_ours(args, rank, world, dist):
     traffic = load_traffic(dom_launch)
     cpu = cpu_baseline(args.cpu_sample_scale) if (world == 1 and not args.skip_cpu) else None
     line = {
-        "metric": METRIC, "value": world * STEP_TOKENS * args.steps / (ms_max * 1e-3),
+        "metric": METRIC, "value": job_tokens_per_s(world, STEP_TOKENS, args.steps, ms_max),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch CPU generator)",
@@ -277,7 +292,7 @@ def run_ours(args, rank, world, dist):
                      "frac": round(achieved / hbm, 4), "traffic": traffic},
         "parts": parts,
         "cpu_baseline": cpu,
-        "e2e": {"value": world * STEP_TOKENS / (e2e_max * 1e-3), "unit": UNIT,
+        "e2e": {"value": job_tokens_per_s(world, STEP_TOKENS, 1, e2e_max), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": Workload.launches_per_step * args.steps,
         "clocks": sampler.summary(t_wall0, t_wall1),
