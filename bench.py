@@ -171,7 +171,10 @@ class Workload:
         run("wkv6_decode", lambda: ops.wkv6_forward(d["r"], d["k"], d["v"], d["w"], d["u"],
                                                     s0=d["s0"], y=d["y"], sT=d["s0"]))
 
-    launches_per_step = 12 + 1 + 4 + 1
+    # 12 WKV-4 layers, the Finch prefill, 4 long-context calls of two launches each (the
+    # state-only and full passes of the sequence split at 64 heads), the decode step; the
+    # ncu launch list of this step counts the same (profiles/launch_list_bench_step.md)
+    launches_per_step = 12 + 1 + 4 * 2 + 1
 
 
 def max_over_ranks(values, dist, device=None):
@@ -245,6 +248,7 @@ def run_ours(args, rank, world, dist):
 
     # end to end through the public API with host buffers: H2D of every input, D2H of results
     e2e_ms, h2d, d2h = run_e2e(torch, ops, wl, stream, dev, max(3, min(args.steps, 10)), barrier)
+    next_rows = measure_next_rows(torch, inputs, ops, dev, stream)
 
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], dist, device=dev)
     status = ops.device_status()
@@ -295,10 +299,39 @@ def run_ours(args, rank, world, dist):
         "e2e": {"value": job_tokens_per_s(world, STEP_TOKENS, 1, e2e_max), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": Workload.launches_per_step * args.steps,
+        "next_rows": next_rows,
         "clocks": sampler.summary(t_wall0, t_wall1),
         "device_status": status,
     }
     return line
+
+
+def measure_next_rows(torch, inputs, ops, dev, stream, reps=50):
+    """Rows beyond the step, timed on their own (not part of the step's metric): the RWKV-4
+    decode step (T = 1) at the width of a 7B model, state updated in place."""
+    hbm, _ = load_peaks()
+    B, C = 2048, 4096
+    x = inputs.wkv4_inputs(B, 1, C, "bf16", seed=5, wu_seed=6)
+    w, u, k, v = (x[n].to(dev) for n in ("w", "u", "k", "v"))
+    st = torch.zeros(B, 3, C, dtype=torch.float32, device=dev)
+    st[:, 0] = torch.randn(B, C, device=dev)
+    st[:, 1] = 1.0 + torch.rand(B, C, device=dev)
+    y = torch.empty_like(k)
+    for _ in range(3):
+        ops.wkv4_forward(w, u, k, v, s0=st, sT=st, y=y, want_state=True)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        ops.wkv4_forward(w, u, k, v, s0=st, sT=st, y=y, want_state=True)
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    us = a.elapsed_time(b) * 1e3 / reps
+    nbytes = B * C * (2 * 2 + 2 + 2 * 3 * 4) + 2 * C * 4  # k, v, y bf16; state in and out; w, u
+    gbs = nbytes / (us * 1e-6) / 1e9
+    return {"wkv4_decode_B2048_C4096": {"avg_us": round(us, 2), "algorithmic_bytes": nbytes,
+                                        "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                                        "state_bytes": 2 * B * 3 * C * 4, "launches": reps}}
 
 
 def run_e2e(torch, ops, wl, stream, dev, steps, barrier):

@@ -153,3 +153,36 @@ def test_wkv4_state_chaining_full_tiles(dtype):
     ga, gb = wkv4_state_views(f64(s2))
     ra, rb = wkv4_state_views(ref_s)
     assert rel_inf(ga, ra) <= 1e-4 and np.max(np.abs(gb - rb)) <= 1e-3
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("C", [96, 37])
+def test_wkv4_decode_chained_in_place_matches_the_oracle(dtype, C):
+    """40 single-token calls (the T = 1 decode kernel), the state updated in place, equal
+    the oracle over all 40 tokens: every y and the final (a, b, p) state."""
+    B, T = 4, 40
+    x = inputs.wkv4_inputs(B, T, C, dtype, seed=21)
+    w, u, k, v = dev(x["w"]), dev(x["u"]), dev(x["k"]), dev(x["v"])
+    y0, s = ops.wkv4_forward(w, u, k[:, :1].contiguous(), v[:, :1].contiguous(), want_state=True)
+    ys = [y0]
+    for t in range(1, T):
+        yt, s2 = ops.wkv4_forward(w, u, k[:, t:t + 1].contiguous(), v[:, t:t + 1].contiguous(), s0=s, sT=s,
+                                  want_state=True)
+        assert s2.data_ptr() == s.data_ptr()
+        ys.append(yt)
+    torch.cuda.synchronize()
+    ref_y, ref_s = oracle.wkv4(f64(x["w"]), f64(x["u"]), f64(x["k"]), f64(x["v"]), want_state=True)
+    assert rel_inf(f64(torch.cat(ys, 1)), ref_y) <= TOL[k.dtype]
+    ga, gb = wkv4_state_views(f64(s))
+    ra, rb = wkv4_state_views(ref_s)
+    assert rel_inf(ga, ra) <= 1e-4 and np.max(np.abs(gb - rb)) <= 1e-3
+
+
+def test_wkv4_decode_large_keys_and_fresh_state():
+    """One token from an empty state is v exactly (to fp32 rounding), for any key size."""
+    x = inputs.wkv4_inputs(3, 1, 130, "fp32", seed=22)
+    k = dev(x["k"]) * 40.0
+    y, s = ops.wkv4_forward(dev(x["w"]), dev(x["u"]), k, dev(x["v"]), want_state=True)
+    torch.cuda.synchronize()
+    assert rel_inf(f64(y), f64(x["v"])) <= 1e-6
+    assert torch.all(s[:, 1] == 1.0)  # one weight, referenced to itself

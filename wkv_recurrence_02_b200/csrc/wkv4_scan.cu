@@ -969,6 +969,67 @@ bool tma_usable(const Wkv4Args &a)
            tensor_map_encoder() != nullptr;
 }
 
+// ======================================================================= decode (T = 1)
+// One token per call (serving): one thread per (batch row, NV adjacent channels) applies the
+// output and running-maximum update steps above to each (a, b, p) state, which may be
+// updated in place (sT == s0).  Grid: x over channel groups, y over batch rows (a loop
+// covers rows beyond 65535); loads and stores are coalesced along the channel.
+template <typename T, int NV>
+__global__ void __launch_bounds__(256)
+wkv4_decode_kernel(int64_t B, int64_t C, const float *__restrict__ w, const float *__restrict__ u,
+                   const T *__restrict__ k, const T *__restrict__ v, const float *s0, T *__restrict__ y, float *sT)
+{
+    const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * NV;
+    if (c0 >= C) return;
+    float w2[NV], u2[NV];
+#pragma unroll
+    for (int j = 0; j < NV; ++j) {
+        w2[j] = w[c0 + j] * kLog2e;
+        u2[j] = u[c0 + j] * kLog2e;
+    }
+    for (int64_t b = blockIdx.y; b < B; b += gridDim.y) {
+        const int64_t i = b * C + c0;
+        const float *sp = s0 ? s0 + b * 3 * C : nullptr;
+        float *tp = sT ? sT + b * 3 * C : nullptr;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+            const float k2 = Elem<T>::get(k + i + j) * kLog2e, vx = Elem<T>::get(v + i + j);
+            St st{0.f, 0.f, kPEmpty};
+            if (sp) {
+                const float sb = sp[C + c0 + j];
+                if (sb != 0.f) st = {sp[c0 + j], sb, fmaxf(sp[2 * C + c0 + j] * kLog2e, kPEmpty)};
+            }
+            Elem<T>::put(y + i + j, output(st, k2, vx, u2[j]));
+            update(st, k2, vx, w2[j]);
+            if (tp) {
+                tp[c0 + j] = st.a;
+                tp[C + c0 + j] = st.b;
+                tp[2 * C + c0 + j] = st.b == 0.f ? kPEmpty : st.p * kLn2;
+            }
+        }
+    }
+}
+
+template <typename T, int NV>
+cudaError_t launch_decode_v(const Wkv4Args &a, cudaStream_t s)
+{
+    const int64_t groups = (a.C + NV - 1) / NV;
+    const int64_t bx = (groups + 255) / 256;
+    if (bx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const unsigned by = static_cast<unsigned>(a.B < 65535 ? a.B : 65535);
+    wkv4_decode_kernel<T, NV><<<dim3(static_cast<unsigned>(bx), by), 256, 0, s>>>(
+        a.B, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
+        static_cast<T *>(a.y), a.sT);
+    return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_decode(const Wkv4Args &a, cudaStream_t s)
+{
+    if (a.B == 0 || a.C == 0) return cudaSuccess;
+    return a.C % 2 == 0 ? launch_decode_v<T, 2>(a, s) : launch_decode_v<T, 1>(a, s);
+}
+
 template <typename T, int L>
 cudaError_t launch_L(const Wkv4Args &a, cudaStream_t s)
 {
@@ -1006,6 +1067,7 @@ cudaError_t launch_T(const Wkv4Args &a, cudaStream_t s)
 
 cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s)
 {
+    if (a.T == 1) return a.bf16 ? launch_decode<__nv_bfloat16>(a, s) : launch_decode<float>(a, s);
     if (a.B * ((a.C + kCh - 1) / kCh) > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     if (tma_usable(a)) {
         const int lmax = a.bf16 ? 32 : 16;

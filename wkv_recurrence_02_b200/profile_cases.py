@@ -11,6 +11,7 @@ Every case first makes one untimed call (so a profiler can skip it with ``-s``),
   long          WKV-6 chunked prefill with sequence split, B1 T4096 H64 (state-only pass
                 then full pass)
   decode        WKV-6 T=1 decode, B256 H64 with the state updated in place (268 MB of state)
+  wkv4_decode   RWKV-4 T=1 decode, B2048 C4096 bf16, (a, b, p) state updated in place
 
 Inputs come from the seeded generators in ``inputs``; nothing here checks results.
 """
@@ -20,7 +21,7 @@ import torch
 
 from . import inputs, ops
 
-CASES = ("wkv4", "finch", "long", "decode")
+CASES = ("wkv4", "finch", "long", "decode", "wkv4_decode")
 
 
 def _wkv4(reps):
@@ -29,6 +30,16 @@ def _wkv4(reps):
     y = torch.empty_like(a[2])
     for _ in range(1 + reps):
         ops.wkv4_forward(*a, y=y)
+
+
+def _wkv4_decode(reps):
+    x = inputs.wkv4_inputs(2048, 1, 4096, "bf16", seed=5, wu_seed=6)
+    a = [x[n].cuda() for n in ("w", "u", "k", "v")]
+    st = torch.zeros(2048, 3, 4096, dtype=torch.float32, device="cuda")
+    st[:, 1] = 1.0
+    y = torch.empty_like(a[2])
+    for _ in range(1 + reps):
+        ops.wkv4_forward(*a, s0=st, sT=st, y=y, want_state=True)
 
 
 def _wkv6(B, T, H, reps, s0_std=0.1):
@@ -50,6 +61,8 @@ def run(case, reps=1):
         _wkv6(1, 4096, 64, reps)
     elif case == "decode":
         _wkv6(256, 1, 64, reps)
+    elif case == "wkv4_decode":
+        _wkv4_decode(reps)
     else:
         raise ValueError(f"unknown case {case!r}; choose from {CASES}")
 
