@@ -15,6 +15,9 @@ Sources:
     time-dependent softmax).
   * WKV-6: "RWKV-5/6 (Eagle and Finch)" summary, sections 4 (row-vector
     convention), 4.1.2 (Eagle time mixing) and 4.2.2 (Finch per-token decay).
+  * Head LayerNorm and SiLU gate on the WKV-6 output: the same summary, section 4
+    (architecture overview: LayerNorm on the heads, SiLU attention gating) and 4.1.2
+    (the LayerNorm acts on each head separately, i.e. GroupNorm over the heads).
 """
 import ctypes
 import os
@@ -38,6 +41,9 @@ class Oracle:
         lib.oracle_wkv4.restype = None
         lib.oracle_wkv6.argtypes = [_I64, _I64, _I64, _I64, _DP, _DP, _DP, _DP, _DP,
                                     _DP, _DP, _DP, _DP]
+        lib.oracle_head_norm_gate.argtypes = [_I64, _I64, _I64, _I64, _DP, _DP, _DP, _DP,
+                                              ctypes.c_double, _DP]
+        lib.oracle_head_norm_gate.restype = None
         lib.oracle_wkv6.restype = None
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_threads.restype = ctypes.c_int
@@ -101,6 +107,27 @@ class Oracle:
         return y, sT
 
 
+    def head_norm_gate(self, o, g, ln_w, ln_b, eps):
+        """y = SiLU(g) * (ln_w * (o - mean) / sqrt(var + eps) + ln_b) per (b, t, head).
+
+        o, g: [B,T,H,N]; ln_w, ln_b: [H,N].  Returns y [B,T,H,N] in float64.
+        """
+        o, op = self._f64(o)
+        g, gp = self._f64(g)
+        ln_w, wp = self._f64(ln_w)
+        ln_b, bp = self._f64(ln_b)
+        B, T, H, N = o.shape
+        assert g.shape == o.shape and ln_w.shape == (H, N) and ln_b.shape == (H, N)
+        y = np.empty_like(o)
+        self._lib.oracle_head_norm_gate(B, T, H, N, op, gp, wp, bp, float(eps), y.ctypes.data_as(_DP))
+        return y
+
+    def wkv6_gated(self, r, k, v, w, u, g, ln_w, ln_b, eps, s0=None):
+        """WKV-6 forward followed by the head LayerNorm and SiLU gate: (y, sT)."""
+        o, sT = self.wkv6(r, k, v, w, u, s0=s0)
+        return self.head_norm_gate(o, g, ln_w, ln_b, eps), sT
+
+
 _DEFAULT = None
 
 
@@ -120,6 +147,14 @@ def wkv4(w, u, k, v, s0=None, want_state=False):
 
 def wkv6(r, k, v, w, u, s0=None):
     return get().wkv6(r, k, v, w, u, s0=s0)
+
+
+def head_norm_gate(o, g, ln_w, ln_b, eps):
+    return get().head_norm_gate(o, g, ln_w, ln_b, eps)
+
+
+def wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=None):
+    return get().wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=s0)
 
 
 def set_threads(n: int = 0) -> int:

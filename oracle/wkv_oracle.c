@@ -177,3 +177,40 @@ void oracle_wkv6(int64_t B, int64_t T, int64_t H, int64_t N,
                 sT[n * N * N + e] = S[e];
     }
 }
+
+/* Eagle time mixing ("RWKV-5/6 (Eagle and Finch)" summary, section 4.1.2, and the
+ * architecture overview of section 4): the WKV output of each head is normalised by a
+ * LayerNorm over that head's N channels (equivalently GroupNorm over H groups), with a
+ * per-channel scale ln_w and shift ln_b, and multiplied by the SiLU attention gate:
+ *
+ *   y = SiLU(g) * (ln_w * (o - mean) / sqrt(var + eps) + ln_b),   SiLU(g) = g / (1 + e^-g)
+ *
+ * mean and var (the mean of squared deviations) are taken over the N channels of one
+ * (b, t, h).  o, g, y: [B,T,H,N]; ln_w, ln_b: [H,N].  The output projection that follows
+ * in the model is a dense GEMM and is not part of the recurrence.
+ */
+void oracle_head_norm_gate(int64_t B, int64_t T, int64_t H, int64_t N, const double *o, const double *g,
+                           const double *ln_w, const double *ln_b, double eps, double *y)
+{
+    const int64_t rows = B * T * H;
+#pragma omp parallel for schedule(static)
+    for (int64_t row = 0; row < rows; ++row) {
+        const int64_t h = row % H;
+        const double *x = o + row * N;
+        double mean = 0.0;
+        for (int64_t n = 0; n < N; ++n) mean += x[n];
+        mean /= (double)N;
+        double var = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+            const double d = x[n] - mean;
+            var += d * d;
+        }
+        var /= (double)N;
+        const double rstd = 1.0 / sqrt(var + eps);
+        for (int64_t n = 0; n < N; ++n) {
+            const double gn = g[row * N + n];
+            const double gate = gn / (1.0 + exp(-gn));
+            y[row * N + n] = gate * (ln_w[h * N + n] * (x[n] - mean) * rstd + ln_b[h * N + n]);
+        }
+    }
+}

@@ -11,7 +11,10 @@ Kinds of pin used (none retypes the oracle's recurrence):
     linear attention as a masked matmul);
   * hand-worked examples with exact rational values (tests/golden/);
   * invariants: WKV-4 shift invariance in k and convex-hull bounds, WKV-6
-    linearity in (v, s0) and head independence, split-sequence chaining.
+    linearity in (v, s0) and head independence, split-sequence chaining;
+  * head LayerNorm + SiLU gate: the two-channel closed form, SiLU at +-ln 3 (sigmoid 3/4
+    and 1/4), shift/scale invariance and unit moments, affinity in the per-channel
+    parameters, per-head parameter rows.
 """
 import json
 import os
@@ -269,11 +272,87 @@ def pin_wkv6_golden(O):
     assert np.array_equal(sT[0, 0], s_exp), ("wkv6 golden sT", sT[0, 0], s_exp)
 
 
+# ----------------------------------------------------------- head LayerNorm + SiLU gate
+# SiLU at two points with closed forms: sigma(ln 3) = 3/4, sigma(-ln 3) = 1/4.
+_LN3 = float(np.log(3.0))
+_SILU_LN3, _SILU_MLN3 = 0.75 * _LN3, -0.25 * _LN3
+
+
+def pin_norm_gate_two_channels(O):
+    """N = 2: the deviations from the mean are +-d with d = (a - b) / 2, so the normalised
+    pair is +-d / sqrt(d^2 + eps) -- exactly +-1 for eps = 0."""
+    rng = np.random.default_rng(41)
+    B, T, H, N = 2, 3, 2, 2
+    o = rng.normal(0, 2, (B, T, H, N))
+    g = np.empty_like(o)
+    g[..., 0], g[..., 1] = _LN3, -_LN3
+    gam = rng.uniform(0.5, 2, (H, N))
+    bet = rng.normal(0, 1, (H, N))
+    for eps in (0.0, 0.3):
+        y = O.head_norm_gate(o, g, gam, bet, eps)
+        d = (o[..., 0] - o[..., 1]) / 2
+        xh0 = d / np.sqrt(d * d + eps)
+        exp0 = _SILU_LN3 * (gam[None, None, :, 0] * xh0 + bet[None, None, :, 0])
+        exp1 = _SILU_MLN3 * (gam[None, None, :, 1] * -xh0 + bet[None, None, :, 1])
+        assert _rel(y[..., 0], exp0) < 1e-12 and _rel(y[..., 1], exp1) < 1e-12, ("two-channel closed form", eps)
+
+
+def pin_norm_gate_invariants(O):
+    """eps = 0: the normalised part is unchanged by a per-row shift or positive scale of o,
+    and has zero mean and unit mean square over the head's channels."""
+    rng = np.random.default_rng(42)
+    B, T, H, N = 2, 4, 3, 8
+    o = rng.normal(0, 1, (B, T, H, N))
+    g = np.full_like(o, _LN3)
+    one, zero = np.ones((H, N)), np.zeros((H, N))
+    y = O.head_norm_gate(o, g, one, zero, 0.0)
+    xh = y / _SILU_LN3
+    assert np.max(np.abs(xh.mean(-1))) < 1e-12, "normalised mean"
+    assert np.max(np.abs((xh * xh).mean(-1) - 1.0)) < 1e-12, "normalised mean square"
+    shift = rng.normal(0, 5, (B, T, H, 1))
+    scale = rng.uniform(0.1, 10, (B, T, H, 1))
+    assert _rel(O.head_norm_gate(o + shift, g, one, zero, 0.0), y) < 1e-10, "shift invariance"
+    assert _rel(O.head_norm_gate(o * scale, g, one, zero, 0.0), y) < 1e-10, "scale invariance"
+
+
+def pin_norm_gate_affine(O):
+    """Linear in (ln_w, ln_b): y(w, b) = y(w, 0) + y(0, b), and y(0, b) = SiLU(g) * b."""
+    rng = np.random.default_rng(43)
+    B, T, H, N = 1, 3, 2, 8
+    o = rng.normal(0, 1, (B, T, H, N))
+    g = np.where(rng.uniform(size=o.shape) < 0.5, _LN3, -_LN3)
+    silu = np.where(g > 0, _SILU_LN3, _SILU_MLN3)
+    gam = rng.normal(0, 1, (H, N))
+    bet = rng.normal(0, 1, (H, N))
+    zero = np.zeros((H, N))
+    y = O.head_norm_gate(o, g, gam, bet, 1e-3)
+    yw = O.head_norm_gate(o, g, gam, zero, 1e-3)
+    yb = O.head_norm_gate(o, g, zero, bet, 1e-3)
+    assert _rel(y, yw + yb) < 1e-12, "additivity in (w, b)"
+    assert _rel(yb, silu * bet[None, None]) < 1e-12, "shift term is SiLU(g) * b"
+
+
+def pin_norm_gate_heads(O):
+    """Each head uses its own row of (ln_w, ln_b): permuting the heads of o and g together
+    with those rows permutes y."""
+    rng = np.random.default_rng(44)
+    B, T, H, N = 2, 2, 4, 8
+    o = rng.normal(0, 1, (B, T, H, N))
+    g = rng.normal(0, 2, (B, T, H, N))
+    gam = rng.normal(0, 1, (H, N))
+    bet = rng.normal(0, 1, (H, N))
+    perm = np.array([2, 0, 3, 1])
+    y = O.head_norm_gate(o, g, gam, bet, 1e-5)
+    yp = O.head_norm_gate(o[:, :, perm], g[:, :, perm], gam[perm], bet[perm], 1e-5)
+    assert _rel(yp, y[:, :, perm]) < 1e-12, "per-head parameters"
+
+
 ALL_PINS = [
     pin_wkv4_bruteforce, pin_wkv4_T1, pin_wkv4_fast_decay, pin_wkv4_invariants,
     pin_wkv4_chaining, pin_wkv4_golden,
     pin_wkv6_bruteforce, pin_wkv6_T1, pin_wkv6_fast_decay, pin_wkv6_no_decay,
     pin_wkv6_chaining, pin_wkv6_linearity, pin_wkv6_head_independence, pin_wkv6_golden,
+    pin_norm_gate_two_channels, pin_norm_gate_invariants, pin_norm_gate_affine, pin_norm_gate_heads,
 ]
 
 

@@ -28,6 +28,13 @@ MUTANTS = [
     ("wkv4_output_after_decay", "double e_past = exp(p - q);", "double e_past = exp(p - w - q);"),
     ("wkv4_ignore_s0_max", "p = s0[(bi * 3 + 2) * C + c];", "p = 0.0;"),
     ("wkv4_denominator_uses_v", "(e_past * b + e_now)", "(e_past * b + e_now * vt)"),
+    ("norm_unbiased_variance", "var /= (double)N;", "var /= (double)(N - 1);"),
+    ("norm_drops_eps", "rstd = 1.0 / sqrt(var + eps);", "rstd = 1.0 / sqrt(var);"),
+    ("gate_sigmoid_not_silu", "gn / (1.0 + exp(-gn))", "1.0 / (1.0 + exp(-gn))"),
+    ("norm_shared_head_params", "ln_w[h * N + n] * (x[n] - mean)", "ln_w[n] * (x[n] - mean)"),
+    ("norm_no_centering", "(x[n] - mean) * rstd", "x[n] * rstd"),
+    ("gate_skips_shift", "gate * (ln_w[h * N + n] * (x[n] - mean) * rstd + ln_b[h * N + n])",
+     "gate * ln_w[h * N + n] * (x[n] - mean) * rstd + ln_b[h * N + n]"),
 ]
 
 
