@@ -248,7 +248,7 @@ def run_ours(args, rank, world, dist):
 
     # end to end through the public API with host buffers: H2D of every input, D2H of results
     e2e_ms, h2d, d2h = run_e2e(torch, ops, wl, stream, dev, max(3, min(args.steps, 10)), barrier)
-    next_rows = measure_next_rows(torch, inputs, ops, dev, stream)
+    next_rows = measure_next_rows(torch, inputs, ops, dev, stream, wl)
 
     ms_max, e2e_max = max_over_ranks([ms, e2e_ms], dist, device=dev)
     status = ops.device_status()
@@ -306,10 +306,40 @@ def run_ours(args, rank, world, dist):
     return line
 
 
-def measure_next_rows(torch, inputs, ops, dev, stream, reps=50):
-    """Rows beyond the step, timed on their own (not part of the step's metric): the RWKV-4
-    decode step (T = 1) at the width of a 7B model, state updated in place."""
+def _time_us(torch, stream, dev, fn, reps):
+    for _ in range(3):
+        fn()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize(dev)
+    return a.elapsed_time(b) * 1e3 / reps
+
+
+def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
+    """Rows beyond the step, timed on their own (not part of the step's metric):
+      * the RWKV-4 decode step (T = 1) at the width of a 7B model, state updated in place;
+      * the Finch prefill with the time-mixing output stage (head LayerNorm, SiLU gate)
+        fused into the chunked kernel's epilogue, against the same call without it."""
     hbm, _ = load_peaks()
+    rows = {}
+    f = wl.finch
+    ng = inputs.norm_gate_inputs(8, 4096, 32, 64, seed=3)
+    g, lw, lb = (ng[n].to(dev) for n in ("g", "ln_w", "ln_b"))
+    plain = _time_us(torch, stream, dev, lambda: ops.wkv6_forward(
+        f["r"], f["k"], f["v"], f["w"], f["u"], s0=f["s0"], y=f["y"], sT=f["sT"]), 20)
+    gated = _time_us(torch, stream, dev, lambda: ops.wkv6_forward_gated(
+        f["r"], f["k"], f["v"], f["w"], f["u"], g, lw, lb, eps=1e-5, s0=f["s0"], y=f["y"], sT=f["sT"]), 20)
+    nbytes = BYTES["wkv6_chunked_finch"] + g.numel() * 2 + 2 * 32 * 64 * 4
+    separate = 3 * f["y"].numel() * 2  # an unfused stage reads y and g and writes y again
+    rows["wkv6_finch_gated_B8_T4096_H32"] = {
+        "avg_us": round(gated, 2), "ungated_avg_us": round(plain, 2), "algorithmic_bytes": nbytes,
+        "GBps": round(nbytes / (gated * 1e-6) / 1e9, 1),
+        "frac_hbm": round(nbytes / (gated * 1e-6) / 1e9 / hbm, 4),
+        "separate_stage_floor_us": round(separate / (hbm * 1e9) * 1e6, 2)}
     B, C = 2048, 4096
     x = inputs.wkv4_inputs(B, 1, C, "bf16", seed=5, wu_seed=6)
     w, u, k, v = (x[n].to(dev) for n in ("w", "u", "k", "v"))
@@ -329,9 +359,10 @@ def measure_next_rows(torch, inputs, ops, dev, stream, reps=50):
     us = a.elapsed_time(b) * 1e3 / reps
     nbytes = B * C * (2 * 2 + 2 + 2 * 3 * 4) + 2 * C * 4  # k, v, y bf16; state in and out; w, u
     gbs = nbytes / (us * 1e-6) / 1e9
-    return {"wkv4_decode_B2048_C4096": {"avg_us": round(us, 2), "algorithmic_bytes": nbytes,
-                                        "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
-                                        "state_bytes": 2 * B * 3 * C * 4, "launches": reps}}
+    rows["wkv4_decode_B2048_C4096"] = {"avg_us": round(us, 2), "algorithmic_bytes": nbytes,
+                                       "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                                       "state_bytes": 2 * B * 3 * C * 4, "launches": reps}
+    return rows
 
 
 def run_e2e(torch, ops, wl, stream, dev, steps, barrier):

@@ -118,6 +118,25 @@ int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
                            const uint16_t *w, const float *u, const float *s0,
                            uint16_t *y, float *sT);
 
+/* WKV-6 with the time-mixing output stage fused into the epilogue ([E412]: LayerNorm on
+ * each head, i.e. GroupNorm over the H heads, then the SiLU attention gate):
+ *   o = the rwkv_wkv6_forward_bf16 output (fp32 before rounding),
+ *   y[b,t,h,:] = SiLU(g[b,t,h,:]) * ( ln_w[h,:] * (o - mean) / sqrt(var + eps) + ln_b[h,:] )
+ * with mean and var (mean of squared deviations) over the N channels of o[b,t,h,:] and
+ * SiLU(x) = x / (1 + e^-x).  y is written once, in bf16; the state is as in
+ * rwkv_wkv6_forward_bf16.
+ *   g             : [B, T, H, N] bf16, the gate before its activation; must not overlap y.
+ *   ln_w, ln_b    : [H, N] fp32, the per-channel scale and shift (not NULL).
+ *   eps           : >= 0 (RWKV_ERR_ARG otherwise).
+ * T > 1 runs the chunked kernel, T == 1 the decode kernel, each with the fused epilogue
+ * (the rwkv_set_wkv6_algo choice does not apply).  Other arguments, layouts, aliasing
+ * rules and errors are those of rwkv_wkv6_forward_bf16. */
+int rwkv_wkv6_forward_gated_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
+                                 const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                                 const uint16_t *w, const float *u, const float *s0,
+                                 const uint16_t *g, const float *ln_w, const float *ln_b, float eps,
+                                 uint16_t *y, float *sT);
+
 /* Kernel choice for WKV-6 on the calling thread: RWKV_WKV6_AUTO (default, as above),
  * RWKV_WKV6_SERIAL (always the serial kernel), RWKV_WKV6_CHUNKED (the chunked kernel
  * for bf16 whatever T; ignored for fp32).  Returns RWKV_OK or RWKV_ERR_ARG. */
@@ -133,8 +152,8 @@ int rwkv_get_wkv6_algo(void);
  * side: a first state-only pass gives each segment's local end state and decay product,
  * and each segment then starts from its exact incoming state.  The result equals the
  * unsplit evaluation up to fp32 rounding order.  The split needs B*H*(G-1)*(N*N+N)*4 bytes
- * of scratch, taken stream-ordered from the device's current memory pool
- * (cudaMallocAsync / cudaFreeAsync on the calling thread's stream) within the call.
+ * of scratch, taken stream-ordered (on the calling thread's stream, within the call) from
+ * a memory pool the library keeps per device, which holds up to 64 MB between calls.
  *   segments = 0 (default): choose G;  1: never split;  n >= 2: split into at most n.
  * Returns RWKV_OK or RWKV_ERR_ARG. */
 int rwkv_set_wkv6_segments(int segments);

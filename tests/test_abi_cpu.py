@@ -84,6 +84,28 @@ def test_wkv6_validation(lib):
     assert f(2, 4, 0, 64, *([None] * 8)) == 0
 
 
+def test_wkv6_gated_validation(lib):
+    """Gate, LayerNorm parameters and eps are checked on the host like the other tensors."""
+    f = lib.rwkv_wkv6_forward_gated_bf16
+    r, k, v, w, u, s0, g, lw, lb, y, sT = (_p(i << 24) for i in range(11))
+
+    def call(eps=1e-5, **kw):
+        a = dict(r=r, k=k, v=v, w=w, u=u, s0=s0, g=g, lw=lw, lb=lb, y=y, sT=sT)
+        a.update(kw)
+        return f(1, 4, 2, 64, a["r"], a["k"], a["v"], a["w"], a["u"], a["s0"], a["g"], a["lw"], a["lb"],
+                 ctypes.c_float(eps), a["y"], a["sT"])
+
+    assert call(g=None) == -1                     # gate null
+    assert call(lw=None) == -1                    # LayerNorm scale null
+    assert call(lb=None) == -1
+    assert call(eps=-1.0) == -8                   # eps < 0
+    assert call(eps=float("nan")) == -8
+    assert call(g=_p((6 << 24) + 4)) == -7        # misaligned gate
+    assert call(y=g) == -4                        # y == g
+    assert call(sT=lw) == -4                      # sT over the LayerNorm scale
+    assert f(0, 4, 2, 64, *([None] * 9), ctypes.c_float(1e-5), None, None) == 0  # empty
+
+
 def test_algo_selection(lib):
     assert lib.rwkv_set_wkv6_algo(7) == -8
     for a in (1, 2, 0):

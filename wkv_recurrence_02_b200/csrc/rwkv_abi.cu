@@ -123,7 +123,8 @@ int wkv4_entry(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
 
 int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
                const void *v, const void *w, const float *u, const float *s0, void *y,
-               float *sT, bool bf16)
+               float *sT, bool bf16, const void *g = nullptr, const float *ln_w = nullptr,
+               const float *ln_b = nullptr, float eps = 0.f, bool gated = false)
 {
     tl_err[0] = 0;
     if (B < 0 || T < 0 || H < 0 || N < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
@@ -137,12 +138,18 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
     if (n > 0 && (!r || !k || !v || !w || !y))
         return fail(RWKV_ERR_NULL, "r, k, v, w and y must be non-null%s");
     if (BH > 0 && !u) return fail(RWKV_ERR_NULL, "u must be non-null%s");
-    const void *ptrs[] = {r, k, v, w, u, s0, y, sT};
+    if (gated) {
+        if (n > 0 && !g) return fail(RWKV_ERR_NULL, "g must be non-null%s");
+        if (H * N > 0 && (!ln_w || !ln_b)) return fail(RWKV_ERR_NULL, "ln_w and ln_b must be non-null%s");
+        if (!(eps >= 0.f) || eps > 3.0e38f) return fail(RWKV_ERR_ARG, "eps must be finite and >= 0%s");
+    }
+    const void *ptrs[] = {r, k, v, w, u, s0, y, sT, g, ln_w, ln_b};
     for (const void *p : ptrs)
         if (p && !aligned16(p)) return fail(RWKV_ERR_ALIGN, "tensor pointers must be 16-byte aligned%s");
     Span sy{y, n * esz}, sr{r, n * esz}, sk{k, n * esz}, sv{v, n * esz}, sw{w, n * esz};
     Span su{u, H * N * 4}, ss0{s0, ns * 4}, ssT{sT, ns * 4};
-    const Span ins[] = {sr, sk, sv, sw, su};
+    Span sg{g, n * esz}, slw{ln_w, H * N * 4}, slb{ln_b, H * N * 4};
+    const Span ins[] = {sr, sk, sv, sw, su, sg, slw, slb};
     for (const Span &s : ins)
         if (overlap(sy, s)) return fail(RWKV_ERR_ALIAS, "y overlaps an input%s");
     if (overlap(sy, ss0) || overlap(sy, ssT)) return fail(RWKV_ERR_ALIAS, "y overlaps a state%s");
@@ -163,6 +170,15 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
     }
     wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, bf16, status, tl_wkv6_segments};
     cudaError_t e;
+    if (gated) {  // fused output stage: chunked for T > 1, decode for T == 1
+        a.g = g;
+        a.ln_w = ln_w;
+        a.ln_b = ln_b;
+        a.eps = eps;
+        e = T > 1 ? wkv::wkv6_chunked_launch(a, tl_stream) : wkv::wkv6_decode_launch(a, tl_stream);
+        if (e != cudaSuccess) return cuda_fail(e, "wkv6 gated launch");
+        return RWKV_OK;
+    }
     int algo = tl_wkv6_algo;
     if (algo == RWKV_WKV6_SERIAL || !bf16)
         e = (T == 1 && algo != RWKV_WKV6_SERIAL) ? wkv::wkv6_decode_launch(a, tl_stream)
@@ -273,6 +289,15 @@ int rwkv_wkv6_forward_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uin
                            const float *u, const float *s0, uint16_t *y, float *sT)
 {
     return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, true);
+}
+
+extern "C" int rwkv_wkv6_forward_gated_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,
+                                            const uint16_t *k, const uint16_t *v, const uint16_t *w,
+                                            const float *u, const float *s0, const uint16_t *g,
+                                            const float *ln_w, const float *ln_b, float eps, uint16_t *y,
+                                            float *sT)
+{
+    return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, true, g, ln_w, ln_b, eps, true);
 }
 
 int rwkv_wkv6_forward_bf16_noalloc(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,

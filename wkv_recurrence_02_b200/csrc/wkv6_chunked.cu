@@ -68,7 +68,8 @@ constexpr int OFF_UB = OFF_D + kStages * 64 * 4;      // [stage][64] bonus diago
 constexpr int OFF_DD = OFF_UB + kStages * 64 * 4;     // [4][16][16] exact diagonal blocks
 constexpr int OFF_BAR = OFF_DD + 4 * 16 * 16 * 4;     // mbarriers (8 bytes each)
 constexpr int OFF_MISC = OFF_BAR + 16 * 8;            // tmem base, flags
-constexpr int kSmemBytes = OFF_MISC + 64 + 1024;      // + alignment slack
+constexpr int OFF_LN = OFF_MISC + 64;                 // [2][64] LayerNorm scale, shift of the head
+constexpr int kSmemBytes = OFF_LN + 2 * 64 * 4 + 1024; // + alignment slack
 
 // TMEM columns (fp32 accumulators, M = 64 layout: row m -> lane (m % 16) + 32 (m / 16))
 constexpr uint32_t COL_S = 0, COL_AD = 64, COL_AO = 128, COL_O = 192, kTmemCols = 256;
@@ -236,6 +237,13 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32])
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 __device__ __forceinline__ float rcp_approx(float x)
 {
     float y;
@@ -388,6 +396,10 @@ struct ChunkedParams {
     int state_only;        // 1: only the segment's local end state (from zero) and decay
     float *seg;            // [B*H][segments-1][N*N + N]: local end state, then decay product
     int nseg;              // segments per sequence
+    // fused output stage (null gate: plain y): y = SiLU(g) (ln_w (o - mean) rstd + ln_b)
+    const __nv_bfloat16 *gate;
+    const float *ln_w, *ln_b;
+    float eps;
 };
 constexpr int kSegStride = kN * kN + kN;
 
@@ -449,6 +461,59 @@ __device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t c
     }
 }
 
+// y row of token tok, head h: this thread's 32 of the 64 channels, the other 32 in lane
+// ^ 16.  With a gate, the head's LayerNorm (statistics over both halves) and the SiLU gate
+// are applied first.  Every lane of the warp calls this (the statistics pair lanes); only
+// `valid` rows read g and store.
+template <bool GATED>
+__device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[32], int64_t tok, int64_t b,
+                                            int64_t h, int colh, bool valid, const float *lns)
+{
+    if (GATED) {
+        float s = 0.f;
+#pragma unroll
+        for (int n = 0; n < 32; ++n) s += ov[n];
+        s += __shfl_xor_sync(0xffffffffu, s, 16);
+        const float mean = s * (1.f / kN);
+        float q = 0.f;
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+            const float d = ov[n] - mean;
+            q = fmaf(d, d, q);
+        }
+        q += __shfl_xor_sync(0xffffffffu, q, 16);
+        const float rstd = rsqrtf(q * (1.f / kN) + p.eps);
+        if (valid) {
+            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + ((b * p.T + tok) * p.H + h) * kN + colh);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+                const uint4 gw = gp[v4];
+                const uint32_t wd[4] = {gw.x, gw.y, gw.z, gw.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int n = 8 * v4 + e;
+                    const float gv = __uint_as_float(e & 1 ? (wd[e >> 1] & 0xFFFF0000u) : (wd[e >> 1] << 16));
+                    // SiLU(g) = g / (1 + 2^(-g log2 e)), approximate exponential and reciprocal
+                    const float gate = gv * rcp_approx(1.f + ex2_approx(-gv * 1.4426950408889634f));
+                    ov[n] = gate * fmaf(lns[colh + n] * (ov[n] - mean), rstd, lns[kN + colh + n]);
+                }
+            }
+        }
+    }
+    if (valid) {
+        uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * p.T + tok) * p.H + h) * kN + colh);
+#pragma unroll
+        for (int v4 = 0; v4 < 4; ++v4) {
+            uint4 x;
+            x.x = pack_bf16(ov[8 * v4 + 0], ov[8 * v4 + 1]);
+            x.y = pack_bf16(ov[8 * v4 + 2], ov[8 * v4 + 3]);
+            x.z = pack_bf16(ov[8 * v4 + 4], ov[8 * v4 + 5]);
+            x.w = pack_bf16(ov[8 * v4 + 6], ov[8 * v4 + 7]);
+            dst[v4] = x;
+        }
+    }
+}
+
 // Warp roles (256 threads):
 //   warps 0-3  prep group: warp a builds the operand rows of 16-token sub-block a, running
 //              up to two chunks ahead of the TMEM group;
@@ -461,6 +526,7 @@ __device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t c
 // Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue), scores
 // done, O done, state done and stage empty (tcgen05.commit).  Per-chunk bookkeeping (bonus
 // diagonal, decay, path flags) lives beside the chunk's stage.
+template <bool GATED>
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
@@ -473,6 +539,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     float *Dv = reinterpret_cast<float *>(sm + OFF_D);   // [stage][64]
     float *UB = reinterpret_cast<float *>(sm + OFF_UB);  // [stage][64]
     float *DD = reinterpret_cast<float *>(sm + OFF_DD);
+    float *lns = reinterpret_cast<float *>(sm + OFF_LN);  // gated output: [scale, shift][64]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC);
     // misc: [0] TMEM base, [1] abort, [2+s] sub-block path, [5+s] exact diagonal (s = stage),
@@ -712,6 +779,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         const bool iss_o = issuer, iss_s = tid == kPrepThreads + 32, iss_a = tid == kPrepThreads + 64;
         const bool iss_t = tid == kPrepThreads + 96;
         int issued = misc[8];
+        if (GATED && !so) {  // the head's LayerNorm scale and shift (read after the loop's first barrier)
+            const int t = tid - kPrepThreads;
+            lns[t] = t < kN ? p.ln_w[h * kN + t] : p.ln_b[h * kN + t - kN];
+        }
 
         // scores of chunk c into TMEM (issuer only)
         auto issue_scores = [&](int c) -> int {
@@ -883,17 +954,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 if (c > 0) {
                     float ov[32];
                     tmem_ld32(tlane + COL_O, ov);
-                    const int64_t tp = t0 - kC + row;
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + tp) * p.H + h) * kN + colh);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint4 x;
-                        x.x = pack_bf16(ov[8 * v4 + 0], ov[8 * v4 + 1]);
-                        x.y = pack_bf16(ov[8 * v4 + 2], ov[8 * v4 + 3]);
-                        x.z = pack_bf16(ov[8 * v4 + 4], ov[8 * v4 + 5]);
-                        x.w = pack_bf16(ov[8 * v4 + 6], ov[8 * v4 + 7]);
-                        dst[v4] = x;
-                    }
+                    store_y_row<GATED>(p, ov, t0 - kC + row, b, h, colh, true, lns);
                 }
                 float va[32];
                 tmem_ld32(tlane + COL_AD, va);
@@ -1001,18 +1062,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 tmem_ld32(tlane + COL_O, ov);
                 const int64_t t0 = static_cast<int64_t>(cb + nchunks - 1) * kC;
                 const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
-                if (row < tv) {
-                    uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * T + t0 + row) * p.H + h) * kN + colh);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint4 x;
-                        x.x = pack_bf16(ov[8 * v4 + 0], ov[8 * v4 + 1]);
-                        x.y = pack_bf16(ov[8 * v4 + 2], ov[8 * v4 + 3]);
-                        x.z = pack_bf16(ov[8 * v4 + 4], ov[8 * v4 + 5]);
-                        x.w = pack_bf16(ov[8 * v4 + 6], ov[8 * v4 + 7]);
-                        dst[v4] = x;
-                    }
-                }
+                store_y_row<GATED>(p, ov, t0 + row, b, h, colh, row < tv, lns);
                 if (p.sT && g == p.nseg - 1) {
                     float sv[32];
                     tmem_ld32(tlane + COL_S, sv);
@@ -1105,11 +1155,14 @@ cudaError_t configure_kernel()
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (done[dev]) return cudaSuccess;
-    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(wkv6_chunked_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e == cudaSuccess) done[dev] = true;
-    return e;
+    for (auto kern : {wkv6_chunked_kernel<false>, wkv6_chunked_kernel<true>}) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+    }
+    done[dev] = true;
+    return cudaSuccess;
 }
 
 // Stream-ordered pool for the sequence-split scratch, one per device, owned by the library.
@@ -1182,7 +1235,8 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
 
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
-                      static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G)};
+                      static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G),
+                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     float *seg = nullptr;
     if (G > 1) {
         cudaMemPool_t pool = nullptr;
@@ -1194,14 +1248,15 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
         ChunkedParams pa = prm;
         pa.state_only = 1;
         pa.seg = seg;
-        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes,
-                              s>>>(mr, mk, mv, mw, pa);
+        wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads,
+                                     kSmemBytes, s>>>(mr, mk, mv, mw, pa);
         e = cudaGetLastError();
         prm.seg = seg;
     }
     if (e == cudaSuccess) {
-        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes,
-                              s>>>(mr, mk, mv, mw, prm);
+        auto kern = prm.gate ? wkv6_chunked_kernel<true> : wkv6_chunked_kernel<false>;
+        kern<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(mr, mk, mv,
+                                                                                                   mw, prm);
         e = cudaGetLastError();
     }
     if (seg) {
@@ -1284,18 +1339,19 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     if (e != cudaSuccess) return e;
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
-                      static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G)};
+                      static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G),
+                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     if (G > 1) {
         // the state-only pass writes every scratch entry the full pass reads: nothing in the
         // array has to start at zero, and what an earlier call left there is never read
         ChunkedParams pa = prm;
         pa.state_only = 1;
-        wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes,
-                              s>>>(mr, mk, mv, mw, pa);
+        wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads,
+                                     kSmemBytes, s>>>(mr, mk, mv, mw, pa);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    wkv6_chunked_kernel<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(
+    wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(
         mr, mk, mv, mw, prm);
     return cudaGetLastError();
 }

@@ -18,7 +18,8 @@
 //  * wkv6_decode_kernel -- T == 1: one (b, h) per 256-thread CTA; thread (ig, j4) owns
 //    rows 4ig..4ig+3 x columns 4j4..4j4+3 of S and moves them with 16-byte loads and
 //    stores, so the 2 x 16 KB state stream per head is fully coalesced.  Partial
-//    outputs are reduced over the 16 row groups through shared memory.
+//    outputs are reduced over the 16 row groups through shared memory.  With a gate g the
+//    64 outputs of the head go through the fused LayerNorm + SiLU gate before the store.
 #include "wkv_internal.cuh"
 
 namespace wkv {
@@ -133,10 +134,13 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ w,
-                   const float *__restrict__ u, const float *s0, T *__restrict__ y, float *sT)
+                   const float *__restrict__ u, const float *s0, T *__restrict__ y, float *sT,
+                   const T *__restrict__ g, const float *__restrict__ ln_w, const float *__restrict__ ln_b,
+                   float eps)
 {
     __shared__ __align__(16) float red[16][kN];
     __shared__ float bred[16];
+    __shared__ float stat[2][2];
 
     const int64_t n = blockIdx.x;  // b * H + h; with T == 1 the token row is n * N
     const int64_t h = n % H;
@@ -185,7 +189,27 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
             acc += red[g][tid];
             bsum += bred[g];
         }
-        st(y + vbase + tid, fmaf(bsum, ld(v + vbase + tid), acc));
+        float o = fmaf(bsum, ld(v + vbase + tid), acc);
+        if (g) {
+            // fused output stage: LayerNorm over the head's 64 outputs (two warps), SiLU gate
+            float s = o;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) s += __shfl_xor_sync(0xffffffffu, s, m);
+            if ((tid & 31) == 0) stat[0][tid >> 5] = s;
+            asm volatile("bar.sync 1, 64;" ::: "memory");
+            const float mean = (stat[0][0] + stat[0][1]) * (1.f / kN);
+            const float d = o - mean;
+            float q = d * d;
+#pragma unroll
+            for (int m = 16; m >= 1; m >>= 1) q += __shfl_xor_sync(0xffffffffu, q, m);
+            if ((tid & 31) == 0) stat[1][tid >> 5] = q;
+            asm volatile("bar.sync 1, 64;" ::: "memory");
+            const float rstd = rsqrtf((stat[1][0] + stat[1][1]) * (1.f / kN) + eps);
+            const float gv = ld(g + vbase + tid);
+            const float gate = __fdividef(gv, 1.f + __expf(-gv));  // SiLU, fast intrinsics
+            o = gate * fmaf(ln_w[h * kN + tid] * d, rstd, ln_b[h * kN + tid]);
+        }
+        st(y + vbase + tid, o);
     }
 }
 
@@ -222,12 +246,12 @@ cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s)
         wkv6_decode_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k),
             static_cast<const T *>(a.v), static_cast<const T *>(a.w), a.u, a.s0,
-            static_cast<T *>(a.y), a.sT);
+            static_cast<T *>(a.y), a.sT, static_cast<const T *>(a.g), a.ln_w, a.ln_b, a.eps);
     } else {
         wkv6_decode_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const float *>(a.r), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), static_cast<const float *>(a.w), a.u, a.s0,
-            static_cast<float *>(a.y), a.sT);
+            static_cast<float *>(a.y), a.sT, nullptr, nullptr, nullptr, 0.f);
     }
     return cudaGetLastError();
 }

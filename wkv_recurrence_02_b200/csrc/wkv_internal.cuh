@@ -40,6 +40,11 @@ struct Wkv6Args {
     bool bf16;
     int *status;
     int segments;               // chunked kernel: 0 = choose the sequence split, n = at most n
+    // fused output stage (bf16 only): y = SiLU(g) * (ln_w * (o - mean) / sqrt(var + eps) + ln_b)
+    // per (b, t, h) when g is non-null
+    const void *g = nullptr;    // [B,T,H,N] bf16
+    const float *ln_w = nullptr, *ln_b = nullptr;  // [H,N]
+    float eps = 0.f;
 };
 
 // cuTensorMapEncodeTiled from the driver (null if unavailable).

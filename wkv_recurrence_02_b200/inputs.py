@@ -83,6 +83,21 @@ def wkv6_inputs(B: int, T: int, H: int, N: int = 64, dtype: str = "fp32", seed: 
     return {"r": r.to(dt), "k": k.to(dt), "v": v.to(dt), "w": w.to(dt), "u": u, "s0": s0}
 
 
+def norm_gate_inputs(B: int, T: int, H: int, N: int = 64, seed: int = 0):
+    """Inputs of the WKV-6 output stage (head LayerNorm, SiLU gate).
+
+    Draw order (generator seeded with `seed`):
+      ln_w ~ U(0.5, 1.5)   [H, N] fp32 (per-channel scale)
+      ln_b ~ N(0, 0.2)     [H, N] fp32 (per-channel shift)
+      g    ~ N(0, 1.5)     [B, T, H, N], cast to bf16 (the gate before its SiLU)
+    """
+    gen = _gen(seed)
+    ln_w = torch.rand(H, N, generator=gen) + 0.5
+    ln_b = torch.randn(H, N, generator=gen) * 0.2
+    g = (torch.randn(B, T, H, N, generator=gen) * 1.5).to(torch.bfloat16)
+    return {"g": g, "ln_w": ln_w, "ln_b": ln_b}
+
+
 @dataclass(frozen=True)
 class Workload:
     name: str

@@ -69,6 +69,8 @@ def load(path: str = LIB_PATH):
     lib.rwkv_get_wkv6_algo.argtypes = []
     lib.rwkv_get_wkv6_algo.restype = ctypes.c_int
     lib.rwkv_wkv6_forward_bf16_noalloc.argtypes = wkv6 + [ctypes.c_int]
+    lib.rwkv_wkv6_forward_gated_bf16.argtypes = wkv6[:10] + [_vp, _vp, _vp, ctypes.c_float] + wkv6[10:]
+    lib.rwkv_wkv6_forward_gated_bf16.restype = ctypes.c_int
     lib.rwkv_wkv6_forward_bf16_noalloc.restype = ctypes.c_int
     lib.rwkv_set_wkv6_segments.argtypes = [ctypes.c_int]
     lib.rwkv_set_wkv6_segments.restype = ctypes.c_int
@@ -187,6 +189,33 @@ def wkv6_forward(r, k, v, w, u, s0=None, want_state=True, y=None, sT=None, algo=
             lib.rwkv_set_wkv6_algo(prev)
         if prev_seg is not None:
             lib.rwkv_set_wkv6_segments(prev_seg)
+    return (y, sT) if want_state else y
+
+
+def wkv6_forward_gated(r, k, v, w, u, g, ln_w, ln_b, eps=1e-5, s0=None, want_state=True, y=None,
+                       sT=None):
+    """WKV-6 (bf16) with the fused output stage: y = SiLU(g) * LayerNorm_head(o; ln_w, ln_b, eps).
+
+    r,k,v,w,g: [B,T,H,N] bf16; u, ln_w, ln_b: [H,N] fp32; s0: [B,H,N,N] fp32.
+    """
+    lib = load()
+    _cuda(r, "r", torch.bfloat16)
+    B, T, H, N = r.shape
+    for name, t in (("k", k), ("v", v), ("w", w), ("g", g)):
+        _cuda(t, name, torch.bfloat16, (B, T, H, N))
+    for name, t in (("u", u), ("ln_w", ln_w), ("ln_b", ln_b)):
+        _cuda(t, name, torch.float32, (H, N))
+    _cuda(s0, "s0", torch.float32, (B, H, N, N))
+    if y is None:
+        y = torch.empty_like(r)
+    _cuda(y, "y", torch.bfloat16, (B, T, H, N))
+    if sT is None and want_state:
+        sT = torch.empty(B, H, N, N, device=r.device, dtype=torch.float32)
+    _cuda(sT, "sT", torch.float32, (B, H, N, N))
+    _use_current_stream(lib, r.device)
+    _check(lib.rwkv_wkv6_forward_gated_bf16(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
+                                             _ptr(s0), _ptr(g), _ptr(ln_w), _ptr(ln_b), float(eps),
+                                             _ptr(y), _ptr(sT)))
     return (y, sT) if want_state else y
 
 
