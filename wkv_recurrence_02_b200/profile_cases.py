@@ -12,6 +12,8 @@ Every case first makes one untimed call (so a profiler can skip it with ``-s``),
                 then full pass)
   decode        WKV-6 T=1 decode, B256 H64 with the state updated in place (268 MB of state)
   wkv4_decode   RWKV-4 T=1 decode, B2048 C4096 bf16, (a, b, p) state updated in place
+  finch_gated   the finch case through rwkv_wkv6_forward_gated_bf16 (head LayerNorm and
+                SiLU gate fused into the epilogue)
 
 Inputs come from the seeded generators in ``inputs``; nothing here checks results.
 """
@@ -21,7 +23,7 @@ import torch
 
 from . import inputs, ops
 
-CASES = ("wkv4", "finch", "long", "decode", "wkv4_decode")
+CASES = ("wkv4", "finch", "long", "decode", "wkv4_decode", "finch_gated")
 
 
 def _wkv4(reps):
@@ -40,6 +42,18 @@ def _wkv4_decode(reps):
     y = torch.empty_like(a[2])
     for _ in range(1 + reps):
         ops.wkv4_forward(*a, s0=st, sT=st, y=y, want_state=True)
+
+
+def _wkv6_gated(B, T, H, reps):
+    x = inputs.wkv6_inputs(B, T, H, 64, "bf16", seed=0, s0_std=0.1)
+    a = [x[n].cuda() for n in ("r", "k", "v", "w", "u")]
+    ng = inputs.norm_gate_inputs(B, T, H, 64, seed=1)
+    g, lw, lb = (ng[n].cuda() for n in ("g", "ln_w", "ln_b"))
+    s0 = x["s0"].cuda()
+    y = torch.empty_like(a[0])
+    sT = torch.empty_like(s0)
+    for _ in range(1 + reps):
+        ops.wkv6_forward_gated(*a, g, lw, lb, eps=1e-5, s0=s0, y=y, sT=sT)
 
 
 def _wkv6(B, T, H, reps, s0_std=0.1):
@@ -63,6 +77,8 @@ def run(case, reps=1):
         _wkv6(256, 1, 64, reps)
     elif case == "wkv4_decode":
         _wkv4_decode(reps)
+    elif case == "finch_gated":
+        _wkv6_gated(8, 1024, 32, reps)
     else:
         raise ValueError(f"unknown case {case!r}; choose from {CASES}")
 
