@@ -18,6 +18,9 @@ Sources:
   * Head LayerNorm and SiLU gate on the WKV-6 output: the same summary, section 4
     (architecture overview: LayerNorm on the heads, SiLU attention gating) and 4.1.2
     (the LayerNorm acts on each head separately, i.e. GroupNorm over the heads).
+  * Decay from its logit, w = exp(-exp(omega)): the same summary, section 4.1.2
+    (Eagle: omega is the trainable per-head parameter) and 4.2.2 (Finch: w_t varies
+    per token; section 4.2.1 gives the LoRA offset that makes omega_t per token).
 """
 import ctypes
 import os
@@ -44,6 +47,8 @@ class Oracle:
         lib.oracle_head_norm_gate.argtypes = [_I64, _I64, _I64, _I64, _DP, _DP, _DP, _DP,
                                               ctypes.c_double, _DP]
         lib.oracle_head_norm_gate.restype = None
+        lib.oracle_decay_from_logit.argtypes = [_I64, _DP, _DP]
+        lib.oracle_decay_from_logit.restype = None
         lib.oracle_wkv6.restype = None
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_threads.restype = ctypes.c_int
@@ -127,6 +132,23 @@ class Oracle:
         o, sT = self.wkv6(r, k, v, w, u, s0=s0)
         return self.head_norm_gate(o, g, ln_w, ln_b, eps), sT
 
+    def decay_from_logit(self, omega):
+        """w = exp(-exp(omega)) elementwise (any shape), in float64."""
+        omega, op = self._f64(omega)
+        w = np.empty_like(omega)
+        self._lib.oracle_decay_from_logit(omega.size, op, w.ctypes.data_as(_DP))
+        return w
+
+    def wkv6_logit(self, r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None, eps=1e-5):
+        """WKV-6 with the decay given by its logit omega_t (w_t = exp(-exp(omega_t))): (y, sT).
+
+        With g, ln_w and ln_b the head LayerNorm and SiLU gate follow, as in wkv6_gated.
+        """
+        w = self.decay_from_logit(omega)
+        if g is None:
+            return self.wkv6(r, k, v, w, u, s0=s0)
+        return self.wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=s0)
+
 
 _DEFAULT = None
 
@@ -155,6 +177,14 @@ def head_norm_gate(o, g, ln_w, ln_b, eps):
 
 def wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=None):
     return get().wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=s0)
+
+
+def decay_from_logit(omega):
+    return get().decay_from_logit(omega)
+
+
+def wkv6_logit(r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None, eps=1e-5):
+    return get().wkv6_logit(r, k, v, omega, u, s0=s0, g=g, ln_w=ln_w, ln_b=ln_b, eps=eps)
 
 
 def set_threads(n: int = 0) -> int:

@@ -214,3 +214,18 @@ void oracle_head_norm_gate(int64_t B, int64_t T, int64_t H, int64_t N, const dou
         }
     }
 }
+
+/*
+ * Decay from its logit, [E412] and [F422].
+ *
+ * Eagle obtains the per-channel decay as w = exp(-exp(omega)) from the trainable logit
+ * omega, which puts w in (0,1); Finch adds a per-token, data-dependent offset (a LoRA of
+ * the token-shifted input, section 4.2.1) to omega before the same map, giving w_t per
+ * token and channel.  This evaluates the map elementwise: w[i] = exp(-exp(omega[i])),
+ * n elements.  omega = -inf gives 1, omega = +inf gives 0.
+ */
+void oracle_decay_from_logit(int64_t n, const double *omega, double *w)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) w[i] = exp(-exp(omega[i]));
+}

@@ -14,7 +14,10 @@ Kinds of pin used (none retypes the oracle's recurrence):
     linearity in (v, s0) and head independence, split-sequence chaining;
   * head LayerNorm + SiLU gate: the two-channel closed form, SiLU at +-ln 3 (sigmoid 3/4
     and 1/4), shift/scale invariance and unit moments, affinity in the per-channel
-    parameters, per-head parameter rows.
+    parameters, per-head parameter rows;
+  * decay from its logit, w = exp(-exp(omega)): points with closed forms (ln ln 2 -> 1/2),
+    inversion by numpy's logarithms, monotonicity and range, the slow-decay asymptote,
+    and the -inf / +inf limits through the recurrence (no decay, instant forgetting).
 """
 import json
 import os
@@ -347,12 +350,62 @@ def pin_norm_gate_heads(O):
     assert _rel(yp, y[:, :, perm]) < 1e-12, "per-head parameters"
 
 
+# ------------------------------------------------------------ decay from its logit omega
+def pin_logit_closed_forms(O):
+    """w = exp(-exp(omega)): omega = ln ln 2 gives 1/2, ln ln 4 gives 1/4, 0 gives 1/e,
+    ln 3 gives e^-3; the limits -inf and +inf give 1 and 0."""
+    om = np.array([np.log(np.log(2.0)), np.log(np.log(4.0)), 0.0, np.log(3.0), -np.inf, np.inf])
+    w = O.decay_from_logit(om)
+    expect = np.array([0.5, 0.25, np.exp(-1.0), np.exp(-3.0), 1.0, 0.0])
+    assert np.max(np.abs(w - expect)) < 1e-15, ("logit closed forms", w)
+
+
+def pin_logit_inverse_and_shape(O):
+    """omega = ln(-ln w) inverts the map (numpy's logarithms, not the map), the map keeps
+    the array's shape, is strictly decreasing and stays in (0, 1); for omega << 0,
+    -ln w = e^omega, i.e. the decay distance 1 - w is about e^omega."""
+    rng = np.random.default_rng(45)
+    w_true = rng.uniform(1e-6, 1 - 1e-9, (3, 5, 2, 4))
+    w = O.decay_from_logit(np.log(-np.log(w_true)))
+    assert w.shape == w_true.shape, "shape"
+    assert np.max(np.abs(w - w_true) / w_true) < 1e-13, "inverse"
+    om = np.linspace(-30.0, 3.0, 331)
+    ws = O.decay_from_logit(om)
+    assert np.all(np.diff(ws) < 0) and np.all((ws > 0) & (ws < 1)), "monotone, in (0, 1)"
+    small = np.array([-12.0, -16.0, -20.0])
+    assert _rel(-np.log(O.decay_from_logit(small)), np.exp(small)) < 1e-6, "slow-decay asymptote"
+
+
+def pin_wkv6_logit_limits(O):
+    """Through the WKV-6 recurrence: omega = -inf everywhere is the no-decay case (causal
+    linear attention, masked matmul); omega = +inf is the instant-forget case,
+    o_t = (r_t.k_{t-1}) v_{t-1} + (r_t.(u*k_t)) v_t; omega = ln ln 2 halves the state."""
+    rng = np.random.default_rng(46)
+    B, T, H, N = 1, 10, 2, 8
+    r, k, v, w, u, s0 = _wkv6_rand(rng, B, T, H, N, True)
+    y, sT = O.wkv6_logit(r, k, v, np.full_like(w, -np.inf), u, s0=s0)
+    for h in range(H):
+        o_ref, s_ref = ref_defs.causal_linear_attention(r[0, :, h], k[0, :, h], v[0, :, h],
+                                                       u[h], s0[0, h])
+        assert _rel(y[0, :, h], o_ref) < 1e-12 and _rel(sT[0, h], s_ref) < 1e-12, "logit no decay"
+    y, sT = O.wkv6_logit(r, k, v, np.full_like(w, np.inf), u, s0=s0)
+    for t in range(1, T):
+        expect = (np.einsum("bhi,bhi->bh", r[:, t], k[:, t - 1])[..., None] * v[:, t - 1]
+                  + np.einsum("bhi,hi,bhi->bh", r[:, t], u, k[:, t])[..., None] * v[:, t])
+        assert _rel(y[:, t], expect) < 1e-13, ("logit instant forget", t)
+    # T = 1 with w = 1/2 on every channel: sT = s0 / 2 + k^T v
+    r1, k1, v1 = r[:, :1], k[:, :1], v[:, :1]
+    _, sT = O.wkv6_logit(r1, k1, v1, np.full_like(r1, np.log(np.log(2.0))), u, s0=s0)
+    assert _rel(sT, 0.5 * s0 + np.einsum("bhi,bhj->bhij", k1[:, 0], v1[:, 0])) < 1e-14, "logit halving"
+
+
 ALL_PINS = [
     pin_wkv4_bruteforce, pin_wkv4_T1, pin_wkv4_fast_decay, pin_wkv4_invariants,
     pin_wkv4_chaining, pin_wkv4_golden,
     pin_wkv6_bruteforce, pin_wkv6_T1, pin_wkv6_fast_decay, pin_wkv6_no_decay,
     pin_wkv6_chaining, pin_wkv6_linearity, pin_wkv6_head_independence, pin_wkv6_golden,
     pin_norm_gate_two_channels, pin_norm_gate_invariants, pin_norm_gate_affine, pin_norm_gate_heads,
+    pin_logit_closed_forms, pin_logit_inverse_and_shape, pin_wkv6_logit_limits,
 ]
 
 

@@ -35,6 +35,11 @@ MUTANTS = [
     ("norm_no_centering", "(x[n] - mean) * rstd", "x[n] * rstd"),
     ("gate_skips_shift", "gate * (ln_w[h * N + n] * (x[n] - mean) * rstd + ln_b[h * N + n])",
      "gate * ln_w[h * N + n] * (x[n] - mean) * rstd + ln_b[h * N + n]"),
+    ("logit_single_exponential", "w[i] = exp(-exp(omega[i]));", "w[i] = exp(-omega[i]);"),
+    ("logit_outer_sign", "w[i] = exp(-exp(omega[i]));", "w[i] = exp(exp(omega[i]));"),
+    ("logit_inner_sign", "w[i] = exp(-exp(omega[i]));", "w[i] = exp(-exp(-omega[i]));"),
+    ("logit_base_two", "w[i] = exp(-exp(omega[i]));", "w[i] = exp2(-exp(omega[i]));"),
+    ("logit_skips_last", "for (int64_t i = 0; i < n; ++i) w[i]", "for (int64_t i = 0; i < n - 1; ++i) w[i]"),
 ]
 
 

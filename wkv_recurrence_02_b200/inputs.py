@@ -53,7 +53,7 @@ def wkv4_inputs(B: int, T: int, C: int, dtype: str = "fp32", seed: int = 0, wu_s
 
 
 def wkv6_inputs(B: int, T: int, H: int, N: int = 64, dtype: str = "fp32", seed: int = 0,
-                s0_std: float = None):
+                s0_std: float = None, decay: str = "w"):
     """One WKV-6 call, Finch-style per-token decay.
 
     Draw order (generator seeded with `seed`):
@@ -62,8 +62,12 @@ def wkv6_inputs(B: int, T: int, H: int, N: int = 64, dtype: str = "fp32", seed: 
       r, k, v ~ N(0, 1) / sqrt(N) [B, T, H, N] each, in that order
       xi      ~ N(0, 1)          [B, T, H, N];  omega_t = omega_h + 0.3 xi
       s0      ~ N(0, s0_std)     [B, H, N, N]  (only when s0_std is given)
-    w = exp(-exp(omega_t)) is formed in fp32 and then cast with r, k, v; u and s0 stay fp32.
+    decay="w": w = exp(-exp(omega_t)) is formed in fp32 and then cast with r, k, v;
+    decay="omega": the logit omega_t itself is returned (key "omega", cast like r, k, v)
+    instead of w, for the entry points that take the logit.  u and s0 stay fp32.
     """
+    if decay not in ("w", "omega"):
+        raise ValueError(f"decay must be 'w' or 'omega', not {decay!r}")
     g = _gen(seed)
     omega_h = torch.rand(H, N, generator=g) * 5.5 - 6.0
     u = torch.randn(H, N, generator=g) * 0.5
@@ -74,13 +78,16 @@ def wkv6_inputs(B: int, T: int, H: int, N: int = 64, dtype: str = "fp32", seed: 
     xi = torch.randn(B, T, H, N, generator=g)
     omega_t = omega_h + 0.3 * xi
     del xi
-    w = torch.exp(-torch.exp(omega_t))
+    dt = _DTYPES[dtype]
+    if decay == "w":
+        dec = {"w": torch.exp(-torch.exp(omega_t)).to(dt)}
+    else:
+        dec = {"omega": omega_t.to(dt)}
     del omega_t
     s0 = None
     if s0_std is not None:
         s0 = torch.randn(B, H, N, N, generator=g) * float(s0_std)
-    dt = _DTYPES[dtype]
-    return {"r": r.to(dt), "k": k.to(dt), "v": v.to(dt), "w": w.to(dt), "u": u, "s0": s0}
+    return {"r": r.to(dt), "k": k.to(dt), "v": v.to(dt), **dec, "u": u, "s0": s0}
 
 
 def norm_gate_inputs(B: int, T: int, H: int, N: int = 64, seed: int = 0):
