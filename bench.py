@@ -323,7 +323,9 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
     """Rows beyond the step, timed on their own (not part of the step's metric):
       * the RWKV-4 decode step (T = 1) at the width of a 7B model, state updated in place;
       * the Finch prefill with the time-mixing output stage (head LayerNorm, SiLU gate)
-        fused into the chunked kernel's epilogue, against the same call without it."""
+        fused into the chunked kernel's epilogue, against the same call without it;
+      * the Finch prefill fed the decay logit omega_t (w_t = exp(-exp(omega_t)) formed in
+        the kernel), plain and with the fused output stage."""
     hbm, _ = load_peaks()
     rows = {}
     f = wl.finch
@@ -340,6 +342,22 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
         "GBps": round(nbytes / (gated * 1e-6) / 1e9, 1),
         "frac_hbm": round(nbytes / (gated * 1e-6) / 1e9 / hbm, 4),
         "separate_stage_floor_us": round(separate / (hbm * 1e9) * 1e6, 2)}
+    # decay given by its logit: omega_t = omega_h + 0.3 xi, the recipe the step's w comes from
+    gen = torch.Generator(device=dev)
+    gen.manual_seed(7)
+    om = ((torch.rand(32, 64, device=dev, generator=gen) * 5.5 - 6.0)
+          + 0.3 * torch.randn(8, 4096, 32, 64, device=dev, generator=gen)).to(torch.bfloat16)
+    omega = _time_us(torch, stream, dev, lambda: ops.wkv6_forward_omega(
+        f["r"], f["k"], f["v"], om, f["u"], s0=f["s0"], y=f["y"], sT=f["sT"]), 20)
+    omega_gated = _time_us(torch, stream, dev, lambda: ops.wkv6_forward_omega(
+        f["r"], f["k"], f["v"], om, f["u"], s0=f["s0"], g=g, ln_w=lw, ln_b=lb, y=f["y"], sT=f["sT"]), 20)
+    nb = BYTES["wkv6_chunked_finch"]
+    rows["wkv6_finch_omega_B8_T4096_H32"] = {
+        "avg_us": round(omega, 2), "w_input_avg_us": round(plain, 2), "gated_avg_us": round(omega_gated, 2),
+        "algorithmic_bytes": nb, "GBps": round(nb / (omega * 1e-6) / 1e9, 1),
+        "frac_hbm": round(nb / (omega * 1e-6) / 1e9 / hbm, 4),
+        "separate_map_floor_us": round(2 * om.numel() * 2 / (hbm * 1e9) * 1e6, 2)}
+    del om
     B, C = 2048, 4096
     x = inputs.wkv4_inputs(B, 1, C, "bf16", seed=5, wu_seed=6)
     w, u, k, v = (x[n].to(dev) for n in ("w", "u", "k", "v"))

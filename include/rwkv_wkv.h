@@ -137,6 +137,30 @@ int rwkv_wkv6_forward_gated_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
                                  const uint16_t *g, const float *ln_w, const float *ln_b, float eps,
                                  uint16_t *y, float *sT);
 
+/* WKV-6 fed the decay LOGIT instead of the decay ([E412]: w = exp(-exp(omega)) with omega
+ * the trainable per-head parameter; [F422]: omega_t per token, the learned omega plus the
+ * data-dependent LoRA offset of the Finch token shift, section 4.2.1).  The kernels form
+ *   w_t[i] = exp(-exp(omega_t[i]))
+ * in fp32 as they load each tile and then run the recurrence of rwkv_wkv6_forward_bf16.
+ * Passing omega_t saves the caller a separate elementwise pass over [B, T, H, N], and a decay
+ * close to 1 keeps its distance from 1: a bf16 w cannot hold one (the largest bf16 value
+ * below 1 is 1 - 2^-8), so slowly decaying channels of a bf16 w round to w = 1 or to
+ * 1 - 2^-8.  Any omega, +-inf included, gives w in [0, 1]; NaN is outside the contract.
+ *   omega         : [B, T, H, N] bf16 (in place of w).
+ *   g, ln_w, ln_b : all NULL = plain output (as rwkv_wkv6_forward_bf16);  all non-NULL =
+ *                   the fused head LayerNorm + SiLU gate of rwkv_wkv6_forward_gated_bf16,
+ *                   with eps as there.  Some but not all NULL: RWKV_ERR_NULL.  eps is
+ *                   ignored without the gate.
+ * Kernels, the rwkv_set_wkv6_algo choice (plain output only), layouts, aliasing rules and
+ * errors are those of rwkv_wkv6_forward_bf16 / rwkv_wkv6_forward_gated_bf16.  The chunked
+ * kernel forms w_t with the hardware's approximate base-2 exponential (relative error of
+ * order 1e-7 on w_t); the serial and decode kernels with the accurate one. */
+int rwkv_wkv6_forward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
+                                 const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                                 const uint16_t *omega, const float *u, const float *s0,
+                                 const uint16_t *g, const float *ln_w, const float *ln_b, float eps,
+                                 uint16_t *y, float *sT);
+
 /* Kernel choice for WKV-6 on the calling thread: RWKV_WKV6_AUTO (default, as above),
  * RWKV_WKV6_SERIAL (always the serial kernel), RWKV_WKV6_CHUNKED (the chunked kernel
  * for bf16 whatever T; ignored for fp32).  Returns RWKV_OK or RWKV_ERR_ARG. */

@@ -106,6 +106,32 @@ def test_wkv6_gated_validation(lib):
     assert f(0, 4, 2, 64, *([None] * 9), ctypes.c_float(1e-5), None, None) == 0  # empty
 
 
+def test_wkv6_omega_validation(lib):
+    """The logit entry: the output-stage trio is all-or-nothing, eps is checked only with the
+    gate, and the logit is an input like w."""
+    f = lib.rwkv_wkv6_forward_omega_bf16
+    r, k, v, om, u, s0, g, lw, lb, y, sT = (_p(i << 24) for i in range(11))
+
+    def call(eps=1e-5, **kw):
+        a = dict(r=r, k=k, v=v, om=om, u=u, s0=s0, g=g, lw=lw, lb=lb, y=y, sT=sT)
+        a.update(kw)
+        return f(1, 4, 2, 64, a["r"], a["k"], a["v"], a["om"], a["u"], a["s0"], a["g"], a["lw"], a["lb"],
+                 ctypes.c_float(eps), a["y"], a["sT"])
+
+    assert call(om=None) == -1                     # logit null
+    assert call(g=None) == -1                      # gate missing, LayerNorm given
+    assert call(g=None, lw=None) == -1             # shift alone
+    assert call(lw=None, lb=None) == -1            # gate alone
+    assert call(eps=-1.0) == -8                    # eps < 0 with the gate
+    assert call(om=_p((3 << 24) + 8)) == -7        # misaligned logit
+    assert call(y=om) == -4                        # y == omega
+    assert call(sT=_p((3 << 24) + 512)) == -4      # sT over the logit
+    assert f(2, 4, 0, 64, *([None] * 9), ctypes.c_float(1e-5), None, None) == 0  # empty
+    if not torch.cuda.is_available():
+        # without the gate, eps is ignored: a valid call gets as far as CUDA
+        assert call(g=None, lw=None, lb=None, eps=-1.0) == -5
+
+
 def test_algo_selection(lib):
     assert lib.rwkv_set_wkv6_algo(7) == -8
     for a in (1, 2, 0):

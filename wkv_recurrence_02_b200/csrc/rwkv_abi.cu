@@ -124,7 +124,7 @@ int wkv4_entry(int64_t B, int64_t T, int64_t C, const float *w, const float *u,
 int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
                const void *v, const void *w, const float *u, const float *s0, void *y,
                float *sT, bool bf16, const void *g = nullptr, const float *ln_w = nullptr,
-               const float *ln_b = nullptr, float eps = 0.f, bool gated = false)
+               const float *ln_b = nullptr, float eps = 0.f, bool gated = false, bool omega = false)
 {
     tl_err[0] = 0;
     if (B < 0 || T < 0 || H < 0 || N < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
@@ -169,6 +169,7 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
         return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "T=0 state copy");
     }
     wkv::Wkv6Args a{B, T, H, N, r, k, v, w, u, s0, y, sT, bf16, status, tl_wkv6_segments};
+    a.omega = omega;
     cudaError_t e;
     if (gated) {  // fused output stage: chunked for T > 1, decode for T == 1
         a.g = g;
@@ -298,6 +299,18 @@ extern "C" int rwkv_wkv6_forward_gated_bf16(int64_t B, int64_t T, int64_t H, int
                                             float *sT)
 {
     return wkv6_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, true, g, ln_w, ln_b, eps, true);
+}
+
+int rwkv_wkv6_forward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,
+                                 const uint16_t *k, const uint16_t *v, const uint16_t *omega,
+                                 const float *u, const float *s0, const uint16_t *g, const float *ln_w,
+                                 const float *ln_b, float eps, uint16_t *y, float *sT)
+{
+    // the output stage is fused when any of its three tensors is given; the gated checks then
+    // reject a missing one
+    const bool gated = g || ln_w || ln_b;
+    return wkv6_entry(B, T, H, N, r, k, v, omega, u, s0, y, sT, true, g, ln_w, ln_b, gated ? eps : 0.f, gated,
+                      true);
 }
 
 int rwkv_wkv6_forward_bf16_noalloc(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,

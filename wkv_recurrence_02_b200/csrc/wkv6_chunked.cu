@@ -383,6 +383,17 @@ __device__ __forceinline__ float bonus4(Q4 r, Q4 u, Q4 k)
     return lo(acc) + hi(acc);
 }
 
+// Decay from its logit (section 4.1.2: w = exp(-exp(omega))), as 2^(-2^(omega log2 e) log2 e)
+// with two approximate base-2 exponentials.  omega = -inf gives 1, +inf gives 0; fp32 keeps a
+// decay close to 1 apart from 1, which a bf16 w cannot (its largest value below 1 is 1 - 2^-8).
+__device__ __forceinline__ float decay_of_logit(float om)
+{
+    constexpr float kLog2e = 1.4426950408889634f;
+    return ex2_approx(-ex2_approx(om * kLog2e) * kLog2e);
+}
+__device__ __forceinline__ P2 decay2(P2 om) { return pk(decay_of_logit(lo(om)), decay_of_logit(hi(om))); }
+__device__ __forceinline__ Q4 decay4(Q4 om) { return {decay2(om.a), decay2(om.b)}; }
+
 struct ChunkedParams {
     int64_t T, H;
     const float *u, *s0;
@@ -526,7 +537,7 @@ __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[
 // Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue), scores
 // done, O done, state done and stage empty (tcgen05.commit).  Per-chunk bookkeeping (bonus
 // diagonal, decay, path flags) lives beside the chunk's stage.
-template <bool GATED>
+template <bool GATED, bool OMEGA>
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                     const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
@@ -630,7 +641,12 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int t = t0h + m;
-                w[m] = t < tv ? unpack4(ld_u2(st + SLOT_W, swz(t, cbyte))) : one4();
+                if (t < tv) {
+                    const Q4 x = unpack4(ld_u2(st + SLOT_W, swz(t, cbyte)));
+                    w[m] = OMEGA ? decay4(x) : x;
+                } else {
+                    w[m] = one4();
+                }
                 Gh = mul4(Gh, w[m]);
             }
             const Q4 Go = shfl_xor4(Gh, 16);
@@ -709,7 +725,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                                 const float2 rt = ld_bf2(st + SLOT_R, swz(t, 2 * cc));
                                 const float2 ki = ld_bf2(st + SLOT_K, swz(i, 2 * cc));
                                 float2 f = one;
-                                for (int j = i + 1; j < t; ++j) f = mul2(f, ld_bf2(st + SLOT_W, swz(j, 2 * cc)));
+                                for (int j = i + 1; j < t; ++j) {
+                                    float2 wj = ld_bf2(st + SLOT_W, swz(j, 2 * cc));
+                                    if (OMEGA) wj = make_float2(decay_of_logit(wj.x), decay_of_logit(wj.y));
+                                    f = mul2(f, wj);
+                                }
                                 acc += rt.x * ki.x * f.x + rt.y * ki.y * f.y;
                             }
                         }
@@ -1155,7 +1175,8 @@ cudaError_t configure_kernel()
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (done[dev]) return cudaSuccess;
-    for (auto kern : {wkv6_chunked_kernel<false>, wkv6_chunked_kernel<true>}) {
+    for (auto kern : {wkv6_chunked_kernel<false, false>, wkv6_chunked_kernel<true, false>,
+                      wkv6_chunked_kernel<false, true>, wkv6_chunked_kernel<true, true>}) {
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
@@ -1248,13 +1269,15 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
         ChunkedParams pa = prm;
         pa.state_only = 1;
         pa.seg = seg;
-        wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads,
-                                     kSmemBytes, s>>>(mr, mk, mv, mw, pa);
+        auto kso = a.omega ? wkv6_chunked_kernel<false, true> : wkv6_chunked_kernel<false, false>;
+        kso<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes, s>>>(mr, mk, mv,
+                                                                                                      mw, pa);
         e = cudaGetLastError();
         prm.seg = seg;
     }
     if (e == cudaSuccess) {
-        auto kern = prm.gate ? wkv6_chunked_kernel<true> : wkv6_chunked_kernel<false>;
+        auto kern = prm.gate ? (a.omega ? wkv6_chunked_kernel<true, true> : wkv6_chunked_kernel<true, false>)
+                             : (a.omega ? wkv6_chunked_kernel<false, true> : wkv6_chunked_kernel<false, false>);
         kern<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(mr, mk, mv,
                                                                                                    mw, prm);
         e = cudaGetLastError();
@@ -1346,12 +1369,13 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
         // array has to start at zero, and what an earlier call left there is never read
         ChunkedParams pa = prm;
         pa.state_only = 1;
-        wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads,
-                                     kSmemBytes, s>>>(mr, mk, mv, mw, pa);
+        wkv6_chunked_kernel<false, false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)),
+                                            kThreads, kSmemBytes, s>>>(mr, mk, mv, mw, pa);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
-    wkv6_chunked_kernel<false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads, kSmemBytes, s>>>(
+    wkv6_chunked_kernel<false, false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads,
+                                        kSmemBytes, s>>>(
         mr, mk, mv, mw, prm);
     return cudaGetLastError();
 }

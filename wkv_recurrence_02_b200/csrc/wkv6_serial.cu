@@ -20,6 +20,8 @@
 //    stores, so the 2 x 16 KB state stream per head is fully coalesced.  Partial
 //    outputs are reduced over the 16 row groups through shared memory.  With a gate g the
 //    64 outputs of the head go through the fused LayerNorm + SiLU gate before the store.
+// Both kernels can take the decay as its logit omega_t and form w_t = exp(-exp(omega_t)) as
+// they load it.
 #include "wkv_internal.cuh"
 
 namespace wkv {
@@ -40,11 +42,15 @@ template <> __device__ __forceinline__ void st<__nv_bfloat16>(__nv_bfloat16 *p, 
     *p = __float2bfloat16_rn(x);
 }
 
+// Decay from its logit, w = exp(-exp(omega)) (section 4.1.2), with the accurate exponential:
+// omega = -inf gives 1, +inf gives 0.
+__device__ __forceinline__ float decay_of_logit(float om) { return expf(-expf(om)); }
+
 template <typename T>
 __global__ void __launch_bounds__(kN)
 wkv6_serial_kernel(int64_t T_len, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
-                   const float *s0, T *__restrict__ y, float *sT)
+                   const float *s0, T *__restrict__ y, float *sT, int omega)
 {
     __shared__ __align__(16) float sr[2][kN], sk[2][kN], sw[2][kN];
     __shared__ __align__(16) float su[kN];
@@ -67,7 +73,7 @@ wkv6_serial_kernel(int64_t T_len, int64_t H, const T *__restrict__ r, const T *_
         const int buf = static_cast<int>(t & 1);
         sr[buf][j] = rn;
         sk[buf][j] = kn;
-        sw[buf][j] = wn;
+        sw[buf][j] = omega ? decay_of_logit(wn) : wn;
         const float vj = vn;
         __syncthreads();
         if (t + 1 < T_len) {
@@ -136,7 +142,7 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ w,
                    const float *__restrict__ u, const float *s0, T *__restrict__ y, float *sT,
                    const T *__restrict__ g, const float *__restrict__ ln_w, const float *__restrict__ ln_b,
-                   float eps)
+                   float eps, int omega)
 {
     __shared__ __align__(16) float red[16][kN];
     __shared__ float bred[16];
@@ -149,7 +155,9 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
 
     const float4 rr = ld4(r + vbase + 4 * ig);
     const float4 kk = ld4(k + vbase + 4 * ig);
-    const float4 ww = ld4(w + vbase + 4 * ig);
+    float4 ww = ld4(w + vbase + 4 * ig);
+    if (omega)
+        ww = make_float4(decay_of_logit(ww.x), decay_of_logit(ww.y), decay_of_logit(ww.z), decay_of_logit(ww.w));
     const float4 uu = __ldg(reinterpret_cast<const float4 *>(u + h * kN + 4 * ig));
     const float4 vv = ld4(v + vbase + 4 * j4);
 
@@ -185,9 +193,9 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
     if (tid < kN) {
         float acc = 0.f, bsum = 0.f;
 #pragma unroll
-        for (int g = 0; g < 16; ++g) {
-            acc += red[g][tid];
-            bsum += bred[g];
+        for (int rg = 0; rg < 16; ++rg) {
+            acc += red[rg][tid];
+            bsum += bred[rg];
         }
         float o = fmaf(bsum, ld(v + vbase + tid), acc);
         if (g) {
@@ -225,12 +233,12 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s)
         wkv6_serial_kernel<T><<<static_cast<unsigned>(blocks), kN, 0, s>>>(
             a.T, a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k),
             static_cast<const T *>(a.v), static_cast<const T *>(a.w), a.u, a.s0,
-            static_cast<T *>(a.y), a.sT);
+            static_cast<T *>(a.y), a.sT, a.omega ? 1 : 0);
     } else {
         wkv6_serial_kernel<float><<<static_cast<unsigned>(blocks), kN, 0, s>>>(
             a.T, a.H, static_cast<const float *>(a.r), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), static_cast<const float *>(a.w), a.u, a.s0,
-            static_cast<float *>(a.y), a.sT);
+            static_cast<float *>(a.y), a.sT, a.omega ? 1 : 0);
     }
     return cudaGetLastError();
 }
@@ -246,12 +254,12 @@ cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s)
         wkv6_decode_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k),
             static_cast<const T *>(a.v), static_cast<const T *>(a.w), a.u, a.s0,
-            static_cast<T *>(a.y), a.sT, static_cast<const T *>(a.g), a.ln_w, a.ln_b, a.eps);
+            static_cast<T *>(a.y), a.sT, static_cast<const T *>(a.g), a.ln_w, a.ln_b, a.eps, a.omega ? 1 : 0);
     } else {
         wkv6_decode_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const float *>(a.r), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), static_cast<const float *>(a.w), a.u, a.s0,
-            static_cast<float *>(a.y), a.sT, nullptr, nullptr, nullptr, 0.f);
+            static_cast<float *>(a.y), a.sT, nullptr, nullptr, nullptr, 0.f, a.omega ? 1 : 0);
     }
     return cudaGetLastError();
 }

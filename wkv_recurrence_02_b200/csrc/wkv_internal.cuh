@@ -45,6 +45,8 @@ struct Wkv6Args {
     const void *g = nullptr;    // [B,T,H,N] bf16
     const float *ln_w = nullptr, *ln_b = nullptr;  // [H,N]
     float eps = 0.f;
+    // decay given by its logit: w holds omega_t and the kernels form w_t = exp(-exp(omega_t))
+    bool omega = false;
 };
 
 // cuTensorMapEncodeTiled from the driver (null if unavailable).

@@ -71,6 +71,8 @@ def load(path: str = LIB_PATH):
     lib.rwkv_wkv6_forward_bf16_noalloc.argtypes = wkv6 + [ctypes.c_int]
     lib.rwkv_wkv6_forward_gated_bf16.argtypes = wkv6[:10] + [_vp, _vp, _vp, ctypes.c_float] + wkv6[10:]
     lib.rwkv_wkv6_forward_gated_bf16.restype = ctypes.c_int
+    lib.rwkv_wkv6_forward_omega_bf16.argtypes = wkv6[:10] + [_vp, _vp, _vp, ctypes.c_float] + wkv6[10:]
+    lib.rwkv_wkv6_forward_omega_bf16.restype = ctypes.c_int
     lib.rwkv_wkv6_forward_bf16_noalloc.restype = ctypes.c_int
     lib.rwkv_set_wkv6_segments.argtypes = [ctypes.c_int]
     lib.rwkv_set_wkv6_segments.restype = ctypes.c_int
@@ -216,6 +218,43 @@ def wkv6_forward_gated(r, k, v, w, u, g, ln_w, ln_b, eps=1e-5, s0=None, want_sta
     _check(lib.rwkv_wkv6_forward_gated_bf16(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u),
                                              _ptr(s0), _ptr(g), _ptr(ln_w), _ptr(ln_b), float(eps),
                                              _ptr(y), _ptr(sT)))
+    return (y, sT) if want_state else y
+
+
+def wkv6_forward_omega(r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None, eps=1e-5,
+                       want_state=True, y=None, sT=None, algo=None):
+    """WKV-6 (bf16) fed the decay logit omega_t; the kernels form w_t = exp(-exp(omega_t)).
+
+    r,k,v,omega (and g): [B,T,H,N] bf16; u (and ln_w, ln_b): [H,N] fp32; s0: [B,H,N,N] fp32.
+    With g, ln_w and ln_b the fused head LayerNorm + SiLU gate is applied as in
+    wkv6_forward_gated.  algo (plain output only): as in wkv6_forward.
+    """
+    lib = load()
+    _cuda(r, "r", torch.bfloat16)
+    B, T, H, N = r.shape
+    for name, t in (("k", k), ("v", v), ("omega", omega), ("g", g)):
+        _cuda(t, name, torch.bfloat16, (B, T, H, N))
+    for name, t in (("u", u), ("ln_w", ln_w), ("ln_b", ln_b)):
+        _cuda(t, name, torch.float32, (H, N))
+    _cuda(s0, "s0", torch.float32, (B, H, N, N))
+    if y is None:
+        y = torch.empty_like(r)
+    _cuda(y, "y", torch.bfloat16, (B, T, H, N))
+    if sT is None and want_state:
+        sT = torch.empty(B, H, N, N, device=r.device, dtype=torch.float32)
+    _cuda(sT, "sT", torch.float32, (B, H, N, N))
+    _use_current_stream(lib, r.device)
+    prev = None
+    if algo is not None:
+        prev = lib.rwkv_get_wkv6_algo()
+        _check(lib.rwkv_set_wkv6_algo(ALGOS[algo]))
+    try:
+        _check(lib.rwkv_wkv6_forward_omega_bf16(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(omega),
+                                                 _ptr(u), _ptr(s0), _ptr(g), _ptr(ln_w), _ptr(ln_b),
+                                                 float(eps), _ptr(y), _ptr(sT)))
+    finally:
+        if prev is not None:
+            lib.rwkv_set_wkv6_algo(prev)
     return (y, sT) if want_state else y
 
 
