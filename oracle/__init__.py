@@ -49,6 +49,10 @@ class Oracle:
         lib.oracle_head_norm_gate.restype = None
         lib.oracle_decay_from_logit.argtypes = [_I64, _DP, _DP]
         lib.oracle_decay_from_logit.restype = None
+        lib.oracle_decay_from_logit_grad.argtypes = [_I64, _DP, _DP, _DP]
+        lib.oracle_decay_from_logit_grad.restype = None
+        lib.oracle_wkv6_backward.argtypes = [_I64, _I64, _I64, _I64] + [_DP] * 15
+        lib.oracle_wkv6_backward.restype = None
         lib.oracle_wkv6.restype = None
         lib.oracle_set_threads.argtypes = [ctypes.c_int]
         lib.oracle_set_threads.restype = ctypes.c_int
@@ -139,6 +143,50 @@ class Oracle:
         self._lib.oracle_decay_from_logit(omega.size, op, w.ctypes.data_as(_DP))
         return w
 
+    def decay_from_logit_grad(self, omega, dw):
+        """dL/domega from dL/dw through w = exp(-exp(omega)), elementwise, in float64."""
+        omega, op = self._f64(omega)
+        dw, dp = self._f64(dw)
+        assert dw.shape == omega.shape
+        out = np.empty_like(omega)
+        self._lib.oracle_decay_from_logit_grad(omega.size, op, dp, out.ctypes.data_as(_DP))
+        return out
+
+    def wkv6_backward(self, r, k, v, w, u, dy, s0=None, dsT=None):
+        """WKV-6 backward: given dL/dy (and dL/dsT, None = 0), returns the dict of float64
+        gradients dr, dk, dv, dw [B,T,H,N], du [H,N] and ds0 [B,H,N,N]."""
+        r, rp = self._f64(r)
+        k, kp = self._f64(k)
+        v, vp = self._f64(v)
+        w, wp = self._f64(w)
+        u, up = self._f64(u)
+        dy, gp = self._f64(dy)
+        B, T, H, N = r.shape
+        for x in (k, v, w, dy):
+            assert x.shape == (B, T, H, N)
+        assert u.shape == (H, N)
+        s0p = dsp = None
+        if s0 is not None:
+            s0, s0p = self._f64(s0)
+            assert s0.shape == (B, H, N, N)
+        if dsT is not None:
+            dsT, dsp = self._f64(dsT)
+            assert dsT.shape == (B, H, N, N)
+        out = {n: np.empty((B, T, H, N), np.float64) for n in ("dr", "dk", "dv", "dw")}
+        out["du"] = np.empty((H, N), np.float64)
+        out["ds0"] = np.empty((B, H, N, N), np.float64)
+        work = np.empty(H * (T + 1) * N * N + H * N * N, np.float64)
+        p = lambda a: a.ctypes.data_as(_DP)  # noqa: E731
+        self._lib.oracle_wkv6_backward(B, T, H, N, rp, kp, vp, wp, up, s0p, gp, dsp, p(out["dr"]), p(out["dk"]),
+                                       p(out["dv"]), p(out["dw"]), p(out["du"]), p(out["ds0"]), p(work))
+        return out
+
+    def wkv6_logit_backward(self, r, k, v, omega, u, dy, s0=None, dsT=None):
+        """Backward of wkv6_logit (plain output): as wkv6_backward, with domega in place of dw."""
+        out = self.wkv6_backward(r, k, v, self.decay_from_logit(omega), u, dy, s0=s0, dsT=dsT)
+        out["domega"] = self.decay_from_logit_grad(omega, out.pop("dw"))
+        return out
+
     def wkv6_logit(self, r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None, eps=1e-5):
         """WKV-6 with the decay given by its logit omega_t (w_t = exp(-exp(omega_t))): (y, sT).
 
@@ -181,6 +229,18 @@ def wkv6_gated(r, k, v, w, u, g, ln_w, ln_b, eps, s0=None):
 
 def decay_from_logit(omega):
     return get().decay_from_logit(omega)
+
+
+def decay_from_logit_grad(omega, dw):
+    return get().decay_from_logit_grad(omega, dw)
+
+
+def wkv6_backward(r, k, v, w, u, dy, s0=None, dsT=None):
+    return get().wkv6_backward(r, k, v, w, u, dy, s0=s0, dsT=dsT)
+
+
+def wkv6_logit_backward(r, k, v, omega, u, dy, s0=None, dsT=None):
+    return get().wkv6_logit_backward(r, k, v, omega, u, dy, s0=s0, dsT=dsT)
 
 
 def wkv6_logit(r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None, eps=1e-5):

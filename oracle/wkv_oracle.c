@@ -229,3 +229,91 @@ void oracle_decay_from_logit(int64_t n, const double *omega, double *w)
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < n; ++i) w[i] = exp(-exp(omega[i]));
 }
+
+/*
+ * WKV-6 backward: the reverse-mode derivative of oracle_wkv6 ([E412], [F422]) for a loss
+ * L whose gradients with respect to the outputs are dy = dL/dy [B,T,H,N] and
+ * dsT = dL/dsT [B,H,N,N] (NULL = zero).  The forward pass is walked first and every state
+ * it passes through is kept; then, with Lambda = dL/dS for the state after token t
+ * (Lambda = dsT after the last token), the chain rule through the two forward lines
+ *   o_t[j] = sum_i r_t[i] (S[i][j] + u[i] k_t[i] v_t[j]),   S' = diag(w_t) S + k_t^T v_t
+ * gives, for t = T-1 down to 0 with S = the state before token t:
+ *   dr_t[i] = sum_j dy_t[j] (S[i][j] + u[i] k_t[i] v_t[j])
+ *   dk_t[i] = sum_j Lambda[i][j] v_t[j] + sum_j dy_t[j] r_t[i] u[i] v_t[j]
+ *   dv_t[j] = sum_i Lambda[i][j] k_t[i] + sum_i dy_t[j] r_t[i] u[i] k_t[i]
+ *   dw_t[i] = sum_j Lambda[i][j] S[i][j]
+ *   du[i]  += sum_j dy_t[j] r_t[i] k_t[i] v_t[j]
+ *   Lambda[i][j] <- w_t[i] Lambda[i][j] + r_t[i] dy_t[j]    (the gradient reaching S)
+ * and ds0 = Lambda after token 0 is undone.  du is summed over the batch rows (u is
+ * shared by them).  Outputs dr, dk, dv, dw: [B,T,H,N]; du: [H,N]; ds0: [B,H,N,N] or NULL.
+ * work: H*(T+1)*N*N + H*N*N doubles of caller-owned scratch.
+ */
+void oracle_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N,
+                          const double *r, const double *k, const double *v, const double *w,
+                          const double *u, const double *s0, const double *dy, const double *dsT,
+                          double *dr, double *dk, double *dv, double *dw, double *du, double *ds0,
+                          double *work)
+{
+    const int64_t NN = N * N, stride = H * N;
+#pragma omp parallel for schedule(static)
+    for (int64_t h = 0; h < H; ++h) {
+        double *Sall = work + h * (T + 1) * NN;  /* Sall[t] = state before token t */
+        double *L = work + H * (T + 1) * NN + h * NN;
+        const double *uh = u + h * N;
+        for (int64_t i = 0; i < N; ++i) du[h * N + i] = 0.0;
+        for (int64_t bi = 0; bi < B; ++bi) {
+            const int64_t n = bi * H + h, base = (bi * T * H + h) * N;
+            for (int64_t e = 0; e < NN; ++e) Sall[e] = s0 ? s0[n * NN + e] : 0.0;
+            for (int64_t t = 0; t < T; ++t) {
+                const double *kt = k + base + t * stride, *vt = v + base + t * stride;
+                const double *wt = w + base + t * stride;
+                const double *S = Sall + t * NN;
+                double *Sn = Sall + (t + 1) * NN;
+                for (int64_t i = 0; i < N; ++i)
+                    for (int64_t j = 0; j < N; ++j) Sn[i * N + j] = kt[i] * vt[j] + wt[i] * S[i * N + j];
+            }
+            for (int64_t e = 0; e < NN; ++e) L[e] = dsT ? dsT[n * NN + e] : 0.0;
+            for (int64_t t = T - 1; t >= 0; --t) {
+                const int64_t o = base + t * stride;
+                const double *rt = r + o, *kt = k + o, *vt = v + o, *wt = w + o, *gt = dy + o;
+                const double *S = Sall + t * NN;
+                for (int64_t i = 0; i < N; ++i) {
+                    double a = 0.0, b = 0.0, c = 0.0, d = 0.0;
+                    for (int64_t j = 0; j < N; ++j) {
+                        a += gt[j] * (S[i * N + j] + uh[i] * kt[i] * vt[j]);
+                        b += L[i * N + j] * vt[j] + gt[j] * rt[i] * uh[i] * vt[j];
+                        c += L[i * N + j] * S[i * N + j];
+                        d += gt[j] * rt[i] * kt[i] * vt[j];
+                    }
+                    dr[o + i] = a;
+                    dk[o + i] = b;
+                    dw[o + i] = c;
+                    du[h * N + i] += d;
+                }
+                for (int64_t j = 0; j < N; ++j) {
+                    double a = 0.0;
+                    for (int64_t i = 0; i < N; ++i) a += L[i * N + j] * kt[i] + gt[j] * rt[i] * uh[i] * kt[i];
+                    dv[o + j] = a;
+                }
+                for (int64_t i = 0; i < N; ++i)
+                    for (int64_t j = 0; j < N; ++j) L[i * N + j] = wt[i] * L[i * N + j] + rt[i] * gt[j];
+            }
+            if (ds0)
+                for (int64_t e = 0; e < NN; ++e) ds0[n * NN + e] = L[e];
+        }
+    }
+}
+
+/*
+ * Chain rule through the decay map of oracle_decay_from_logit:
+ * d/domega exp(-exp(omega)) = -exp(omega) exp(-exp(omega)), so
+ * domega[i] = dw[i] * (-exp(omega[i]) * exp(-exp(omega[i]))).  n elements.
+ */
+void oracle_decay_from_logit_grad(int64_t n, const double *omega, const double *dw, double *domega)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const double e = exp(omega[i]);
+        domega[i] = dw[i] * (-e * exp(-e));
+    }
+}

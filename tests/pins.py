@@ -17,7 +17,10 @@ Kinds of pin used (none retypes the oracle's recurrence):
     parameters, per-head parameter rows;
   * decay from its logit, w = exp(-exp(omega)): points with closed forms (ln ln 2 -> 1/2),
     inversion by numpy's logarithms, monotonicity and range, the slow-decay asymptote,
-    and the -inf / +inf limits through the recurrence (no decay, instant forgetting).
+    and the -inf / +inf limits through the recurrence (no decay, instant forgetting);
+  * WKV-6 backward: central finite differences of the pinned forward oracle, element by
+    element on a tiny case and along random directions at head size 64; the chain rule
+    through the decay map against differences of the map and of the logit forward.
 """
 import json
 import os
@@ -399,6 +402,89 @@ def pin_wkv6_logit_limits(O):
     assert _rel(sT, 0.5 * s0 + np.einsum("bhi,bhj->bhij", k1[:, 0], v1[:, 0])) < 1e-14, "logit halving"
 
 
+# ------------------------------------------------------------------- WKV-6 backward
+# The backward is pinned against central finite differences of the (separately pinned)
+# forward oracle: L = sum(dy * y) + sum(dsT * sT), so dL/dx is what the backward returns.
+def _wkv6_loss(O, r, k, v, w, u, s0, dy, dsT):
+    y, sT = O.wkv6(r, k, v, w, u, s0=s0)
+    return float(np.sum(dy * y) + np.sum(dsT * sT))
+
+
+def pin_wkv6_backward_fd_elementwise(O):
+    """Every element of every input of a tiny case against its central difference."""
+    rng = np.random.default_rng(47)
+    B, T, H, N = 2, 4, 2, 3
+    r, k, v, w, u, s0 = _wkv6_rand(rng, B, T, H, N, True)
+    dy = rng.normal(0, 1, r.shape)
+    dsT = rng.normal(0, 1, s0.shape)
+    g = O.wkv6_backward(r, k, v, w, u, dy, s0=s0, dsT=dsT)
+    args = {"r": r, "k": k, "v": v, "w": w, "u": u, "s0": s0}
+    h = 1e-6
+    for name, grad in (("r", "dr"), ("k", "dk"), ("v", "dv"), ("w", "dw"), ("u", "du"), ("s0", "ds0")):
+        x = args[name]
+        fd = np.empty_like(x)
+        for idx in np.ndindex(x.shape):
+            a = dict(args)
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            a[name] = xp
+            lp = _wkv6_loss(O, **a, dy=dy, dsT=dsT)
+            a[name] = xm
+            lm = _wkv6_loss(O, **a, dy=dy, dsT=dsT)
+            fd[idx] = (lp - lm) / (2 * h)
+        assert _rel(g[grad], fd) < 1e-6, ("backward vs finite differences", name, _rel(g[grad], fd))
+
+
+def pin_wkv6_backward_fd_directional(O):
+    """Head size 64, no initial state, no state gradient: directional derivatives along a
+    random direction per input."""
+    rng = np.random.default_rng(48)
+    B, T, H, N = 1, 5, 2, 64
+    r, k, v, w, u, _ = _wkv6_rand(rng, B, T, H, N, False)
+    s0 = np.zeros((B, H, N, N))
+    dy = rng.normal(0, 1, r.shape)
+    dsT = np.zeros_like(s0)
+    g = O.wkv6_backward(r, k, v, w, u, dy)
+    args = {"r": r, "k": k, "v": v, "w": w, "u": u, "s0": s0}
+    h = 1e-5
+    for name, grad in (("r", "dr"), ("k", "dk"), ("v", "dv"), ("w", "dw"), ("u", "du"), ("s0", "ds0")):
+        d = rng.normal(0, 1, args[name].shape)
+        a = dict(args)
+        a[name] = args[name] + h * d
+        lp = _wkv6_loss(O, **a, dy=dy, dsT=dsT)
+        a[name] = args[name] - h * d
+        lm = _wkv6_loss(O, **a, dy=dy, dsT=dsT)
+        fd = (lp - lm) / (2 * h)
+        an = float(np.sum(g[grad] * d))
+        assert abs(an - fd) <= 1e-7 * max(1.0, abs(fd)), ("directional derivative", name, an, fd)
+
+
+def pin_logit_backward_fd(O):
+    """The chain rule through w = exp(-exp(omega)): elementwise against central differences
+    of the map, and through the recurrence against differences of wkv6_logit."""
+    om = np.linspace(-8.0, 3.0, 45)
+    h = 1e-6
+    fd = (O.decay_from_logit(om + h) - O.decay_from_logit(om - h)) / (2 * h)
+    dw = np.linspace(-2.0, 2.0, 45)
+    assert _rel(O.decay_from_logit_grad(om, dw), dw * fd) < 1e-7, "map derivative"
+    rng = np.random.default_rng(49)
+    B, T, H, N = 1, 3, 1, 4
+    r, k, v, w, u, s0 = _wkv6_rand(rng, B, T, H, N, True)
+    omega = rng.uniform(-3.0, 1.0, r.shape)
+    dy = rng.normal(0, 1, r.shape)
+    g = O.wkv6_logit_backward(r, k, v, omega, u, dy, s0=s0)
+    fd = np.empty_like(omega)
+    for idx in np.ndindex(omega.shape):
+        op, omm = omega.copy(), omega.copy()
+        op[idx] += h
+        omm[idx] -= h
+        yp, _ = O.wkv6_logit(r, k, v, op, u, s0=s0)
+        ym, _ = O.wkv6_logit(r, k, v, omm, u, s0=s0)
+        fd[idx] = np.sum(dy * (yp - ym)) / (2 * h)
+    assert _rel(g["domega"], fd) < 1e-6, ("logit backward", _rel(g["domega"], fd))
+
+
 ALL_PINS = [
     pin_wkv4_bruteforce, pin_wkv4_T1, pin_wkv4_fast_decay, pin_wkv4_invariants,
     pin_wkv4_chaining, pin_wkv4_golden,
@@ -406,6 +492,7 @@ ALL_PINS = [
     pin_wkv6_chaining, pin_wkv6_linearity, pin_wkv6_head_independence, pin_wkv6_golden,
     pin_norm_gate_two_channels, pin_norm_gate_invariants, pin_norm_gate_affine, pin_norm_gate_heads,
     pin_logit_closed_forms, pin_logit_inverse_and_shape, pin_wkv6_logit_limits,
+    pin_wkv6_backward_fd_elementwise, pin_wkv6_backward_fd_directional, pin_logit_backward_fd,
 ]
 
 

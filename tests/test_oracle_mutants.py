@@ -40,6 +40,19 @@ MUTANTS = [
     ("logit_inner_sign", "w[i] = exp(-exp(omega[i]));", "w[i] = exp(-exp(-omega[i]));"),
     ("logit_base_two", "w[i] = exp(-exp(omega[i]));", "w[i] = exp2(-exp(omega[i]));"),
     ("logit_skips_last", "for (int64_t i = 0; i < n; ++i) w[i]", "for (int64_t i = 0; i < n - 1; ++i) w[i]"),
+    ("bwd_dk_drops_bonus", "b += L[i * N + j] * vt[j] + gt[j] * rt[i] * uh[i] * vt[j];", "b += L[i * N + j] * vt[j];"),
+    ("bwd_dw_uses_next_state", "c += L[i * N + j] * S[i * N + j];",
+     "c += L[i * N + j] * Sall[(t + 1) * NN + i * N + j];"),
+    ("bwd_adjoint_transposed", "L[i * N + j] = wt[i] * L[i * N + j] + rt[i] * gt[j];",
+     "L[i * N + j] = wt[i] * L[i * N + j] + rt[j] * gt[i];"),
+    ("bwd_adjoint_decay_wrong_axis", "L[i * N + j] = wt[i] * L[i * N + j] + rt[i] * gt[j];",
+     "L[i * N + j] = wt[j] * L[i * N + j] + rt[i] * gt[j];"),
+    ("bwd_du_not_summed_over_batch", "du[h * N + i] += d;", "du[h * N + i] = d;"),
+    ("bwd_ds0_not_propagated", "ds0[n * NN + e] = L[e];", "ds0[n * NN + e] = dsT ? dsT[n * NN + e] : 0.0;"),
+    ("bwd_dv_bonus_without_u", "+ gt[j] * rt[i] * uh[i] * kt[i];", "+ gt[j] * rt[i] * kt[i];"),
+    ("bwd_dr_decayed_state", "a += gt[j] * (S[i * N + j] + uh[i] * kt[i] * vt[j]);",
+     "a += gt[j] * (wt[i] * S[i * N + j] + uh[i] * kt[i] * vt[j]);"),
+    ("bwd_logit_grad_sign", "domega[i] = dw[i] * (-e * exp(-e));", "domega[i] = dw[i] * (e * exp(-e));"),
 ]
 
 
