@@ -62,6 +62,10 @@ BYTES = {
 }
 
 
+# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA per clock x 2 flops x 1.965 GHz
+SIMT_FP32_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 2)
+
+
 def load_peaks():
     p = os.path.join(HERE, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -325,7 +329,8 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
       * the Finch prefill with the time-mixing output stage (head LayerNorm, SiLU gate)
         fused into the chunked kernel's epilogue, against the same call without it;
       * the Finch prefill fed the decay logit omega_t (w_t = exp(-exp(omega_t)) formed in
-        the kernel), plain and with the fused output stage."""
+        the kernel), plain and with the fused output stage;
+      * the WKV-6 backward pass at the Finch shape."""
     hbm, _ = load_peaks()
     rows = {}
     f = wl.finch
@@ -358,6 +363,25 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
         "frac_hbm": round(nb / (omega * 1e-6) / 1e9 / hbm, 4),
         "separate_map_floor_us": round(2 * om.numel() * 2 / (hbm * 1e9) * 1e6, 2)}
     del om
+    # WKV-6 backward at the Finch shape (fp32 gradients; SIMT kernels)
+    gen.manual_seed(8)
+    dy = (torch.randn(8, 4096, 32, 64, device=dev, generator=gen)).to(torch.bfloat16)
+    dsT = torch.randn(8, 32, 64, 64, device=dev, generator=gen) * 0.1
+    ws = torch.empty(ops.wkv6_backward_workspace_bytes(8, 4096, 32), device=dev, dtype=torch.uint8)
+    bwd_ms = _time_us(torch, stream, dev, lambda: ops.wkv6_backward(
+        f["r"], f["k"], f["v"], f["w"], f["u"], dy, s0=f["s0"], dsT=dsT, workspace=ws), 3) / 1e3
+    n_el, n_st = dy.numel(), dsT.numel()
+    bwd_bytes = 5 * n_el * 2 + 4 * n_el * 4 + 3 * n_st * 4 + 2 * 32 * 64 * 4
+    bwd_flops = 2 * 6 * 64 * n_el  # six 64-term products per token and channel, 2 flops per FMA
+    alu_peak = SIMT_FP32_TFLOPS
+    rows["wkv6_finch_backward_B8_T4096_H32"] = {
+        "avg_ms": round(bwd_ms, 3), "algorithmic_bytes": bwd_bytes, "algorithmic_flops": bwd_flops,
+        "GBps": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
+        "TFLOPs": round(bwd_flops / (bwd_ms * 1e-3) / 1e12, 2),
+        "bound": "alu", "peak_tflops_fp32_simt": alu_peak,
+        "frac_alu": round(bwd_flops / (bwd_ms * 1e-3) / 1e12 / alu_peak, 4),
+        "workspace_bytes": ws.numel(), "launches_per_call": 4}
+    del dy, dsT, ws
     B, C = 2048, 4096
     x = inputs.wkv4_inputs(B, 1, C, "bf16", seed=5, wu_seed=6)
     w, u, k, v = (x[n].to(dev) for n in ("w", "u", "k", "v"))

@@ -41,6 +41,7 @@
 #ifndef RWKV_WKV_H
 #define RWKV_WKV_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -160,6 +161,54 @@ int rwkv_wkv6_forward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
                                  const uint16_t *omega, const float *u, const float *s0,
                                  const uint16_t *g, const float *ln_w, const float *ln_b, float eps,
                                  uint16_t *y, float *sT);
+
+/* WKV-6 backward pass, for training ([E412], [F422]; the gradients of the recurrence of
+ * rwkv_wkv6_forward by the chain rule, walked backwards in time).  Given the gradients of a
+ * loss L with respect to the forward's outputs,
+ *   dy  = dL/dy  [B, T, H, N] (dtype of r),   dsT = dL/dsT [B, H, N, N] fp32 (NULL = 0),
+ * it writes, all fp32:
+ *   dr, dk, dv, dw : [B, T, H, N]   dL/dr, dL/dk, dL/dv, dL/dw per token and channel
+ *                    (rwkv_wkv6_backward_omega_bf16: domega = dL/domega_t in place of dw);
+ *   du             : [H, N]         dL/du, summed over the batch rows in a fixed order
+ *                                   (deterministic);
+ *   ds0            : [B, H, N, N]   dL/ds0, or NULL = not written.  ds0 may be the very
+ *                                   same array as dsT (in place).
+ * With L_t = dL/d(state after token t), L_{T-1} = dsT and S = the state before token t:
+ *   dr_t[i] = sum_j dy_t[j] (S[i][j] + u[i] k_t[i] v_t[j])
+ *   dk_t[i] = sum_j L_t[i][j] v_t[j] + u[i] r_t[i] (dy_t . v_t)
+ *   dv_t[j] = sum_i L_t[i][j] k_t[i] + (sum_i r_t[i] u[i] k_t[i]) dy_t[j]
+ *   dw_t[i] = sum_j L_t[i][j] S[i][j]           domega_t[i] = -dw_t[i] exp(omega_t[i]) w_t[i]
+ *   du[i]   = sum_{b,t} r_t[i] k_t[i] (dy_t . v_t)
+ *   L_{t-1} = diag(w_t) L_t + r_t^T dy_t,       ds0 = L_{-1}.
+ * Inputs r, k, v, w (or omega), u, s0 are those of the forward call; the forward states
+ * are recomputed, not read.
+ *   workspace : device scratch owned by the caller, 16-byte aligned, of at least the size
+ *               rwkv_wkv6_backward_workspace_bytes reports (B*H*(ceil(T/8)*N*N + N)*4 bytes:
+ *               a checkpoint of the state every 8 tokens); it must not overlap any tensor.
+ *               A smaller workspace_bytes is refused with RWKV_ERR_ARG before any launch.
+ * Runs on CUDA cores in fp32 (four launches: a forward pass for dr, du and the
+ * checkpoints; a backward pass over state rows for dk, dw; one over state columns for
+ * dv, ds0; the sum of du over b).  N must be 64.  T = 0 writes du = 0 and ds0 = dsT.
+ * Aliasing: no output may overlap an input, the workspace or another output (except
+ * ds0 == dsT).  Other rules and errors as rwkv_wkv6_forward. */
+int rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, size_t *bytes);
+int rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N,
+                       const float *r, const float *k, const float *v, const float *w,
+                       const float *u, const float *s0, const float *dy, const float *dsT,
+                       float *dr, float *dk, float *dv, float *dw, float *du, float *ds0,
+                       void *workspace, size_t workspace_bytes);
+int rwkv_wkv6_backward_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
+                            const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                            const uint16_t *w, const float *u, const float *s0,
+                            const uint16_t *dy, const float *dsT,
+                            float *dr, float *dk, float *dv, float *dw, float *du, float *ds0,
+                            void *workspace, size_t workspace_bytes);
+int rwkv_wkv6_backward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
+                                  const uint16_t *r, const uint16_t *k, const uint16_t *v,
+                                  const uint16_t *omega, const float *u, const float *s0,
+                                  const uint16_t *dy, const float *dsT,
+                                  float *dr, float *dk, float *dv, float *domega, float *du,
+                                  float *ds0, void *workspace, size_t workspace_bytes);
 
 /* Kernel choice for WKV-6 on the calling thread: RWKV_WKV6_AUTO (default, as above),
  * RWKV_WKV6_SERIAL (always the serial kernel), RWKV_WKV6_CHUNKED (the chunked kernel

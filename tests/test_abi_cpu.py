@@ -132,6 +132,38 @@ def test_wkv6_omega_validation(lib):
         assert call(g=None, lw=None, lb=None, eps=-1.0) == -5
 
 
+def test_wkv6_backward_validation(lib):
+    """The backward's host checks: workspace size, nulls, alignment and aliasing."""
+    f = lib.rwkv_wkv6_backward_bf16
+    names = ["r", "k", "v", "w", "u", "s0", "dy", "dsT", "dr", "dk", "dv", "dw", "du", "ds0", "ws"]
+    B, T, H = 1, 20, 2
+    need = ops.wkv6_backward_workspace_bytes(B, T, H)
+    assert need == B * H * (3 * 64 * 64 + 64) * 4  # ceil(20 / 8) = 3 checkpoints per (b, h)
+    assert ops.wkv6_backward_workspace_bytes(B, 0, H) == 0
+    with pytest.raises(ops.WkvError):
+        ops.wkv6_backward_workspace_bytes(-1, T, H)
+
+    def call(wbytes=need, **kw):
+        a = {n: _p(i << 24) for i, n in enumerate(names)}
+        a.update(kw)
+        return f(B, T, H, 64, *[a[n] for n in names], ctypes.c_size_t(wbytes))
+
+    assert call(wbytes=need - 1) == -8            # workspace too small
+    assert call(ws=None) == -1                    # workspace missing
+    assert call(dy=None) == -1
+    assert call(dw=None) == -1
+    assert call(du=None) == -1
+    assert call(dr=_p((8 << 24) + 8)) == -7       # misaligned gradient
+    assert call(ws=_p((14 << 24) + 4)) == -7      # misaligned workspace
+    assert call(dk=_p(1 << 24)) == -4             # dk over k
+    assert call(ws=_p(8 << 24)) == -4             # workspace over dr
+    assert call(du=_p((9 << 24) + 64)) == -4      # du inside dk
+    assert call(ds0=_p(7 << 24)) != -4            # ds0 == dsT is allowed (in place)
+    assert call(ds0=_p((7 << 24) + 16)) == -4     # but not a partial overlap
+    assert f(B, T, H, 32, *[_p(i << 24) for i in range(15)], ctypes.c_size_t(need)) == -3
+    assert f(0, T, 0, 64, *([None] * 15), ctypes.c_size_t(0)) == 0  # nothing to produce
+
+
 def test_algo_selection(lib):
     assert lib.rwkv_set_wkv6_algo(7) == -8
     for a in (1, 2, 0):

@@ -192,6 +192,77 @@ int wkv6_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const 
     return RWKV_OK;
 }
 
+// ---- WKV-6 backward -----------------------------------------------------------------
+
+int wkv6_bwd_sizes(int64_t B, int64_t T, int64_t H, int64_t N, int64_t *n, int64_t *ns, int64_t *hn)
+{
+    if (B < 0 || T < 0 || H < 0 || N < 0) return fail(RWKV_ERR_SHAPE, "negative size%s");
+    int64_t BT, BTH, BH;
+    if (!mul_ok(B, T, &BT) || !mul_ok(BT, H, &BTH) || !mul_ok(BTH, N, n) || !mul_ok(B, H, &BH) ||
+        !mul_ok(BH, N * N, ns) || !mul_ok(H, N, hn))
+        return fail(RWKV_ERR_SHAPE, "size product overflows%s");
+    const int64_t nblk = (T + 7) / 8;
+    int64_t cells;
+    if (!mul_ok(BH, nblk * 4096 + 64, &cells)) return fail(RWKV_ERR_SHAPE, "workspace size overflows%s");
+    return RWKV_OK;
+}
+
+int wkv6_bwd_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k, const void *v,
+                   const void *w, const float *u, const float *s0, const void *dy, const float *dsT, float *dr,
+                   float *dk, float *dv, float *dw, float *du, float *ds0, void *workspace, size_t wbytes,
+                   bool bf16, bool omega)
+{
+    tl_err[0] = 0;
+    int64_t n, ns, hn;
+    int rc = wkv6_bwd_sizes(B, T, H, N, &n, &ns, &hn);
+    if (rc) return rc;
+    if (n == 0 && hn == 0 && !(ds0 && ns > 0)) return RWKV_OK;
+    if (N != 64) return fail(RWKV_ERR_UNSUPPORTED, "head size N must be 64%s");
+    if (n > 0 && (!r || !k || !v || !w || !dy))
+        return fail(RWKV_ERR_NULL, "r, k, v, w (or omega) and dy must be non-null%s");
+    if (n > 0 && (!dr || !dk || !dv || !dw)) return fail(RWKV_ERR_NULL, "dr, dk, dv and dw must be non-null%s");
+    if (hn > 0 && (!u || !du)) return fail(RWKV_ERR_NULL, "u and du must be non-null%s");
+    const size_t need = n > 0 ? wkv::wkv6_backward_workspace_bytes(B, T, H) : 0;
+    if (need > 0 && !workspace) return fail(RWKV_ERR_NULL, "workspace must be non-null%s");
+    if (wbytes < need) {
+        snprintf(tl_err, sizeof(tl_err), "workspace holds %zu bytes; this call needs %zu", wbytes, need);
+        return RWKV_ERR_ARG;
+    }
+    const void *ptrs[] = {r, k, v, w, u, s0, dy, dsT, dr, dk, dv, dw, du, ds0, workspace};
+    for (const void *p : ptrs)
+        if (p && !aligned16(p)) return fail(RWKV_ERR_ALIGN, "tensor pointers must be 16-byte aligned%s");
+    const int64_t esz = bf16 ? 2 : 4;
+    const Span ins[] = {{r, n * esz}, {k, n * esz}, {v, n * esz}, {w, n * esz}, {u, hn * 4}, {s0, ns * 4},
+                        {dy, n * esz}, {dsT, ns * 4}};
+    const Span outs[] = {{dr, n * 4}, {dk, n * 4}, {dv, n * 4}, {dw, n * 4}, {du, hn * 4},
+                         {ds0, ns * 4}, {workspace, static_cast<int64_t>(need)}};
+    const int n_outs = sizeof(outs) / sizeof(outs[0]);
+    for (int a = 0; a < n_outs; ++a) {
+        for (const Span &x : ins) {
+            // ds0 may be the very same array as dsT (in place); any other overlap is refused
+            if (outs[a].p == ds0 && x.p == dsT && ds0 == dsT) continue;
+            if (overlap(outs[a], x)) return fail(RWKV_ERR_ALIAS, "a gradient or the workspace overlaps an input%s");
+        }
+        for (int c = a + 1; c < n_outs; ++c)
+            if (overlap(outs[a], outs[c])) return fail(RWKV_ERR_ALIAS, "two outputs overlap%s");
+    }
+    int *status = nullptr;
+    rc = status_word(&status);
+    if (rc) return rc;
+    cudaError_t e = cudaSuccess;
+    if (n == 0) {  // no token: du = 0, ds0 = dsT (or 0)
+        if (hn > 0) e = cudaMemsetAsync(du, 0, hn * 4, tl_stream);
+        if (e == cudaSuccess && ds0 && ns > 0 && ds0 != dsT)
+            e = dsT ? cudaMemcpyAsync(ds0, dsT, ns * 4, cudaMemcpyDeviceToDevice, tl_stream)
+                    : cudaMemsetAsync(ds0, 0, ns * 4, tl_stream);
+        return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "wkv6 backward without tokens");
+    }
+    wkv::Wkv6BwdArgs a{B, T, H, N, r, k, v, w, u, s0, dy, dsT, dr, dk, dv, dw, du, ds0, workspace, bf16, omega};
+    e = wkv::wkv6_backward_launch(a, tl_stream);
+    if (e != cudaSuccess) return cuda_fail(e, "wkv6 backward launch");
+    return RWKV_OK;
+}
+
 // Allocation-free WKV-6 (bf16): same validation as wkv6_entry, chunked kernel only, the
 // split's scratch in the library's fixed device array.
 int wkv6_noalloc_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, const void *k,
@@ -319,6 +390,45 @@ int rwkv_wkv6_forward_bf16_noalloc(int64_t B, int64_t T, int64_t H, int64_t N, c
                                    int segments)
 {
     return wkv6_noalloc_entry(B, T, H, N, r, k, v, w, u, s0, y, sT, segments);
+}
+
+int rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, size_t *bytes)
+{
+    tl_err[0] = 0;
+    if (!bytes) return fail(RWKV_ERR_NULL, "bytes must be non-null%s");
+    int64_t n, ns, hn;
+    int rc = wkv6_bwd_sizes(B, T, H, N, &n, &ns, &hn);
+    if (rc) return rc;
+    *bytes = n > 0 ? wkv::wkv6_backward_workspace_bytes(B, T, H) : 0;
+    return RWKV_OK;
+}
+
+int rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N, const float *r, const float *k,
+                       const float *v, const float *w, const float *u, const float *s0, const float *dy,
+                       const float *dsT, float *dr, float *dk, float *dv, float *dw, float *du, float *ds0,
+                       void *workspace, size_t workspace_bytes)
+{
+    return wkv6_bwd_entry(B, T, H, N, r, k, v, w, u, s0, dy, dsT, dr, dk, dv, dw, du, ds0, workspace,
+                          workspace_bytes, false, false);
+}
+
+int rwkv_wkv6_backward_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r, const uint16_t *k,
+                            const uint16_t *v, const uint16_t *w, const float *u, const float *s0,
+                            const uint16_t *dy, const float *dsT, float *dr, float *dk, float *dv, float *dw,
+                            float *du, float *ds0, void *workspace, size_t workspace_bytes)
+{
+    return wkv6_bwd_entry(B, T, H, N, r, k, v, w, u, s0, dy, dsT, dr, dk, dv, dw, du, ds0, workspace,
+                          workspace_bytes, true, false);
+}
+
+int rwkv_wkv6_backward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N, const uint16_t *r,
+                                  const uint16_t *k, const uint16_t *v, const uint16_t *omega, const float *u,
+                                  const float *s0, const uint16_t *dy, const float *dsT, float *dr, float *dk,
+                                  float *dv, float *domega, float *du, float *ds0, void *workspace,
+                                  size_t workspace_bytes)
+{
+    return wkv6_bwd_entry(B, T, H, N, r, k, v, omega, u, s0, dy, dsT, dr, dk, dv, domega, du, ds0, workspace,
+                          workspace_bytes, true, true);
 }
 
 int rwkv_set_wkv6_algo(int algo)

@@ -49,6 +49,24 @@ struct Wkv6Args {
     bool omega = false;
 };
 
+// WKV-6 backward: gradients (fp32) of a loss with dL/dy = dy and dL/dsT = dsT (null = 0).
+struct Wkv6BwdArgs {
+    int64_t B, T, H, N;
+    const void *r, *k, *v, *w;  // [B,T,H,N] fp32 or bf16; w holds omega_t when omega is set
+    const float *u;             // [H,N]
+    const float *s0;            // [B,H,N,N] or null
+    const void *dy;             // [B,T,H,N], dtype of r
+    const float *dsT;           // [B,H,N,N] or null
+    float *dr, *dk, *dv, *dw;   // [B,T,H,N]; dw is domega when omega is set
+    float *du;                  // [H,N]
+    float *ds0;                 // [B,H,N,N] or null
+    void *workspace;            // wkv6_backward_workspace_bytes(B, T, H) bytes, 16-byte aligned
+    bool bf16, omega;
+};
+
+size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H);
+cudaError_t wkv6_backward_launch(const Wkv6BwdArgs &a, cudaStream_t s);
+
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
 

@@ -73,6 +73,13 @@ def load(path: str = LIB_PATH):
     lib.rwkv_wkv6_forward_gated_bf16.restype = ctypes.c_int
     lib.rwkv_wkv6_forward_omega_bf16.argtypes = wkv6[:10] + [_vp, _vp, _vp, ctypes.c_float] + wkv6[10:]
     lib.rwkv_wkv6_forward_omega_bf16.restype = ctypes.c_int
+    bwd = [_i64] * 4 + [_vp] * 14 + [_vp, ctypes.c_size_t]
+    for name in ("rwkv_wkv6_backward", "rwkv_wkv6_backward_bf16", "rwkv_wkv6_backward_omega_bf16"):
+        fn = getattr(lib, name)
+        fn.argtypes = bwd
+        fn.restype = ctypes.c_int
+    lib.rwkv_wkv6_backward_workspace_bytes.argtypes = [_i64] * 4 + [ctypes.POINTER(ctypes.c_size_t)]
+    lib.rwkv_wkv6_backward_workspace_bytes.restype = ctypes.c_int
     lib.rwkv_wkv6_forward_bf16_noalloc.restype = ctypes.c_int
     lib.rwkv_set_wkv6_segments.argtypes = [ctypes.c_int]
     lib.rwkv_set_wkv6_segments.restype = ctypes.c_int
@@ -256,6 +263,56 @@ def wkv6_forward_omega(r, k, v, omega, u, s0=None, g=None, ln_w=None, ln_b=None,
         if prev is not None:
             lib.rwkv_set_wkv6_algo(prev)
     return (y, sT) if want_state else y
+
+
+def wkv6_backward_workspace_bytes(B, T, H, N=64) -> int:
+    """Device scratch (bytes) that a WKV-6 backward call of this shape needs."""
+    lib = load()
+    out = ctypes.c_size_t(0)
+    _check(lib.rwkv_wkv6_backward_workspace_bytes(int(B), int(T), int(H), int(N), ctypes.byref(out)))
+    return int(out.value)
+
+
+def wkv6_backward(r, k, v, w, u, dy, s0=None, dsT=None, omega=False, want_ds0=True, workspace=None):
+    """WKV-6 backward: gradients of a loss with dL/dy = dy and dL/dsT = dsT (None = 0).
+
+    r,k,v,w,dy: [B,T,H,N] fp32|bf16 (with omega=True, w holds omega_t and bf16 is required);
+    u: [H,N] fp32; s0, dsT: [B,H,N,N] fp32.  Returns a dict of fp32 tensors dr, dk, dv,
+    dw (or domega), du, and ds0 (when want_ds0).  workspace: optional uint8 CUDA tensor of at
+    least wkv6_backward_workspace_bytes bytes; allocated here when not given.
+    """
+    lib = load()
+    _cuda(r, "r")
+    B, T, H, N = r.shape
+    dt = r.dtype
+    if dt not in (torch.float32, torch.bfloat16):
+        raise TypeError("r must be float32 or bfloat16")
+    if omega and dt != torch.bfloat16:
+        raise TypeError("the logit backward takes bf16 inputs")
+    for name, t in (("k", k), ("v", v), ("w", w), ("dy", dy)):
+        _cuda(t, name, dt, (B, T, H, N))
+    _cuda(u, "u", torch.float32, (H, N))
+    _cuda(s0, "s0", torch.float32, (B, H, N, N))
+    _cuda(dsT, "dsT", torch.float32, (B, H, N, N))
+    dev = r.device
+    out = {n: torch.empty(B, T, H, N, device=dev, dtype=torch.float32) for n in ("dr", "dk", "dv")}
+    dwn = "domega" if omega else "dw"
+    out[dwn] = torch.empty(B, T, H, N, device=dev, dtype=torch.float32)
+    out["du"] = torch.empty(H, N, device=dev, dtype=torch.float32)
+    out["ds0"] = torch.empty(B, H, N, N, device=dev, dtype=torch.float32) if want_ds0 else None
+    need = wkv6_backward_workspace_bytes(B, T, H, N)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), device=dev, dtype=torch.uint8)
+    _cuda(workspace, "workspace", torch.uint8)
+    _use_current_stream(lib, dev)
+    fn = (lib.rwkv_wkv6_backward_omega_bf16 if omega else
+          lib.rwkv_wkv6_backward_bf16 if dt == torch.bfloat16 else lib.rwkv_wkv6_backward)
+    _check(fn(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(dy), _ptr(dsT),
+              _ptr(out["dr"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out[dwn]), _ptr(out["du"]),
+              _ptr(out["ds0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel())))
+    if not want_ds0:
+        del out["ds0"]
+    return out
 
 
 def device_status() -> int:
