@@ -17,294 +17,421 @@
 // domega_t = dw_t * (-exp(omega_t) w_t).
 //
 // Each term is a dot product along one axis of a 64 x 64 matrix, so each kernel keeps the
-// matrix it walks in registers with that axis local to a thread pair:
-//   wkv6_bwd_forward_kernel  rows of S (thread pair per key channel i), forward in time:
-//                            dr, du, and a checkpoint of S every kBlock tokens;
+// matrix it walks in registers with that axis local to a group of TPR consecutive lanes:
+//   wkv6_bwd_forward_kernel  rows of S, forward in time: dr, du, and a checkpoint of S
+//                            every kBlock tokens;
 //   wkv6_bwd_rows_kernel     rows of L, backward in time: dk and dw.  dw needs the state
 //                            before every token: each block of kBlock tokens is recomputed
 //                            forward from its checkpoint into shared memory first;
-//   wkv6_bwd_cols_kernel     columns of L (thread pair per value channel j), backward in
-//                            time: dv and ds0;
+//   wkv6_bwd_cols_kernel     columns of L, backward in time: dv and ds0;
 //   wkv6_bwd_du_kernel       du summed over the batch rows (fixed order: deterministic).
-// One CTA of 128 threads per (b, h).  A thread pair shares one row (or column) and splits
-// its 64 entries into interleaved float4 groups (pair half p owns entries 8m + 4p .. +3), so
-// the pair's shared-memory reads of a broadcast vector fall in different banks.
+// Rows of S and of L evolve independently of one another (row i sees only w[i], k[i] or
+// r[i]), and so do the columns of L, so each (b, h) is split over several CTAs of 128
+// threads (TPR threads per row or column, 64 / TPR entries per thread).  Inputs reach
+// shared memory 32 tokens at a time by cp.async, a chunk ahead of their use.
 #include "wkv_internal.cuh"
 
 #include <algorithm>
+#include <mutex>
 
 namespace wkv {
 namespace {
 
 constexpr int kN = 64;
 constexpr int kThreads = 128;
-constexpr int kBlock = 8;  // tokens per checkpoint
-constexpr int kStashBytes = kBlock * kThreads * 32 * 4;  // states of one block, per CTA
-
-template <typename T> __device__ __forceinline__ float ldf(const T *p);
-template <> __device__ __forceinline__ float ldf<float>(const float *p) { return __ldg(p); }
-template <> __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16 *p)
-{
-    return __bfloat162float(*p);
-}
+constexpr int kBlock = 8;                 // tokens per checkpoint
 
 // Decay from its logit, w = exp(-exp(omega)), with the accurate exponential.
 __device__ __forceinline__ float decay(float x, bool omega) { return omega ? expf(-expf(x)) : x; }
 
-__device__ __forceinline__ float pair_sum(float x) { return x + __shfl_xor_sync(0xffffffffu, x, 1); }
+// sum over the TPR consecutive lanes that share a row (or column)
+template <int TPR> __device__ __forceinline__ float group_sum(float x)
+{
+#pragma unroll
+    for (int m = 1; m < TPR; m <<= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
 
-// index of the e-th entry of group m owned by pair half p
-__device__ __forceinline__ int col(int m, int p, int e) { return 8 * m + 4 * p + e; }
+// With TPR threads per row (or column), a thread owns E = 64 / TPR of its entries in float4
+// groups: group m holds entries 4 TPR m + 4p .. + 3 for part p = lane % TPR.  The TPR parts
+// of a row read a broadcast vector from disjoint bank groups.
+template <int TPR> __device__ __forceinline__ int ent(int p, int e) { return 4 * TPR * (e >> 2) + 4 * p + (e & 3); }
+
+// ------------------------------------------------------------------ staging in shared memory
+// Inputs reach the kernels through shared memory, kChunk tokens at a time, copied with
+// cp.async into the second of two buffers while the first is being used: every load is
+// issued a whole chunk before its data is needed.  U is the storage type (the bits of a
+// bf16 or an fp32 value); values are widened to fp32 when read.
+constexpr int kChunk = 32;
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void cp16(void *dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_one() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait_all() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
+
+template <typename T> struct Store;
+template <> struct Store<float> {
+    using type = float;
+};
+template <> struct Store<__nv_bfloat16> {
+    using type = unsigned short;
+};
+
+__device__ __forceinline__ float sm1(const float *p) { return *p; }
+__device__ __forceinline__ float sm1(const unsigned short *p) { return __uint_as_float(static_cast<uint32_t>(*p) << 16); }
+__device__ __forceinline__ float4 sm4(const float *p) { return *reinterpret_cast<const float4 *>(p); }
+__device__ __forceinline__ float4 sm4(const unsigned short *p)
+{
+    const uint2 x = *reinterpret_cast<const uint2 *>(p);
+    return make_float4(__uint_as_float(x.x << 16), __uint_as_float(x.x & 0xFFFF0000u), __uint_as_float(x.y << 16),
+                       __uint_as_float(x.y & 0xFFFF0000u));
+}
+// the thread's entries (see ent) of a 64-vector in shared memory
+template <int TPR, typename U, int E> __device__ __forceinline__ void smv(const U *vec, int p, float (&o)[E])
+{
+#pragma unroll
+    for (int m = 0; m < E / 4; ++m) {
+        const float4 a = sm4(vec + 4 * TPR * m + 4 * p);
+        o[4 * m] = a.x, o[4 * m + 1] = a.y, o[4 * m + 2] = a.z, o[4 * m + 3] = a.w;
+    }
+}
+
+// Copy cnt elements at element offset off of each token t0 .. t0 + nt - 1 (global layout
+// base + t stride) into dst[tt][cnt].  cnt * sizeof(U) is a multiple of 16 bytes and every
+// source address is 16-byte aligned (token rows are 64 elements apart, off a multiple of 16).
+template <typename U>
+__device__ __forceinline__ void stage(U *dst, const void *src, int64_t base, int64_t stride, int64_t t0, int nt,
+                                      int off, int cnt, int tid)
+{
+    constexpr int per = 16 / sizeof(U);
+    const int pieces = cnt / per;
+    const U *g = static_cast<const U *>(src);
+    for (int q = tid; q < nt * pieces; q += kThreads) {
+        const int tt = q / pieces, x = (q % pieces) * per;
+        cp16(dst + tt * cnt + x, g + base + (t0 + tt) * stride + off + x);
+    }
+}
+
+// a chunk of the row-walking kernels as copied: all 64 channels of v and dy, the CTA's rows
+// of r, k, w
+template <typename U, int R> struct RowStage {
+    U v[kChunk][kN], g[kChunk][kN];
+    U r[kChunk][R], k[kChunk][R], w[kChunk][R];
+};
+// a chunk of the column-walking kernel as copied: all 64 channels of r, k, w, the CTA's
+// columns of dy
+template <typename U, int R> struct ColStage {
+    U r[kChunk][kN], k[kChunk][kN], w[kChunk][kN];
+    U g[kChunk][R];
+};
+// the same in fp32, with bon[t] = sum_i r_t[i] u[i] k_t[i]
+template <int R> struct ColWork {
+    float r[kChunk][kN], k[kChunk][kN], w[kChunk][kN];
+    float g[kChunk][R];
+    float bon[kChunk];
+};
+
+template <typename U, int R>
+__device__ __forceinline__ void issue_rows(RowStage<U, R> &st, const void *r, const void *k, const void *v,
+                                           const void *w, const void *dy, int64_t base, int64_t stride, int64_t t0,
+                                           int nt, int rg, int tid)
+{
+    stage(&st.v[0][0], v, base, stride, t0, nt, 0, kN, tid);
+    stage(&st.g[0][0], dy, base, stride, t0, nt, 0, kN, tid);
+    stage(&st.r[0][0], r, base, stride, t0, nt, R * rg, R, tid);
+    stage(&st.k[0][0], k, base, stride, t0, nt, R * rg, R, tid);
+    stage(&st.w[0][0], w, base, stride, t0, nt, R * rg, R, tid);
+    cp_commit();
+}
+
+// widen cnt4 groups of 4 values (x 4 = nt * row length) from src into dst; with dec, form the
+// decay from its logit
+template <typename U>
+__device__ __forceinline__ void widen(float *dst, const U *src, int cnt4, int tid, bool dec)
+{
+    for (int q = tid; q < cnt4; q += kThreads) {
+        float4 x = sm4(src + 4 * q);
+        if (dec) x = make_float4(decay(x.x, true), decay(x.y, true), decay(x.z, true), decay(x.w, true));
+        *reinterpret_cast<float4 *>(dst + 4 * q) = x;
+    }
+}
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int m = 16; m >= 1; m >>= 1) x += __shfl_xor_sync(0xffffffffu, x, m);
+    return x;
+}
 
 // ------------------------------------------------------------------ forward: dr, du, checkpoints
-template <typename T>
+// CTA (n = b*H + h, row group rg): rows i = R rg .. R rg + R - 1 of S, TPR threads per row.
+// Rows of S evolve independently, so the row groups of one head run as separate CTAs.
+// Chunks are double-buffered: chunk c + 1 is copied while chunk c is walked.  Checkpoints
+// are written row-major (entry i*64 + j of a 64 x 64 block).
+template <typename T, int TPR>
 __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_forward_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                         const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                         const float *__restrict__ s0, const T *__restrict__ dy, float *__restrict__ dr,
                         float *__restrict__ ckpt, float *__restrict__ du_part, int omega)
 {
-    __shared__ __align__(16) float vs[2][kN], gs[2][kN];
+    using U = typename Store<T>::type;
+    constexpr int R = kThreads / TPR, E = kN / TPR;
+    extern __shared__ __align__(16) unsigned char smem[];
+    RowStage<U, R> *stg = reinterpret_cast<RowStage<U, R> *>(smem);  // [2]
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
-    const int tid = threadIdx.x, i = tid >> 1, p = tid & 1;
+    const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
+    const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
+    const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
     const float ui = u[h * kN + i];
-
-    float S[32];
-#pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) S[4 * m + e] = s0 ? s0[n * kN * kN + i * kN + col(m, p, e)] : 0.f;
-
     const int64_t stride = H * kN;
     const int64_t base = (b * Tlen * H + h) * kN;
-    float du_acc = 0.f;
-    for (int64_t t = 0; t < Tlen; ++t) {
-        const int buf = static_cast<int>(t & 1);
-        const int64_t o = base + t * stride;
-        if (tid < kN) vs[buf][tid] = ldf(v + o + tid);
-        else gs[buf][tid - kN] = ldf(dy + o + tid - kN);
-        const float ri = ldf(r + o + i), ki = ldf(k + o + i), wi = decay(ldf(w + o + i), omega);
-        if (t % kBlock == 0) {  // checkpoint: the state before this token, in register order
-            float4 *cp = reinterpret_cast<float4 *>(ckpt + (n * nblk + t / kBlock) * (kN * kN));
+
+    float S[E];
 #pragma unroll
-            for (int m = 0; m < 8; ++m)
-                cp[m * kThreads + tid] = make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+    for (int e = 0; e < E; ++e) S[e] = s0 ? s0[n * kN * kN + i * kN + ent<TPR>(p, e)] : 0.f;
+
+    float du_acc = 0.f;
+    issue_rows(stg[0], r, k, v, w, dy, base, stride, 0, static_cast<int>(std::min<int64_t>(kChunk, Tlen)), rg, tid);
+    for (int64_t c = 0; c < nchunks; ++c) {
+        const int64_t t0 = c * kChunk;
+        const int nt = static_cast<int>(std::min<int64_t>(kChunk, Tlen - t0));
+        if (c + 1 < nchunks) {
+            issue_rows(stg[(c + 1) & 1], r, k, v, w, dy, base, stride, t0 + kChunk,
+                       static_cast<int>(std::min<int64_t>(kChunk, Tlen - t0 - kChunk)), rg, tid);
+            cp_wait_one();
+        } else {
+            cp_wait_all();
         }
         __syncthreads();
-        float sd = 0.f, dot = 0.f;
+        const RowStage<U, R> &st = stg[c & 1];
+        for (int tt = 0; tt < nt; ++tt) {
+            const int64_t t = t0 + tt;
+            if (t % kBlock == 0) {  // checkpoint: the state before this token
+                float *cp = ckpt + (n * nblk + t / kBlock) * (kN * kN) + i * kN;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float4 g4 = *reinterpret_cast<const float4 *>(&gs[buf][col(m, p, 0)]);
-            const float4 v4 = *reinterpret_cast<const float4 *>(&vs[buf][col(m, p, 0)]);
-            sd = fmaf(S[4 * m], g4.x, sd);
-            sd = fmaf(S[4 * m + 1], g4.y, sd);
-            sd = fmaf(S[4 * m + 2], g4.z, sd);
-            sd = fmaf(S[4 * m + 3], g4.w, sd);
-            dot = fmaf(g4.x, v4.x, dot);
-            dot = fmaf(g4.y, v4.y, dot);
-            dot = fmaf(g4.z, v4.z, dot);
-            dot = fmaf(g4.w, v4.w, dot);
-            S[4 * m] = fmaf(wi, S[4 * m], ki * v4.x);
-            S[4 * m + 1] = fmaf(wi, S[4 * m + 1], ki * v4.y);
-            S[4 * m + 2] = fmaf(wi, S[4 * m + 2], ki * v4.z);
-            S[4 * m + 3] = fmaf(wi, S[4 * m + 3], ki * v4.w);
+                for (int m = 0; m < E / 4; ++m)
+                    *reinterpret_cast<float4 *>(cp + ent<TPR>(p, 4 * m)) =
+                        make_float4(S[4 * m], S[4 * m + 1], S[4 * m + 2], S[4 * m + 3]);
+            }
+            float xv[E], xg[E];
+            smv<TPR>(st.v[tt], p, xv);
+            smv<TPR>(st.g[tt], p, xg);
+            const float xr = sm1(&st.r[tt][il]), xk = sm1(&st.k[tt][il]);
+            const float xw = decay(sm1(&st.w[tt][il]), omega);
+            float sd = 0.f, dot = 0.f;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                sd = fmaf(S[e], xg[e], sd);
+                dot = fmaf(xg[e], xv[e], dot);
+                S[e] = fmaf(xw, S[e], xk * xv[e]);
+            }
+            sd = group_sum<TPR>(sd);
+            dot = group_sum<TPR>(dot);
+            if (p == 0) dr[base + t * stride + i] = fmaf(ui * xk, dot, sd);
+            du_acc = fmaf(xr * xk, dot, du_acc);
         }
-        sd = pair_sum(sd);
-        dot = pair_sum(dot);
-        if (p == 0) dr[o + i] = fmaf(ui * ki, dot, sd);
-        du_acc = fmaf(ri * ki, dot, du_acc);
+        __syncthreads();  // this buffer is refilled for chunk c + 2 next
     }
     if (p == 0) du_part[n * kN + i] = du_acc;
 }
 
 // ------------------------------------------------------------------ backward, rows: dk, dw
-template <typename T>
+// Same CTA and thread layout as the forward kernel; chunks (double-buffered) and the tokens
+// in them are walked last to first.  For each block of kBlock tokens, the states before
+// its tokens are first recomputed from the block's checkpoint into a per-thread
+// shared-memory stash.
+template <typename T, int TPR>
 __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                      const T *__restrict__ dy, const float *__restrict__ dsT, const float *__restrict__ ckpt,
                      float *__restrict__ dk, float *__restrict__ dw, int omega)
 {
+    using U = typename Store<T>::type;
+    constexpr int R = kThreads / TPR, E = kN / TPR, G = E / 4;
     extern __shared__ __align__(16) unsigned char smem[];
-    float4 *stash = reinterpret_cast<float4 *>(smem);                                // [kBlock][8][kThreads]
-    float *vs = reinterpret_cast<float *>(smem + kStashBytes);                       // [kBlock][kN]
-    float *gs = vs + kBlock * kN;                                                    // [kBlock][kN]
+    RowStage<U, R> *stg = reinterpret_cast<RowStage<U, R> *>(smem);  // [2]
+    float4(*stash)[G][kThreads] = reinterpret_cast<float4(*)[G][kThreads]>(smem + 2 * sizeof(RowStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
-    const int tid = threadIdx.x, i = tid >> 1, p = tid & 1;
+    const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
+    const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
+    const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
     const float ui = u[h * kN + i];
     const int64_t stride = H * kN;
     const int64_t base = (b * Tlen * H + h) * kN;
 
-    float L[32];
+    float L[E];
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) L[4 * m + e] = dsT ? dsT[n * kN * kN + i * kN + col(m, p, e)] : 0.f;
+    for (int e = 0; e < E; ++e) L[e] = dsT ? dsT[n * kN * kN + i * kN + ent<TPR>(p, e)] : 0.f;
 
-    for (int64_t c = nblk - 1; c >= 0; --c) {
-        const int64_t t0 = c * kBlock;
-        const int tv = static_cast<int>(std::min<int64_t>(kBlock, Tlen - t0));
-        __syncthreads();  // the previous block's v, do are no longer read
-        for (int q = tid; q < 2 * kBlock * kN; q += kThreads) {
-            const int tt = q / (2 * kN), x = q % (2 * kN);
-            float val = 0.f;
-            if (tt < tv) {
-                const int64_t o = base + (t0 + tt) * stride;
-                val = x < kN ? ldf(v + o + x) : ldf(dy + o + x - kN);
+    // this thread's part of a block's checkpoint, loaded one block ahead
+    float4 nx[G];
+    auto ck = [&](int64_t cb) {
+        const float *cp = ckpt + (n * nblk + cb) * (kN * kN) + i * kN;
+#pragma unroll
+        for (int m = 0; m < G; ++m) nx[m] = *reinterpret_cast<const float4 *>(cp + ent<TPR>(p, 4 * m));
+    };
+    ck(nblk - 1);
+    {
+        const int64_t t0 = (nchunks - 1) * kChunk;
+        issue_rows(stg[(nchunks - 1) & 1], r, k, v, w, dy, base, stride, t0, static_cast<int>(Tlen - t0), rg, tid);
+    }
+    for (int64_t c = nchunks - 1; c >= 0; --c) {
+        const int64_t t0 = c * kChunk;
+        const int nt = static_cast<int>(std::min<int64_t>(kChunk, Tlen - t0));
+        if (c > 0) {
+            issue_rows(stg[(c - 1) & 1], r, k, v, w, dy, base, stride, t0 - kChunk, kChunk, rg, tid);
+            cp_wait_one();
+        } else {
+            cp_wait_all();
+        }
+        __syncthreads();
+        const RowStage<U, R> &st = stg[c & 1];
+        for (int blk = (nt - 1) / kBlock; blk >= 0; --blk) {
+            const int64_t cb = t0 / kBlock + blk;  // global block index
+            const int tb = kBlock * blk;           // first token of the block within the chunk
+            const int tv = nt - tb < kBlock ? nt - tb : kBlock;
+            float sv[E];
+#pragma unroll
+            for (int m = 0; m < G; ++m) {
+                sv[4 * m] = nx[m].x, sv[4 * m + 1] = nx[m].y, sv[4 * m + 2] = nx[m].z, sv[4 * m + 3] = nx[m].w;
             }
-            (x < kN ? vs : gs)[tt * kN + (x % kN)] = val;
-        }
-        float rr[kBlock], kk[kBlock], ww[kBlock], om[kBlock];
+            if (cb > 0) ck(cb - 1);
 #pragma unroll
-        for (int m = 0; m < kBlock; ++m) {
-            rr[m] = kk[m] = om[m] = 0.f;
-            ww[m] = 1.f;
-            if (m < tv) {
-                const int64_t o = base + (t0 + m) * stride + i;
-                rr[m] = ldf(r + o);
-                kk[m] = ldf(k + o);
-                om[m] = ldf(w + o);
-                ww[m] = decay(om[m], omega);
+            for (int tt = 0; tt < kBlock; ++tt) {
+                if (tt < tv) {
+#pragma unroll
+                    for (int m = 0; m < G; ++m)
+                        stash[tt][m][tid] = make_float4(sv[4 * m], sv[4 * m + 1], sv[4 * m + 2], sv[4 * m + 3]);
+                    if (tt + 1 < tv) {
+                        float xv[E];
+                        smv<TPR>(st.v[tb + tt], p, xv);
+                        const float xk = sm1(&st.k[tb + tt][il]);
+                        const float xw = decay(sm1(&st.w[tb + tt][il]), omega);
+#pragma unroll
+                        for (int e = 0; e < E; ++e) sv[e] = fmaf(xw, sv[e], xk * xv[e]);
+                    }
+                }
             }
-        }
-        // the states before each token of the block, from the checkpoint (own entries only)
-        const float4 *cp = reinterpret_cast<const float4 *>(ckpt + (n * nblk + c) * (kN * kN));
-        float s[32];
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float4 x = cp[m * kThreads + tid];
-            s[4 * m] = x.x;
-            s[4 * m + 1] = x.y;
-            s[4 * m + 2] = x.z;
-            s[4 * m + 3] = x.w;
-        }
-        __syncthreads();  // v, do of the block in shared memory
+            for (int tt = kBlock - 1; tt >= 0; --tt) {
+                if (tt < tv) {
+                    float sp[E], xv[E], xg[E];
 #pragma unroll
-        for (int tt = 0; tt < kBlock; ++tt) {
-            if (tt < tv) {
+                    for (int m = 0; m < G; ++m) {
+                        const float4 a = stash[tt][m][tid];
+                        sp[4 * m] = a.x, sp[4 * m + 1] = a.y, sp[4 * m + 2] = a.z, sp[4 * m + 3] = a.w;
+                    }
+                    smv<TPR>(st.v[tb + tt], p, xv);
+                    smv<TPR>(st.g[tb + tt], p, xg);
+                    const float xr = sm1(&st.r[tb + tt][il]), om = sm1(&st.w[tb + tt][il]);
+                    const float xw = decay(om, omega);
+                    float dwp = 0.f, dkp = 0.f, dot = 0.f;
 #pragma unroll
-                for (int m = 0; m < 8; ++m)
-                    stash[(tt * 8 + m) * kThreads + tid] =
-                        make_float4(s[4 * m], s[4 * m + 1], s[4 * m + 2], s[4 * m + 3]);
-                if (tt + 1 < tv) {
-#pragma unroll
-                    for (int m = 0; m < 8; ++m) {
-                        const float4 v4 = *reinterpret_cast<const float4 *>(&vs[tt * kN + col(m, p, 0)]);
-                        s[4 * m] = fmaf(ww[tt], s[4 * m], kk[tt] * v4.x);
-                        s[4 * m + 1] = fmaf(ww[tt], s[4 * m + 1], kk[tt] * v4.y);
-                        s[4 * m + 2] = fmaf(ww[tt], s[4 * m + 2], kk[tt] * v4.z);
-                        s[4 * m + 3] = fmaf(ww[tt], s[4 * m + 3], kk[tt] * v4.w);
+                    for (int e = 0; e < E; ++e) {
+                        dwp = fmaf(L[e], sp[e], dwp);
+                        dkp = fmaf(L[e], xv[e], dkp);
+                        dot = fmaf(xg[e], xv[e], dot);
+                        L[e] = fmaf(xw, L[e], xr * xg[e]);
+                    }
+                    dwp = group_sum<TPR>(dwp);
+                    dkp = group_sum<TPR>(dkp);
+                    dot = group_sum<TPR>(dot);
+                    if (p == 0) {
+                        const int64_t o = base + (t0 + tb + tt) * stride + i;
+                        dk[o] = fmaf(ui * xr, dot, dkp);
+                        // with the logit: dw/domega = -exp(omega) w
+                        dw[o] = omega ? dwp * (-expf(om) * xw) : dwp;
                     }
                 }
             }
         }
-#pragma unroll
-        for (int tt = kBlock - 1; tt >= 0; --tt) {
-            if (tt < tv) {
-                float dwp = 0.f, dkp = 0.f, dot = 0.f;
-#pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const float4 s4 = stash[(tt * 8 + m) * kThreads + tid];
-                    const float4 v4 = *reinterpret_cast<const float4 *>(&vs[tt * kN + col(m, p, 0)]);
-                    const float4 g4 = *reinterpret_cast<const float4 *>(&gs[tt * kN + col(m, p, 0)]);
-                    dwp = fmaf(L[4 * m], s4.x, dwp);
-                    dwp = fmaf(L[4 * m + 1], s4.y, dwp);
-                    dwp = fmaf(L[4 * m + 2], s4.z, dwp);
-                    dwp = fmaf(L[4 * m + 3], s4.w, dwp);
-                    dkp = fmaf(L[4 * m], v4.x, dkp);
-                    dkp = fmaf(L[4 * m + 1], v4.y, dkp);
-                    dkp = fmaf(L[4 * m + 2], v4.z, dkp);
-                    dkp = fmaf(L[4 * m + 3], v4.w, dkp);
-                    dot = fmaf(g4.x, v4.x, dot);
-                    dot = fmaf(g4.y, v4.y, dot);
-                    dot = fmaf(g4.z, v4.z, dot);
-                    dot = fmaf(g4.w, v4.w, dot);
-                    L[4 * m] = fmaf(ww[tt], L[4 * m], rr[tt] * g4.x);
-                    L[4 * m + 1] = fmaf(ww[tt], L[4 * m + 1], rr[tt] * g4.y);
-                    L[4 * m + 2] = fmaf(ww[tt], L[4 * m + 2], rr[tt] * g4.z);
-                    L[4 * m + 3] = fmaf(ww[tt], L[4 * m + 3], rr[tt] * g4.w);
-                }
-                dwp = pair_sum(dwp);
-                dkp = pair_sum(dkp);
-                dot = pair_sum(dot);
-                if (p == 0) {
-                    const int64_t o = base + (t0 + tt) * stride + i;
-                    dk[o] = fmaf(ui * rr[tt], dot, dkp);
-                    // with the logit: dw/domega = -exp(omega) w
-                    dw[o] = omega ? dwp * (-expf(om[tt]) * ww[tt]) : dwp;
-                }
-            }
-        }
+        __syncthreads();  // this buffer is refilled for chunk c - 2 next
     }
 }
 
 // ------------------------------------------------------------------ backward, columns: dv, ds0
-template <typename T>
+// CTA (n, column group cg): columns j = R cg .. + R - 1 of the state gradient, TPR threads
+// per column, each holding E of its rows (columns evolve independently).
+template <typename T, int TPR>
 __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ w, const float *__restrict__ u, const T *__restrict__ dy,
                      const float *__restrict__ dsT, float *__restrict__ dv, float *__restrict__ ds0, int omega)
 {
-    __shared__ __align__(16) float rs[2][kN], ks[2][kN], ws[2][kN], rus[2][kN];
-    __shared__ __align__(16) float us[kN];
+    using U = typename Store<T>::type;
+    constexpr int R = kThreads / TPR, E = kN / TPR;
+    extern __shared__ __align__(16) unsigned char smem[];
+    ColStage<U, R> &st = *reinterpret_cast<ColStage<U, R> *>(smem);
+    ColWork<R> &wk = *reinterpret_cast<ColWork<R> *>(smem + sizeof(ColStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
-    const int tid = threadIdx.x, j = tid >> 1, p = tid & 1;
-    if (tid < kN) us[tid] = u[h * kN + tid];
+    const int cg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, jl = tid / TPR;
+    const int j = R * cg + jl;
+    const int warp = tid / 32, lane = tid % 32;
+    const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
     const int64_t stride = H * kN;
     const int64_t base = (b * Tlen * H + h) * kN;
-
-    // L[i][j] for this thread's rows i = col(m, p, e)
-    float L[32];
+    float L[E];
 #pragma unroll
-    for (int m = 0; m < 8; ++m)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) L[4 * m + e] = dsT ? dsT[n * kN * kN + col(m, p, e) * kN + j] : 0.f;
-    __syncthreads();
-
-    for (int64_t t = Tlen - 1; t >= 0; --t) {
-        const int buf = static_cast<int>(t & 1);
-        const int64_t o = base + t * stride;
-        if (tid < kN) {
-            const float rv = ldf(r + o + tid);
-            rs[buf][tid] = rv;
-            rus[buf][tid] = rv * us[tid];
-            ws[buf][tid] = decay(ldf(w + o + tid), omega);
-        } else {
-            ks[buf][tid - kN] = ldf(k + o + tid - kN);
+    for (int e = 0; e < E; ++e) L[e] = dsT ? dsT[n * kN * kN + ent<TPR>(p, e) * kN + j] : 0.f;
+    const float u0 = u[h * kN + 2 * lane], u1 = u[h * kN + 2 * lane + 1];
+    auto issue = [&](int64_t t0, int nt) {
+        stage(&st.r[0][0], r, base, stride, t0, nt, 0, kN, tid);
+        stage(&st.k[0][0], k, base, stride, t0, nt, 0, kN, tid);
+        stage(&st.w[0][0], w, base, stride, t0, nt, 0, kN, tid);
+        stage(&st.g[0][0], dy, base, stride, t0, nt, R * cg, R, tid);
+        cp_commit();
+    };
+    {
+        const int64_t t0 = (nchunks - 1) * kChunk;
+        issue(t0, static_cast<int>(Tlen - t0));
+    }
+    for (int64_t c = nchunks - 1; c >= 0; --c) {
+        const int64_t t0 = c * kChunk;
+        const int nt = static_cast<int>(std::min<int64_t>(kChunk, Tlen - t0));
+        cp_wait_all();
+        __syncthreads();  // chunk c copied; the previous chunk's working copy no longer read
+        widen(&wk.r[0][0], &st.r[0][0], nt * kN / 4, tid, false);
+        widen(&wk.k[0][0], &st.k[0][0], nt * kN / 4, tid, false);
+        widen(&wk.w[0][0], &st.w[0][0], nt * kN / 4, tid, omega != 0);
+        widen(&wk.g[0][0], &st.g[0][0], nt * R / 4, tid, false);
+        for (int tt = warp; tt < nt; tt += kThreads / 32) {
+            const float q = sm1(&st.r[tt][2 * lane]) * u0 * sm1(&st.k[tt][2 * lane]) +
+                            sm1(&st.r[tt][2 * lane + 1]) * u1 * sm1(&st.k[tt][2 * lane + 1]);
+            const float sum = warp_sum(q);
+            if (lane == 0) wk.bon[tt] = sum;
         }
-        const float gj = ldf(dy + o + j);
-        __syncthreads();
-        float dvp = 0.f, bon = 0.f;
+        __syncthreads();  // working copy ready; the copy buffer is free
+        if (c > 0) issue(t0 - kChunk, kChunk);
+        for (int tt = nt - 1; tt >= 0; --tt) {
+            float xr[E], xk[E], xw[E];
+            smv<TPR>(wk.r[tt], p, xr);
+            smv<TPR>(wk.k[tt], p, xk);
+            smv<TPR>(wk.w[tt], p, xw);
+            const float xg = wk.g[tt][jl];
+            float dvp = 0.f;
 #pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const float4 k4 = *reinterpret_cast<const float4 *>(&ks[buf][col(m, p, 0)]);
-            const float4 r4 = *reinterpret_cast<const float4 *>(&rs[buf][col(m, p, 0)]);
-            const float4 w4 = *reinterpret_cast<const float4 *>(&ws[buf][col(m, p, 0)]);
-            const float4 q4 = *reinterpret_cast<const float4 *>(&rus[buf][col(m, p, 0)]);
-            dvp = fmaf(L[4 * m], k4.x, dvp);
-            dvp = fmaf(L[4 * m + 1], k4.y, dvp);
-            dvp = fmaf(L[4 * m + 2], k4.z, dvp);
-            dvp = fmaf(L[4 * m + 3], k4.w, dvp);
-            bon = fmaf(q4.x, k4.x, bon);
-            bon = fmaf(q4.y, k4.y, bon);
-            bon = fmaf(q4.z, k4.z, bon);
-            bon = fmaf(q4.w, k4.w, bon);
-            L[4 * m] = fmaf(w4.x, L[4 * m], r4.x * gj);
-            L[4 * m + 1] = fmaf(w4.y, L[4 * m + 1], r4.y * gj);
-            L[4 * m + 2] = fmaf(w4.z, L[4 * m + 2], r4.z * gj);
-            L[4 * m + 3] = fmaf(w4.w, L[4 * m + 3], r4.w * gj);
+            for (int e = 0; e < E; ++e) {
+                dvp = fmaf(L[e], xk[e], dvp);
+                L[e] = fmaf(xw[e], L[e], xr[e] * xg);
+            }
+            dvp = group_sum<TPR>(dvp);
+            if (p == 0) dv[base + (t0 + tt) * stride + j] = fmaf(wk.bon[tt], xg, dvp);
         }
-        dvp = pair_sum(dvp);
-        bon = pair_sum(bon);
-        if (p == 0) dv[o + j] = fmaf(bon, gj, dvp);
     }
     if (ds0) {
 #pragma unroll
-        for (int m = 0; m < 8; ++m)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) ds0[n * kN * kN + col(m, p, e) * kN + j] = L[4 * m + e];
+        for (int e = 0; e < E; ++e) ds0[n * kN * kN + ent<TPR>(p, e) * kN + j] = L[e];
     }
 }
 
@@ -319,45 +446,75 @@ __global__ void __launch_bounds__(kN) wkv6_bwd_du_kernel(int64_t B, int64_t H, c
     du[h * kN + i] = acc;
 }
 
-cudaError_t configure_rows()
+// threads per row (column) of each kernel: the row walk backwards keeps a stash of kBlock
+// states per row in shared memory, so it spreads a row over more threads
+constexpr int kFwdTPR = 4, kRowsTPR = 8, kColsTPR = 4;
+
+template <typename T> constexpr int fwd_smem()
 {
-    static bool done[64] = {};
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (done[dev]) return cudaSuccess;
-    const int bytes = kStashBytes + 2 * kBlock * kN * 4;
-    e = cudaFuncSetAttribute(wkv6_bwd_rows_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(wkv6_bwd_rows_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             bytes);
-    if (e != cudaSuccess) return e;
-    done[dev] = true;
-    return cudaSuccess;
+    return 2 * static_cast<int>(sizeof(RowStage<typename Store<T>::type, kThreads / kFwdTPR>));
+}
+template <typename T> constexpr int rows_smem()
+{
+    return 2 * static_cast<int>(sizeof(RowStage<typename Store<T>::type, kThreads / kRowsTPR>)) +
+           kBlock * kThreads * (kN / kRowsTPR) * 4;
+}
+template <typename T> constexpr int cols_smem()
+{
+    constexpr int R = kThreads / kColsTPR;
+    return static_cast<int>(sizeof(ColStage<typename Store<T>::type, R>) + sizeof(ColWork<R>));
+}
+
+template <typename T> cudaError_t configure()
+{
+    cudaError_t e = cudaFuncSetAttribute(wkv6_bwd_forward_kernel<T, kFwdTPR>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, fwd_smem<T>());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(wkv6_bwd_rows_kernel<T, kRowsTPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 rows_smem<T>());
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(wkv6_bwd_cols_kernel<T, kColsTPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 cols_smem<T>());
+    return e;
 }
 
 template <typename T>
 cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
 {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!done[dev]) {
+            e = configure<T>();
+            if (e != cudaSuccess) return e;
+            done[dev] = true;
+        }
+    }
     const int64_t bh = a.B * a.H;
     const int64_t nblk = (a.T + kBlock - 1) / kBlock;
     float *ckpt = static_cast<float *>(a.workspace);
     float *du_part = ckpt + bh * nblk * kN * kN;
     const int om = a.omega ? 1 : 0;
-    const unsigned grid = static_cast<unsigned>(bh);
+    const unsigned nbh = static_cast<unsigned>(bh);
     const T *r = static_cast<const T *>(a.r), *k = static_cast<const T *>(a.k);
     const T *v = static_cast<const T *>(a.v), *w = static_cast<const T *>(a.w);
     const T *dy = static_cast<const T *>(a.dy);
-    wkv6_bwd_forward_kernel<T><<<grid, kThreads, 0, s>>>(a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt,
-                                                         du_part, om);
-    cudaError_t e = cudaGetLastError();
+    // grid: (b, h) x the row (column) groups of a head, kN / (kThreads / TPR) = TPR / 2 of them
+    wkv6_bwd_forward_kernel<T, kFwdTPR><<<dim3(nbh, kFwdTPR / 2), kThreads, fwd_smem<T>(), s>>>(
+        a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om);
+    e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_rows_kernel<T><<<grid, kThreads, kStashBytes + 2 * kBlock * kN * 4, s>>>(
+    wkv6_bwd_rows_kernel<T, kRowsTPR><<<dim3(nbh, kRowsTPR / 2), kThreads, rows_smem<T>(), s>>>(
         a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_cols_kernel<T><<<grid, kThreads, 0, s>>>(a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om);
+    wkv6_bwd_cols_kernel<T, kColsTPR><<<dim3(nbh, kColsTPR / 2), kThreads, cols_smem<T>(), s>>>(
+        a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_du_kernel<<<static_cast<unsigned>(a.H), kN, 0, s>>>(a.B, a.H, du_part, a.du);
@@ -376,8 +533,6 @@ cudaError_t wkv6_backward_launch(const Wkv6BwdArgs &a, cudaStream_t s)
 {
     if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
     if (a.B * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    cudaError_t e = configure_rows();
-    if (e != cudaSuccess) return e;
     return a.bf16 ? launch_all<__nv_bfloat16>(a, s) : launch_all<float>(a, s);
 }
 

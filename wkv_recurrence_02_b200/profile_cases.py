@@ -14,6 +14,9 @@ Every case first makes one untimed call (so a profiler can skip it with ``-s``),
   wkv4_decode   RWKV-4 T=1 decode, B2048 C4096 bf16, (a, b, p) state updated in place
   finch_gated   the finch case through rwkv_wkv6_forward_gated_bf16 (head LayerNorm and
                 SiLU gate fused into the epilogue)
+  finch_backward  the WKV-6 backward pass at the finch shape (B8 T4096 H32 bf16 inputs,
+                fp32 gradients, random s0 and dsT): four launches per call
+  small_backward  the same at B8 T1024 H32 (for ncu captures)
 
 Inputs come from the seeded generators in ``inputs``; nothing here checks results.
 """
@@ -23,7 +26,7 @@ import torch
 
 from . import inputs, ops
 
-CASES = ("wkv4", "finch", "long", "decode", "wkv4_decode", "finch_gated")
+CASES = ("wkv4", "finch", "long", "decode", "wkv4_decode", "finch_gated", "finch_backward", "small_backward")
 
 
 def _wkv4(reps):
@@ -56,6 +59,19 @@ def _wkv6_gated(B, T, H, reps):
         ops.wkv6_forward_gated(*a, g, lw, lb, eps=1e-5, s0=s0, y=y, sT=sT)
 
 
+def _wkv6_backward(B, T, H, reps):
+    x = inputs.wkv6_inputs(B, T, H, 64, "bf16", seed=0, s0_std=0.1)
+    a = [x[n].cuda() for n in ("r", "k", "v", "w", "u")]
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    dy = torch.randn(B, T, H, 64, device="cuda", generator=g).to(torch.bfloat16)
+    dsT = torch.randn(B, H, 64, 64, device="cuda", generator=g) * 0.1
+    s0 = x["s0"].cuda()
+    ws = torch.empty(ops.wkv6_backward_workspace_bytes(B, T, H), device="cuda", dtype=torch.uint8)
+    for _ in range(1 + reps):
+        ops.wkv6_backward(*a, dy, s0=s0, dsT=dsT, workspace=ws)
+
+
 def _wkv6(B, T, H, reps, s0_std=0.1):
     x = inputs.wkv6_inputs(B, T, H, 64, "bf16", seed=0, s0_std=s0_std)
     a = [x[n].cuda() for n in ("r", "k", "v", "w", "u")]
@@ -79,6 +95,10 @@ def run(case, reps=1):
         _wkv4_decode(reps)
     elif case == "finch_gated":
         _wkv6_gated(8, 1024, 32, reps)
+    elif case == "finch_backward":
+        _wkv6_backward(8, 4096, 32, reps)
+    elif case == "small_backward":
+        _wkv6_backward(8, 1024, 32, reps)
     else:
         raise ValueError(f"unknown case {case!r}; choose from {CASES}")
 
