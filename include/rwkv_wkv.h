@@ -34,9 +34,11 @@
  *    call failed; rwkv_last_error() has the text.  Faults inside a kernel that the
  *    kernel itself detects (e.g. a bounded wait that ran out) are reported through the
  *    device status word, read with rwkv_get_device_status().
- *  - The library keeps no device memory of its own beyond its status word (a statically
- *    allocated __device__ variable).  The only per-call allocation is the stream-ordered
- *    scratch of a split chunked WKV-6 call (see rwkv_set_wkv6_segments).
+ *  - The library keeps no device memory of its own beyond its status word and the fixed
+ *    scratch array of rwkv_wkv6_forward_bf16_noalloc (statically allocated __device__
+ *    variables).  The only per-call allocation is the stream-ordered scratch of a split
+ *    chunked WKV-6 call (see rwkv_set_wkv6_segments); the backward pass takes its
+ *    workspace from the caller.
  */
 #ifndef RWKV_WKV_H
 #define RWKV_WKV_H
