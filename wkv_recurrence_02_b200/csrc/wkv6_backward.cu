@@ -361,29 +361,33 @@ wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
 }
 
 // ------------------------------------------------------------------ backward, columns: dv, ds0
-// CTA (n, column group cg): columns j = R cg .. + R - 1 of the state gradient, TPR threads
-// per column, each holding E of its rows (columns evolve independently).
-template <typename T, int TPR>
+// CTA (n, column group cg): R = CPT kThreads / TPR columns of the state gradient.  TPR
+// threads share a column and each holds E of its rows; a thread serves CPT columns
+// (jl + m kThreads / TPR), so every r, k, w value it reads from shared memory feeds CPT
+// columns (columns evolve independently).
+template <typename T, int TPR, int CPT>
 __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ w, const float *__restrict__ u, const T *__restrict__ dy,
                      const float *__restrict__ dsT, float *__restrict__ dv, float *__restrict__ ds0, int omega)
 {
     using U = typename Store<T>::type;
-    constexpr int R = kThreads / TPR, E = kN / TPR;
+    constexpr int S = kThreads / TPR, R = S * CPT, E = kN / TPR;
     extern __shared__ __align__(16) unsigned char smem[];
     ColStage<U, R> &st = *reinterpret_cast<ColStage<U, R> *>(smem);
     ColWork<R> &wk = *reinterpret_cast<ColWork<R> *>(smem + sizeof(ColStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
     const int cg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, jl = tid / TPR;
-    const int j = R * cg + jl;
     const int warp = tid / 32, lane = tid % 32;
     const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
     const int64_t stride = H * kN;
     const int64_t base = (b * Tlen * H + h) * kN;
-    float L[E];
+    float L[CPT][E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) L[e] = dsT ? dsT[n * kN * kN + ent<TPR>(p, e) * kN + j] : 0.f;
+    for (int c = 0; c < CPT; ++c)
+#pragma unroll
+        for (int e = 0; e < E; ++e)
+            L[c][e] = dsT ? dsT[n * kN * kN + ent<TPR>(p, e) * kN + R * cg + jl + S * c] : 0.f;
     const float u0 = u[h * kN + 2 * lane], u1 = u[h * kN + 2 * lane + 1];
     auto issue = [&](int64_t t0, int nt) {
         stage(&st.r[0][0], r, base, stride, t0, nt, 0, kN, tid);
@@ -396,11 +400,11 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
         const int64_t t0 = (nchunks - 1) * kChunk;
         issue(t0, static_cast<int>(Tlen - t0));
     }
-    for (int64_t c = nchunks - 1; c >= 0; --c) {
-        const int64_t t0 = c * kChunk;
+    for (int64_t ch = nchunks - 1; ch >= 0; --ch) {
+        const int64_t t0 = ch * kChunk;
         const int nt = static_cast<int>(std::min<int64_t>(kChunk, Tlen - t0));
         cp_wait_all();
-        __syncthreads();  // chunk c copied; the previous chunk's working copy no longer read
+        __syncthreads();  // chunk ch copied; the previous chunk's working copy no longer read
         widen(&wk.r[0][0], &st.r[0][0], nt * kN / 4, tid, false);
         widen(&wk.k[0][0], &st.k[0][0], nt * kN / 4, tid, false);
         widen(&wk.w[0][0], &st.w[0][0], nt * kN / 4, tid, omega != 0);
@@ -412,26 +416,31 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
             if (lane == 0) wk.bon[tt] = sum;
         }
         __syncthreads();  // working copy ready; the copy buffer is free
-        if (c > 0) issue(t0 - kChunk, kChunk);
+        if (ch > 0) issue(t0 - kChunk, kChunk);
         for (int tt = nt - 1; tt >= 0; --tt) {
             float xr[E], xk[E], xw[E];
             smv<TPR>(wk.r[tt], p, xr);
             smv<TPR>(wk.k[tt], p, xk);
             smv<TPR>(wk.w[tt], p, xw);
-            const float xg = wk.g[tt][jl];
-            float dvp = 0.f;
 #pragma unroll
-            for (int e = 0; e < E; ++e) {
-                dvp = fmaf(L[e], xk[e], dvp);
-                L[e] = fmaf(xw[e], L[e], xr[e] * xg);
+            for (int c = 0; c < CPT; ++c) {
+                const float xg = wk.g[tt][jl + S * c];
+                float dvp = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    dvp = fmaf(L[c][e], xk[e], dvp);
+                    L[c][e] = fmaf(xw[e], L[c][e], xr[e] * xg);
+                }
+                dvp = group_sum<TPR>(dvp);
+                if (p == 0) dv[base + (t0 + tt) * stride + R * cg + jl + S * c] = fmaf(wk.bon[tt], xg, dvp);
             }
-            dvp = group_sum<TPR>(dvp);
-            if (p == 0) dv[base + (t0 + tt) * stride + j] = fmaf(wk.bon[tt], xg, dvp);
         }
     }
     if (ds0) {
 #pragma unroll
-        for (int e = 0; e < E; ++e) ds0[n * kN * kN + ent<TPR>(p, e) * kN + j] = L[e];
+        for (int c = 0; c < CPT; ++c)
+#pragma unroll
+            for (int e = 0; e < E; ++e) ds0[n * kN * kN + ent<TPR>(p, e) * kN + R * cg + jl + S * c] = L[c][e];
     }
 }
 
@@ -448,7 +457,7 @@ __global__ void __launch_bounds__(kN) wkv6_bwd_du_kernel(int64_t B, int64_t H, c
 
 // threads per row (column) of each kernel: the row walk backwards keeps a stash of kBlock
 // states per row in shared memory, so it spreads a row over more threads
-constexpr int kFwdTPR = 4, kRowsTPR = 8, kColsTPR = 4;
+constexpr int kFwdTPR = 4, kRowsTPR = 8, kColsTPR = 8, kColsCPT = 2;
 
 template <typename T> constexpr int fwd_smem()
 {
@@ -461,7 +470,7 @@ template <typename T> constexpr int rows_smem()
 }
 template <typename T> constexpr int cols_smem()
 {
-    constexpr int R = kThreads / kColsTPR;
+    constexpr int R = kThreads / kColsTPR * kColsCPT;
     return static_cast<int>(sizeof(ColStage<typename Store<T>::type, R>) + sizeof(ColWork<R>));
 }
 
@@ -473,8 +482,8 @@ template <typename T> cudaError_t configure()
         e = cudaFuncSetAttribute(wkv6_bwd_rows_kernel<T, kRowsTPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  rows_smem<T>());
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(wkv6_bwd_cols_kernel<T, kColsTPR>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 cols_smem<T>());
+        e = cudaFuncSetAttribute(wkv6_bwd_cols_kernel<T, kColsTPR, kColsCPT>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, cols_smem<T>());
     return e;
 }
 
@@ -504,7 +513,7 @@ cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
     const T *r = static_cast<const T *>(a.r), *k = static_cast<const T *>(a.k);
     const T *v = static_cast<const T *>(a.v), *w = static_cast<const T *>(a.w);
     const T *dy = static_cast<const T *>(a.dy);
-    // grid: (b, h) x the row (column) groups of a head, kN / (kThreads / TPR) = TPR / 2 of them
+    // grid: (b, h) x the row (column) groups of a head
     wkv6_bwd_forward_kernel<T, kFwdTPR><<<dim3(nbh, kFwdTPR / 2), kThreads, fwd_smem<T>(), s>>>(
         a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om);
     e = cudaGetLastError();
@@ -513,7 +522,8 @@ cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
         a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    wkv6_bwd_cols_kernel<T, kColsTPR><<<dim3(nbh, kColsTPR / 2), kThreads, cols_smem<T>(), s>>>(
+    wkv6_bwd_cols_kernel<T, kColsTPR, kColsCPT><<<dim3(nbh, kN / (kThreads / kColsTPR * kColsCPT)), kThreads,
+                                                   cols_smem<T>(), s>>>(
         a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
