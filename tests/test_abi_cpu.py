@@ -142,6 +142,8 @@ def test_wkv6_backward_validation(lib):
     assert ops.wkv6_backward_workspace_bytes(B, 0, H) == 0
     with pytest.raises(ops.WkvError):
         ops.wkv6_backward_workspace_bytes(-1, T, H)
+    with pytest.raises(ops.WkvError):  # checkpoint count x 64 x 64 overflows
+        ops.wkv6_backward_workspace_bytes(1, 1 << 56, 1, 1)
 
     def call(wbytes=need, **kw):
         a = {n: _p(i << 24) for i, n in enumerate(names)}

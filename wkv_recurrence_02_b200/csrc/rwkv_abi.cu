@@ -201,9 +201,11 @@ int wkv6_bwd_sizes(int64_t B, int64_t T, int64_t H, int64_t N, int64_t *n, int64
     if (!mul_ok(B, T, &BT) || !mul_ok(BT, H, &BTH) || !mul_ok(BTH, N, n) || !mul_ok(B, H, &BH) ||
         !mul_ok(BH, N * N, ns) || !mul_ok(H, N, hn))
         return fail(RWKV_ERR_SHAPE, "size product overflows%s");
+    // workspace: per (b, h), a 64 x 64 fp32 checkpoint every 8 tokens and 64 floats
     const int64_t nblk = (T + 7) / 8;
-    int64_t cells;
-    if (!mul_ok(BH, nblk * 4096 + 64, &cells)) return fail(RWKV_ERR_SHAPE, "workspace size overflows%s");
+    int64_t per_head, cells;
+    if (!mul_ok(nblk, 4096, &per_head) || !mul_ok(BH, per_head + 64, &cells))
+        return fail(RWKV_ERR_SHAPE, "workspace size overflows%s");
     return RWKV_OK;
 }
 
