@@ -466,8 +466,8 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
 // Used when a 16-channel block of k, v, y can be addressed by the tensor-memory
 // accelerator (row pitch C * element size a multiple of 16 bytes, 16-byte aligned bases).
 // Same algorithm and segment structure as above, different data movement:
-//   * one CTA = one batch row x 16 channels; warp h = one 16-byte unit of channels
-//     (8 bf16 or 4 fp32, carried as f32x2 pairs), lane = segment;
+//   * one CTA = one batch row x 16 channels; warp h = one 8-byte half of a 16-byte unit
+//     of channels (4 bf16 or 2 fp32, carried as f32x2 pairs: 4 or 8 warps), lane = segment;
 //   * the tile is held token-index-major: block i (128-byte aligned, as tensor copies
 //     require) holds row i of all 32 segments, 16 channels each, and arrives as one TMA
 //     box over a 4-D view (channel, i, segment, batch) of [B, T, C] -- exact when L
@@ -477,26 +477,10 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
 //   * two tile buffers: tile tau+1 is loaded while tile tau is scanned, and tile tau's
 //     store drains while tile tau+1 is scanned.
 
+// Scalar access to the channels of a lane (the exact fallback paths) and the tensor-map
+// element type.
 template <typename T> struct Unit;
 template <> struct Unit<__nv_bfloat16> {
-    static constexpr int NC = 8;  // channels per 16-byte unit
-    __device__ static void unpack(uint4 u, P2 (&x)[4])
-    {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            asm("mov.b64 %0, {%1, %2};" : "=l"(x[q].r) : "r"(w[q] << 16), "r"(w[q] & 0xFFFF0000u));
-    }
-    __device__ static uint4 pack(const P2 (&x)[4])
-    {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-            asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.bf16x2.f32 %0, h, l;\n\t}"
-                : "=r"(w[q])
-                : "l"(x[q].r));
-        return make_uint4(w[0], w[1], w[2], w[3]);
-    }
     __device__ static float get(const unsigned char *unit, int n)
     {
         return __bfloat162float(reinterpret_cast<const __nv_bfloat16 *>(unit)[n]);
@@ -508,68 +492,82 @@ template <> struct Unit<__nv_bfloat16> {
     static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
 };
 template <> struct Unit<float> {
-    static constexpr int NC = 4;
-    __device__ static void unpack(uint4 u, P2 (&x)[2])
-    {
-        x[0] = pk(__uint_as_float(u.x), __uint_as_float(u.y));
-        x[1] = pk(__uint_as_float(u.z), __uint_as_float(u.w));
-    }
-    __device__ static uint4 pack(const P2 (&x)[2])
-    {
-        return make_uint4(__float_as_uint(lo(x[0])), __float_as_uint(hi(x[0])), __float_as_uint(lo(x[1])),
-                          __float_as_uint(hi(x[1])));
-    }
     __device__ static float get(const unsigned char *unit, int n) { return reinterpret_cast<const float *>(unit)[n]; }
     __device__ static void put(unsigned char *unit, int n, float x) { reinterpret_cast<float *>(unit)[n] = x; }
     static constexpr CUtensorMapDataType kMapType = CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
 };
 
-// running min / max of the keys of one unit (bf16: two channels per instruction)
-template <typename T> struct KeyRange;
-template <> struct KeyRange<__nv_bfloat16> {
-    __nv_bfloat162 mx[4], mn[4];
+// The channels one lane owns in a token row: one 8-byte half of a 16-byte unit (4 bf16 or 2
+// fp32 channels).  Two warps share each unit, so a CTA of 16 channels runs 4 (bf16) or 8
+// (fp32) warps and each lane carries half the registers of a whole-unit lane.
+template <typename T> struct Lane;
+template <> struct Lane<__nv_bfloat16> {
+    static constexpr int NC = 4;
+    __device__ static uint2 load(const unsigned char *p) { return *reinterpret_cast<const uint2 *>(p); }
+    __device__ static void store(unsigned char *p, uint2 x) { *reinterpret_cast<uint2 *>(p) = x; }
+    __device__ static void unpack(uint2 u, P2 (&x)[2])
+    {
+        const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            asm("mov.b64 %0, {%1, %2};" : "=l"(x[q].r) : "r"(w[q] << 16), "r"(w[q] & 0xFFFF0000u));
+    }
+    __device__ static uint2 pack(const P2 (&x)[2])
+    {
+        uint32_t w[2];
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+            asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.bf16x2.f32 %0, h, l;\n\t}"
+                : "=r"(w[q])
+                : "l"(x[q].r));
+        return make_uint2(w[0], w[1]);
+    }
+};
+template <> struct Lane<float> {
+    static constexpr int NC = 2;
+    __device__ static uint2 load(const unsigned char *p) { return *reinterpret_cast<const uint2 *>(p); }
+    __device__ static void store(unsigned char *p, uint2 x) { *reinterpret_cast<uint2 *>(p) = x; }
+    __device__ static void unpack(uint2 u, P2 (&x)[1]) { x[0] = pk(__uint_as_float(u.x), __uint_as_float(u.y)); }
+    __device__ static uint2 pack(const P2 (&x)[1]) { return make_uint2(__float_as_uint(lo(x[0])), __float_as_uint(hi(x[0]))); }
+};
+
+// running min / max of a lane's keys
+template <typename T> struct LaneRange;
+template <> struct LaneRange<__nv_bfloat16> {
+    __nv_bfloat162 mx[2], mn[2];
     __device__ void init()
     {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             mx[q] = __floats2bfloat162_rn(-3.0e38f, -3.0e38f);
             mn[q] = __floats2bfloat162_rn(3.0e38f, 3.0e38f);
         }
     }
-    __device__ void add(uint4 u)
+    __device__ void add(uint2 u)
     {
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+        const uint32_t w[2] = {u.x, u.y};
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < 2; ++q) {
             const __nv_bfloat162 x = *reinterpret_cast<const __nv_bfloat162 *>(&w[q]);
             mx[q] = __hmax2(mx[q], x);
             mn[q] = __hmin2(mn[q], x);
         }
     }
-    __device__ float max(int n) const
-    {
-        return n & 1 ? __high2float(mx[n >> 1]) : __low2float(mx[n >> 1]);
-    }
-    __device__ float min(int n) const
-    {
-        return n & 1 ? __high2float(mn[n >> 1]) : __low2float(mn[n >> 1]);
-    }
+    __device__ float max(int n) const { return n & 1 ? __high2float(mx[n >> 1]) : __low2float(mx[n >> 1]); }
+    __device__ float min(int n) const { return n & 1 ? __high2float(mn[n >> 1]) : __low2float(mn[n >> 1]); }
 };
-template <> struct KeyRange<float> {
-    float mx[4], mn[4];
+template <> struct LaneRange<float> {
+    float mx[2], mn[2];
     __device__ void init()
     {
-#pragma unroll
-        for (int n = 0; n < 4; ++n) {
-            mx[n] = -3.4e38f;
-            mn[n] = 3.4e38f;
-        }
+        mx[0] = mx[1] = -3.4e38f;
+        mn[0] = mn[1] = 3.4e38f;
     }
-    __device__ void add(uint4 u)
+    __device__ void add(uint2 u)
     {
-        const float x[4] = {__uint_as_float(u.x), __uint_as_float(u.y), __uint_as_float(u.z), __uint_as_float(u.w)};
+        const float x[2] = {__uint_as_float(u.x), __uint_as_float(u.y)};
 #pragma unroll
-        for (int n = 0; n < 4; ++n) {
+        for (int n = 0; n < 2; ++n) {
             mx[n] = fmaxf(mx[n], x[n]);
             mn[n] = fminf(mn[n], x[n]);
         }
@@ -631,11 +629,11 @@ struct TmaParams {
 };
 
 template <typename T, int L, int NB>
-__global__ void __launch_bounds__(32 * (kCh / Unit<T>::NC), 3)
+__global__ void __launch_bounds__(32 * (kCh / Lane<T>::NC), 3)
 wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
                 const __grid_constant__ CUtensorMap map_y, const TmaParams p)
 {
-    constexpr int NC = Unit<T>::NC;              // channels per lane
+    constexpr int NC = Lane<T>::NC;              // channels per lane
     constexpr int NP = NC / 2;                   // f32x2 pairs per lane
     constexpr int RB = kCh * sizeof(T);          // bytes of one token row (16 channels)
     constexpr int BLK = kSegs * RB;              // bytes of block i: row i of every segment
@@ -710,13 +708,13 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         abort = __syncthreads_or(!mbar_wait(bar0 + 8 * (tile % NB), (tile / NB) & 1, p.spin_limit));
         if (abort) break;
         // this lane's unit in row 0 of its segment; row i is BLK bytes further
-        unsigned char *uk = sk + lane * RB + 16 * h;
-        const unsigned char *uv = sv + lane * RB + 16 * h;
+        unsigned char *uk = sk + lane * RB + NC * static_cast<int>(sizeof(T)) * h;
+        const unsigned char *uv = sv + lane * RB + NC * static_cast<int>(sizeof(T)) * h;
         const int nv = seg0 + lane < nsegs ? L : 0;
 
         // pass 1: local summaries against the segment's last key; key range
         St la[NC];
-        KeyRange<T> kr;
+        LaneRange<T> kr;
         kr.init();
 #pragma unroll
         for (int n = 0; n < NC; ++n) la[n] = empty;
@@ -724,7 +722,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             P2 nF[NP], A[NP], Bs[NP];
             {
                 P2 kl[NP];
-                Unit<T>::unpack(*reinterpret_cast<const uint4 *>(uk + (nv - 1) * BLK), kl);
+                Lane<T>::unpack(Lane<T>::load(uk + (nv - 1) * BLK), kl);
 #pragma unroll
                 for (int q = 0; q < NP; ++q) {
                     nF[q] = mul2(kl[q], nl2e);
@@ -735,12 +733,12 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int i = 0; i < L; ++i) {
                 if (i < nv) {
-                    const uint4 ku = *reinterpret_cast<const uint4 *>(uk + i * BLK);
-                    const uint4 vu = *reinterpret_cast<const uint4 *>(uv + i * BLK);
+                    const uint2 ku = Lane<T>::load(uk + i * BLK);
+                    const uint2 vu = Lane<T>::load(uv + i * BLK);
                     kr.add(ku);
                     P2 kk[NP], vv[NP];
-                    Unit<T>::unpack(ku, kk);
-                    Unit<T>::unpack(vu, vv);
+                    Lane<T>::unpack(ku, kk);
+                    Lane<T>::unpack(vu, vv);
 #pragma unroll
                     for (int q = 0; q < NP; ++q) {
                         const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
@@ -813,11 +811,11 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             for (int i = 0; i < L; ++i) {
                 if (i < nv) {
                     unsigned char *ui = uk + i * BLK;
-                    const uint4 ku = *reinterpret_cast<const uint4 *>(ui);
-                    const uint4 vu = *reinterpret_cast<const uint4 *>(uv + i * BLK);
+                    const uint2 ku = Lane<T>::load(ui);
+                    const uint2 vu = Lane<T>::load(uv + i * BLK);
                     P2 kk[NP], vv[NP], o[NP];
-                    Unit<T>::unpack(ku, kk);
-                    Unit<T>::unpack(vu, vv);
+                    Lane<T>::unpack(ku, kk);
+                    Lane<T>::unpack(vu, vv);
 #pragma unroll
                     for (int q = 0; q < NP; ++q) {
                         const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
@@ -826,7 +824,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
                         Bs[q] = fma2(dd[q], Bs[q], E);
                     }
-                    *reinterpret_cast<uint4 *>(ui) = Unit<T>::pack(o);
+                    Lane<T>::store(ui, Lane<T>::pack(o));
                 }
             }
         } else {
@@ -876,7 +874,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 template <typename T, int L, int NB>
 cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
 {
-    constexpr int NC = Unit<T>::NC;
+    constexpr int NC = Lane<T>::NC;
     constexpr int RB = kCh * sizeof(T);
     constexpr int BLK = kSegs * RB;
     constexpr int kThr = 32 * (kCh / NC);
