@@ -484,48 +484,65 @@ def load_traffic(kernel):
 
 # --------------------------------------------------------------------------- CPU oracle
 
-def oracle_sample(scale=1.0):
-    """Time the fp64 oracle on a bounded sample of each part of the step.
+_SAMPLE_INPUTS = {}
 
-    Returns (seconds for the full step extrapolated by tokens, threads, description).
+
+def _sample_inputs(n4, hs):
+    """The oracle sample's inputs as float64 arrays, drawn once per size (the draws are not timed)."""
+    key = (n4, hs)
+    if key not in _SAMPLE_INPUTS:
+        from wkv_recurrence_02_b200 import inputs
+        f64 = lambda t: t.float().double().numpy()  # noqa: E731
+        kv = inputs.wkv4_kv(8, 1024, 768, 0, "bf16")
+        wu = [tuple(f64(t) for t in inputs.wkv4_wu(768, layer + 1)) for layer in range(n4)]
+        x = inputs.wkv6_inputs(1, 4096, hs, 64, "bf16", seed=0, s0_std=0.1)
+        d = inputs.wkv6_inputs(256, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
+        _SAMPLE_INPUTS[key] = {
+            "kv": (f64(kv[0]), f64(kv[1])), "wu": wu,
+            "pre": [f64(x[n]) for n in ("r", "k", "v", "w", "u", "s0")],
+            "dec": [f64(d[n]) for n in ("r", "k", "v", "w", "u", "s0")]}
+    return _SAMPLE_INPUTS[key]
+
+
+def oracle_sample(scale=1.0):
+    """Time the fp64 oracle on a bounded sample of each part of the step, on all the
+    host's cores (the oracle runs independent units on OpenMP threads).
+
+    Sizes at scale 1: two WKV-4 layers at the full batch (B8 T1024 C768); 8 heads per thread
+    of a T=4096 WKV-6 sequence (so every thread has whole heads to walk); the full decode
+    step (B256 H64).  Returns (seconds for the full step extrapolated by tokens, threads,
+    description).
     """
-    import numpy as np
     import oracle
-    from wkv_recurrence_02_b200 import inputs
 
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
-    f64 = lambda t: t.float().double().numpy()  # noqa: E731
+    n4 = max(1, int(round(2 * scale)))
+    hs = threads * max(1, int(round(8 * scale)))
+    x = _sample_inputs(n4, hs)
     total = 0.0
     desc = []
-    # WKV-4: layer 0 on B=1 of 8 (1024 tokens x 768 channels)
-    b4 = max(1, int(round(1 * scale)))
-    kv = inputs.wkv4_kv(b4, 1024, 768, 0, "bf16")
-    w, u = inputs.wkv4_wu(768, 1)
-    a = [f64(w), f64(u), f64(kv[0]), f64(kv[1])]
+    # WKV-4: n4 layers of the full batch (each layer its own w, u)
+    dt = 0.0
+    for w, u in x["wu"]:
+        t0 = time.perf_counter()
+        oracle.wkv4(w, u, *x["kv"])
+        dt += time.perf_counter() - t0
+    total += dt * TOKENS_WKV4 / (n4 * 8 * 1024)
+    desc.append(f"wkv4 B8 T1024 C768 x{n4} layers")
+    # WKV-6 prefill: hs heads of a T=4096 sequence, scaled to Finch (H=32, B=8) and 7B (H=64, B=1)
+    r, k, v, w, u, s0 = x["pre"]
     t0 = time.perf_counter()
-    oracle.wkv4(*a)
+    oracle.wkv6(r, k, v, w, u, s0=s0)
     dt = time.perf_counter() - t0
-    total += dt * TOKENS_WKV4 / (b4 * 1024)
-    desc.append(f"wkv4 B{b4} T1024 C768 x1 layer")
-    # WKV-6 prefill: H heads of a T=4096 sequence, scaled to Finch (H=32, B=8) and 7B (H=64, B=1)
-    hs = max(1, int(round(4 * scale)))
-    x = inputs.wkv6_inputs(1, 4096, hs, 64, "bf16", seed=0, s0_std=0.1)
-    a = [f64(x[n]) for n in ("r", "k", "v", "w")]
-    t0 = time.perf_counter()
-    oracle.wkv6(*a, f64(x["u"]), s0=np.asarray(x["s0"].double().numpy()))
-    dt = time.perf_counter() - t0
-    per_head_token = dt / (hs * 4096)
-    total += per_head_token * (TOKENS_FINCH * 32 + TOKENS_LONG * 64)
+    total += dt / (hs * 4096) * (TOKENS_FINCH * 32 + TOKENS_LONG * 64)
     desc.append(f"wkv6 B1 T4096 H{hs}")
-    # decode: B rows of a T=1 step
-    bd = max(1, int(round(32 * scale)))
-    x = inputs.wkv6_inputs(bd, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
+    # decode: the full T=1 step
+    r, k, v, w, u, s0 = x["dec"]
     t0 = time.perf_counter()
-    oracle.wkv6(*[f64(x[n]) for n in ("r", "k", "v", "w")], f64(x["u"]), s0=x["s0"].double().numpy())
-    dt = time.perf_counter() - t0
-    total += dt * TOKENS_DECODE / bd
-    desc.append(f"wkv6 decode B{bd} H64")
+    oracle.wkv6(r, k, v, w, u, s0=s0)
+    total += time.perf_counter() - t0
+    desc.append("wkv6 decode B256 H64 (the whole decode part)")
     return total, threads, "; ".join(desc) + "; extrapolated to one step by tokens (x heads)"
 
 
