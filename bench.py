@@ -518,7 +518,9 @@ def oracle_sample(scale=1.0):
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
     n4 = max(1, int(round(2 * scale)))
-    hs = threads * max(1, int(round(8 * scale)))
+    # whole heads for every thread, at most 128 heads (1.6 GB of fp64 inputs) unless there
+    # are more threads than that
+    hs = min(threads * max(1, int(round(8 * scale))), max(threads, 128))
     x = _sample_inputs(n4, hs)
     total = 0.0
     desc = []
