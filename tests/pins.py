@@ -19,8 +19,9 @@ Kinds of pin used (none retypes the oracle's recurrence):
     inversion by numpy's logarithms, monotonicity and range, the slow-decay asymptote,
     and the -inf / +inf limits through the recurrence (no decay, instant forgetting);
   * WKV-6 backward: central finite differences of the pinned forward oracle, element by
-    element on a tiny case and along random directions at head size 64; the chain rule
-    through the decay map against differences of the map and of the logit forward.
+    element on a tiny case and along random directions at head size 64; an exact hand-worked
+    scalar example (tests/golden); the chain rule through the decay map against differences
+    of the map and of the logit forward.
 """
 import json
 import os
@@ -460,6 +461,21 @@ def pin_wkv6_backward_fd_directional(O):
         assert abs(an - fd) <= 1e-7 * max(1.0, abs(fd)), ("directional derivative", name, an, fd)
 
 
+def pin_wkv6_backward_golden(O):
+    """Exact hand-worked gradients of a scalar two-token case (tests/golden), derived from the
+    loss written out as a polynomial; every value is dyadic, so fp64 must match exactly."""
+    with open(os.path.join(GOLDEN, "wkv6_backward_hand_example.json")) as f:
+        g = json.load(f)
+    q = lambda x: float(Fraction(str(x)))  # noqa: E731
+    seq = lambda xs: np.array([q(x) for x in xs]).reshape(1, 2, 1, 1)  # noqa: E731
+    out = O.wkv6_backward(seq(g["r"]), seq(g["k"]), seq(g["v"]), seq(g["w"]), np.array([[q(g["u"])]]),
+                          seq(g["dy"]), s0=np.array([[[[q(g["s0"])]]]]), dsT=np.array([[[[q(g["dsT"])]]]]))
+    for name in ("dr", "dk", "dv", "dw"):
+        assert np.array_equal(out[name].reshape(2), np.array([q(x) for x in g[name]])), ("backward golden", name)
+    assert out["du"].reshape(()) == q(g["du"]), ("backward golden du", out["du"])
+    assert out["ds0"].reshape(()) == q(g["ds0"]), ("backward golden ds0", out["ds0"])
+
+
 def pin_logit_backward_fd(O):
     """The chain rule through w = exp(-exp(omega)): elementwise against central differences
     of the map, and through the recurrence against differences of wkv6_logit."""
@@ -492,7 +508,8 @@ ALL_PINS = [
     pin_wkv6_chaining, pin_wkv6_linearity, pin_wkv6_head_independence, pin_wkv6_golden,
     pin_norm_gate_two_channels, pin_norm_gate_invariants, pin_norm_gate_affine, pin_norm_gate_heads,
     pin_logit_closed_forms, pin_logit_inverse_and_shape, pin_wkv6_logit_limits,
-    pin_wkv6_backward_fd_elementwise, pin_wkv6_backward_fd_directional, pin_logit_backward_fd,
+    pin_wkv6_backward_fd_elementwise, pin_wkv6_backward_fd_directional, pin_wkv6_backward_golden,
+    pin_logit_backward_fd,
 ]
 
 
