@@ -59,9 +59,10 @@ template <int TPR> __device__ __forceinline__ int ent(int p, int e) { return 4 *
 
 // ------------------------------------------------------------------ staging in shared memory
 // Inputs reach the kernels through shared memory, kChunk tokens at a time, copied with
-// cp.async into the second of two buffers while the first is being used: every load is
-// issued a whole chunk before its data is needed.  U is the storage type (the bits of a
-// bf16 or an fp32 value); values are widened to fp32 when read.
+// cp.async a whole chunk before their data is needed: the row walks alternate two copy
+// buffers; the column walk widens each copied chunk into an fp32 working copy once and
+// refills the copy buffer while it walks the working copy.  U is the storage type (the bits
+// of a bf16 or an fp32 value); values are widened to fp32 when read.
 constexpr int kChunk = 32;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
