@@ -16,7 +16,7 @@ independent sequences/heads with no exchange step: weak scaling, no collective o
 data path); `value` is the tokens of all ranks over the max-over-ranks device time.
 
 --impl reference times the fp64 CPU oracle (the only other implementation this method
-has here) on a bounded sample of the same workload, on the host's cores.
+has here) on whole steps of the same workload, on the host's cores.
 """
 import argparse
 import json
@@ -61,6 +61,8 @@ BYTES = {
     "wkv6_decode": wkv6_bytes(256, 1, 64),
 }
 
+
+NOMINAL_HBM_GBS = 8000.0  # the 8 TB/s denominator the workload's roofline is stated against
 
 # fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA per clock x 2 flops x 1.965 GHz
 SIMT_FP32_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 2)
@@ -177,8 +179,15 @@ class Workload:
 
     # 12 WKV-4 layers, the Finch prefill, 4 long-context calls of two launches each (the
     # state-only and full passes of the sequence split at 64 heads), the decode step; the
-    # ncu launch list of this step counts the same (profiles/launch_list_bench_step.md)
+    # ncu launch list of this step counts the same
     launches_per_step = 12 + 1 + 4 * 2 + 1
+
+
+def step_config(world):
+    """The `config` object of the JSON line (the same for both arms)."""
+    return {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
+            "l2": "inputs larger than L2 (~2.4 GB per step per GPU); no flush",
+            "parallelism": f"replicas x{world} (independent sequences, no collective)"}
 
 
 def max_over_ranks(values, dist, device=None):
@@ -269,35 +278,24 @@ def run_ours(args, rank, world, dist):
         f["launches"] += len(ts)
     total_kernel_ms = sum(f["ms"] for f in fam.values())
     dom = max(fam, key=lambda k: fam[k]["ms"])
-    # roofline of the dominant kernel on one fixed launch: its largest workload in the step
-    # (the chunked kernel: the Finch-1.6B prefill launch, B8 T4096 H32)
-    dom_launch = max((n for n in per if (n.startswith(dom) if dom == "wkv6_chunked" else n == dom)),
-                     key=lambda n: BYTES[n])
-    dom_avg_ms = sum(per[dom_launch]) / len(per[dom_launch])
-    achieved = BYTES[dom_launch] / (dom_avg_ms * 1e-3) / 1e9
     parts = {}
     for name, ts in sorted(per.items()):
         avg = sum(ts) / len(ts)
         gbs = BYTES[name] / (avg * 1e-3) / 1e9
         parts[name] = {"avg_us": round(avg * 1e3, 2), "launches": len(ts),
-                       "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4)}
+                       "GBps": round(gbs, 1), "frac_hbm": round(gbs / hbm, 4),
+                       "frac_8TBps": round(gbs / NOMINAL_HBM_GBS, 4)}
     for k, f in fam.items():
         parts.setdefault("share", {})[k] = round(f["ms"] / total_kernel_ms, 4)
-    traffic = load_traffic(dom_launch)
-    cpu = cpu_baseline(args.cpu_sample_scale) if (world == 1 and not args.skip_cpu) else None
+    roofline = dominant_roofline(dom, fam[dom], per, hbm, peak_kind)
+    cpu = cpu_baseline() if (world == 1 and not args.skip_cpu) else None
     line = {
         "metric": METRIC, "value": job_tokens_per_s(world, STEP_TOKENS, args.steps, ms_max),
         "unit": UNIT, "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch CPU generator)",
-        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
-                   "l2": "inputs larger than L2 (~2.4 GB per step per GPU); no flush",
-                   "parallelism": f"replicas x{world} (independent sequences, no collective)"},
-        "roofline": {"bound": "hbm", "kernel": dom, "launch": dom_launch,
-                     "algorithmic_bytes": BYTES[dom_launch], "avg_us": round(dom_avg_ms * 1e3, 2),
-                     "achieved": round(achieved, 1),
-                     "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 4), "traffic": traffic},
+        "config": step_config(world),
+        "roofline": roofline,
         "parts": parts,
         "cpu_baseline": cpu,
         "e2e": {"value": job_tokens_per_s(world, STEP_TOKENS, 1, e2e_max), "unit": UNIT,
@@ -308,6 +306,29 @@ def run_ours(args, rank, world, dist):
         "device_status": status,
     }
     return line
+
+
+def dominant_roofline(kern, fam, per, hbm, peak_kind):
+    """Roofline of the dominant kernel over ALL its launches in the step: algorithmic bytes
+    of every timed call of the kernel over their summed CUDA-event durations (the average
+    launch).  Each call of the kernel is also listed on its own.  `traffic` is the DRAM
+    read + write of the average call, from committed ncu captures (see load_traffic)."""
+    names = sorted(n for n in per if (n.startswith(kern) if kern == "wkv6_chunked" else n == kern))
+    achieved = fam["bytes"] / (fam["ms"] * 1e-3) / 1e9
+    calls = {}
+    for n in names:
+        avg = sum(per[n]) / len(per[n])
+        gbs = BYTES[n] / (avg * 1e-3) / 1e9
+        calls[n] = {"algorithmic_bytes": BYTES[n], "avg_us": round(avg * 1e3, 2), "calls": len(per[n]),
+                    "achieved": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                    "frac_8TBps": round(gbs / NOMINAL_HBM_GBS, 4)}
+    traffic, note = load_traffic(names, per)
+    return {"bound": "hbm", "kernel": kern, "scope": "every launch of the kernel in the timed steps",
+            "algorithmic_bytes_per_launch": round(fam["bytes"] / fam["launches"]),
+            "avg_us_per_launch": round(fam["ms"] / fam["launches"] * 1e3, 2),
+            "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "frac_8TBps": round(achieved / NOMINAL_HBM_GBS, 4),
+            "traffic": traffic, "traffic_note": note, "calls": calls}
 
 
 def _time_us(torch, stream, dev, fn, reps):
@@ -472,111 +493,158 @@ def run_e2e(torch, ops, wl, stream, dev, steps, barrier):
     return e0.elapsed_time(e1) / steps, h2d, d2h
 
 
-def load_traffic(kernel):
-    """DRAM bytes per launch of `kernel` from the committed ncu summary, if present."""
+def load_traffic(names, per):
+    """DRAM bytes (read + write) of the average launch of the calls `names`, weighted by how
+    often each ran, from the committed ncu figures in profiles/traffic.json; None if any call
+    has no figure.  Returns (bytes, the file's note on how the figures were taken)."""
     p = os.path.join(HERE, "profiles", "traffic.json")
     if not os.path.exists(p):
-        return None
+        return None, None
     with open(p) as f:
         d = json.load(f)
-    return d.get(kernel)
+    if any(d.get(n) is None for n in names):
+        return None, d.get("_note")
+    n_calls = sum(len(per[n]) for n in names)
+    return round(sum(d[n] * len(per[n]) for n in names) / n_calls), d.get("_note")
 
 
 # --------------------------------------------------------------------------- CPU oracle
 
-_SAMPLE_INPUTS = {}
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
-def _sample_inputs(n4, hs):
-    """The oracle sample's inputs as float64 arrays, drawn once per size (the draws are not timed)."""
-    key = (n4, hs)
-    if key not in _SAMPLE_INPUTS:
+class OracleStep:
+    """The fp64 CPU oracle on the inputs of one whole step (drawn once, widened to float64
+    exactly; the draws are not timed).  full() runs the step as the GPU arm does: 12 WKV-4
+    layers, the Finch prefill, the four chained long-context calls and the decode step."""
+
+    def __init__(self):
         from wkv_recurrence_02_b200 import inputs
         f64 = lambda t: t.float().double().numpy()  # noqa: E731
         kv = inputs.wkv4_kv(8, 1024, 768, 0, "bf16")
-        wu = [tuple(f64(t) for t in inputs.wkv4_wu(768, layer + 1)) for layer in range(n4)]
-        x = inputs.wkv6_inputs(1, 4096, hs, 64, "bf16", seed=0, s0_std=0.1)
-        d = inputs.wkv6_inputs(256, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
-        _SAMPLE_INPUTS[key] = {
-            "kv": (f64(kv[0]), f64(kv[1])), "wu": wu,
-            "pre": [f64(x[n]) for n in ("r", "k", "v", "w", "u", "s0")],
-            "dec": [f64(d[n]) for n in ("r", "k", "v", "w", "u", "s0")]}
-    return _SAMPLE_INPUTS[key]
+        self.kv = (f64(kv[0]), f64(kv[1]))
+        self.wu = [tuple(f64(t) for t in inputs.wkv4_wu(768, layer + 1)) for layer in range(12)]
+        x = inputs.wkv6_inputs(8, 4096, 32, 64, "bf16", seed=0, s0_std=0.1)
+        self.finch = [f64(x[n]) for n in ("r", "k", "v", "w", "u", "s0")]
+        x = inputs.wkv6_inputs(1, 16384, 64, 64, "bf16", seed=0)
+        self.long = [f64(x[n]) for n in ("r", "k", "v", "w", "u")]
+        x = inputs.wkv6_inputs(256, 1, 64, 64, "bf16", seed=7, s0_std=0.1)
+        self.dec = [f64(x[n]) for n in ("r", "k", "v", "w", "u", "s0")]
+        del x
 
+    def _long(self, T):
+        r, k, v, w, u = self.long
+        s = None
+        for c in range(0, T, 4096):
+            sl = slice(c, min(c + 4096, T))  # B = 1: a slice of T is contiguous
+            _, s = oracle_mod().wkv6(r[:, sl], k[:, sl], v[:, sl], w[:, sl], u, s0=s)
 
-def oracle_sample(scale=1.0):
-    """Time the fp64 oracle on a bounded sample of each part of the step, on all the
-    host's cores (the oracle runs independent units on OpenMP threads).
-
-    Sizes at scale 1: two WKV-4 layers at the full batch (B8 T1024 C768); 8 heads per thread
-    of a T=4096 WKV-6 sequence (so every thread has whole heads to walk); the full decode
-    step (B256 H64).  Returns (seconds for the full step extrapolated by tokens, threads,
-    description).
-    """
-    import oracle
-
-    threads = len(os.sched_getaffinity(0))
-    oracle.set_threads(threads)
-    n4 = max(1, int(round(2 * scale)))
-    # whole heads for every thread, at most 128 heads (1.6 GB of fp64 inputs) unless there
-    # are more threads than that
-    hs = min(threads * max(1, int(round(8 * scale))), max(threads, 128))
-    x = _sample_inputs(n4, hs)
-    total = 0.0
-    desc = []
-    # WKV-4: n4 layers of the full batch (each layer its own w, u)
-    dt = 0.0
-    for w, u in x["wu"]:
+    def full(self):
+        """One whole step; returns its wall time in seconds."""
+        o = oracle_mod()
         t0 = time.perf_counter()
-        oracle.wkv4(w, u, *x["kv"])
-        dt += time.perf_counter() - t0
-    total += dt * TOKENS_WKV4 / (n4 * 8 * 1024)
-    desc.append(f"wkv4 B8 T1024 C768 x{n4} layers")
-    # WKV-6 prefill: hs heads of a T=4096 sequence, scaled to Finch (H=32, B=8) and 7B (H=64, B=1)
-    r, k, v, w, u, s0 = x["pre"]
-    t0 = time.perf_counter()
-    oracle.wkv6(r, k, v, w, u, s0=s0)
-    dt = time.perf_counter() - t0
-    total += dt / (hs * 4096) * (TOKENS_FINCH * 32 + TOKENS_LONG * 64)
-    desc.append(f"wkv6 B1 T4096 H{hs}")
-    # decode: the full T=1 step
-    r, k, v, w, u, s0 = x["dec"]
-    t0 = time.perf_counter()
-    oracle.wkv6(r, k, v, w, u, s0=s0)
-    total += time.perf_counter() - t0
-    desc.append("wkv6 decode B256 H64 (the whole decode part)")
-    return total, threads, "; ".join(desc) + "; extrapolated to one step by tokens (x heads)"
+        for w, u in self.wu:
+            o.wkv4(w, u, *self.kv)
+        r, k, v, w, u, s0 = self.finch
+        o.wkv6(r, k, v, w, u, s0=s0)
+        self._long(16384)
+        r, k, v, w, u, s0 = self.dec
+        o.wkv6(r, k, v, w, u, s0=s0)
+        return time.perf_counter() - t0
+
+    def sample(self):
+        """A bounded part of each piece of the step: one WKV-4 layer, Finch batch row 0 (of 8),
+        the first 512 tokens of the long context (of 16384) and the whole decode step.
+        Returns (the step's time extrapolated from the pieces by tokens, description)."""
+        o = oracle_mod()
+        t0 = time.perf_counter()
+        o.wkv4(*self.wu[0], *self.kv)
+        t1 = time.perf_counter()
+        r, k, v, w, u, s0 = self.finch
+        o.wkv6(r[:1], k[:1], v[:1], w[:1], u, s0=s0[:1])
+        t2 = time.perf_counter()
+        self._long(512)
+        t3 = time.perf_counter()
+        r, k, v, w, u, s0 = self.dec
+        o.wkv6(r, k, v, w, u, s0=s0)
+        t4 = time.perf_counter()
+        step = 12 * (t1 - t0) + 8 * (t2 - t1) + 32 * (t3 - t2) + (t4 - t3)
+        desc = ("wkv4 one layer (x12), wkv6 Finch batch row 0 (x8), wkv6 7B long context first "
+                "512 tokens (x32), the whole decode step; extrapolated to one step by tokens")
+        return step, desc
 
 
-def cpu_baseline(scale):
-    step_s, threads, desc = oracle_sample(scale)
+def oracle_mod():
+    import oracle
+    return oracle
+
+
+def cpu_figures(ostep, full_steps):
+    """All-thread figure: `full_steps` whole steps of the oracle on every host thread (after
+    one untimed step); single-thread figure: the bounded sample on one thread."""
+    o = oracle_mod()
+    threads = len(os.sched_getaffinity(0))
+    o.set_threads(threads)
+    times = [ostep.full() for _ in range(full_steps)]
+    o.set_threads(1)
+    one, desc1 = ostep.sample()
+    o.set_threads(threads)
+    return times, threads, {"value": STEP_TOKENS / one, "unit": UNIT, "cores": 1, "sample": desc1}
+
+
+def cpu_baseline(full_steps=2):
+    """The oracle timed on the host's cores: measured whole steps on every thread (the
+    reported value), and the single-thread figure on a bounded sample."""
+    ostep = OracleStep()
+    o = oracle_mod()
+    o.set_threads(len(os.sched_getaffinity(0)))
+    ostep.full()  # untimed: pages in the outputs
+    times, threads, single = cpu_figures(ostep, full_steps)
+    step_s = statistics.median(times)
     return {"value": STEP_TOKENS / step_s, "unit": UNIT, "cores": threads, "kind": "oracle",
-            "sample": desc}
+            "sample": f"the whole step, measured ({full_steps} steps, median {step_s:.3f} s)",
+            "cpu_model": cpu_model(), "single_thread": single}
 
 
 def run_reference(args, rank, world):
+    """The oracle as the reference arm: W untimed whole steps, then K whole steps timed with
+    the host clock (every host thread), then the single-thread figure on the bounded sample."""
     if rank != 0:
         return None
+    ostep = OracleStep()
+    o = oracle_mod()
+    threads = len(os.sched_getaffinity(0))
+    o.set_threads(threads)
     for _ in range(args.warmup):
-        oracle_sample(args.cpu_sample_scale * 0.25)
-    times = []
-    threads, desc = None, None
+        ostep.full()
     t0 = time.perf_counter()
-    for _ in range(args.steps):
-        s, threads, desc = oracle_sample(args.cpu_sample_scale * 0.25)
-        times.append(s)
+    times = [ostep.full() for _ in range(args.steps)]
     wall = time.perf_counter() - t0
-    step_s = sum(times) / len(times)
-    value = STEP_TOKENS / step_s
+    o.set_threads(1)
+    one, desc1 = ostep.sample()
+    o.set_threads(threads)
+    ms = wall * 1e3 / args.steps
+    value = STEP_TOKENS * args.steps / wall
     return {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded torch CPU generator)",
         "impl": "reference",
-        "config": {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
-                   "sampled_wall_s": round(wall, 2)},
+        "config": step_config(world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                         "sample": desc},
+                         "sample": f"the whole step, {args.steps} steps measured "
+                                   f"(median {statistics.median(times) * 1e3:.1f} ms)",
+                         "cpu_model": cpu_model(),
+                         "single_thread": {"value": STEP_TOKENS / one, "unit": UNIT, "cores": 1,
+                                           "sample": desc1}},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
@@ -587,7 +655,6 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-sample-scale", type=float, default=1.0)
     ap.add_argument("--skip-cpu", action="store_true", help="omit the CPU oracle baseline")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -227,8 +227,11 @@ int rwkv_get_wkv6_algo(void);
  * side: a first state-only pass gives each segment's local end state and decay product,
  * and each segment then starts from its exact incoming state.  The result equals the
  * unsplit evaluation up to fp32 rounding order.  The split needs B*H*(G-1)*(N*N+N)*4 bytes
- * of scratch, taken stream-ordered (on the calling thread's stream, within the call) from
- * a memory pool the library keeps per device, which holds up to 64 MB between calls.
+ * of scratch, plus B*H*N*N*4 bytes for a copy of s0 when the state is updated in place
+ * (sT == s0: the copy is taken before any segment runs, so no segment can read an s0 that
+ * the last segment has already overwritten).  The scratch is taken stream-ordered (on the
+ * calling thread's stream, within the call) from a memory pool the library keeps per
+ * device, which holds up to 64 MB between calls.
  *   segments = 0 (default): choose G;  1: never split;  n >= 2: split into at most n.
  * Returns RWKV_OK or RWKV_ERR_ARG. */
 int rwkv_set_wkv6_segments(int segments);
@@ -244,8 +247,9 @@ int rwkv_get_wkv6_segments(void);
  * that loads the library until the process exits) and never allocates or frees memory.
  *   segments: 0 = choose the split as rwkv_wkv6_forward_bf16 does, capped to what the
  *             array holds; n >= 1 = split into at most n segments.  A split needing more
- *             than RWKV_NOALLOC_SCRATCH_BYTES (B*H*(segments-1)*(N*N+N)*4 bytes) is
- *             rejected with RWKV_ERR_SHAPE before any launch; rwkv_last_error() says why.
+ *             than RWKV_NOALLOC_SCRATCH_BYTES (B*H*(G-1)*(N*N+N)*4 bytes for G segments,
+ *             plus B*H*N*N*4 bytes for the copy of s0 when sT == s0) is rejected with
+ *             RWKV_ERR_SHAPE before any launch; rwkv_last_error() says why.
  * Arguments, layouts and the result are otherwise those of rwkv_wkv6_forward_bf16 (always
  * the chunked kernel, whatever T).
  *   - The first call on each device looks up the array's device address (a CUDA runtime

@@ -1,3 +1,4 @@
+import json
 import os
 import sys
 
@@ -29,3 +30,13 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_sessionfinish(session, exitstatus):
+    """Write the parity comparisons made through gpu_util.rel_inf to $WKV_PARITY_RECORD."""
+    path = os.environ.get("WKV_PARITY_RECORD")
+    mod = sys.modules.get("gpu_util")
+    if not path or mod is None:
+        return
+    with open(path, "w") as f:
+        json.dump(mod.RECORDS, f)

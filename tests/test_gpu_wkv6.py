@@ -109,6 +109,22 @@ def test_wkv6_in_place_state_and_T0():
     assert rel_inf(f64(y), ry) <= 2e-2 and rel_inf(f64(s), rs) <= 2e-2
 
 
+def test_wkv6_in_place_state_of_split_sequences_over_several_waves():
+    """sT == s0 with every sequence cut into 4 segments and 512 CTAs per pass (more than one
+    wave at two CTAs per SM): no segment may start from an s0 that the last segment has
+    already overwritten.  Bit-identical to the out-of-place call with the same split."""
+    x = _inputs(4, 1024, 32, "bf16", 19, s0_std=0.1)
+    y_ref, s_ref = _gpu(x, s0=x["s0"], algo="chunked", segments=4)
+    s = dev(x["s0"]).clone()
+    y, s_out = ops.wkv6_forward(*(dev(x[n]) for n in ("r", "k", "v", "w")), dev(x["u"]), s0=s, sT=s,
+                                algo="chunked", segments=4)
+    torch.cuda.synchronize()
+    assert s_out.data_ptr() == s.data_ptr()
+    assert torch.equal(y, y_ref) and torch.equal(s, s_ref)
+    ry, rs = _ref(x, x["s0"])
+    assert rel_inf(f64(y), ry) <= 2e-2 and rel_inf(f64(s), rs) <= 2e-2
+
+
 @pytest.mark.parametrize("algo", ["serial", "chunked"])
 def test_wkv6_extreme_decays(algo):
     """w rounded to exactly 1.0 in bf16 on some channels, tiny w (1e-30) on others."""

@@ -28,11 +28,18 @@
 // Both channels of a lane are carried in 64-bit register pairs and advanced with packed
 // f32x2 arithmetic.
 //
-// Layout: one CTA = one batch row x 16 channels; warp = channel pair (2 channels per
-// lane), lane = segment.  k and v tiles (32 x L tokens x 16 channels) are copied with
-// cp.async straight into a [pair][segment][L+1] layout (the +1 pad and a 4-word skew per
-// pair make both the row-contiguous fill and the lane-strided reads conflict-free).
-// y overwrites k's words in place and is written back with row-contiguous stores.
+// Two kernels share this scan; both use one CTA per batch row x 16 channels and
+// lane = segment:
+//   wkv4_tma_kernel (the default, used when the row pitch is a multiple of 16 bytes, the
+//     segment length L divides T and T/L >= 32): the k and v tiles arrive by TMA as
+//     token-index-major blocks (block i = token i of all 32 segments); each warp holds one
+//     8-byte half of a 16-byte unit of channels; y replaces k in place and leaves by TMA
+//     store.
+//   wkv4_scan_kernel (every other shape: odd C, unaligned pointers, L not dividing T):
+//     warp = channel pair (2 channels per lane); k and v tiles are copied with cp.async
+//     into a [pair][segment][L+1] layout (the +1 pad and a 4-word skew per pair make both
+//     the row-contiguous fill and the lane-strided reads conflict-free); y overwrites k's
+//     words in place and is written back with row-contiguous stores.
 #include "wkv_internal.cuh"
 
 #include <mutex>

@@ -8,29 +8,28 @@
 // S <- diag(w_t) S + k_t^T v_t.  The RWKV-4 paper's parallelisation section motivates
 // evaluating the recurrence in time-parallel blocks.
 //
-// One CTA owns one (batch row, head) and walks its sequence in 64-token chunks.  The
-// fp32 state S (64x64) lives in tensor memory for the whole sequence.  Per chunk:
+// One CTA owns one (batch row, head) -- or one segment of it when sequences are split --
+// and walks its sequence in 64-token chunks.  The fp32 state S (64x64) lives in tensor
+// memory for the whole sequence.  Per chunk, with every decay referenced to the chunk end
+// (running products of w on CUDA cores -- no logarithms):
 //
-//   decay bookkeeping  Each 64-token chunk is 4 sub-blocks of 16.  With P_t the product of
-//                      w from the start of t's sub-block through t (running products on
-//                      CUDA cores -- no logarithms, no exponentials), every factor used
-//                      below is a product of w's and therefore <= 1, except the inverse
-//                      1/P_i of the diagonal sub-blocks (guarded, see below).
-//   intra-chunk scores A[t][i] = r_t . (k_i * prod_{j=i+1}^{t-1} w_j)  (i < t):
-//     off-diagonal     key sub-block b < query sub-block a: reference at the end of b,
-//                      Qo_b[t] = r_t * prod_{j=e_b+1}^{t-1} w_j,  Kb[i] = k_i * prod_{j=i+1}^{e_b} w_j,
-//                      three tcgen05 MMAs (M=64, N=16, K=64) into TMEM;
-//     diagonal         Qd[t] = r_t P_{t-1}, Kd[i] = k_i / P_i, one MMA (N=64), the four
-//                      16x16 diagonal blocks used.  If some P in the chunk falls below
-//                      2^-60 (very fast decay) the diagonal blocks are instead computed
-//                      exactly on CUDA cores from running products of w.
-//     A[t][t]          = sum_c r_t[c] u[c] k_t[c]  (the bonus term), on CUDA cores.
-//   O  = P V + Qi S_prev        P = causal-masked A in bf16, Qi[t] = r_t * prod_{j<t} w_j
-//   S  = diag(D) S_prev + Kh^T V,   Kh[i] = k_i * prod_{j>i} w_j,  D = prod_j w_j
-// The five products are tcgen05.mma kind::f16 (bf16 operands from swizzled shared
-// memory, fp32 accumulators in TMEM); S_prev is read from TMEM, copied to a bf16
-// operand tile and scaled by D in place.  r, k, v, w tiles arrive by TMA (4-D tensor
-// maps over [B, T, H, N], 128-byte swizzle, zero fill past T) into a 2-stage ring.
+//   Qx[t] = r_t / prod_{j>=t} w_j      (written over the r tile)
+//   Kh[i] = k_i * prod_{j>i} w_j       (written over the k tile; every factor <= 1)
+//   A     = Qx Kh^T                    scores: A[t][i] = r_t . (k_i prod_{j=i+1}^{t-1} w_j)
+//   P     = causal mask of A with the bonus sum_c r_t[c] u[c] k_t[c] on the diagonal (bf16)
+//   O     = P V + Qx . bf16(D (.) S_prev)      (Qx (.) D = r_t prod_{j<t} w_j)
+//   S     = diag(D) S_prev + Kh^T V,   D = prod_j w_j over the chunk
+//
+// If some channel's chunk decay D falls below 2^-100, 1/prod could overflow: that chunk
+// takes the sub-block path instead, with each 16-token query sub-block referenced to its
+// own start (all off-diagonal factors <= 1, three extra MMAs of N = 16 into TMEM), and the
+// 16x16 diagonal blocks either factored about the sub-block start or, when a 16-token
+// product is below 2^-60, computed exactly on CUDA cores.
+//
+// The products are tcgen05.mma kind::f16 (bf16 operands from 128-byte-swizzled shared
+// memory, fp32 accumulators in TMEM); S_prev is read from TMEM into a bf16 operand tile.
+// r, k, v, w tiles arrive by TMA (4-D tensor maps over [B, T, H, N], 128-byte swizzle,
+// zero fill past T) into a 3-stage ring.
 //
 // Every mbarrier wait is bounded; on expiry the CTA records RWKV_ERR_TIMEOUT in the
 // device status word, waits (bounded) for its own copies and MMAs, frees its tensor
@@ -407,6 +406,10 @@ struct ChunkedParams {
     int state_only;        // 1: only the segment's local end state (from zero) and decay
     float *seg;            // [B*H][segments-1][N*N + N]: local end state, then decay product
     int nseg;              // segments per sequence
+    // in-place state update of a split sequence (sT == s0): the state-only pass copies s0
+    // here (segment 0's CTAs) and the full pass reads the copy, so no CTA can read s0 after
+    // the last segment has overwritten it
+    float *s0copy;         // [B*H][N*N] or null
     // fused output stage (null gate: plain y): y = SiLU(g) (ln_w (o - mean) rstd + ln_b)
     const __nv_bfloat16 *gate;
     const float *ln_w, *ln_b;
@@ -830,6 +833,12 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 
         int ok = 1;
         if (iss_a && !abort && !so) ok = issue_scores(0);
+        if (so && p.s0copy && g == 0) {  // in-place split: keep s0 for the full pass
+            const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
+            float4 *dst = reinterpret_cast<float4 *>(p.s0copy + (bh * kN + row) * kN + colh);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) dst[i] = src[i];
+        }
         {   // initial state into TMEM: s0 advanced over the earlier segments (zero for a
             // state-only pass, which wants the segment's local contribution)
             float v[32];
@@ -1164,6 +1173,9 @@ int sm_count()
     return n;
 }
 
+// A split call that updates its state in place (sT == s0) needs a copy of s0 in scratch.
+bool split_state_copy(const Wkv6Args &a) { return a.s0 != nullptr && a.sT == a.s0; }
+
 // Kernel attributes (shared memory size, carveout), set once per device.
 cudaError_t configure_kernel()
 {
@@ -1257,18 +1269,24 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
                       static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G),
-                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
+                      nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     float *seg = nullptr;
     if (G > 1) {
+        const size_t seg_floats = static_cast<size_t>(bh) * (G - 1) * kSegStride;
+        const size_t copy_floats = split_state_copy(a) ? static_cast<size_t>(bh) * kN * kN : 0;
         cudaMemPool_t pool = nullptr;
         e = scratch_pool(&pool);
         if (e != cudaSuccess) return e;
-        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&seg),
-                                    static_cast<size_t>(bh) * (G - 1) * kSegStride * sizeof(float), pool, s);
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&seg), (seg_floats + copy_floats) * sizeof(float),
+                                    pool, s);
         if (e != cudaSuccess) return e;
         ChunkedParams pa = prm;
         pa.state_only = 1;
         pa.seg = seg;
+        if (copy_floats) {
+            pa.s0copy = seg + seg_floats;
+            prm.s0 = pa.s0copy;
+        }
         auto kso = a.omega ? wkv6_chunked_kernel<false, true> : wkv6_chunked_kernel<false, false>;
         kso<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes, s>>>(mr, mk, mv,
                                                                                                       mw, pa);
@@ -1334,11 +1352,14 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
         return cudaErrorInvalidConfiguration;
     const int64_t nchunks = (a.T + kC - 1) / kC;
     const int64_t per_segment = static_cast<int64_t>(kSegStride) * sizeof(float) * bh;
+    // an in-place split also keeps a copy of s0 in the array
+    const int64_t copy_bytes = split_state_copy(a) ? bh * kN * kN * static_cast<int64_t>(sizeof(float)) : 0;
+    const int64_t cap = static_cast<int64_t>(kNoAllocScratchBytes);
     int64_t G = 1;
     if (segments == 0) {  // as the allocating entry point, capped to what the array holds
         const int64_t slots = 2LL * sm_count();
         if (bh < slots) G = std::min<int64_t>(slots / bh, nchunks / 4);
-        G = std::min<int64_t>(G, static_cast<int64_t>(kNoAllocScratchBytes) / per_segment + 1);
+        G = std::min<int64_t>(G, cap >= copy_bytes ? (cap - copy_bytes) / per_segment + 1 : 1);
     } else {
         G = std::min<int64_t>(segments, nchunks);
     }
@@ -1346,7 +1367,7 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     const int64_t seg_chunks = (nchunks + G - 1) / G;
     G = (nchunks + seg_chunks - 1) / seg_chunks;
     if (G > 65535) return cudaErrorInvalidConfiguration;
-    *scratch_needed = static_cast<size_t>((G - 1) * per_segment);
+    *scratch_needed = G > 1 ? static_cast<size_t>((G - 1) * per_segment + copy_bytes) : 0;
     if (*scratch_needed > kNoAllocScratchBytes) return cudaErrorInvalidValue;
 
     float *seg = nullptr;
@@ -1363,12 +1384,17 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
                       static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G),
-                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
+                      nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     if (G > 1) {
-        // the state-only pass writes every scratch entry the full pass reads: nothing in the
-        // array has to start at zero, and what an earlier call left there is never read
+        // the state-only pass writes every scratch entry the full pass reads (the s0 copy of
+        // an in-place call included): nothing in the array has to start at zero, and what an
+        // earlier call left there is never read
         ChunkedParams pa = prm;
         pa.state_only = 1;
+        if (copy_bytes) {
+            pa.s0copy = seg + (G - 1) * per_segment / static_cast<int64_t>(sizeof(float));
+            prm.s0 = pa.s0copy;
+        }
         wkv6_chunked_kernel<false, false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)),
                                             kThreads, kSmemBytes, s>>>(mr, mk, mv, mw, pa);
         e = cudaGetLastError();
