@@ -138,7 +138,10 @@ def test_wkv6_backward_validation(lib):
     names = ["r", "k", "v", "w", "u", "s0", "dy", "dsT", "dr", "dk", "dv", "dw", "du", "ds0", "ws"]
     B, T, H = 1, 20, 2
     need = ops.wkv6_backward_workspace_bytes(B, T, H)
-    assert need == B * H * (3 * 64 * 64 + 64) * 4  # ceil(20 / 8) = 3 checkpoints per (b, h)
+    bh, nblk, nch = B * H, 3, 1  # ceil(20 / 8) walk checkpoints, ceil(20 / 64) chunks per (b, h)
+    walks = bh * nblk * 64 * 64 * 4                       # fp32 state every 8 tokens
+    chunked = bh * ((nch + 1) + nch) * 64 * 64 * 2 + bh * nch * 64 * 4  # bf16 states, row dots
+    assert need == max(walks, chunked) + bh * 64 * 4 + bh * nch * 64 * 4 + 16  # du shares, flags
     assert ops.wkv6_backward_workspace_bytes(B, 0, H) == 0
     with pytest.raises(ops.WkvError):
         ops.wkv6_backward_workspace_bytes(-1, T, H)

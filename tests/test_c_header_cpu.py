@@ -27,7 +27,9 @@ int main(void)
     if (rwkv_wkv6_forward(1, 4, 2, 32, 0, 0, 0, 0, 0, 0, 0, 0) != RWKV_ERR_UNSUPPORTED) fails |= 8;
     if (rwkv_wkv6_forward_bf16(0, 4, 2, 64, 0, 0, 0, 0, 0, 0, 0, 0) != RWKV_OK) fails |= 16;
     if (rwkv_wkv6_backward_workspace_bytes(2, 20, 3, 64, &bytes) != RWKV_OK ||
-        bytes != (size_t)2 * 3 * (3 * 64 * 64 + 64) * 4) fails |= 32;
+        /* the walks' three fp32 checkpoints per (b, h), then du shares per (b, h) and per
+           (b, h, chunk), then the (b, h) flags rounded up to 16 bytes */
+        bytes != (size_t)2 * 3 * (3 * 64 * 64) * 4 + 2 * 3 * 64 * 4 + 2 * 3 * 1 * 64 * 4 + 32) fails |= 32;
     if (rwkv_set_wkv6_algo(99) != RWKV_ERR_ARG) fails |= 64;
     printf("fails=%d\n", fails);
     return fails;

@@ -260,6 +260,8 @@ int wkv6_bwd_entry(int64_t B, int64_t T, int64_t H, int64_t N, const void *r, co
         return e == cudaSuccess ? RWKV_OK : cuda_fail(e, "wkv6 backward without tokens");
     }
     wkv::Wkv6BwdArgs a{B, T, H, N, r, k, v, w, u, s0, dy, dsT, dr, dk, dv, dw, du, ds0, workspace, bf16, omega};
+    a.chunked = bf16 && tl_wkv6_algo != RWKV_WKV6_SERIAL;
+    a.status = status;
     e = wkv::wkv6_backward_launch(a, tl_stream);
     if (e != cudaSuccess) return cuda_fail(e, "wkv6 backward launch");
     return RWKV_OK;

@@ -181,13 +181,14 @@ __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_forward_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                         const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                         const float *__restrict__ s0, const T *__restrict__ dy, float *__restrict__ dr,
-                        float *__restrict__ ckpt, float *__restrict__ du_part, int omega)
+                        float *__restrict__ ckpt, float *__restrict__ du_part, int omega, const int *only)
 {
     using U = typename Store<T>::type;
     constexpr int R = kThreads / TPR, E = kN / TPR;
     extern __shared__ __align__(16) unsigned char smem[];
     RowStage<U, R> *stg = reinterpret_cast<RowStage<U, R> *>(smem);  // [2]
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
+    if (only && !only[n]) return;
     const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
     const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
@@ -255,7 +256,7 @@ __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                      const T *__restrict__ dy, const float *__restrict__ dsT, const float *__restrict__ ckpt,
-                     float *__restrict__ dk, float *__restrict__ dw, int omega)
+                     float *__restrict__ dk, float *__restrict__ dw, int omega, const int *only)
 {
     using U = typename Store<T>::type;
     constexpr int R = kThreads / TPR, E = kN / TPR, G = E / 4;
@@ -263,6 +264,7 @@ wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     RowStage<U, R> *stg = reinterpret_cast<RowStage<U, R> *>(smem);  // [2]
     float4(*stash)[G][kThreads] = reinterpret_cast<float4(*)[G][kThreads]>(smem + 2 * sizeof(RowStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
+    if (only && !only[n]) return;
     const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
     const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
@@ -370,7 +372,8 @@ template <typename T, int TPR, int CPT>
 __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ w, const float *__restrict__ u, const T *__restrict__ dy,
-                     const float *__restrict__ dsT, float *__restrict__ dv, float *__restrict__ ds0, int omega)
+                     const float *__restrict__ dsT, float *__restrict__ dv, float *__restrict__ ds0, int omega,
+                     const int *only)
 {
     using U = typename Store<T>::type;
     constexpr int S = kThreads / TPR, R = S * CPT, E = kN / TPR;
@@ -378,6 +381,7 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     ColStage<U, R> &st = *reinterpret_cast<ColStage<U, R> *>(smem);
     ColWork<R> &wk = *reinterpret_cast<ColWork<R> *>(smem + sizeof(ColStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
+    if (only && !only[n]) return;
     const int cg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, jl = tid / TPR;
     const int warp = tid / 32, lane = tid % 32;
     const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
@@ -445,14 +449,28 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     }
 }
 
-// du[h][i] = sum over batch rows b of du_part[b][h][i], in order of b
-__global__ void __launch_bounds__(kN) wkv6_bwd_du_kernel(int64_t B, int64_t H, const float *__restrict__ du_part,
-                                                        float *__restrict__ du)
+// du[h][i] = sum over batch rows b, in order of b, of the (b, h) sequence's share: du_part[b][h][i]
+// from the walks, or, where the chunked path served the sequence (flags given and the
+// sequence's flag clear), the sum over its chunks of du_item[b][h][c][i] in order of c.
+// Fixed order throughout: deterministic.
+__global__ void __launch_bounds__(kN) wkv6_bwd_du_kernel(int64_t B, int64_t H, int64_t nch,
+                                                        const float *__restrict__ du_part,
+                                                        const float *__restrict__ du_item,
+                                                        const int *__restrict__ flags, float *__restrict__ du)
 {
     const int64_t h = blockIdx.x;
     const int i = threadIdx.x;
     float acc = 0.f;
-    for (int64_t b = 0; b < B; ++b) acc += du_part[(b * H + h) * kN + i];
+    for (int64_t b = 0; b < B; ++b) {
+        const int64_t n = b * H + h;
+        if (!flags || flags[n]) {
+            acc += du_part[n * kN + i];
+        } else {
+            float part = 0.f;
+            for (int64_t c = 0; c < nch; ++c) part += du_item[(n * nch + c) * kN + i];
+            acc += part;
+        }
+    }
     du[h * kN + i] = acc;
 }
 
@@ -489,7 +507,7 @@ template <typename T> cudaError_t configure()
 }
 
 template <typename T>
-cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
+cudaError_t launch_all(const Wkv6BwdArgs &a, const BwdLayout &L, const int *only, cudaStream_t s)
 {
     static std::mutex mu;
     static bool done[64] = {};
@@ -506,9 +524,9 @@ cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
         }
     }
     const int64_t bh = a.B * a.H;
-    const int64_t nblk = (a.T + kBlock - 1) / kBlock;
-    float *ckpt = static_cast<float *>(a.workspace);
-    float *du_part = ckpt + bh * nblk * kN * kN;
+    unsigned char *ws = static_cast<unsigned char *>(a.workspace);
+    float *ckpt = reinterpret_cast<float *>(ws);
+    float *du_part = reinterpret_cast<float *>(ws + L.du_part);
     const int om = a.omega ? 1 : 0;
     const unsigned nbh = static_cast<unsigned>(bh);
     const T *r = static_cast<const T *>(a.r), *k = static_cast<const T *>(a.k);
@@ -516,35 +534,68 @@ cudaError_t launch_all(const Wkv6BwdArgs &a, cudaStream_t s)
     const T *dy = static_cast<const T *>(a.dy);
     // grid: (b, h) x the row (column) groups of a head
     wkv6_bwd_forward_kernel<T, kFwdTPR><<<dim3(nbh, kFwdTPR / 2), kThreads, fwd_smem<T>(), s>>>(
-        a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om);
+        a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om, only);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_rows_kernel<T, kRowsTPR><<<dim3(nbh, kRowsTPR / 2), kThreads, rows_smem<T>(), s>>>(
-        a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om);
+        a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om, only);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_cols_kernel<T, kColsTPR, kColsCPT><<<dim3(nbh, kN / (kThreads / kColsTPR * kColsCPT)), kThreads,
                                                    cols_smem<T>(), s>>>(
-        a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    wkv6_bwd_du_kernel<<<static_cast<unsigned>(a.H), kN, 0, s>>>(a.B, a.H, du_part, a.du);
+        a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om, only);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H)
+BwdLayout wkv6_backward_layout(int64_t B, int64_t T, int64_t H)
 {
-    const int64_t nblk = (T + kBlock - 1) / kBlock;
-    return static_cast<size_t>(B * H) * static_cast<size_t>(nblk * kN * kN + kN) * sizeof(float);
+    const size_t bh = static_cast<size_t>(B * H);
+    const size_t nblk = static_cast<size_t>((T + kBlock - 1) / kBlock);
+    const size_t nch = static_cast<size_t>((T + 63) / 64);
+    BwdLayout L{};
+    L.nch = static_cast<int64_t>(nch);
+    const size_t walks = bh * nblk * kN * kN * sizeof(float);  // fp32 checkpoints every kBlock tokens
+    L.sck = 0;                                                 // bf16 [bh][nch + 1][64][64]
+    L.dsck = L.sck + bh * (nch + 1) * kN * kN * 2;             // bf16 [bh][nch][64][64]
+    L.rowdot = L.dsck + bh * nch * kN * kN * 2;                // fp32 [bh][nch][64]
+    const size_t chunked = L.rowdot + bh * nch * kN * sizeof(float);
+    L.du_part = std::max(walks, chunked);                      // fp32 [bh][64]
+    L.du_item = L.du_part + bh * kN * sizeof(float);           // fp32 [bh][nch][64]
+    L.flags = L.du_item + bh * nch * kN * sizeof(float);       // int [bh]
+    L.total = L.flags + ((bh * sizeof(int) + 15) & ~static_cast<size_t>(15));
+    return L;
+}
+
+size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H) { return wkv6_backward_layout(B, T, H).total; }
+
+cudaError_t wkv6_backward_walks_launch(const Wkv6BwdArgs &a, const BwdLayout &L, const int *only, cudaStream_t s)
+{
+    return a.bf16 ? launch_all<__nv_bfloat16>(a, L, only, s) : launch_all<float>(a, L, only, s);
 }
 
 cudaError_t wkv6_backward_launch(const Wkv6BwdArgs &a, cudaStream_t s)
 {
     if (a.B * a.H == 0 || a.T == 0) return cudaSuccess;
     if (a.B * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    return a.bf16 ? launch_all<__nv_bfloat16>(a, s) : launch_all<float>(a, s);
+    const BwdLayout L = wkv6_backward_layout(a.B, a.T, a.H);
+    unsigned char *ws = static_cast<unsigned char *>(a.workspace);
+    const int *flags = nullptr;
+    cudaError_t e;
+    if (a.chunked && a.bf16) {
+        // the tensor-core path; the sequences it flags (decay too fast for its chunk algebra)
+        // are then served by the exact walks
+        e = wkv6_backward_tc_launch(a, L, s);
+        if (e != cudaSuccess) return e;
+        flags = reinterpret_cast<const int *>(ws + L.flags);
+    }
+    e = wkv6_backward_walks_launch(a, L, flags, s);
+    if (e != cudaSuccess) return e;
+    wkv6_bwd_du_kernel<<<static_cast<unsigned>(a.H), kN, 0, s>>>(
+        a.B, a.H, L.nch, reinterpret_cast<const float *>(ws + L.du_part),
+        reinterpret_cast<const float *>(ws + L.du_item), flags, a.du);
+    return cudaGetLastError();
 }
 
 }  // namespace wkv

@@ -1,0 +1,784 @@
+// wkv6_backward_tc.cu -- Eagle/Finch WKV-6 backward pass on B200 tensor cores (tcgen05 + TMA
+// + TMEM), in 64-token chunks.
+//
+// Source: "RWKV-5/6 (Eagle and Finch)", section 4.1.2 (time mixing: S is a sum of k^T v, each
+// key channel decayed by w every step, gain u on the current token, receptance r applied like a
+// query; w = exp(-exp(omega))) and section 4.2.2 (Finch: w_t per token).  Forward, per (b, h):
+//   y_t = r_t (S + diag(u) k_t^T v_t),   S <- diag(w_t) S + k_t^T v_t.
+// The gradients are those of the fp32 walks in wkv6_backward.cu (the chain rule walked
+// backwards in time), regrouped by chunk.  Within a chunk, with every decay referenced to the
+// chunk end (D = prod_j w_j; Qfac_t = prod_{j>=t} w_j; Kfac_i = prod_{j>i} w_j):
+//   Qx = r / Qfac,  Kh = k * Kfac,  A = Qx Kh^T (scores),  dA = dO V^T,
+//   Am  = causal part of A with the bonus sum_c r_t u k_t on the diagonal,  dAm = dA strictly
+//         below the diagonal,  dd_t = dO_t . v_t (the diagonal of dA),
+//   dR  = (dAm Kh + dO (D S_prev)^T) / Qfac + u k_t dd_t
+//   dK  = (dAm^T Qx + V dS_end^T) * Kfac + u r_t dd_t
+//   dV  = Am^T dO + Kh dS_end
+//   dS_prev = diag(D) dS_end + Qi^T dO,  Qi_t = r_t prod_{j<t} w_j
+// and the decay gradient in log space, d(log w_j) = sum_{m>=j} dL_m with
+//   dL_m = (Qx dRacc)_{m+1} - (Kh dKacc)_m  (+ rowdot(dS_end, S_end) on the chunk's last token),
+// where dRacc and dKacc are the accumulators above before their row scaling: each pair of
+// tokens appears once on each side with the same bf16 operands, so the pairs inside the chunk
+// cancel exactly.  Then dw = d(log w) / w, or domega = -exp(omega) d(log w).
+//
+// Three kernels:
+//   wkv6_bwd_state_kernel<false>  forward over chunks (k, v, w): the state before every chunk
+//                                 and after the last, in bf16; flags (b, h) sequences whose
+//                                 decay is too fast for the chunk-end reference;
+//   wkv6_bwd_state_kernel<true>   backward over chunks (r, dO, w): the state gradient after
+//                                 every chunk in bf16, rowdot(dS_end, S_end) per chunk, ds0;
+//   wkv6_bwd_chunk_kernel         one CTA per (b, h, chunk), all chunks in parallel: the
+//                                 products above on tcgen05 (bf16 operands from swizzled shared
+//                                 memory, fp32 accumulators in TMEM), dr, dk, dv, dw and the
+//                                 chunk's share of du.
+// A flagged sequence (some channel's chunk decay below 2^-100, where 1/Qfac could overflow,
+// or, for a w input, some w below 2^-5, where d(log w) / w would magnify the rounding of
+// d(log w)) is skipped by the chunk kernels and served by the exact fp32 walks.
+//
+// Every mbarrier wait is bounded; on expiry the CTA records RWKV_ERR_TIMEOUT in the device
+// status word, waits (bounded) for its own copies and MMAs, frees its tensor memory and returns.
+#include "tc_common.cuh"
+
+#include <algorithm>
+#include <mutex>
+
+namespace wkv {
+namespace {
+using namespace tc;
+
+constexpr int kC = 64;                                // tokens per chunk
+constexpr int kN = 64;                                // head size
+constexpr float kFastMin = 7.888609052210118e-31f;    // 2^-100: chunk-end reference guard
+constexpr float kWMin = 0.03125f;                     // 2^-5: smallest w the w-input path divides by
+
+__device__ __forceinline__ unsigned char *align1024(unsigned char *p)
+{
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+}
+
+// sum over the four channels of a * b
+__device__ __forceinline__ float dot4(Q4 a, Q4 b)
+{
+    const P2 acc = fma2(a.b, b.b, mul2(a.a, b.a));
+    return lo(acc) + hi(acc);
+}
+
+// Sum over the 16 lanes of a half-warp of 8 per-lane partials (one per token m = 0..7).
+// Returns the total for token (lane >> 1) & 7 (valid in every lane).
+__device__ __forceinline__ float half_sum8(const float (&part)[8], int lane)
+{
+    float v4[4], v2[2];
+    const bool b8 = lane & 8, b4 = lane & 4, b2 = lane & 2;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        v4[i] = (b8 ? part[4 + i] : part[i]) + __shfl_xor_sync(0xffffffffu, b8 ? part[i] : part[4 + i], 8);
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        v2[i] = (b4 ? v4[2 + i] : v4[i]) + __shfl_xor_sync(0xffffffffu, b4 ? v4[i] : v4[2 + i], 4);
+    float v = (b2 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b2 ? v2[0] : v2[1], 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
+}
+
+// 8 bf16 (16 bytes) -> 8 fp32
+__device__ __forceinline__ void unpack8(uint4 x, float *o)
+{
+    const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        o[2 * e] = __uint_as_float(w[e] << 16);
+        o[2 * e + 1] = __uint_as_float(w[e] & 0xFFFF0000u);
+    }
+}
+
+// 8 consecutive bf16 of row `row` from byte column `colbyte` (a multiple of 16) of a swizzled tile
+__device__ __forceinline__ void ld_row8(const unsigned char *tile, int row, int colbyte, float *o)
+{
+    unpack8(*reinterpret_cast<const uint4 *>(tile + swz(row, colbyte)), o);
+}
+
+__device__ __forceinline__ void st_f32x32(float *dst, const float (&v)[32])
+{
+    float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
+__device__ __forceinline__ void st_bf16x32(__nv_bfloat16 *dst, const float (&v)[32])
+{
+    uint4 *d = reinterpret_cast<uint4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+        d[i] = make_uint4(pack_bf16(v[8 * i], v[8 * i + 1]), pack_bf16(v[8 * i + 2], v[8 * i + 3]),
+                          pack_bf16(v[8 * i + 4], v[8 * i + 5]), pack_bf16(v[8 * i + 6], v[8 * i + 7]));
+}
+
+// ================================================================ state passes (K0 / K1)
+// 128 threads = 4 warps.  Warp a prepares the operand rows of 16-token sub-block a (lane:
+// 8-token half hf, channel quad cq); the same warp then serves TMEM lanes 32a.. of the state
+// (rows 16a .. 16a + 15, two 32-column halves).  One elected thread issues the TMA copies
+// (a 3-stage ring of X | Y | W tiles) and the four MMAs per chunk.
+constexpr int kSThreads = 128;
+constexpr int kSStages = 3;
+constexpr int kSStage = 3 * kTile;                     // X | Y | W
+constexpr int S_H = kSStages * kSStage;                // [4][64] sub-block decay products
+constexpr int S_D = S_H + 4 * 64 * 4;                  // [stage][64] chunk decay
+constexpr int S_BAR = S_D + kSStages * 64 * 4;         // full[3], mma
+constexpr int S_MISC = S_BAR + 64;                     // TMEM base
+constexpr int kStateSmem = S_MISC + 64 + 1024;
+
+struct StateParams {
+    int64_t T, H;
+    int nch;
+    const float *init;            // [bh][N][N] fp32: s0 (forward) or dsT (backward); null = 0
+    __nv_bfloat16 *ck;            // forward: [bh][nch + 1][N][N]; backward: [bh][nch][N][N]
+    const __nv_bfloat16 *sck;     // backward: the forward checkpoints (for the row dots)
+    float *rowdot;                // backward: [bh][nch][N]
+    int *flags;                   // forward: written; backward: read (flagged sequences skipped)
+    float *fin;                   // backward: ds0 [bh][N][N] fp32, or null
+    int *status;
+    uint32_t spin_limit;
+};
+
+// REV = false: S <- diag(D) S + Kh^T V over chunks 0..nch-1 (X = k, Y = v), writing the state
+//              entering each chunk and the final state.
+// REV = true:  dS <- diag(D) dS + Qi^T dO over chunks nch-1..0 (X = r, Y = dO), writing the
+//              state gradient leaving each chunk, its row dot with the state there, and ds0.
+template <bool REV, bool OMEGA>
+__global__ void __launch_bounds__(kSThreads)
+wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_y,
+                      const __grid_constant__ CUtensorMap map_w, const StateParams p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = align1024(smem_raw);
+    float *Hs = reinterpret_cast<float *>(sm + S_H);
+    float *Dv = reinterpret_cast<float *>(sm + S_D);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S_BAR);
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + S_MISC);
+    const uint32_t bar_full0 = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[kSStages]);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
+    const int nch = p.nch;
+    const int nck = REV ? nch : nch + 1;
+    const uint32_t limit = p.spin_limit;
+    if (REV && p.flags[bh]) return;  // served by the exact walks
+
+    if (tid == 0) {
+        for (int s = 0; s < kSStages; ++s) bar_init(bar_full0 + 8 * s, 1);
+        bar_init(bar_mma, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(const_cast<uint32_t *>(misc))),
+                     "r"(64));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tbase = misc[0];
+
+    int issued = 0, committed = 0;  // meaningful in thread 0
+    auto issue = [&](int n) {
+        const int cc = REV ? nch - 1 - n : n;
+        const int s = n % kSStages;
+        const uint32_t dst = smem_u32(sm + s * kSStage), bar = bar_full0 + 8 * s;
+        bar_expect_tx(bar, kSStage);
+        tma_load_4d(dst, &map_x, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
+        tma_load_4d(dst + kTile, &map_y, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
+        tma_load_4d(dst + 2 * kTile, &map_w, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
+    };
+    if (tid == 0)
+        for (; issued < kSStages && issued < nch; ++issued) issue(issued);
+
+    // TMEM lane group of this warp: rows 16 warp .. + 15, columns [colh, colh + 32)
+    const int lr = lane & 15, hi = lane >> 4, row = 16 * warp + lr, colh = 32 * hi;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * warp) << 16);
+    {
+        float v[32];
+        if (p.init) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = src[i];
+                v[4 * i] = x.x, v[4 * i + 1] = x.y, v[4 * i + 2] = x.z, v[4 * i + 3] = x.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.f;
+        }
+        tmem_st32(tl, v);
+    }
+
+    // prep lanes: warp a = 16-token sub-block, hf = 8-token half, cq = channel quad
+    const int a = warp, hf = lane >> 4, cq = lane & 15, t0h = 16 * a + 8 * hf;
+    const uint32_t cbyte = 8 * cq;
+    int hazard = 0, abort = 0;
+    for (int n = 0; n < nch; ++n) {
+        const int cc = REV ? nch - 1 - n : n;
+        const int s = n % kSStages;
+        unsigned char *st = sm + s * kSStage;
+        const int64_t t0 = static_cast<int64_t>(cc) * kC;
+        const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+        int ok = bar_wait(bar_full0 + 8 * s, (n / kSStages) & 1, limit);
+        if (__syncthreads_or(!ok)) {
+            abort = 1;
+            break;
+        }
+        // decays of this half (1 past the end) and their products
+        Q4 w[8];
+        Q4 Gh = one4();
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int t = t0h + m;
+            if (t < tv) {
+                const Q4 x = unpack4(ld_u2(st + 2 * kTile, swz(t, cbyte)));
+                w[m] = OMEGA ? decay4(x) : x;
+                if (!REV && !OMEGA) hazard |= any_below(w[m], kWMin);
+            } else {
+                w[m] = one4();
+            }
+            Gh = mul4(Gh, w[m]);
+        }
+        const Q4 Go = shfl_xor4(Gh, 16);
+        if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
+        __syncthreads();
+        Q4 D = one4(), before = one4(), aft = one4();
+#pragma unroll
+        for (int be = 0; be < 4; ++be) {
+            const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
+            D = mul4(D, g);
+            before = be < a ? mul4(before, g) : before;
+            aft = be > a ? mul4(aft, g) : aft;
+        }
+        if (!REV) hazard |= any_below(D, kFastMin);
+        if (!REV) {  // Kh[i] = k_i prod_{j>i} w_j (chunk-end reference, every factor <= 1)
+            Q4 run = mul4(aft, hf ? one4() : Go);
+#pragma unroll
+            for (int m = 7; m >= 0; --m) {
+                const uint32_t off = swz(t0h + m, cbyte);
+                st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
+                run = mul4(run, w[m]);
+            }
+        } else {     // Qi[t] = r_t prod_{j<t} w_j (chunk-start reference, every factor <= 1)
+            Q4 run = mul4(before, hf ? Go : one4());
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const uint32_t off = swz(t0h + m, cbyte);
+                st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
+                run = mul4(run, w[m]);
+            }
+        }
+        if (warp == 0 && hf == 0) st_q4(Dv + s * 64 + 4 * cq, D);
+        fence_async_smem();
+        // the previous chunk's update must be complete before the state is read
+        ok = n > 0 ? bar_wait(bar_mma, (n - 1) & 1, limit) : 1;
+        if (__syncthreads_or(!ok)) {
+            abort = 1;
+            break;
+        }
+        if (tid == 0 && n > 0 && issued < nch) issue(issued++);  // the stage of chunk n - 1 is free
+        fence_after();
+        {
+            float v[32];
+            tmem_ld32(tl, v);
+            st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, v);
+            if (REV) {  // rowdot(dS_end, S_end), S_end = the forward checkpoint after chunk cc
+                const uint4 *src = reinterpret_cast<const uint4 *>(
+                    p.sck + ((bh * (nch + 1) + cc + 1) * kN + row) * kN + colh);
+                float part = 0.f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float x[8];
+                    unpack8(src[i], x);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) part = fmaf(v[8 * i + e], x[e], part);
+                }
+                part += __shfl_xor_sync(0xffffffffu, part, 16);
+                if (hi == 0) p.rowdot[(bh * nch + cc) * kN + row] = part;
+            }
+            const float d = Dv[s * 64 + row];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] *= d;
+            tmem_st32(tl, v);
+        }
+        fence_before();
+        __syncthreads();
+        fence_after();
+        if (tid == 0) {
+            const uint32_t aX = smem_u32(st), aY = smem_u32(st + kTile);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+                mma(tbase, desc_mn(aX + 2048 * ks), desc_mn(aY + 2048 * ks), idesc(64, 1, 1), 1);
+            mma_commit(bar_mma);
+            ++committed;
+        }
+    }
+    if (!abort) {
+        const int ok = bar_wait(bar_mma, (nch - 1) & 1, limit);
+        abort = __syncthreads_or(!ok);
+    }
+    if (!abort) {
+        fence_after();
+        float v[32];
+        tmem_ld32(tl, v);
+        if (!REV)
+            st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, v);
+        else if (p.fin)
+            st_f32x32(p.fin + (bh * kN + row) * kN + colh, v);
+    }
+    if (!REV) {
+        const int hz = __syncthreads_or(hazard);
+        if (tid == 0) p.flags[bh] = hz;
+    }
+    if (abort) {
+        record_status(p.status, kStatusTimeout);
+        if (tid == 0) {
+            for (int n = issued - kSStages < 0 ? 0 : issued - kSStages; n < issued; ++n)
+                bar_wait(bar_full0 + 8 * (n % kSStages), (n / kSStages) & 1, limit);
+            if (committed > 0) bar_wait(bar_mma, (committed - 1) & 1, limit);
+        }
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(64));
+}
+
+// ================================================================ per-chunk gradients (K2)
+// 128 threads = 4 warps, one (b, h, chunk) per CTA, two CTAs per SM.  Shared memory: the seven
+// input tiles (r, k, v, w, dO, the bf16 state before the chunk, the bf16 state gradient after
+// it), four operand tiles built here (Qx, Kh, Am, dAm), and the fp32 prefix decay products.
+// TMEM (256 columns): A at 0 and dA at 64, then dV at 0 (after A is read), dR at 128, dK at 192.
+constexpr int G_R = 0, G_K = 1, G_V = 2, G_W = 3, G_G = 4, G_S = 5, G_DS = 6, G_QX = 7, G_KH = 8, G_AM = 9,
+              G_DAM = 10;                              // tile slots (x kTile bytes)
+constexpr int kPreStride = 68;                         // fp32 row stride of the prefix products (pad)
+constexpr int G_PRE = 11 * kTile;                      // [64][68] fp32: prod_{j<t} w_j
+constexpr int G_SMALL = G_PRE + 64 * kPreStride * 4;
+constexpr int G_HS = G_SMALL;                          // [4][64] sub-block products; later column totals
+constexpr int G_DV = G_HS + 4 * 64 * 4;                // [64] chunk decay D
+constexpr int G_IDV = G_DV + 64 * 4;                   // [64] 1 / D
+constexpr int G_UB = G_IDV + 64 * 4;                   // [64] bonus sum_c r u k per token
+constexpr int G_DD = G_UB + 64 * 4;                    // [64] dO_t . v_t
+constexpr int G_U = G_DD + 64 * 4;                     // [64] u of the head
+constexpr int G_RD = G_U + 64 * 4;                     // [64] rowdot(dS_end, S_end)
+constexpr int G_DU = G_RD + 64 * 4;                    // [4][64] du partials
+constexpr int G_BAR = G_DU + 4 * 64 * 4;               // full, mma1, mma2
+constexpr int G_MISC = G_BAR + 64;
+constexpr int kChunkSmem = G_MISC + 64 + 1024;
+constexpr uint32_t T_A = 0, T_DA = 64, T_DV = 0, T_DR = 128, T_DK = 192, kChunkTmem = 256;
+
+struct GradParams {
+    int64_t T, H;
+    int nch;
+    const float *u;                  // [H][N]
+    const float *rowdot;             // [bh][nch][N]
+    const int *flags;                // [bh]
+    float *dr, *dk, *dv, *dw;        // [B][T][H][N] fp32 (dw holds domega with the decay logit)
+    float *du_item;                  // [bh][nch][N]
+    int *status;
+    uint32_t spin_limit;
+};
+
+template <bool OMEGA>
+__global__ void __launch_bounds__(128, 2)
+wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
+                      const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
+                      const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_s,
+                      const __grid_constant__ CUtensorMap map_ds, const GradParams p)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = align1024(smem_raw);
+    unsigned char *TR = sm + G_R * kTile, *TK = sm + G_K * kTile, *TV = sm + G_V * kTile, *TW = sm + G_W * kTile;
+    unsigned char *TG = sm + G_G * kTile, *TS = sm + G_S * kTile, *TDS = sm + G_DS * kTile;
+    unsigned char *TQX = sm + G_QX * kTile, *TKH = sm + G_KH * kTile, *TAM = sm + G_AM * kTile;
+    unsigned char *TDAM = sm + G_DAM * kTile;
+    float *PRE = reinterpret_cast<float *>(sm + G_PRE);
+    float *Hs = reinterpret_cast<float *>(sm + G_HS);
+    float *Dv = reinterpret_cast<float *>(sm + G_DV), *iDv = reinterpret_cast<float *>(sm + G_IDV);
+    float *UB = reinterpret_cast<float *>(sm + G_UB), *DD = reinterpret_cast<float *>(sm + G_DD);
+    float *U = reinterpret_cast<float *>(sm + G_U), *RD = reinterpret_cast<float *>(sm + G_RD);
+    float *DU = reinterpret_cast<float *>(sm + G_DU);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + G_BAR);
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + G_MISC);
+    const uint32_t bar_full = smem_u32(&bars[0]), bar_m1 = smem_u32(&bars[1]), bar_m2 = smem_u32(&bars[2]);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nch = p.nch;
+    const int64_t item = blockIdx.x, bh = item / nch, b = bh / p.H, h = bh % p.H;
+    const int cc = static_cast<int>(item % nch);
+    const int64_t t0 = static_cast<int64_t>(cc) * kC;
+    const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+    const uint32_t limit = p.spin_limit;
+    if (p.flags[bh]) return;  // served by the exact walks
+
+    if (tid == 0) {
+        bar_init(bar_full, 1);
+        bar_init(bar_m1, 1);
+        bar_init(bar_m2, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(const_cast<uint32_t *>(misc))),
+                     "r"(kChunkTmem));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    const uint32_t tbase = misc[0];
+
+    if (tid == 0) {
+        bar_expect_tx(bar_full, 7 * kTile);
+        const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
+        tma_load_4d(smem_u32(TR), &map_r, 0, hh, tt, bb, bar_full);
+        tma_load_4d(smem_u32(TK), &map_k, 0, hh, tt, bb, bar_full);
+        tma_load_4d(smem_u32(TV), &map_v, 0, hh, tt, bb, bar_full);
+        tma_load_4d(smem_u32(TW), &map_w, 0, hh, tt, bb, bar_full);
+        tma_load_4d(smem_u32(TG), &map_g, 0, hh, tt, bb, bar_full);
+        tma_load_2d(smem_u32(TS), &map_s, 0, static_cast<int>((bh * (nch + 1) + cc) * kC), bar_full);
+        tma_load_2d(smem_u32(TDS), &map_ds, 0, static_cast<int>((bh * nch + cc) * kC), bar_full);
+    }
+    if (tid < 64) {
+        U[tid] = p.u[h * kN + tid];
+        RD[tid] = p.rowdot[(bh * nch + cc) * kN + tid];
+    }
+    int waited = 0;  // 1: copies landed; 2: first MMA group done; 3: second (for the drain)
+    int ok = bar_wait(bar_full, 0, limit);
+    int abort = __syncthreads_or(!ok);
+    if (!abort) {
+        waited = 1;
+        // ---------------------------------------------------------------- operand rows
+        const int a = warp, hf = lane >> 4, cq = lane & 15, t0h = 16 * a + 8 * hf;
+        const uint32_t cbyte = 8 * cq;
+        const Q4 u4 = ld_q4(U + 4 * cq);
+        Q4 w[8];
+        Q4 Gh = one4();
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int t = t0h + m;
+            if (t < tv) {
+                const Q4 x = unpack4(ld_u2(TW, swz(t, cbyte)));
+                w[m] = OMEGA ? decay4(x) : x;
+            } else {
+                w[m] = one4();
+            }
+            Gh = mul4(Gh, w[m]);
+        }
+        const Q4 Go = shfl_xor4(Gh, 16);
+        if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
+        __syncthreads();
+        Q4 D = one4(), before = one4(), aft = one4();
+#pragma unroll
+        for (int be = 0; be < 4; ++be) {
+            const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
+            D = mul4(D, g);
+            before = be < a ? mul4(before, g) : before;
+            aft = be > a ? mul4(aft, g) : aft;
+        }
+        // suffix products prod_{j>t} w_j of this half's tokens
+        Q4 suf[8];
+        {
+            Q4 run = mul4(aft, hf ? one4() : Go);
+#pragma unroll
+            for (int m = 7; m >= 0; --m) {
+                suf[m] = run;
+                run = mul4(run, w[m]);
+            }
+        }
+        Q4 pre = mul4(before, hf ? Go : one4());  // prod_{j<t} w_j
+        float pu[8], pd[8];
+#pragma unroll
+        for (int m = 0; m < 8; ++m) {
+            const int t = t0h + m;
+            const uint32_t off = swz(t, cbyte);
+            const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
+            const Q4 v = unpack4(ld_u2(TV, off)), g = unpack4(ld_u2(TG, off));
+            const Q4 qf = mul4(suf[m], w[m]);  // prod_{j>=t} w_j
+            st_u2(TQX, off, pack4({mul2(r.a, rcp2(qf.a)), mul2(r.b, rcp2(qf.b))}));
+            st_u2(TKH, off, pack4(mul4(k, suf[m])));
+            st_q4(PRE + t * kPreStride + 4 * cq, pre);
+            pu[m] = bonus4(r, u4, k);
+            pd[m] = dot4(g, v);
+            pre = mul4(pre, w[m]);
+        }
+        const float ub = half_sum8(pu, lane), dd = half_sum8(pd, lane);
+        if ((lane & 1) == 0) {
+            UB[t0h + ((lane >> 1) & 7)] = ub;
+            DD[t0h + ((lane >> 1) & 7)] = dd;
+        }
+        if (warp == 0 && hf == 0) {
+            st_q4(Dv + 4 * cq, D);
+            iDv[4 * cq] = 1.f / lo(D.a);
+            iDv[4 * cq + 1] = 1.f / hi(D.a);
+            iDv[4 * cq + 2] = 1.f / lo(D.b);
+            iDv[4 * cq + 3] = 1.f / hi(D.b);
+        }
+        __syncthreads();
+        // du share of this chunk: sum_t r_t k_t dd_t per channel
+        {
+            P2 acc0 = pk(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int t = t0h + m;
+                const uint32_t off = swz(t, cbyte);
+                const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
+                const P2 d2 = pk(DD[t], DD[t]);
+                acc0 = fma2(mul2(r.a, k.a), d2, acc0);
+                acc1 = fma2(mul2(r.b, k.b), d2, acc1);
+            }
+            Q4 acc = {acc0, acc1};
+            const Q4 oth = shfl_xor4(acc, 16);
+            acc = {pk(lo(acc.a) + lo(oth.a), hi(acc.a) + hi(oth.a)), pk(lo(acc.b) + lo(oth.b), hi(acc.b) + hi(oth.b))};
+            if (hf == 0) st_q4(DU + a * 64 + 4 * cq, acc);
+        }
+        // D (.) S_prev in place: row c of the state scaled by D[c]
+        {
+            const int c = tid >> 1, half = tid & 1;
+            const float d = Dv[c];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint4 *x = reinterpret_cast<uint4 *>(TS + swz(c, 64 * half + 16 * i));
+                float f[8];
+                unpack8(*x, f);
+                *x = make_uint4(pack_bf16(f[0] * d, f[1] * d), pack_bf16(f[2] * d, f[3] * d),
+                                pack_bf16(f[4] * d, f[5] * d), pack_bf16(f[6] * d, f[7] * d));
+            }
+        }
+        fence_async_smem();
+        fence_before();
+        __syncthreads();
+        fence_after();
+        if (tid < 64) p.du_item[(bh * nch + cc) * kN + tid] = DU[tid] + DU[64 + tid] + DU[128 + tid] + DU[192 + tid];
+        if (tid == 0) {
+            const uint32_t aR = smem_u32(TQX), aK = smem_u32(TKH), aV = smem_u32(TV), aG = smem_u32(TG);
+            const uint32_t aS = smem_u32(TS), aDS = smem_u32(TDS);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // A = Qx Kh^T
+                mma(tbase + T_A, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dA = dO V^T
+                mma(tbase + T_DA, desc_k(aG + 32 * ks), desc_k(aV + 32 * ks), idesc(64, 0, 0), ks > 0);
+            mma_commit(bar_m1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dR = dO (D S_prev)^T
+                mma(tbase + T_DR, desc_k(aG + 32 * ks), desc_k(aS + 32 * ks), idesc(64, 0, 0), ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dK = V dS_end^T
+                mma(tbase + T_DK, desc_k(aV + 32 * ks), desc_k(aDS + 32 * ks), idesc(64, 0, 0), ks > 0);
+        }
+        ok = bar_wait(bar_m1, 0, limit);
+        abort = __syncthreads_or(!ok);
+    }
+
+    // TMEM lane group of this warp: rows 16 warp .. + 15, columns [colh, colh + 32)
+    const int lr = lane & 15, hi = lane >> 4, t = 16 * warp + lr, colh = 32 * hi;
+    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * warp) << 16);
+    if (!abort) {
+        waited = 2;
+        fence_after();
+        // ------------------------------------------------------------ Am and dAm
+        float x[32];
+        tmem_ld32(tl + T_A, x);
+        const float ubt = UB[t];
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+            const int i = colh + n;
+            x[n] = i < t ? x[n] : (i == t ? ubt : 0.f);
+        }
+        st_row16_bf16(TAM, t, 2 * colh, *reinterpret_cast<float(*)[16]>(&x[0]));
+        st_row16_bf16(TAM, t, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&x[16]));
+        tmem_ld32(tl + T_DA, x);
+#pragma unroll
+        for (int n = 0; n < 32; ++n) x[n] = colh + n < t ? x[n] : 0.f;
+        st_row16_bf16(TDAM, t, 2 * colh, *reinterpret_cast<float(*)[16]>(&x[0]));
+        st_row16_bf16(TDAM, t, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&x[16]));
+        fence_async_smem();
+        fence_before();
+        __syncthreads();
+        fence_after();
+        if (tid == 0) {
+            const uint32_t aQ = smem_u32(TQX), aK = smem_u32(TKH), aG = smem_u32(TG), aDS = smem_u32(TDS);
+            const uint32_t aAm = smem_u32(TAM), aDAm = smem_u32(TDAM);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dR += dAm Kh
+                mma(tbase + T_DR, desc_k(aDAm + 32 * ks), desc_mn(aK + 2048 * ks), idesc(64, 0, 1), 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dK += dAm^T Qx
+                mma(tbase + T_DK, desc_mn(aDAm + 2048 * ks), desc_mn(aQ + 2048 * ks), idesc(64, 1, 1), 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dV = Am^T dO
+                mma(tbase + T_DV, desc_mn(aAm + 2048 * ks), desc_mn(aG + 2048 * ks), idesc(64, 1, 1), ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)  // dV += Kh dS_end
+                mma(tbase + T_DV, desc_k(aK + 32 * ks), desc_mn(aDS + 2048 * ks), idesc(64, 0, 1), 1);
+            mma_commit(bar_m2);
+        }
+        ok = bar_wait(bar_m2, 0, limit);
+        abort = __syncthreads_or(!ok);
+    }
+    if (!abort) {
+        waited = 3;
+        fence_after();
+        // ------------------------------------------------------------ gradients of row t
+        const bool valid = t < tv;
+        const int64_t go = ((b * p.T + t0 + t) * p.H + h) * kN + colh;
+        const float ddt = DD[t];
+        const float *pre = PRE + t * kPreStride + colh;
+        float x[32];
+        tmem_ld32(tl + T_DV, x);
+        if (valid) st_f32x32(p.dv + go, x);
+        float rdr[32], e[32];
+        tmem_ld32(tl + T_DR, x);
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+            float kk[8], qx[8];
+            ld_row8(TK, t, 2 * colh + 16 * g8, kk);
+            ld_row8(TQX, t, 2 * colh + 16 * g8, qx);
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8) {
+                const int n = 8 * g8 + e8, c = colh + n;
+                rdr[n] = qx[e8] * x[n];
+                x[n] = fmaf(x[n], pre[n] * iDv[c], U[c] * kk[e8] * ddt);
+            }
+        }
+        if (valid) st_f32x32(p.dr + go, x);
+        tmem_ld32(tl + T_DK, x);
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+            float rr[8], kh[8], wv[8];
+            ld_row8(TR, t, 2 * colh + 16 * g8, rr);
+            ld_row8(TKH, t, 2 * colh + 16 * g8, kh);
+            ld_row8(TW, t, 2 * colh + 16 * g8, wv);
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8) {
+                const int n = 8 * g8 + e8, c = colh + n;
+                const float wt = t < tv ? (OMEGA ? decay_of_logit(wv[e8]) : wv[e8]) : 1.f;
+                const float kf = Dv[c] * rcp_approx(pre[n] * wt);  // prod_{j>t} w_j
+                e[n] = rdr[n] - kh[e8] * x[n];
+                x[n] = fmaf(x[n], kf, U[c] * rr[e8] * ddt);
+            }
+        }
+        if (valid) st_f32x32(p.dk + go, x);
+        // d(log w_j) = sum_{t>=j} e_t - rdr_j + rowdot: suffix sums down the rows (columns are
+        // independent); rows 16 warp .. + 15 are the 16 lanes of each half-warp
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+            float s = e[n];
+#pragma unroll
+            for (int d = 1; d < 16; d <<= 1) {
+                const float y = __shfl_down_sync(0xffffffffu, s, d, 16);
+                if (lr + d < 16) s += y;
+            }
+            e[n] = s;
+        }
+        if (lr == 0)
+#pragma unroll
+            for (int n = 0; n < 32; ++n) Hs[warp * 64 + colh + n] = e[n];
+        __syncthreads();
+#pragma unroll
+        for (int n = 0; n < 32; ++n) {
+            float add = 0.f;
+            for (int q = warp + 1; q < 4; ++q) add += Hs[q * 64 + colh + n];
+            e[n] += add;
+        }
+#pragma unroll
+        for (int g8 = 0; g8 < 4; ++g8) {
+            float wv[8];
+            ld_row8(TW, t, 2 * colh + 16 * g8, wv);
+#pragma unroll
+            for (int e8 = 0; e8 < 8; ++e8) {
+                const int n = 8 * g8 + e8, c = colh + n;
+                const float dl = e[n] - rdr[n] + RD[c];
+                if (OMEGA)  // domega = -exp(omega) d(log w)
+                    x[n] = -ex2_approx(wv[e8] * 1.4426950408889634f) * dl;
+                else        // dw = d(log w) / w; w >= 2^-5 on this path
+                    x[n] = dl / wv[e8];
+            }
+        }
+        if (valid) st_f32x32(p.dw + go, x);
+    }
+    if (abort) {
+        record_status(p.status, kStatusTimeout);
+        if (tid == 0) {
+            if (waited < 1) bar_wait(bar_full, 0, limit);
+            if (waited == 1) bar_wait(bar_m1, 0, limit);
+            if (waited >= 1 && waited < 3) bar_wait(bar_m2, 0, limit);
+        }
+    }
+    fence_before();
+    __syncthreads();
+    fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(kChunkTmem));
+}
+
+cudaError_t configure_tc()
+{
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    for (auto kern : {wkv6_bwd_state_kernel<false, false>, wkv6_bwd_state_kernel<false, true>,
+                      wkv6_bwd_state_kernel<true, false>, wkv6_bwd_state_kernel<true, true>}) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+        if (e != cudaSuccess) return e;
+    }
+    for (auto kern : {wkv6_bwd_chunk_kernel<false>, wkv6_bwd_chunk_kernel<true>}) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kChunkSmem);
+        if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        if (e != cudaSuccess) return e;
+    }
+    done[dev] = true;
+    return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cudaStream_t s)
+{
+    const int64_t bh = a.B * a.H, nch = L.nch;
+    if (bh * nch > 0x7fffffffLL || bh * (nch + 1) * kC > 0x7fffffffLL || a.T > 0x7fffffffLL - kC)
+        return cudaErrorInvalidConfiguration;
+    unsigned char *ws = static_cast<unsigned char *>(a.workspace);
+    __nv_bfloat16 *sck = reinterpret_cast<__nv_bfloat16 *>(ws + L.sck);
+    __nv_bfloat16 *dsck = reinterpret_cast<__nv_bfloat16 *>(ws + L.dsck);
+    float *rowdot = reinterpret_cast<float *>(ws + L.rowdot);
+    float *du_item = reinterpret_cast<float *>(ws + L.du_item);
+    int *flags = reinterpret_cast<int *>(ws + L.flags);
+
+    CUtensorMap mr, mk, mv, mw, mg, ms, mds;
+    if (!make_map(&mr, a.r, a.B, a.T, a.H) || !make_map(&mk, a.k, a.B, a.T, a.H) ||
+        !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H) ||
+        !make_map(&mg, a.dy, a.B, a.T, a.H) || !make_rows_map(&ms, sck, bh * (nch + 1) * kC) ||
+        !make_rows_map(&mds, dsck, bh * nch * kC))
+        return cudaErrorInvalidValue;
+    cudaError_t e = configure_tc();
+    if (e != cudaSuccess) return e;
+    int *status = a.status;
+    const uint32_t spin = 100000u;
+    StateParams fw{a.T, a.H, static_cast<int>(nch), a.s0, sck, nullptr, nullptr, flags, nullptr, status, spin};
+    StateParams bw{a.T, a.H, static_cast<int>(nch), a.dsT, dsck, sck, rowdot, flags, a.ds0, status, spin};
+    GradParams gp{a.T, a.H, static_cast<int>(nch), a.u, rowdot, flags, a.dr, a.dk, a.dv, a.dw, du_item, status, spin};
+    const dim3 gs(static_cast<unsigned>(bh)), gc(static_cast<unsigned>(bh * nch));
+    if (a.omega) {
+        wkv6_bwd_state_kernel<false, true><<<gs, kSThreads, kStateSmem, s>>>(mk, mv, mw, fw);
+        wkv6_bwd_state_kernel<true, true><<<gs, kSThreads, kStateSmem, s>>>(mr, mg, mw, bw);
+        wkv6_bwd_chunk_kernel<true><<<gc, 128, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+    } else {
+        wkv6_bwd_state_kernel<false, false><<<gs, kSThreads, kStateSmem, s>>>(mk, mv, mw, fw);
+        wkv6_bwd_state_kernel<true, false><<<gs, kSThreads, kStateSmem, s>>>(mr, mg, mw, bw);
+        wkv6_bwd_chunk_kernel<false><<<gc, 128, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace wkv

@@ -808,6 +808,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 
 // ---------------------------------------------------------------------------- host side
 
+}  // namespace
+
 // [B, T, H, N] bf16, box = 64 channels x 1 head x 64 tokens x 1 batch row
 bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t H)
 {
@@ -825,7 +827,20 @@ bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t 
     return r == CUDA_SUCCESS;
 }
 
-}  // namespace
+// rows x 64 bf16 (128-byte rows), box = 64 rows, 128-byte swizzle
+bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc || rows <= 0 || rows > 0x7fffffffLL) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(kN), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(kN * 2)};
+    cuuint32_t box[2] = {kN, 64};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
 
 // cuTensorMapEncodeTiled, looked up once through the runtime (no link-time driver dependency)
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()

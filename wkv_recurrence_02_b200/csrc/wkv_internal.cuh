@@ -62,13 +62,39 @@ struct Wkv6BwdArgs {
     float *ds0;                 // [B,H,N,N] or null
     void *workspace;            // wkv6_backward_workspace_bytes(B, T, H) bytes, 16-byte aligned
     bool bf16, omega;
+    bool chunked = false;       // bf16 only: the tensor-core chunked backward (else the fp32 walks)
+    int *status = nullptr;      // device status word (bounded waits that ran out)
 };
+
+// Byte layout of the backward workspace, shared by both backward paths.  The region at
+// offset 0 holds either the fp32 walks' state checkpoints (one every 8 tokens) or the
+// chunked path's bf16 checkpoints (state before each 64-token chunk and after the last,
+// state gradient after each chunk) and its per-chunk row-dot terms; the walks run after
+// the chunked kernels have finished with it (they serve the sequences the chunked path
+// leaves to them).
+struct BwdLayout {
+    int64_t nch;                       // 64-token chunks
+    size_t sck, dsck, rowdot;          // chunked: checkpoints and row dots (inside region 0)
+    size_t du_part, du_item, flags;    // walks' du per (b, h); chunked du per (b, h, chunk); flags
+    size_t total;
+};
+BwdLayout wkv6_backward_layout(int64_t B, int64_t T, int64_t H);
+cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cudaStream_t s);
+// The fp32 walks; with `only` non-null they serve only the (b, h) whose flag is set.
+cudaError_t wkv6_backward_walks_launch(const Wkv6BwdArgs &a, const BwdLayout &L, const int *only,
+                                       cudaStream_t s);
 
 size_t wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H);
 cudaError_t wkv6_backward_launch(const Wkv6BwdArgs &a, cudaStream_t s);
 
 // cuTensorMapEncodeTiled from the driver (null if unavailable).
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder();
+
+// TMA tensor maps with the 128-byte swizzle, for bf16 tiles of 64 rows x 64 channels:
+//   make_map:      a [B, T, H, 64] tensor, box = 64 tokens of one (b, h);
+//   make_rows_map: a [rows, 64] array, box = 64 consecutive rows.
+bool make_map(CUtensorMap *map, const void *base, int64_t B, int64_t T, int64_t H);
+bool make_rows_map(CUtensorMap *map, const void *base, int64_t rows);
 
 // Each launcher returns the cudaError_t of its launch(es).
 cudaError_t wkv4_launch(const Wkv4Args &a, cudaStream_t s);

@@ -273,13 +273,16 @@ def wkv6_backward_workspace_bytes(B, T, H, N=64) -> int:
     return int(out.value)
 
 
-def wkv6_backward(r, k, v, w, u, dy, s0=None, dsT=None, omega=False, want_ds0=True, workspace=None):
+def wkv6_backward(r, k, v, w, u, dy, s0=None, dsT=None, omega=False, want_ds0=True, workspace=None,
+                  algo=None):
     """WKV-6 backward: gradients of a loss with dL/dy = dy and dL/dsT = dsT (None = 0).
 
     r,k,v,w,dy: [B,T,H,N] fp32|bf16 (with omega=True, w holds omega_t and bf16 is required);
     u: [H,N] fp32; s0, dsT: [B,H,N,N] fp32.  Returns a dict of fp32 tensors dr, dk, dv,
     dw (or domega), du, and ds0 (when want_ds0).  workspace: optional uint8 CUDA tensor of at
     least wkv6_backward_workspace_bytes bytes; allocated here when not given.
+    algo: None (library default: bf16 inputs take the chunked tensor-core path), "auto",
+    "serial" (the exact fp32 walks) or "chunked" (this call only).
     """
     lib = load()
     _cuda(r, "r")
@@ -307,9 +310,17 @@ def wkv6_backward(r, k, v, w, u, dy, s0=None, dsT=None, omega=False, want_ds0=Tr
     _use_current_stream(lib, dev)
     fn = (lib.rwkv_wkv6_backward_omega_bf16 if omega else
           lib.rwkv_wkv6_backward_bf16 if dt == torch.bfloat16 else lib.rwkv_wkv6_backward)
-    _check(fn(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(dy), _ptr(dsT),
-              _ptr(out["dr"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out[dwn]), _ptr(out["du"]),
-              _ptr(out["ds0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel())))
+    prev = None
+    if algo is not None:
+        prev = lib.rwkv_get_wkv6_algo()
+        _check(lib.rwkv_set_wkv6_algo(ALGOS[algo]))
+    try:
+        _check(fn(B, T, H, N, _ptr(r), _ptr(k), _ptr(v), _ptr(w), _ptr(u), _ptr(s0), _ptr(dy), _ptr(dsT),
+                  _ptr(out["dr"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out[dwn]), _ptr(out["du"]),
+                  _ptr(out["ds0"]), _ptr(workspace), ctypes.c_size_t(workspace.numel())))
+    finally:
+        if prev is not None:
+            lib.rwkv_set_wkv6_algo(prev)
     if not want_ds0:
         del out["ds0"]
     return out
