@@ -64,8 +64,6 @@ BYTES = {
 
 NOMINAL_HBM_GBS = 8000.0  # the 8 TB/s denominator the workload's roofline is stated against
 
-# fp32 FMA peak of the CUDA cores: 148 SMs x 128 FMA per clock x 2 flops x 1.965 GHz
-SIMT_FP32_TFLOPS = round(148 * 128 * 2 * 1.965e9 / 1e12, 2)
 
 
 def load_peaks():
@@ -351,7 +349,8 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
         fused into the chunked kernel's epilogue, against the same call without it;
       * the Finch prefill fed the decay logit omega_t (w_t = exp(-exp(omega_t)) formed in
         the kernel), plain and with the fused output stage;
-      * the WKV-6 backward pass at the Finch shape."""
+      * the WKV-6 backward pass at the Finch shape (the chunked tensor-core path, with the
+        exact fp32 walks timed beside it)."""
     hbm, _ = load_peaks()
     rows = {}
     f = wl.finch
@@ -384,24 +383,34 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
         "frac_hbm": round(nb / (omega * 1e-6) / 1e9 / hbm, 4),
         "separate_map_floor_us": round(2 * om.numel() * 2 / (hbm * 1e9) * 1e6, 2)}
     del om
-    # WKV-6 backward at the Finch shape (fp32 gradients; SIMT kernels)
+    # WKV-6 backward at the Finch shape (fp32 gradients): the chunked tensor-core path (the
+    # default for bf16 inputs), against the HBM roofline of its algorithmic bytes; the exact
+    # fp32 walks timed beside it
     gen.manual_seed(8)
     dy = (torch.randn(8, 4096, 32, 64, device=dev, generator=gen)).to(torch.bfloat16)
     dsT = torch.randn(8, 32, 64, 64, device=dev, generator=gen) * 0.1
     ws = torch.empty(ops.wkv6_backward_workspace_bytes(8, 4096, 32), device=dev, dtype=torch.uint8)
-    bwd_ms = _time_us(torch, stream, dev, lambda: ops.wkv6_backward(
-        f["r"], f["k"], f["v"], f["w"], f["u"], dy, s0=f["s0"], dsT=dsT, workspace=ws), 3) / 1e3
+
+    def bwd(algo):
+        return lambda: ops.wkv6_backward(f["r"], f["k"], f["v"], f["w"], f["u"], dy, s0=f["s0"], dsT=dsT,
+                                         workspace=ws, algo=algo)
+    bwd_ms = _time_us(torch, stream, dev, bwd("chunked"), 10) / 1e3
+    walks_ms = _time_us(torch, stream, dev, bwd("serial"), 2) / 1e3
     n_el, n_st = dy.numel(), dsT.numel()
+    # r, k, v, w, dy in bf16; dr, dk, dv, dw in fp32; s0, dsT, ds0; u and du
     bwd_bytes = 5 * n_el * 2 + 4 * n_el * 4 + 3 * n_st * 4 + 2 * 32 * 64 * 4
-    bwd_flops = 2 * 6 * 64 * n_el  # six 64-term products per token and channel, 2 flops per FMA
-    alu_peak = SIMT_FP32_TFLOPS
+    # tensor work: 24 products of 64 x 64 x 64 per chunk (A, dA, dR, dK, dV: 5 pairs of 4, dR/dK
+    # second halves 2 x 4) and 4 per chunk in each state pass
+    n_chunks = 8 * 32 * (4096 // 64)
+    bwd_flops = (24 + 8) * 2 * 64 * 16 * 64 * n_chunks
+    gbs = bwd_bytes / (bwd_ms * 1e-3) / 1e9
     rows["wkv6_finch_backward_B8_T4096_H32"] = {
-        "avg_ms": round(bwd_ms, 3), "algorithmic_bytes": bwd_bytes, "algorithmic_flops": bwd_flops,
-        "GBps": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
-        "TFLOPs": round(bwd_flops / (bwd_ms * 1e-3) / 1e12, 2),
-        "bound": "alu", "peak_tflops_fp32_simt": alu_peak,
-        "frac_alu": round(bwd_flops / (bwd_ms * 1e-3) / 1e12 / alu_peak, 4),
-        "workspace_bytes": ws.numel(), "launches_per_call": 4}
+        "avg_ms": round(bwd_ms, 3), "path": "chunked tensor-core (bf16 operands, fp32 accumulation)",
+        "algorithmic_bytes": bwd_bytes, "GBps": round(gbs, 1), "bound": "hbm", "peak_gbs": hbm,
+        "frac_hbm": round(gbs / hbm, 4), "frac_8TBps": round(gbs / NOMINAL_HBM_GBS, 4),
+        "tensor_tflops": round(bwd_flops / (bwd_ms * 1e-3) / 1e12, 2),
+        "exact_walks_avg_ms": round(walks_ms, 3),
+        "workspace_bytes": ws.numel(), "launches_per_call": 7}
     del dy, dsT, ws
     B, C = 2048, 4096
     x = inputs.wkv4_inputs(B, 1, C, "bf16", seed=5, wu_seed=6)

@@ -185,14 +185,27 @@ int rwkv_wkv6_forward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
  * Inputs r, k, v, w (or omega), u, s0 are those of the forward call; the forward states
  * are recomputed, not read.
  *   workspace : device scratch owned by the caller, 16-byte aligned, of at least the size
- *               rwkv_wkv6_backward_workspace_bytes reports (B*H*(ceil(T/8)*N*N + N)*4 bytes:
- *               a checkpoint of the state every 8 tokens); it must not overlap any tensor.
- *               A smaller workspace_bytes is refused with RWKV_ERR_ARG before any launch.
- * Runs on CUDA cores in fp32 (four launches: a forward pass for dr, du and the
- * checkpoints; a backward pass over state rows for dk, dw; one over state columns for
- * dv, ds0; the sum of du over b).  N must be 64.  T = 0 writes du = 0 and ds0 = dsT.
- * Aliasing: no output may overlap an input, the workspace or another output (except
- * ds0 == dsT).  Other rules and errors as rwkv_wkv6_forward. */
+ *               rwkv_wkv6_backward_workspace_bytes reports (about B*H*ceil(T/8)*N*N*4 bytes:
+ *               room for an fp32 checkpoint of the state every 8 tokens, which the exact
+ *               walks below use; the chunked path needs about an eighth of it); it must not
+ *               overlap any tensor.  A smaller workspace_bytes is refused with RWKV_ERR_ARG
+ *               before any launch.  Its contents need no initialisation and are undefined
+ *               after the call.
+ * Two paths (rwkv_set_wkv6_algo on the calling thread chooses):
+ *   - bf16 inputs (default, and RWKV_WKV6_AUTO / RWKV_WKV6_CHUNKED): the chunked tensor-core
+ *     path in 64-token chunks -- a pass over the chunks for the state entering each chunk
+ *     (kept in bf16), a reverse pass for the state gradient leaving each chunk, and one
+ *     kernel over all (b, h, chunk) at once for the gradients, with bf16 MMA operands and
+ *     fp32 accumulation (results within the bf16 tolerance of the exact gradient).  A (b, h)
+ *     sequence with a channel whose 64-token decay product falls below 2^-100, or (w input)
+ *     with a w below 2^-5, is served by the exact walks instead, inside the same call.
+ *   - fp32 inputs, or RWKV_WKV6_SERIAL: the exact walks on CUDA cores in fp32 (a forward
+ *     pass for dr, du and the checkpoints; a backward pass over state rows for dk, dw; one
+ *     over state columns for dv, ds0).
+ * du is summed over the batch rows (and chunks) in a fixed order: results are deterministic.
+ * N must be 64.  T = 0 writes du = 0 and ds0 = dsT.  Aliasing: no output may overlap an
+ * input, the workspace or another output (except ds0 == dsT).  Other rules and errors as
+ * rwkv_wkv6_forward. */
 int rwkv_wkv6_backward_workspace_bytes(int64_t B, int64_t T, int64_t H, int64_t N, size_t *bytes);
 int rwkv_wkv6_backward(int64_t B, int64_t T, int64_t H, int64_t N,
                        const float *r, const float *k, const float *v, const float *w,
@@ -213,8 +226,9 @@ int rwkv_wkv6_backward_omega_bf16(int64_t B, int64_t T, int64_t H, int64_t N,
                                   float *ds0, void *workspace, size_t workspace_bytes);
 
 /* Kernel choice for WKV-6 on the calling thread: RWKV_WKV6_AUTO (default, as above),
- * RWKV_WKV6_SERIAL (always the serial kernel), RWKV_WKV6_CHUNKED (the chunked kernel
- * for bf16 whatever T; ignored for fp32).  Returns RWKV_OK or RWKV_ERR_ARG. */
+ * RWKV_WKV6_SERIAL (always the serial kernel; the backward takes the exact fp32 walks),
+ * RWKV_WKV6_CHUNKED (the chunked kernel for bf16 whatever T; ignored for fp32).  Returns
+ * RWKV_OK or RWKV_ERR_ARG. */
 #define RWKV_WKV6_AUTO 0
 #define RWKV_WKV6_SERIAL 1
 #define RWKV_WKV6_CHUNKED 2

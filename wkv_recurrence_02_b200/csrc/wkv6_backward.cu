@@ -449,29 +449,40 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     }
 }
 
-// du[h][i] = sum over batch rows b, in order of b, of the (b, h) sequence's share: du_part[b][h][i]
-// from the walks, or, where the chunked path served the sequence (flags given and the
-// sequence's flag clear), the sum over its chunks of du_item[b][h][c][i] in order of c.
-// Fixed order throughout: deterministic.
-__global__ void __launch_bounds__(kN) wkv6_bwd_du_kernel(int64_t B, int64_t H, int64_t nch,
-                                                        const float *__restrict__ du_part,
-                                                        const float *__restrict__ du_item,
-                                                        const int *__restrict__ flags, float *__restrict__ du)
+// du[h][i] = the sum over batch rows b of the (b, h) sequence's share: du_part[b][h][i] from
+// the walks, or, where the chunked path served the sequence (flags given and the sequence's
+// flag clear), its chunks' du_item[b][h][c][i].  Four threads per channel each sum a fixed
+// quarter of the terms (chunks c = q mod 4) in order of (b, c), and the quarters are added in
+// order: the result is deterministic.
+constexpr int kDuParts = 4;
+__global__ void __launch_bounds__(kN * kDuParts) wkv6_bwd_du_kernel(int64_t B, int64_t H, int64_t nch,
+                                                                   const float *__restrict__ du_part,
+                                                                   const float *__restrict__ du_item,
+                                                                   const int *__restrict__ flags,
+                                                                   float *__restrict__ du)
 {
+    __shared__ float part[kDuParts][kN];
     const int64_t h = blockIdx.x;
-    const int i = threadIdx.x;
+    const int i = threadIdx.x % kN, q = threadIdx.x / kN;
     float acc = 0.f;
     for (int64_t b = 0; b < B; ++b) {
         const int64_t n = b * H + h;
         if (!flags || flags[n]) {
-            acc += du_part[n * kN + i];
+            if (q == 0) acc += du_part[n * kN + i];
         } else {
-            float part = 0.f;
-            for (int64_t c = 0; c < nch; ++c) part += du_item[(n * nch + c) * kN + i];
-            acc += part;
+            const float *src = du_item + n * nch * kN + i;
+#pragma unroll 4
+            for (int64_t c = q; c < nch; c += kDuParts) acc += src[c * kN];
         }
     }
-    du[h * kN + i] = acc;
+    part[q][i] = acc;
+    __syncthreads();
+    if (q == 0) {
+        float s = part[0][i];
+#pragma unroll
+        for (int j = 1; j < kDuParts; ++j) s += part[j][i];
+        du[h * kN + i] = s;
+    }
 }
 
 // threads per row (column) of each kernel: the row walk backwards keeps a stash of kBlock
@@ -592,7 +603,7 @@ cudaError_t wkv6_backward_launch(const Wkv6BwdArgs &a, cudaStream_t s)
     }
     e = wkv6_backward_walks_launch(a, L, flags, s);
     if (e != cudaSuccess) return e;
-    wkv6_bwd_du_kernel<<<static_cast<unsigned>(a.H), kN, 0, s>>>(
+    wkv6_bwd_du_kernel<<<static_cast<unsigned>(a.H), kN * kDuParts, 0, s>>>(
         a.B, a.H, L.nch, reinterpret_cast<const float *>(ws + L.du_part),
         reinterpret_cast<const float *>(ws + L.du_item), flags, a.du);
     return cudaGetLastError();

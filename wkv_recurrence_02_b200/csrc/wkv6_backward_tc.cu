@@ -114,25 +114,33 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16 *dst, const float (&v)[
 }
 
 // ================================================================ state passes (K0 / K1)
-// 128 threads = 4 warps.  Warp a prepares the operand rows of 16-token sub-block a (lane:
-// 8-token half hf, channel quad cq); the same warp then serves TMEM lanes 32a.. of the state
-// (rows 16a .. 16a + 15, two 32-column halves).  One elected thread issues the TMA copies
-// (a 3-stage ring of X | Y | W tiles) and the four MMAs per chunk.
-constexpr int kSThreads = 128;
+// 256 threads = 8 warps in two groups.
+//   prep group (warps 0-3): warp a builds the operand rows of 16-token sub-block a (lane:
+//     8-token half hf, channel quad cq) and the chunk decay D, running ahead of the state;
+//   state group (warps 4-7): warp 4 + q serves TMEM lanes 32q.. of the state (rows 16q .. +
+//     15, two 32-column halves): per chunk it writes the checkpoint, scales the state by D
+//     and has one elected thread issue the four MMAs of the update; another elected thread
+//     of the group issues the TMA copies of later chunks (a 3-stage ring of X | Y | W tiles,
+//     and for the backward pass the forward checkpoint after the chunk, for the row dots).
+// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> state group), update
+// done (MMA commit -> state group; it also frees the stage of that chunk).
+constexpr int kSThreads = 256;
 constexpr int kSStages = 3;
-constexpr int kSStage = 3 * kTile;                     // X | Y | W
-constexpr int S_H = kSStages * kSStage;                // [4][64] sub-block decay products
-constexpr int S_D = S_H + 4 * 64 * 4;                  // [stage][64] chunk decay
-constexpr int S_BAR = S_D + kSStages * 64 * 4;         // full[3], mma
-constexpr int S_MISC = S_BAR + 64;                     // TMEM base
-constexpr int kStateSmem = S_MISC + 64 + 1024;
+template <bool REV> struct StateLayout {
+    static constexpr int tiles = REV ? 4 : 3;                    // X | Y | W (| S_end)
+    static constexpr int stage = tiles * kTile;
+    static constexpr int hs = kSStages * stage;                  // [4][64] sub-block decay products
+    static constexpr int dv = hs + 4 * 64 * 4;                   // [stage][64] chunk decay
+    static constexpr int bar = dv + kSStages * 64 * 4;           // full[3], prep[3], mma
+    static constexpr int misc = bar + 64;                        // TMEM base, abort flag
+    static constexpr int smem = misc + 64 + 1024;
+};
 
 struct StateParams {
     int64_t T, H;
     int nch;
     const float *init;            // [bh][N][N] fp32: s0 (forward) or dsT (backward); null = 0
     __nv_bfloat16 *ck;            // forward: [bh][nch + 1][N][N]; backward: [bh][nch][N][N]
-    const __nv_bfloat16 *sck;     // backward: the forward checkpoints (for the row dots)
     float *rowdot;                // backward: [bh][nch][N]
     int *flags;                   // forward: written; backward: read (flagged sequences skipped)
     float *fin;                   // backward: ds0 [bh][N][N] fp32, or null
@@ -143,31 +151,39 @@ struct StateParams {
 // REV = false: S <- diag(D) S + Kh^T V over chunks 0..nch-1 (X = k, Y = v), writing the state
 //              entering each chunk and the final state.
 // REV = true:  dS <- diag(D) dS + Qi^T dO over chunks nch-1..0 (X = r, Y = dO), writing the
-//              state gradient leaving each chunk, its row dot with the state there, and ds0.
+//              state gradient leaving each chunk, its row dot with the forward state there
+//              (map_e: the forward checkpoints), and ds0.
 template <bool REV, bool OMEGA>
 __global__ void __launch_bounds__(kSThreads)
 wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_y,
-                      const __grid_constant__ CUtensorMap map_w, const StateParams p)
+                      const __grid_constant__ CUtensorMap map_w, const __grid_constant__ CUtensorMap map_e,
+                      const StateParams p)
 {
+    using L = StateLayout<REV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
-    float *Hs = reinterpret_cast<float *>(sm + S_H);
-    float *Dv = reinterpret_cast<float *>(sm + S_D);
-    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + S_BAR);
-    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + S_MISC);
-    const uint32_t bar_full0 = smem_u32(&bars[0]), bar_mma = smem_u32(&bars[kSStages]);
+    float *Hs = reinterpret_cast<float *>(sm + L::hs);
+    float *Dv = reinterpret_cast<float *>(sm + L::dv);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar);
+    volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + L::misc);
+    const uint32_t bar_full0 = smem_u32(&bars[0]), bar_prep0 = smem_u32(&bars[kSStages]);
+    const uint32_t bar_mma = smem_u32(&bars[2 * kSStages]);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
     const int nch = p.nch;
     const int nck = REV ? nch : nch + 1;
-    const uint32_t limit = p.spin_limit;
+    const uint32_t limit = p.spin_limit, spin = p.spin_limit * 64u;
     if (REV && p.flags[bh]) return;  // served by the exact walks
 
     if (tid == 0) {
-        for (int s = 0; s < kSStages; ++s) bar_init(bar_full0 + 8 * s, 1);
+        for (int s = 0; s < kSStages; ++s) {
+            bar_init(bar_full0 + 8 * s, 1);
+            bar_init(bar_prep0 + 8 * s, 128);
+        }
         bar_init(bar_mma, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        misc[1] = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
@@ -180,119 +196,137 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
     fence_after();
     const uint32_t tbase = misc[0];
 
-    int issued = 0, committed = 0;  // meaningful in thread 0
-    auto issue = [&](int n) {
+    auto issue = [&](int n) {  // TMA of processing step n (one thread)
         const int cc = REV ? nch - 1 - n : n;
         const int s = n % kSStages;
-        const uint32_t dst = smem_u32(sm + s * kSStage), bar = bar_full0 + 8 * s;
-        bar_expect_tx(bar, kSStage);
+        const uint32_t dst = smem_u32(sm + s * L::stage), bar = bar_full0 + 8 * s;
+        bar_expect_tx(bar, L::stage);
         tma_load_4d(dst, &map_x, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
         tma_load_4d(dst + kTile, &map_y, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
         tma_load_4d(dst + 2 * kTile, &map_w, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
+        if (REV)  // the forward state after chunk cc
+            tma_load_2d(dst + 3 * kTile, &map_e, 0, static_cast<int>((bh * (nch + 1) + cc + 1) * kC), bar);
     };
-    if (tid == 0)
+    const int issuer_tma = tid == 128 + 32;  // warp 5
+    int issued = 0, committed = 0;           // meaningful in the issuing threads
+    if (issuer_tma)
         for (; issued < kSStages && issued < nch; ++issued) issue(issued);
 
-    // TMEM lane group of this warp: rows 16 warp .. + 15, columns [colh, colh + 32)
-    const int lr = lane & 15, hi = lane >> 4, row = 16 * warp + lr, colh = 32 * hi;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * warp) << 16);
-    {
-        float v[32];
-        if (p.init) {
-            const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const float4 x = src[i];
-                v[4 * i] = x.x, v[4 * i + 1] = x.y, v[4 * i + 2] = x.z, v[4 * i + 3] = x.w;
+    int abort = 0, hazard = 0;
+    if (warp < 4) {
+        // =============================== prep group ===============================
+        const int a = warp, hf = lane >> 4, cq = lane & 15, t0h = 16 * a + 8 * hf;
+        const uint32_t cbyte = 8 * cq;
+        for (int n = 0; n < nch; ++n) {
+            const int cc = REV ? nch - 1 - n : n;
+            const int s = n % kSStages;
+            unsigned char *st = sm + s * L::stage;
+            const int64_t t0 = static_cast<int64_t>(cc) * kC;
+            const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+            const int ok = tid == 0 ? bar_wait_spin(bar_full0 + 8 * s, (n / kSStages) & 1, spin) : 1;
+            if (named_sync_or(1, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
             }
-        } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.f;
-        }
-        tmem_st32(tl, v);
-    }
-
-    // prep lanes: warp a = 16-token sub-block, hf = 8-token half, cq = channel quad
-    const int a = warp, hf = lane >> 4, cq = lane & 15, t0h = 16 * a + 8 * hf;
-    const uint32_t cbyte = 8 * cq;
-    int hazard = 0, abort = 0;
-    for (int n = 0; n < nch; ++n) {
-        const int cc = REV ? nch - 1 - n : n;
-        const int s = n % kSStages;
-        unsigned char *st = sm + s * kSStage;
-        const int64_t t0 = static_cast<int64_t>(cc) * kC;
-        const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
-        int ok = bar_wait(bar_full0 + 8 * s, (n / kSStages) & 1, limit);
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
-        // decays of this half (1 past the end) and their products
-        Q4 w[8];
-        Q4 Gh = one4();
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int t = t0h + m;
-            if (t < tv) {
-                const Q4 x = unpack4(ld_u2(st + 2 * kTile, swz(t, cbyte)));
-                w[m] = OMEGA ? decay4(x) : x;
-                if (!REV && !OMEGA) hazard |= any_below(w[m], kWMin);
-            } else {
-                w[m] = one4();
-            }
-            Gh = mul4(Gh, w[m]);
-        }
-        const Q4 Go = shfl_xor4(Gh, 16);
-        if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
-        __syncthreads();
-        Q4 D = one4(), before = one4(), aft = one4();
-#pragma unroll
-        for (int be = 0; be < 4; ++be) {
-            const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
-            D = mul4(D, g);
-            before = be < a ? mul4(before, g) : before;
-            aft = be > a ? mul4(aft, g) : aft;
-        }
-        if (!REV) hazard |= any_below(D, kFastMin);
-        if (!REV) {  // Kh[i] = k_i prod_{j>i} w_j (chunk-end reference, every factor <= 1)
-            Q4 run = mul4(aft, hf ? one4() : Go);
-#pragma unroll
-            for (int m = 7; m >= 0; --m) {
-                const uint32_t off = swz(t0h + m, cbyte);
-                st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
-                run = mul4(run, w[m]);
-            }
-        } else {     // Qi[t] = r_t prod_{j<t} w_j (chunk-start reference, every factor <= 1)
-            Q4 run = mul4(before, hf ? Go : one4());
+            bar_try(bar_full0 + 8 * s, (n / kSStages) & 1);
+            Q4 w[8];
+            Q4 Gh = one4();
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
-                const uint32_t off = swz(t0h + m, cbyte);
-                st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
-                run = mul4(run, w[m]);
+                const int t = t0h + m;
+                if (t < tv) {
+                    const Q4 x = unpack4(ld_u2(st + 2 * kTile, swz(t, cbyte)));
+                    w[m] = OMEGA ? decay4(x) : x;
+                    if (!REV && !OMEGA) hazard |= any_below(w[m], kWMin);
+                } else {
+                    w[m] = one4();
+                }
+                Gh = mul4(Gh, w[m]);
             }
+            const Q4 Go = shfl_xor4(Gh, 16);
+            if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
+            named_sync_or(1, 128, 0);
+            Q4 D = one4(), before = one4(), aft = one4();
+#pragma unroll
+            for (int be = 0; be < 4; ++be) {
+                const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
+                D = mul4(D, g);
+                before = be < a ? mul4(before, g) : before;
+                aft = be > a ? mul4(aft, g) : aft;
+            }
+            if (!REV) hazard |= any_below(D, kFastMin);
+            if (!REV) {  // Kh[i] = k_i prod_{j>i} w_j (chunk-end reference, every factor <= 1)
+                Q4 run = mul4(aft, hf ? one4() : Go);
+#pragma unroll
+                for (int m = 7; m >= 0; --m) {
+                    const uint32_t off = swz(t0h + m, cbyte);
+                    st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
+                    run = mul4(run, w[m]);
+                }
+            } else {     // Qi[t] = r_t prod_{j<t} w_j (chunk-start reference, every factor <= 1)
+                Q4 run = mul4(before, hf ? Go : one4());
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const uint32_t off = swz(t0h + m, cbyte);
+                    st_u2(st, off, pack4(mul4(unpack4(ld_u2(st, off)), run)));
+                    run = mul4(run, w[m]);
+                }
+            }
+            if (warp == 0 && hf == 0) st_q4(Dv + s * 64 + 4 * cq, D);
+            // the sub-block products are read again for the next chunk only after every warp
+            // of the group has passed this chunk's first barrier
+            fence_async_smem();
+            bar_arrive(bar_prep0 + 8 * s);
         }
-        if (warp == 0 && hf == 0) st_q4(Dv + s * 64 + 4 * cq, D);
-        fence_async_smem();
-        // the previous chunk's update must be complete before the state is read
-        ok = n > 0 ? bar_wait(bar_mma, (n - 1) & 1, limit) : 1;
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
-        if (tid == 0 && n > 0 && issued < nch) issue(issued++);  // the stage of chunk n - 1 is free
-        fence_after();
+    } else {
+        // =============================== state group ===============================
+        const int q = warp - 4, lr = lane & 15, hi = lane >> 4, row = 16 * q + lr, colh = 32 * hi;
+        const uint32_t tl = tbase + (static_cast<uint32_t>(32 * q) << 16);
+        const bool issuer_mma = tid == 128;
         {
+            float v[32];
+            if (p.init) {
+                const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float4 x = src[i];
+                    v[4 * i] = x.x, v[4 * i + 1] = x.y, v[4 * i + 2] = x.z, v[4 * i + 3] = x.w;
+                }
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            }
+            tmem_st32(tl, v);
+        }
+        for (int n = 0; n < nch; ++n) {
+            const int cc = REV ? nch - 1 - n : n;
+            const int s = n % kSStages;
+            unsigned char *st = sm + s * L::stage;
+            int ok = 1;
+            if (issuer_mma) {
+                ok = bar_wait_spin(bar_prep0 + 8 * s, (n / kSStages) & 1, spin);
+                if (ok && n > 0) ok = bar_wait_spin(bar_mma, (n - 1) & 1, spin);
+            }
+            if (named_sync_or(2, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
+            }
+            bar_try(bar_prep0 + 8 * s, (n / kSStages) & 1);
+            if (n > 0) bar_try(bar_mma, (n - 1) & 1);
+            fence_after();
+            // the stage of step n - 1 is free once its update is done: refill it
+            if (issuer_tma && n > 0 && issued < nch) issue(issued++);
             float v[32];
             tmem_ld32(tl, v);
             st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, v);
-            if (REV) {  // rowdot(dS_end, S_end), S_end = the forward checkpoint after chunk cc
-                const uint4 *src = reinterpret_cast<const uint4 *>(
-                    p.sck + ((bh * (nch + 1) + cc + 1) * kN + row) * kN + colh);
+            if (REV) {  // rowdot(dS_end, S_end): S_end = the forward state after chunk cc
                 float part = 0.f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     float x[8];
-                    unpack8(src[i], x);
+                    ld_row8(st + 3 * kTile, row, 2 * colh + 16 * i, x);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) part = fmaf(v[8 * i + e], x[e], part);
                 }
@@ -303,43 +337,48 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
 #pragma unroll
             for (int i = 0; i < 32; ++i) v[i] *= d;
             tmem_st32(tl, v);
-        }
-        fence_before();
-        __syncthreads();
-        fence_after();
-        if (tid == 0) {
-            const uint32_t aX = smem_u32(st), aY = smem_u32(st + kTile);
+            fence_before();
+            named_sync_or(2, 128, 0);
+            fence_after();
+            if (issuer_mma) {
+                const uint32_t aX = smem_u32(st), aY = smem_u32(st + kTile);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma(tbase, desc_mn(aX + 2048 * ks), desc_mn(aY + 2048 * ks), idesc(64, 1, 1), 1);
-            mma_commit(bar_mma);
-            ++committed;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma(tbase, desc_mn(aX + 2048 * ks), desc_mn(aY + 2048 * ks), idesc(64, 1, 1), 1);
+                mma_commit(bar_mma);
+                ++committed;
+            }
+        }
+        if (!abort) {
+            const int ok = issuer_mma ? bar_wait_spin(bar_mma, (nch - 1) & 1, spin) : 1;
+            if (named_sync_or(2, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+            } else {
+                bar_try(bar_mma, (nch - 1) & 1);
+                fence_after();
+                float v[32];
+                tmem_ld32(tl, v);
+                if (!REV)
+                    st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, v);
+                else if (p.fin)
+                    st_f32x32(p.fin + (bh * kN + row) * kN + colh, v);
+            }
         }
     }
-    if (!abort) {
-        const int ok = bar_wait(bar_mma, (nch - 1) & 1, limit);
-        abort = __syncthreads_or(!ok);
-    }
-    if (!abort) {
-        fence_after();
-        float v[32];
-        tmem_ld32(tl, v);
-        if (!REV)
-            st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, v);
-        else if (p.fin)
-            st_f32x32(p.fin + (bh * kN + row) * kN + colh, v);
-    }
+    fence_before();
+    abort = __syncthreads_or(abort | misc[1]);
+    fence_after();
     if (!REV) {
         const int hz = __syncthreads_or(hazard);
-        if (tid == 0) p.flags[bh] = hz;
+        if (tid == 0 && !abort) p.flags[bh] = hz;
     }
     if (abort) {
         record_status(p.status, kStatusTimeout);
-        if (tid == 0) {
+        if (issuer_tma)
             for (int n = issued - kSStages < 0 ? 0 : issued - kSStages; n < issued; ++n)
                 bar_wait(bar_full0 + 8 * (n % kSStages), (n / kSStages) & 1, limit);
-            if (committed > 0) bar_wait(bar_mma, (committed - 1) & 1, limit);
-        }
+        if (tid == 128 && committed > 0) bar_wait(bar_mma, (committed - 1) & 1, limit);
     }
     fence_before();
     __syncthreads();
@@ -348,24 +387,29 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
 }
 
 // ================================================================ per-chunk gradients (K2)
-// 128 threads = 4 warps, one (b, h, chunk) per CTA, two CTAs per SM.  Shared memory: the seven
+// 256 threads = 8 warps, two persistent CTAs per SM, each walking (b, h, chunk) items in strides
+// of the grid and prefetching the next item's tiles into L2.  Shared memory: the seven
 // input tiles (r, k, v, w, dO, the bf16 state before the chunk, the bf16 state gradient after
 // it), four operand tiles built here (Qx, Kh, Am, dAm), and the fp32 prefix decay products.
 // TMEM (256 columns): A at 0 and dA at 64, then dV at 0 (after A is read), dR at 128, dK at 192.
+// Operand rows: warp w builds tokens 8w .. 8w + 7 (lane: 4-token half, channel quad).
+// Epilogues: warps w and w + 4 share TMEM lanes 32 (w % 4) .. (rows 16 (w % 4) .. + 15) and
+// split the columns: a thread holds 16 columns of one row.
+constexpr int kGThreads = 256;
 constexpr int G_R = 0, G_K = 1, G_V = 2, G_W = 3, G_G = 4, G_S = 5, G_DS = 6, G_QX = 7, G_KH = 8, G_AM = 9,
               G_DAM = 10;                              // tile slots (x kTile bytes)
 constexpr int kPreStride = 68;                         // fp32 row stride of the prefix products (pad)
 constexpr int G_PRE = 11 * kTile;                      // [64][68] fp32: prod_{j<t} w_j
 constexpr int G_SMALL = G_PRE + 64 * kPreStride * 4;
-constexpr int G_HS = G_SMALL;                          // [4][64] sub-block products; later column totals
-constexpr int G_DV = G_HS + 4 * 64 * 4;                // [64] chunk decay D
+constexpr int G_HS = G_SMALL;                          // [8][64] group decay products; later column totals
+constexpr int G_DV = G_HS + 8 * 64 * 4;                // [64] chunk decay D
 constexpr int G_IDV = G_DV + 64 * 4;                   // [64] 1 / D
 constexpr int G_UB = G_IDV + 64 * 4;                   // [64] bonus sum_c r u k per token
 constexpr int G_DD = G_UB + 64 * 4;                    // [64] dO_t . v_t
 constexpr int G_U = G_DD + 64 * 4;                     // [64] u of the head
 constexpr int G_RD = G_U + 64 * 4;                     // [64] rowdot(dS_end, S_end)
-constexpr int G_DU = G_RD + 64 * 4;                    // [4][64] du partials
-constexpr int G_BAR = G_DU + 4 * 64 * 4;               // full, mma1, mma2
+constexpr int G_DU = G_RD + 64 * 4;                    // [8][64] du partials
+constexpr int G_BAR = G_DU + 8 * 64 * 4;               // full, mma1, mma2
 constexpr int G_MISC = G_BAR + 64;
 constexpr int kChunkSmem = G_MISC + 64 + 1024;
 constexpr uint32_t T_A = 0, T_DA = 64, T_DV = 0, T_DR = 128, T_DK = 192, kChunkTmem = 256;
@@ -373,6 +417,7 @@ constexpr uint32_t T_A = 0, T_DA = 64, T_DV = 0, T_DR = 128, T_DK = 192, kChunkT
 struct GradParams {
     int64_t T, H;
     int nch;
+    int64_t nitems;                  // B * H * nch
     const float *u;                  // [H][N]
     const float *rowdot;             // [bh][nch][N]
     const int *flags;                // [bh]
@@ -382,8 +427,30 @@ struct GradParams {
     uint32_t spin_limit;
 };
 
+// Sum over the 16 lanes of a half-warp of 4 per-lane partials (one per token m = 0..3).
+// Returns the total for token 2 ((lane >> 3) & 1) + ((lane >> 2) & 1) (valid in every lane).
+__device__ __forceinline__ float half_sum4(const float (&part)[4], int lane)
+{
+    const bool b8 = lane & 8, b4 = lane & 4;
+    float v2[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+        v2[i] = (b8 ? part[2 + i] : part[i]) + __shfl_xor_sync(0xffffffffu, b8 ? part[i] : part[2 + i], 8);
+    float v = (b4 ? v2[1] : v2[0]) + __shfl_xor_sync(0xffffffffu, b4 ? v2[0] : v2[1], 4);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    return v;
+}
+
+__device__ __forceinline__ void st_f32x16(float *dst, const float (&v)[16])
+{
+    float4 *d = reinterpret_cast<float4 *>(dst);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+}
+
 template <bool OMEGA>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(kGThreads, 2)
 wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                       const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_s,
@@ -407,12 +474,8 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nch = p.nch;
-    const int64_t item = blockIdx.x, bh = item / nch, b = bh / p.H, h = bh % p.H;
-    const int cc = static_cast<int>(item % nch);
-    const int64_t t0 = static_cast<int64_t>(cc) * kC;
-    const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+    const int64_t nitems = p.nitems;
     const uint32_t limit = p.spin_limit;
-    if (p.flags[bh]) return;  // served by the exact walks
 
     if (tid == 0) {
         bar_init(bar_full, 1);
@@ -431,171 +494,213 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
     fence_after();
     const uint32_t tbase = misc[0];
 
-    if (tid == 0) {
-        bar_expect_tx(bar_full, 7 * kTile);
-        const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
-        tma_load_4d(smem_u32(TR), &map_r, 0, hh, tt, bb, bar_full);
-        tma_load_4d(smem_u32(TK), &map_k, 0, hh, tt, bb, bar_full);
-        tma_load_4d(smem_u32(TV), &map_v, 0, hh, tt, bb, bar_full);
-        tma_load_4d(smem_u32(TW), &map_w, 0, hh, tt, bb, bar_full);
-        tma_load_4d(smem_u32(TG), &map_g, 0, hh, tt, bb, bar_full);
-        tma_load_2d(smem_u32(TS), &map_s, 0, static_cast<int>((bh * (nch + 1) + cc) * kC), bar_full);
-        tma_load_2d(smem_u32(TDS), &map_ds, 0, static_cast<int>((bh * nch + cc) * kC), bar_full);
-    }
-    if (tid < 64) {
-        U[tid] = p.u[h * kN + tid];
-        RD[tid] = p.rowdot[(bh * nch + cc) * kN + tid];
-    }
-    int waited = 0;  // 1: copies landed; 2: first MMA group done; 3: second (for the drain)
-    int ok = bar_wait(bar_full, 0, limit);
-    int abort = __syncthreads_or(!ok);
-    if (!abort) {
-        waited = 1;
-        // ---------------------------------------------------------------- operand rows
-        const int a = warp, hf = lane >> 4, cq = lane & 15, t0h = 16 * a + 8 * hf;
-        const uint32_t cbyte = 8 * cq;
-        const Q4 u4 = ld_q4(U + 4 * cq);
-        Q4 w[8];
-        Q4 Gh = one4();
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int t = t0h + m;
-            if (t < tv) {
-                const Q4 x = unpack4(ld_u2(TW, swz(t, cbyte)));
-                w[m] = OMEGA ? decay4(x) : x;
-            } else {
-                w[m] = one4();
-            }
-            Gh = mul4(Gh, w[m]);
-        }
-        const Q4 Go = shfl_xor4(Gh, 16);
-        if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
-        __syncthreads();
-        Q4 D = one4(), before = one4(), aft = one4();
-#pragma unroll
-        for (int be = 0; be < 4; ++be) {
-            const Q4 g = ld_q4(Hs + be * 64 + 4 * cq);
-            D = mul4(D, g);
-            before = be < a ? mul4(before, g) : before;
-            aft = be > a ? mul4(aft, g) : aft;
-        }
-        // suffix products prod_{j>t} w_j of this half's tokens
-        Q4 suf[8];
-        {
-            Q4 run = mul4(aft, hf ? one4() : Go);
-#pragma unroll
-            for (int m = 7; m >= 0; --m) {
-                suf[m] = run;
-                run = mul4(run, w[m]);
-            }
-        }
-        Q4 pre = mul4(before, hf ? Go : one4());  // prod_{j<t} w_j
-        float pu[8], pd[8];
-#pragma unroll
-        for (int m = 0; m < 8; ++m) {
-            const int t = t0h + m;
-            const uint32_t off = swz(t, cbyte);
-            const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
-            const Q4 v = unpack4(ld_u2(TV, off)), g = unpack4(ld_u2(TG, off));
-            const Q4 qf = mul4(suf[m], w[m]);  // prod_{j>=t} w_j
-            st_u2(TQX, off, pack4({mul2(r.a, rcp2(qf.a)), mul2(r.b, rcp2(qf.b))}));
-            st_u2(TKH, off, pack4(mul4(k, suf[m])));
-            st_q4(PRE + t * kPreStride + 4 * cq, pre);
-            pu[m] = bonus4(r, u4, k);
-            pd[m] = dot4(g, v);
-            pre = mul4(pre, w[m]);
-        }
-        const float ub = half_sum8(pu, lane), dd = half_sum8(pd, lane);
-        if ((lane & 1) == 0) {
-            UB[t0h + ((lane >> 1) & 7)] = ub;
-            DD[t0h + ((lane >> 1) & 7)] = dd;
-        }
-        if (warp == 0 && hf == 0) {
-            st_q4(Dv + 4 * cq, D);
-            iDv[4 * cq] = 1.f / lo(D.a);
-            iDv[4 * cq + 1] = 1.f / hi(D.a);
-            iDv[4 * cq + 2] = 1.f / lo(D.b);
-            iDv[4 * cq + 3] = 1.f / hi(D.b);
-        }
-        __syncthreads();
-        // du share of this chunk: sum_t r_t k_t dd_t per channel
-        {
-            P2 acc0 = pk(0.f, 0.f), acc1 = acc0;
-#pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int t = t0h + m;
-                const uint32_t off = swz(t, cbyte);
-                const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
-                const P2 d2 = pk(DD[t], DD[t]);
-                acc0 = fma2(mul2(r.a, k.a), d2, acc0);
-                acc1 = fma2(mul2(r.b, k.b), d2, acc1);
-            }
-            Q4 acc = {acc0, acc1};
-            const Q4 oth = shfl_xor4(acc, 16);
-            acc = {pk(lo(acc.a) + lo(oth.a), hi(acc.a) + hi(oth.a)), pk(lo(acc.b) + lo(oth.b), hi(acc.b) + hi(oth.b))};
-            if (hf == 0) st_q4(DU + a * 64 + 4 * cq, acc);
-        }
-        // D (.) S_prev in place: row c of the state scaled by D[c]
-        {
-            const int c = tid >> 1, half = tid & 1;
-            const float d = Dv[c];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                uint4 *x = reinterpret_cast<uint4 *>(TS + swz(c, 64 * half + 16 * i));
-                float f[8];
-                unpack8(*x, f);
-                *x = make_uint4(pack_bf16(f[0] * d, f[1] * d), pack_bf16(f[2] * d, f[3] * d),
-                                pack_bf16(f[4] * d, f[5] * d), pack_bf16(f[6] * d, f[7] * d));
-            }
-        }
-        fence_async_smem();
-        fence_before();
-        __syncthreads();
-        fence_after();
-        if (tid < 64) p.du_item[(bh * nch + cc) * kN + tid] = DU[tid] + DU[64 + tid] + DU[128 + tid] + DU[192 + tid];
-        if (tid == 0) {
-            const uint32_t aR = smem_u32(TQX), aK = smem_u32(TKH), aV = smem_u32(TV), aG = smem_u32(TG);
-            const uint32_t aS = smem_u32(TS), aDS = smem_u32(TDS);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // A = Qx Kh^T
-                mma(tbase + T_A, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dA = dO V^T
-                mma(tbase + T_DA, desc_k(aG + 32 * ks), desc_k(aV + 32 * ks), idesc(64, 0, 0), ks > 0);
-            mma_commit(bar_m1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dR = dO (D S_prev)^T
-                mma(tbase + T_DR, desc_k(aG + 32 * ks), desc_k(aS + 32 * ks), idesc(64, 0, 0), ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dK = V dS_end^T
-                mma(tbase + T_DK, desc_k(aV + 32 * ks), desc_k(aDS + 32 * ks), idesc(64, 0, 0), ks > 0);
-        }
-        ok = bar_wait(bar_m1, 0, limit);
-        abort = __syncthreads_or(!ok);
-    }
+    // TMEM lanes 32 (warp % 4) .. of this warp: rows 16 (warp % 4) .. + 15; this thread's 16
+    // columns start at col0 (warp / 4 picks the 16-column half of each 32-column half)
+    const int sub = warp & 3, lr = lane & 15, t = 16 * sub + lr;
+    const int col0 = 16 * (warp >> 2) + 32 * (lane >> 4);
+    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * sub) << 16) + static_cast<uint32_t>(16 * (warp >> 2));
 
-    // TMEM lane group of this warp: rows 16 warp .. + 15, columns [colh, colh + 32)
-    const int lr = lane & 15, hi = lane >> 4, t = 16 * warp + lr, colh = 32 * hi;
-    const uint32_t tl = tbase + (static_cast<uint32_t>(32 * warp) << 16);
-    if (!abort) {
+    // items (b, h, chunk) in strides of the grid; the next one's tiles are prefetched into L2
+    // while this one is computed
+    auto item_coords = [&](int64_t it, int64_t &bh_, int64_t &b_, int64_t &h_, int &cc_) {
+        bh_ = it / nch;
+        b_ = bh_ / p.H;
+        h_ = bh_ % p.H;
+        cc_ = static_cast<int>(it % nch);
+    };
+    int abort = 0, waited = 0;  // waited: 1 copies landed; 2 first MMA group done; 3 second
+    uint32_t ph = 0;            // phase of this CTA's barriers (one use each per item)
+    for (int64_t item = blockIdx.x; item < nitems && !abort; item += gridDim.x) {
+        int64_t bh, b, h;
+        int cc;
+        item_coords(item, bh, b, h, cc);
+        if (p.flags[bh]) continue;  // served by the exact walks
+        const int64_t t0 = static_cast<int64_t>(cc) * kC;
+        const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
+        waited = 0;
+        if (tid == 0) {
+            bar_expect_tx(bar_full, 7 * kTile);
+            const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
+            tma_load_4d(smem_u32(TR), &map_r, 0, hh, tt, bb, bar_full);
+            tma_load_4d(smem_u32(TK), &map_k, 0, hh, tt, bb, bar_full);
+            tma_load_4d(smem_u32(TV), &map_v, 0, hh, tt, bb, bar_full);
+            tma_load_4d(smem_u32(TW), &map_w, 0, hh, tt, bb, bar_full);
+            tma_load_4d(smem_u32(TG), &map_g, 0, hh, tt, bb, bar_full);
+            tma_load_2d(smem_u32(TS), &map_s, 0, static_cast<int>((bh * (nch + 1) + cc) * kC), bar_full);
+            tma_load_2d(smem_u32(TDS), &map_ds, 0, static_cast<int>((bh * nch + cc) * kC), bar_full);
+            const int64_t nx = item + gridDim.x;
+            if (nx < nitems) {
+                int64_t nbh, nb, nh;
+                int ncc;
+                item_coords(nx, nbh, nb, nh, ncc);
+                const int hh2 = static_cast<int>(nh), bb2 = static_cast<int>(nb), tt2 = ncc * kC;
+                tma_prefetch_4d(&map_r, 0, hh2, tt2, bb2);
+                tma_prefetch_4d(&map_k, 0, hh2, tt2, bb2);
+                tma_prefetch_4d(&map_v, 0, hh2, tt2, bb2);
+                tma_prefetch_4d(&map_w, 0, hh2, tt2, bb2);
+                tma_prefetch_4d(&map_g, 0, hh2, tt2, bb2);
+                tma_prefetch_2d(&map_s, 0, static_cast<int>((nbh * (nch + 1) + ncc) * kC));
+                tma_prefetch_2d(&map_ds, 0, static_cast<int>((nbh * nch + ncc) * kC));
+            }
+        }
+        if (tid < 64) {
+            U[tid] = p.u[h * kN + tid];
+            RD[tid] = p.rowdot[(bh * nch + cc) * kN + tid];
+        }
+        int ok = bar_wait(bar_full, ph, limit);
+        abort = __syncthreads_or(!ok);
+        if (abort) break;
+        waited = 1;
+        {
+            // ------------------------------------------------------------ operand rows
+            // warp w: tokens 8w .. 8w + 7; lane: half hf (tokens 8w + 4hf .. + 3), channel quad cq
+            const int hf = lane >> 4, cq = lane & 15, t0h = 8 * warp + 4 * hf;
+            const uint32_t cbyte = 8 * cq;
+            const Q4 u4 = ld_q4(U + 4 * cq);
+            Q4 w[4];
+            Q4 Gh = one4();
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int tk = t0h + m;
+                if (tk < tv) {
+                    const Q4 x = unpack4(ld_u2(TW, swz(tk, cbyte)));
+                    w[m] = OMEGA ? decay4(x) : x;
+                } else {
+                    w[m] = one4();
+                }
+                Gh = mul4(Gh, w[m]);
+            }
+            const Q4 Go = shfl_xor4(Gh, 16);
+            if (hf == 0) st_q4(Hs + warp * 64 + 4 * cq, mul4(Gh, Go));
+            __syncthreads();
+            Q4 D = one4(), before = one4(), aft = one4();
+#pragma unroll
+            for (int g = 0; g < 8; ++g) {
+                const Q4 x = ld_q4(Hs + g * 64 + 4 * cq);
+                D = mul4(D, x);
+                before = g < warp ? mul4(before, x) : before;
+                aft = g > warp ? mul4(aft, x) : aft;
+            }
+            // suffix products prod_{j>t} w_j of this half's tokens
+            Q4 suf[4];
+            {
+                Q4 run = mul4(aft, hf ? one4() : Go);
+#pragma unroll
+                for (int m = 3; m >= 0; --m) {
+                    suf[m] = run;
+                    run = mul4(run, w[m]);
+                }
+            }
+            Q4 pre = mul4(before, hf ? Go : one4());  // prod_{j<t} w_j
+            float pu[4], pd[4];
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const int tk = t0h + m;
+                const uint32_t off = swz(tk, cbyte);
+                const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
+                const Q4 v = unpack4(ld_u2(TV, off)), g = unpack4(ld_u2(TG, off));
+                const Q4 qf = mul4(suf[m], w[m]);  // prod_{j>=t} w_j
+                st_u2(TQX, off, pack4({mul2(r.a, rcp2(qf.a)), mul2(r.b, rcp2(qf.b))}));
+                st_u2(TKH, off, pack4(mul4(k, suf[m])));
+                st_q4(PRE + tk * kPreStride + 4 * cq, pre);
+                pu[m] = bonus4(r, u4, k);
+                pd[m] = dot4(g, v);
+                pre = mul4(pre, w[m]);
+            }
+            const float ub = half_sum4(pu, lane), dd = half_sum4(pd, lane);
+            if ((lane & 3) == 0) {
+                const int tk = t0h + 2 * ((lane >> 3) & 1) + ((lane >> 2) & 1);
+                UB[tk] = ub;
+                DD[tk] = dd;
+            }
+            if (warp == 0 && hf == 0) {
+                st_q4(Dv + 4 * cq, D);
+                iDv[4 * cq] = 1.f / lo(D.a);
+                iDv[4 * cq + 1] = 1.f / hi(D.a);
+                iDv[4 * cq + 2] = 1.f / lo(D.b);
+                iDv[4 * cq + 3] = 1.f / hi(D.b);
+            }
+            __syncthreads();
+            // du share of this chunk: sum_t r_t k_t dd_t per channel
+            {
+                P2 acc0 = pk(0.f, 0.f), acc1 = acc0;
+#pragma unroll
+                for (int m = 0; m < 4; ++m) {
+                    const int tk = t0h + m;
+                    const uint32_t off = swz(tk, cbyte);
+                    const Q4 r = unpack4(ld_u2(TR, off)), k = unpack4(ld_u2(TK, off));
+                    const P2 d2 = pk(DD[tk], DD[tk]);
+                    acc0 = fma2(mul2(r.a, k.a), d2, acc0);
+                    acc1 = fma2(mul2(r.b, k.b), d2, acc1);
+                }
+                Q4 acc = {acc0, acc1};
+                const Q4 oth = shfl_xor4(acc, 16);
+                acc = {pk(lo(acc.a) + lo(oth.a), hi(acc.a) + hi(oth.a)),
+                       pk(lo(acc.b) + lo(oth.b), hi(acc.b) + hi(oth.b))};
+                if (hf == 0) st_q4(DU + warp * 64 + 4 * cq, acc);
+            }
+            // D (.) S_prev in place: row c of the state scaled by D[c] (a quarter row per thread)
+            {
+                const int c = tid >> 2, qtr = tid & 3;
+                const float d = Dv[c];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    uint4 *x = reinterpret_cast<uint4 *>(TS + swz(c, 32 * qtr + 16 * i));
+                    float f[8];
+                    unpack8(*x, f);
+                    *x = make_uint4(pack_bf16(f[0] * d, f[1] * d), pack_bf16(f[2] * d, f[3] * d),
+                                    pack_bf16(f[4] * d, f[5] * d), pack_bf16(f[6] * d, f[7] * d));
+                }
+            }
+            fence_async_smem();
+            fence_before();
+            __syncthreads();
+            fence_after();
+            if (tid < 64) {
+                float du = 0.f;
+#pragma unroll
+                for (int g = 0; g < 8; ++g) du += DU[g * 64 + tid];
+                p.du_item[(bh * nch + cc) * kN + tid] = du;
+            }
+            if (tid == 0) {
+                const uint32_t aR = smem_u32(TQX), aK = smem_u32(TKH), aV = smem_u32(TV), aG = smem_u32(TG);
+                const uint32_t aS = smem_u32(TS), aDS = smem_u32(TDS);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // A = Qx Kh^T
+                    mma(tbase + T_A, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // dA = dO V^T
+                    mma(tbase + T_DA, desc_k(aG + 32 * ks), desc_k(aV + 32 * ks), idesc(64, 0, 0), ks > 0);
+                mma_commit(bar_m1);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // dR = dO (D S_prev)^T
+                    mma(tbase + T_DR, desc_k(aG + 32 * ks), desc_k(aS + 32 * ks), idesc(64, 0, 0), ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // dK = V dS_end^T
+                    mma(tbase + T_DK, desc_k(aV + 32 * ks), desc_k(aDS + 32 * ks), idesc(64, 0, 0), ks > 0);
+            }
+        }
+        ok = bar_wait(bar_m1, ph, limit);
+        abort = __syncthreads_or(!ok);
+        if (abort) break;
         waited = 2;
         fence_after();
-        // ------------------------------------------------------------ Am and dAm
-        float x[32];
-        tmem_ld32(tl + T_A, x);
-        const float ubt = UB[t];
+        {
+            // ------------------------------------------------------------ Am and dAm
+            float x[16];
+            tmem_ld16(tl + T_A, x);
+            const float ubt = UB[t];
 #pragma unroll
-        for (int n = 0; n < 32; ++n) {
-            const int i = colh + n;
-            x[n] = i < t ? x[n] : (i == t ? ubt : 0.f);
+            for (int n = 0; n < 16; ++n) {
+                const int i = col0 + n;
+                x[n] = i < t ? x[n] : (i == t ? ubt : 0.f);
+            }
+            st_row16_bf16(TAM, t, 2 * col0, x);
+            tmem_ld16(tl + T_DA, x);
+#pragma unroll
+            for (int n = 0; n < 16; ++n) x[n] = col0 + n < t ? x[n] : 0.f;
+            st_row16_bf16(TDAM, t, 2 * col0, x);
         }
-        st_row16_bf16(TAM, t, 2 * colh, *reinterpret_cast<float(*)[16]>(&x[0]));
-        st_row16_bf16(TAM, t, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&x[16]));
-        tmem_ld32(tl + T_DA, x);
-#pragma unroll
-        for (int n = 0; n < 32; ++n) x[n] = colh + n < t ? x[n] : 0.f;
-        st_row16_bf16(TDAM, t, 2 * colh, *reinterpret_cast<float(*)[16]>(&x[0]));
-        st_row16_bf16(TDAM, t, 2 * colh + 32, *reinterpret_cast<float(*)[16]>(&x[16]));
         fence_async_smem();
         fence_before();
         __syncthreads();
@@ -617,96 +722,102 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
                 mma(tbase + T_DV, desc_k(aK + 32 * ks), desc_mn(aDS + 2048 * ks), idesc(64, 0, 1), 1);
             mma_commit(bar_m2);
         }
-        ok = bar_wait(bar_m2, 0, limit);
+        ok = bar_wait(bar_m2, ph, limit);
         abort = __syncthreads_or(!ok);
-    }
-    if (!abort) {
+        if (abort) break;
         waited = 3;
         fence_after();
-        // ------------------------------------------------------------ gradients of row t
-        const bool valid = t < tv;
-        const int64_t go = ((b * p.T + t0 + t) * p.H + h) * kN + colh;
-        const float ddt = DD[t];
-        const float *pre = PRE + t * kPreStride + colh;
-        float x[32];
-        tmem_ld32(tl + T_DV, x);
-        if (valid) st_f32x32(p.dv + go, x);
-        float rdr[32], e[32];
-        tmem_ld32(tl + T_DR, x);
+        {
+            // ------------------------------------------------------------ gradients of row t
+            const bool valid = t < tv;
+            const int64_t go = ((b * p.T + t0 + t) * p.H + h) * kN + col0;
+            const float ddt = DD[t];
+            const float *pre = PRE + t * kPreStride + col0;
+            float x[16];
+            tmem_ld16(tl + T_DV, x);
+            if (valid) st_f32x16(p.dv + go, x);
+            float rdr[16], e[16];
+            tmem_ld16(tl + T_DR, x);
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-            float kk[8], qx[8];
-            ld_row8(TK, t, 2 * colh + 16 * g8, kk);
-            ld_row8(TQX, t, 2 * colh + 16 * g8, qx);
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float kk[8], qx[8];
+                ld_row8(TK, t, 2 * col0 + 16 * g8, kk);
+                ld_row8(TQX, t, 2 * col0 + 16 * g8, qx);
 #pragma unroll
-            for (int e8 = 0; e8 < 8; ++e8) {
-                const int n = 8 * g8 + e8, c = colh + n;
-                rdr[n] = qx[e8] * x[n];
-                x[n] = fmaf(x[n], pre[n] * iDv[c], U[c] * kk[e8] * ddt);
+                for (int e8 = 0; e8 < 8; ++e8) {
+                    const int n = 8 * g8 + e8, c = col0 + n;
+                    rdr[n] = qx[e8] * x[n];
+                    x[n] = fmaf(x[n], pre[n] * iDv[c], U[c] * kk[e8] * ddt);
+                }
             }
-        }
-        if (valid) st_f32x32(p.dr + go, x);
-        tmem_ld32(tl + T_DK, x);
+            if (valid) st_f32x16(p.dr + go, x);
+            tmem_ld16(tl + T_DK, x);
 #pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-            float rr[8], kh[8], wv[8];
-            ld_row8(TR, t, 2 * colh + 16 * g8, rr);
-            ld_row8(TKH, t, 2 * colh + 16 * g8, kh);
-            ld_row8(TW, t, 2 * colh + 16 * g8, wv);
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float rr[8], kh[8], wv[8];
+                ld_row8(TR, t, 2 * col0 + 16 * g8, rr);
+                ld_row8(TKH, t, 2 * col0 + 16 * g8, kh);
+                ld_row8(TW, t, 2 * col0 + 16 * g8, wv);
 #pragma unroll
-            for (int e8 = 0; e8 < 8; ++e8) {
-                const int n = 8 * g8 + e8, c = colh + n;
-                const float wt = t < tv ? (OMEGA ? decay_of_logit(wv[e8]) : wv[e8]) : 1.f;
-                const float kf = Dv[c] * rcp_approx(pre[n] * wt);  // prod_{j>t} w_j
-                e[n] = rdr[n] - kh[e8] * x[n];
-                x[n] = fmaf(x[n], kf, U[c] * rr[e8] * ddt);
+                for (int e8 = 0; e8 < 8; ++e8) {
+                    const int n = 8 * g8 + e8, c = col0 + n;
+                    const float wt = t < tv ? (OMEGA ? decay_of_logit(wv[e8]) : wv[e8]) : 1.f;
+                    const float kf = Dv[c] * rcp_approx(pre[n] * wt);  // prod_{j>t} w_j
+                    e[n] = rdr[n] - kh[e8] * x[n];
+                    x[n] = fmaf(x[n], kf, U[c] * rr[e8] * ddt);
+                }
             }
-        }
-        if (valid) st_f32x32(p.dk + go, x);
-        // d(log w_j) = sum_{t>=j} e_t - rdr_j + rowdot: suffix sums down the rows (columns are
-        // independent); rows 16 warp .. + 15 are the 16 lanes of each half-warp
+            if (valid) st_f32x16(p.dk + go, x);
+            // d(log w_j) = sum_{t>=j} e_t - rdr_j + rowdot: suffix sums down the rows (columns
+            // are independent); rows 16 sub .. + 15 are the 16 lanes of each half-warp
 #pragma unroll
-        for (int n = 0; n < 32; ++n) {
-            float s = e[n];
+            for (int n = 0; n < 16; ++n) {
+                float sacc = e[n];
 #pragma unroll
-            for (int d = 1; d < 16; d <<= 1) {
-                const float y = __shfl_down_sync(0xffffffffu, s, d, 16);
-                if (lr + d < 16) s += y;
+                for (int d = 1; d < 16; d <<= 1) {
+                    const float y = __shfl_down_sync(0xffffffffu, sacc, d, 16);
+                    if (lr + d < 16) sacc += y;
+                }
+                e[n] = sacc;
             }
-            e[n] = s;
-        }
-        if (lr == 0)
+            if (lr == 0)
 #pragma unroll
-            for (int n = 0; n < 32; ++n) Hs[warp * 64 + colh + n] = e[n];
+                for (int n = 0; n < 16; ++n) Hs[sub * 64 + col0 + n] = e[n];
+            __syncthreads();
+#pragma unroll
+            for (int n = 0; n < 16; ++n) {
+                float add = 0.f;
+                for (int q = sub + 1; q < 4; ++q) add += Hs[q * 64 + col0 + n];
+                e[n] += add;
+            }
+#pragma unroll
+            for (int g8 = 0; g8 < 2; ++g8) {
+                float wv[8];
+                ld_row8(TW, t, 2 * col0 + 16 * g8, wv);
+#pragma unroll
+                for (int e8 = 0; e8 < 8; ++e8) {
+                    const int n = 8 * g8 + e8, c = col0 + n;
+                    const float dl = e[n] - rdr[n] + RD[c];
+                    if (OMEGA)  // domega = -exp(omega) d(log w)
+                        x[n] = -ex2_approx(wv[e8] * 1.4426950408889634f) * dl;
+                    else        // dw = d(log w) / w; w >= 2^-5 on this path
+                        x[n] = dl / wv[e8];
+                }
+            }
+            if (valid) st_f32x16(p.dw + go, x);
+        }
+        // every thread is done with this item's tiles and accumulators before the next one
+        fence_before();
         __syncthreads();
-#pragma unroll
-        for (int n = 0; n < 32; ++n) {
-            float add = 0.f;
-            for (int q = warp + 1; q < 4; ++q) add += Hs[q * 64 + colh + n];
-            e[n] += add;
-        }
-#pragma unroll
-        for (int g8 = 0; g8 < 4; ++g8) {
-            float wv[8];
-            ld_row8(TW, t, 2 * colh + 16 * g8, wv);
-#pragma unroll
-            for (int e8 = 0; e8 < 8; ++e8) {
-                const int n = 8 * g8 + e8, c = colh + n;
-                const float dl = e[n] - rdr[n] + RD[c];
-                if (OMEGA)  // domega = -exp(omega) d(log w)
-                    x[n] = -ex2_approx(wv[e8] * 1.4426950408889634f) * dl;
-                else        // dw = d(log w) / w; w >= 2^-5 on this path
-                    x[n] = dl / wv[e8];
-            }
-        }
-        if (valid) st_f32x32(p.dw + go, x);
+        fence_after();
+        ph ^= 1u;
     }
     if (abort) {
         record_status(p.status, kStatusTimeout);
         if (tid == 0) {
-            if (waited < 1) bar_wait(bar_full, 0, limit);
-            if (waited == 1) bar_wait(bar_m1, 0, limit);
-            if (waited >= 1 && waited < 3) bar_wait(bar_m2, 0, limit);
+            if (waited < 1) bar_wait(bar_full, ph, limit);
+            if (waited == 1) bar_wait(bar_m1, ph, limit);
+            if (waited >= 1 && waited < 3) bar_wait(bar_m2, ph, limit);
         }
     }
     fence_before();
@@ -726,9 +837,12 @@ cudaError_t configure_tc()
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
     if (done[dev]) return cudaSuccess;
-    for (auto kern : {wkv6_bwd_state_kernel<false, false>, wkv6_bwd_state_kernel<false, true>,
-                      wkv6_bwd_state_kernel<true, false>, wkv6_bwd_state_kernel<true, true>}) {
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kStateSmem);
+    for (auto kern : {wkv6_bwd_state_kernel<false, false>, wkv6_bwd_state_kernel<false, true>}) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<false>::smem);
+        if (e != cudaSuccess) return e;
+    }
+    for (auto kern : {wkv6_bwd_state_kernel<true, false>, wkv6_bwd_state_kernel<true, true>}) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, StateLayout<true>::smem);
         if (e != cudaSuccess) return e;
     }
     for (auto kern : {wkv6_bwd_chunk_kernel<false>, wkv6_bwd_chunk_kernel<true>}) {
@@ -765,18 +879,25 @@ cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cu
     if (e != cudaSuccess) return e;
     int *status = a.status;
     const uint32_t spin = 100000u;
-    StateParams fw{a.T, a.H, static_cast<int>(nch), a.s0, sck, nullptr, nullptr, flags, nullptr, status, spin};
-    StateParams bw{a.T, a.H, static_cast<int>(nch), a.dsT, dsck, sck, rowdot, flags, a.ds0, status, spin};
-    GradParams gp{a.T, a.H, static_cast<int>(nch), a.u, rowdot, flags, a.dr, a.dk, a.dv, a.dw, du_item, status, spin};
-    const dim3 gs(static_cast<unsigned>(bh)), gc(static_cast<unsigned>(bh * nch));
+    StateParams fw{a.T, a.H, static_cast<int>(nch), a.s0, sck, nullptr, flags, nullptr, status, spin};
+    StateParams bw{a.T, a.H, static_cast<int>(nch), a.dsT, dsck, rowdot, flags, a.ds0, status, spin};
+    GradParams gp{a.T, a.H, static_cast<int>(nch), bh * nch, a.u, rowdot, flags, a.dr, a.dk, a.dv, a.dw, du_item,
+                  status, spin};
+    // persistent: two CTAs per SM walk the (b, h, chunk) items in strides of the grid
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
+        sms = 148;
+    const dim3 gs(static_cast<unsigned>(bh)),
+        gc(static_cast<unsigned>(std::min<int64_t>(bh * nch, 2LL * sms)));
     if (a.omega) {
-        wkv6_bwd_state_kernel<false, true><<<gs, kSThreads, kStateSmem, s>>>(mk, mv, mw, fw);
-        wkv6_bwd_state_kernel<true, true><<<gs, kSThreads, kStateSmem, s>>>(mr, mg, mw, bw);
-        wkv6_bwd_chunk_kernel<true><<<gc, 128, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+        wkv6_bwd_state_kernel<false, true><<<gs, kSThreads, StateLayout<false>::smem, s>>>(mk, mv, mw, ms, fw);
+        wkv6_bwd_state_kernel<true, true><<<gs, kSThreads, StateLayout<true>::smem, s>>>(mr, mg, mw, ms, bw);
+        wkv6_bwd_chunk_kernel<true><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
     } else {
-        wkv6_bwd_state_kernel<false, false><<<gs, kSThreads, kStateSmem, s>>>(mk, mv, mw, fw);
-        wkv6_bwd_state_kernel<true, false><<<gs, kSThreads, kStateSmem, s>>>(mr, mg, mw, bw);
-        wkv6_bwd_chunk_kernel<false><<<gc, 128, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+        wkv6_bwd_state_kernel<false, false><<<gs, kSThreads, StateLayout<false>::smem, s>>>(mk, mv, mw, ms, fw);
+        wkv6_bwd_state_kernel<true, false><<<gs, kSThreads, StateLayout<true>::smem, s>>>(mr, mg, mw, ms, bw);
+        wkv6_bwd_chunk_kernel<false><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
     }
     return cudaGetLastError();
 }
