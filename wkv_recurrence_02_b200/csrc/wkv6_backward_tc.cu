@@ -449,12 +449,21 @@ __device__ __forceinline__ void st_f32x16(float *dst, const float (&v)[16])
     for (int i = 0; i < 4; ++i) d[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
 }
 
+// Gradient tiles leave through shared memory: each 64 x 64 fp32 tile is staged as two 64 x 32
+// halves with the 128-byte swizzle in tile slots the MMAs no longer read (dV in the V and dO
+// slots, dR in S and dS_end, dK in Am and dAm, then dw in V and dO again) and written by TMA
+// stores, which clip the rows past T.
+struct OutMaps {
+    CUtensorMap dr, dk, dv, dw;  // [B, T, H, 64] fp32, box = 32 channels x 64 tokens
+};
+
 template <bool OMEGA>
 __global__ void __launch_bounds__(kGThreads, 2)
 wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
                       const __grid_constant__ CUtensorMap map_v, const __grid_constant__ CUtensorMap map_w,
                       const __grid_constant__ CUtensorMap map_g, const __grid_constant__ CUtensorMap map_s,
-                      const __grid_constant__ CUtensorMap map_ds, const GradParams p)
+                      const __grid_constant__ CUtensorMap map_ds, const __grid_constant__ OutMaps om,
+                      const GradParams p)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
@@ -477,10 +486,14 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
     const int64_t nitems = p.nitems;
     const uint32_t limit = p.spin_limit;
 
+    // MMA issue is split over four threads (an issue holds its thread for tens of cycles);
+    // each accumulator's chain stays on one thread, so its products run in order:
+    //   warp 0: A, then dV;  warp 1: dA;  warp 2: dR;  warp 3: dK
+    const bool iss = lane == 0 && warp < 4;
     if (tid == 0) {
         bar_init(bar_full, 1);
-        bar_init(bar_m1, 1);
-        bar_init(bar_m2, 1);
+        bar_init(bar_m1, 2);  // A and dA issuers
+        bar_init(bar_m2, 3);  // dR, dK and dV issuers
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
@@ -519,6 +532,7 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
         const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
         waited = 0;
         if (tid == 0) {
+            bulk_wait_read<0>();  // the previous item's gradient stores have read their slots
             bar_expect_tx(bar_full, 7 * kTile);
             const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
             tma_load_4d(smem_u32(TR), &map_r, 0, hh, tt, bb, bar_full);
@@ -662,22 +676,28 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
                 for (int g = 0; g < 8; ++g) du += DU[g * 64 + tid];
                 p.du_item[(bh * nch + cc) * kN + tid] = du;
             }
-            if (tid == 0) {
+            if (iss) {
                 const uint32_t aR = smem_u32(TQX), aK = smem_u32(TKH), aV = smem_u32(TV), aG = smem_u32(TG);
                 const uint32_t aS = smem_u32(TS), aDS = smem_u32(TDS);
+                if (warp == 0) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // A = Qx Kh^T
-                    mma(tbase + T_A, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)  // A = Qx Kh^T
+                        mma(tbase + T_A, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
+                    mma_commit(bar_m1);
+                } else if (warp == 1) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // dA = dO V^T
-                    mma(tbase + T_DA, desc_k(aG + 32 * ks), desc_k(aV + 32 * ks), idesc(64, 0, 0), ks > 0);
-                mma_commit(bar_m1);
+                    for (int ks = 0; ks < 4; ++ks)  // dA = dO V^T
+                        mma(tbase + T_DA, desc_k(aG + 32 * ks), desc_k(aV + 32 * ks), idesc(64, 0, 0), ks > 0);
+                    mma_commit(bar_m1);
+                } else if (warp == 2) {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // dR = dO (D S_prev)^T
-                    mma(tbase + T_DR, desc_k(aG + 32 * ks), desc_k(aS + 32 * ks), idesc(64, 0, 0), ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)  // dR = dO (D S_prev)^T
+                        mma(tbase + T_DR, desc_k(aG + 32 * ks), desc_k(aS + 32 * ks), idesc(64, 0, 0), ks > 0);
+                } else {
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // dK = V dS_end^T
-                    mma(tbase + T_DK, desc_k(aV + 32 * ks), desc_k(aDS + 32 * ks), idesc(64, 0, 0), ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)  // dK = V dS_end^T
+                        mma(tbase + T_DK, desc_k(aV + 32 * ks), desc_k(aDS + 32 * ks), idesc(64, 0, 0), ks > 0);
+                }
             }
         }
         ok = bar_wait(bar_m1, ph, limit);
@@ -705,21 +725,25 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
         fence_before();
         __syncthreads();
         fence_after();
-        if (tid == 0) {
+        if (iss && warp != 1) {
             const uint32_t aQ = smem_u32(TQX), aK = smem_u32(TKH), aG = smem_u32(TG), aDS = smem_u32(TDS);
             const uint32_t aAm = smem_u32(TAM), aDAm = smem_u32(TDAM);
+            if (warp == 2) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dR += dAm Kh
-                mma(tbase + T_DR, desc_k(aDAm + 32 * ks), desc_mn(aK + 2048 * ks), idesc(64, 0, 1), 1);
+                for (int ks = 0; ks < 4; ++ks)  // dR += dAm Kh
+                    mma(tbase + T_DR, desc_k(aDAm + 32 * ks), desc_mn(aK + 2048 * ks), idesc(64, 0, 1), 1);
+            } else if (warp == 3) {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dK += dAm^T Qx
-                mma(tbase + T_DK, desc_mn(aDAm + 2048 * ks), desc_mn(aQ + 2048 * ks), idesc(64, 1, 1), 1);
+                for (int ks = 0; ks < 4; ++ks)  // dK += dAm^T Qx
+                    mma(tbase + T_DK, desc_mn(aDAm + 2048 * ks), desc_mn(aQ + 2048 * ks), idesc(64, 1, 1), 1);
+            } else {
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dV = Am^T dO
-                mma(tbase + T_DV, desc_mn(aAm + 2048 * ks), desc_mn(aG + 2048 * ks), idesc(64, 1, 1), ks > 0);
+                for (int ks = 0; ks < 4; ++ks)  // dV = Am^T dO
+                    mma(tbase + T_DV, desc_mn(aAm + 2048 * ks), desc_mn(aG + 2048 * ks), idesc(64, 1, 1), ks > 0);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)  // dV += Kh dS_end
-                mma(tbase + T_DV, desc_k(aK + 32 * ks), desc_mn(aDS + 2048 * ks), idesc(64, 0, 1), 1);
+                for (int ks = 0; ks < 4; ++ks)  // dV += Kh dS_end
+                    mma(tbase + T_DV, desc_k(aK + 32 * ks), desc_mn(aDS + 2048 * ks), idesc(64, 0, 1), 1);
+            }
             mma_commit(bar_m2);
         }
         ok = bar_wait(bar_m2, ph, limit);
@@ -729,14 +753,22 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
         fence_after();
         {
             // ------------------------------------------------------------ gradients of row t
-            const bool valid = t < tv;
-            const int64_t go = ((b * p.T + t0 + t) * p.H + h) * kN + col0;
+            // staged into two 64 x 32 fp32 halves (128-byte swizzle) of a slot pair
+            const int half = col0 >> 5;
+            const int cb = 4 * (col0 & 31);  // byte column inside the half
+            auto stage16 = [&](unsigned char *lo_half, unsigned char *hi_half, const float (&v)[16]) {
+                unsigned char *tile = half ? hi_half : lo_half;
+#pragma unroll
+                for (int i = 0; i < 4; ++i)
+                    *reinterpret_cast<float4 *>(tile + swz(t, cb + 16 * i)) =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            };
             const float ddt = DD[t];
-            const float *pre = PRE + t * kPreStride + col0;
+            float *pre = PRE + t * kPreStride + col0;
             float x[16];
             tmem_ld16(tl + T_DV, x);
-            if (valid) st_f32x16(p.dv + go, x);
-            float rdr[16], e[16];
+            stage16(TV, TG, x);
+            float rdr[16];
             tmem_ld16(tl + T_DR, x);
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
@@ -750,7 +782,7 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
                     x[n] = fmaf(x[n], pre[n] * iDv[c], U[c] * kk[e8] * ddt);
                 }
             }
-            if (valid) st_f32x16(p.dr + go, x);
+            stage16(TS, TDS, x);
             tmem_ld16(tl + T_DK, x);
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
@@ -763,32 +795,48 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
                     const int n = 8 * g8 + e8, c = col0 + n;
                     const float wt = t < tv ? (OMEGA ? decay_of_logit(wv[e8]) : wv[e8]) : 1.f;
                     const float kf = Dv[c] * rcp_approx(pre[n] * wt);  // prod_{j>t} w_j
-                    e[n] = rdr[n] - kh[e8] * x[n];
+                    const float kdk = kh[e8] * x[n];
                     x[n] = fmaf(x[n], kf, U[c] * rr[e8] * ddt);
+                    const float en = rdr[n] - kdk;
+                    pre[n] = rdr[n];  // the prefix products are no longer needed: keep rdr here
+                    rdr[n] = en;
                 }
             }
-            if (valid) st_f32x16(p.dk + go, x);
-            // d(log w_j) = sum_{t>=j} e_t - rdr_j + rowdot: suffix sums down the rows (columns
-            // are independent); rows 16 sub .. + 15 are the 16 lanes of each half-warp
+            stage16(TAM, TDAM, x);
+            // d(log w_j) = sum_{t>=j} e_t - rdr_j + rowdot with e_t = rdr_t - kdk_t (in rdr[] now):
+            // suffix sums down the rows (columns are independent); rows 16 sub .. + 15 are the
+            // 16 lanes of each half-warp
 #pragma unroll
             for (int n = 0; n < 16; ++n) {
-                float sacc = e[n];
+                float sacc = rdr[n];
 #pragma unroll
                 for (int d = 1; d < 16; d <<= 1) {
                     const float y = __shfl_down_sync(0xffffffffu, sacc, d, 16);
                     if (lr + d < 16) sacc += y;
                 }
-                e[n] = sacc;
+                rdr[n] = sacc;
             }
             if (lr == 0)
 #pragma unroll
-                for (int n = 0; n < 16; ++n) Hs[sub * 64 + col0 + n] = e[n];
+                for (int n = 0; n < 16; ++n) Hs[sub * 64 + col0 + n] = rdr[n];
+            fence_async_smem();
             __syncthreads();
+            if (tid == 0) {  // dv, dr, dk of this chunk
+                const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
+                tma_store_4d(&om.dv, 0, hh, tt, bb, smem_u32(TV));
+                tma_store_4d(&om.dv, 32, hh, tt, bb, smem_u32(TG));
+                bulk_commit();
+                tma_store_4d(&om.dr, 0, hh, tt, bb, smem_u32(TS));
+                tma_store_4d(&om.dr, 32, hh, tt, bb, smem_u32(TDS));
+                tma_store_4d(&om.dk, 0, hh, tt, bb, smem_u32(TAM));
+                tma_store_4d(&om.dk, 32, hh, tt, bb, smem_u32(TDAM));
+                bulk_commit();
+            }
 #pragma unroll
             for (int n = 0; n < 16; ++n) {
                 float add = 0.f;
                 for (int q = sub + 1; q < 4; ++q) add += Hs[q * 64 + col0 + n];
-                e[n] += add;
+                rdr[n] += add;
             }
 #pragma unroll
             for (int g8 = 0; g8 < 2; ++g8) {
@@ -797,14 +845,24 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
 #pragma unroll
                 for (int e8 = 0; e8 < 8; ++e8) {
                     const int n = 8 * g8 + e8, c = col0 + n;
-                    const float dl = e[n] - rdr[n] + RD[c];
+                    const float dl = rdr[n] - pre[n] + RD[c];
                     if (OMEGA)  // domega = -exp(omega) d(log w)
                         x[n] = -ex2_approx(wv[e8] * 1.4426950408889634f) * dl;
                     else        // dw = d(log w) / w; w >= 2^-5 on this path
                         x[n] = dl / wv[e8];
                 }
             }
-            if (valid) st_f32x16(p.dw + go, x);
+            if (tid == 0) bulk_wait_read<1>();  // the dv stores have read V | dO
+            __syncthreads();
+            stage16(TV, TG, x);
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
+                tma_store_4d(&om.dw, 0, hh, tt, bb, smem_u32(TV));
+                tma_store_4d(&om.dw, 32, hh, tt, bb, smem_u32(TG));
+                bulk_commit();
+            }
         }
         // every thread is done with this item's tiles and accumulators before the next one
         fence_before();
@@ -820,6 +878,7 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
             if (waited >= 1 && waited < 3) bar_wait(bar_m2, ph, limit);
         }
     }
+    if (tid == 0) bulk_wait_all();  // the last gradient stores have completed
     fence_before();
     __syncthreads();
     fence_after();
@@ -857,6 +916,23 @@ cudaError_t configure_tc()
 
 }  // namespace
 
+// [B, T, H, 64] fp32 gradient, box = 32 channels x 1 head x 64 tokens x 1 batch row, 128-byte
+// swizzle (TMA stores from the staged halves)
+bool make_out_map(CUtensorMap *map, void *base, int64_t B, int64_t T, int64_t H)
+{
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(kN), static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T),
+                          static_cast<cuuint64_t>(B)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(kN * 4), static_cast<cuuint64_t>(H * kN * 4),
+                             static_cast<cuuint64_t>(T * H * kN * 4)};
+    cuuint32_t box[4] = {32, 1, kC, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cudaStream_t s)
 {
     const int64_t bh = a.B * a.H, nch = L.nch;
@@ -874,6 +950,10 @@ cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cu
         !make_map(&mv, a.v, a.B, a.T, a.H) || !make_map(&mw, a.w, a.B, a.T, a.H) ||
         !make_map(&mg, a.dy, a.B, a.T, a.H) || !make_rows_map(&ms, sck, bh * (nch + 1) * kC) ||
         !make_rows_map(&mds, dsck, bh * nch * kC))
+        return cudaErrorInvalidValue;
+    OutMaps om;
+    if (!make_out_map(&om.dr, a.dr, a.B, a.T, a.H) || !make_out_map(&om.dk, a.dk, a.B, a.T, a.H) ||
+        !make_out_map(&om.dv, a.dv, a.B, a.T, a.H) || !make_out_map(&om.dw, a.dw, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     cudaError_t e = configure_tc();
     if (e != cudaSuccess) return e;
@@ -893,11 +973,11 @@ cudaError_t wkv6_backward_tc_launch(const Wkv6BwdArgs &a, const BwdLayout &L, cu
     if (a.omega) {
         wkv6_bwd_state_kernel<false, true><<<gs, kSThreads, StateLayout<false>::smem, s>>>(mk, mv, mw, ms, fw);
         wkv6_bwd_state_kernel<true, true><<<gs, kSThreads, StateLayout<true>::smem, s>>>(mr, mg, mw, ms, bw);
-        wkv6_bwd_chunk_kernel<true><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+        wkv6_bwd_chunk_kernel<true><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, om, gp);
     } else {
         wkv6_bwd_state_kernel<false, false><<<gs, kSThreads, StateLayout<false>::smem, s>>>(mk, mv, mw, ms, fw);
         wkv6_bwd_state_kernel<true, false><<<gs, kSThreads, StateLayout<true>::smem, s>>>(mr, mg, mw, ms, bw);
-        wkv6_bwd_chunk_kernel<false><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, gp);
+        wkv6_bwd_chunk_kernel<false><<<gc, kGThreads, kChunkSmem, s>>>(mr, mk, mv, mw, mg, ms, mds, om, gp);
     }
     return cudaGetLastError();
 }
