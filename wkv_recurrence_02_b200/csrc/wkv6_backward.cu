@@ -451,10 +451,10 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
 
 // du[h][i] = the sum over batch rows b of the (b, h) sequence's share: du_part[b][h][i] from
 // the walks, or, where the chunked path served the sequence (flags given and the sequence's
-// flag clear), its chunks' du_item[b][h][c][i].  Four threads per channel each sum a fixed
-// quarter of the terms (chunks c = q mod 4) in order of (b, c), and the quarters are added in
-// order: the result is deterministic.
-constexpr int kDuParts = 4;
+// flag clear), its chunks' du_item[b][h][c][i].  kDuParts threads per channel each sum a
+// fixed share of the terms (chunks c = q mod kDuParts) in order of (b, c), and the shares are
+// added in order: the result is deterministic.
+constexpr int kDuParts = 16;
 __global__ void __launch_bounds__(kN * kDuParts) wkv6_bwd_du_kernel(int64_t B, int64_t H, int64_t nch,
                                                                    const float *__restrict__ du_part,
                                                                    const float *__restrict__ du_item,
