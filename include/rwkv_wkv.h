@@ -61,7 +61,9 @@ typedef enum rwkv_status {
     RWKV_ERR_CUDA = -5,        /* a CUDA runtime call or kernel launch failed         */
     RWKV_ERR_TIMEOUT = -6,     /* a bounded device-side wait ran out (device status)  */
     RWKV_ERR_ALIGN = -7,       /* a tensor pointer is not 16-byte aligned             */
-    RWKV_ERR_ARG = -8          /* another invalid argument (e.g. unknown option)      */
+    RWKV_ERR_ARG = -8,         /* another invalid argument (e.g. unknown option)      */
+    RWKV_ERR_BOUNDS = -9       /* debug build only: a kernel's index check failed and
+                                  the access was skipped (device status)              */
 } rwkv_status;
 
 /* ------------------------------------------------------------------ RWKV-4 WKV [R4]
@@ -305,6 +307,13 @@ const char *rwkv_last_error(void);
 
 /* RWKV_ABI_VERSION of the loaded library. */
 int rwkv_abi_version(void);
+
+/* 1 if the loaded library is the bounds-checked debug build (compiled with
+ * WKV_DEBUG_BOUNDS), else 0.  In that build every kernel checks its global, shared-memory and
+ * tensor-memory indices and TMA coordinates; a failed check skips the access and records
+ * RWKV_ERR_BOUNDS in the device status word (rwkv_get_device_status) -- nothing traps.  It
+ * is meant for tests on new shapes; it runs slower. */
+int rwkv_debug_bounds(void);
 
 #ifdef __cplusplus
 }

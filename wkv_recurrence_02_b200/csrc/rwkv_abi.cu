@@ -492,6 +492,7 @@ const char *rwkv_status_string(int status)
     case RWKV_ERR_TIMEOUT: return "device-side wait timed out";
     case RWKV_ERR_ALIGN: return "pointer not 16-byte aligned";
     case RWKV_ERR_ARG: return "invalid argument";
+    case RWKV_ERR_BOUNDS: return "index check failed (debug build)";
     default: return "unknown status";
     }
 }
@@ -499,5 +500,7 @@ const char *rwkv_status_string(int status)
 const char *rwkv_last_error(void) { return tl_err; }
 
 int rwkv_abi_version(void) { return RWKV_ABI_VERSION; }
+
+int rwkv_debug_bounds(void) { return wkv::kDebugBounds ? 1 : 0; }
 
 }  // extern "C"

@@ -300,7 +300,7 @@ template <typename T, int L>
 __global__ void __launch_bounds__(kThreads, 3)
 wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ w,
                  const float *__restrict__ u, const T *__restrict__ k, const T *__restrict__ v,
-                 const float *s0, T *__restrict__ y, float *sT)
+                 const float *s0, T *__restrict__ y, float *sT, int *status)
 {
     using W = typename Word<T>::type;
     extern __shared__ __align__(16) unsigned char smem_raw[];
@@ -314,6 +314,11 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
     const int pr = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int ca = c0 + 2 * pr, cb = ca + 1;
     const bool va = ca < C, vb = cb < C;
+    if (kDebugBounds) {  // the batch row, this lane's shared-memory segment, the state entries
+        const bool ok = in_bounds(status, b, 1, B) && in_bounds(status, widx<L>(pr, lane, 0), L + 1, tile_words<L>()) &&
+                        in_bounds(status, b * 3 * C + 2 * C + (va ? ca : 0), 1, B * 3 * C);
+        if (!__syncthreads_and(ok)) return;
+    }
 
     const float w2a = va ? w[ca] * kLog2e : 0.f, w2b = vb ? w[cb] * kLog2e : 0.f;
     const float u2a = va ? u[ca] * kLog2e : 0.f, u2b = vb ? u[cb] * kLog2e : 0.f;
@@ -341,6 +346,9 @@ wkv4_scan_kernel(int64_t B, int64_t T_len, int64_t C, const float *__restrict__ 
     for (int64_t t0 = 0; t0 < T_len; t0 += TILE) {
         const int64_t rem = T_len - t0;
         const int nt = rem < TILE ? static_cast<int>(rem) : TILE;
+        // debug build: the tile's rows of k, v and y lie inside [B, T, C]
+        if (kDebugBounds && !__syncthreads_and(in_bounds(status, (b * T_len + t0) * C, nt * C, B * T_len * C)))
+            break;
         fetch_tile<T, L>(bk, bv, kb, vbp, t0, nt, C, c0);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();
@@ -628,7 +636,7 @@ __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wa
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 struct TmaParams {
-    int64_t T, C;
+    int64_t T, C, B;
     const float *w, *u, *s0;
     float *sT;
     int *status;
@@ -657,6 +665,13 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     const int c0 = static_cast<int>((blockIdx.x % cblocks) * kCh);
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cb = c0 + NC * h;  // first channel of this lane
+    if (kDebugBounds) {  // the batch row; this lane's state entries; its units inside a buffer
+        const bool ok = in_bounds(p.status, b, 1, p.B) &&
+                        in_bounds(p.status, lane * RB + NC * static_cast<int>(sizeof(T)) * h + (L - 1) * BLK,
+                                  NC * static_cast<int>(sizeof(T)), L * BLK) &&
+                        (cb >= C || in_bounds(p.status, static_cast<int64_t>(b) * 3 * C + 2 * C + cb, 1, p.B * 3 * C));
+        if (!__syncthreads_and(ok)) return;
+    }
 
     const St empty{0.f, 0.f, kPEmpty};
     float w2[NC], u2[NC];
@@ -695,7 +710,10 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         const uint32_t bar = bar0 + 8 * (tl % NB);
         if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
         __syncwarp();
-        if (lane < L) {
+        // debug build: channel block on a 16-byte boundary inside C, the tile's first segment
+        // inside T / L (a copy that fails is not issued; its wait then runs out)
+        if (lane < L && tma_coord_ok(p.status, c0, static_cast<int>(sizeof(T)), C, static_cast<int64_t>(kSegs) * tl,
+                                     T_len / L)) {
             tma_load_4d(smem_u32(bk + lane * BLK), &map_k, c0, lane, kSegs * tl, b, bar);
             tma_load_4d(smem_u32(bk + L * BLK + lane * BLK), &map_v, c0, lane, kSegs * tl, b, bar);
         }
@@ -923,7 +941,7 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
         }
     }
     const int64_t blocks = a.B * ((a.C + kCh - 1) / kCh);
-    const TmaParams prm{a.T, a.C, a.w, a.u, a.s0, a.sT, a.status, 1u << 22};
+    const TmaParams prm{a.T, a.C, a.B, a.w, a.u, a.s0, a.sT, a.status, 1u << 22};
     kern<<<static_cast<unsigned>(blocks), kThr, smem, s>>>(mk, mv, my, prm);
     return cudaGetLastError();
 }
@@ -982,10 +1000,12 @@ bool tma_usable(const Wkv4Args &a)
 template <typename T, int NV>
 __global__ void __launch_bounds__(256)
 wkv4_decode_kernel(int64_t B, int64_t C, const float *__restrict__ w, const float *__restrict__ u,
-                   const T *__restrict__ k, const T *__restrict__ v, const float *s0, T *__restrict__ y, float *sT)
+                   const T *__restrict__ k, const T *__restrict__ v, const float *s0, T *__restrict__ y, float *sT,
+                   int *status)
 {
     const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * NV;
     if (c0 >= C) return;
+    if (!in_bounds(status, c0, NV, C)) return;  // debug build: this thread's channels inside C
     float w2[NV], u2[NV];
 #pragma unroll
     for (int j = 0; j < NV; ++j) {
@@ -1024,7 +1044,7 @@ cudaError_t launch_decode_v(const Wkv4Args &a, cudaStream_t s)
     const unsigned by = static_cast<unsigned>(a.B < 65535 ? a.B : 65535);
     wkv4_decode_kernel<T, NV><<<dim3(static_cast<unsigned>(bx), by), 256, 0, s>>>(
         a.B, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
-        static_cast<T *>(a.y), a.sT);
+        static_cast<T *>(a.y), a.sT, a.status);
     return cudaGetLastError();
 }
 
@@ -1050,7 +1070,7 @@ cudaError_t launch_L(const Wkv4Args &a, cudaStream_t s)
     if (blocks == 0) return cudaSuccess;
     kern<<<static_cast<unsigned>(blocks), kThreads, smem, s>>>(
         a.B, a.T, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
-        static_cast<T *>(a.y), a.sT);
+        static_cast<T *>(a.y), a.sT, a.status);
     return cudaGetLastError();
 }
 

@@ -181,7 +181,8 @@ __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_forward_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                         const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                         const float *__restrict__ s0, const T *__restrict__ dy, float *__restrict__ dr,
-                        float *__restrict__ ckpt, float *__restrict__ du_part, int omega, const int *only)
+                        float *__restrict__ ckpt, float *__restrict__ du_part, int omega, const int *only,
+                        int *status)
 {
     using U = typename Store<T>::type;
     constexpr int R = kThreads / TPR, E = kN / TPR;
@@ -189,6 +190,11 @@ wkv6_bwd_forward_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const 
     RowStage<U, R> *stg = reinterpret_cast<RowStage<U, R> *>(smem);  // [2]
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
     if (only && !only[n]) return;
+    if (kDebugBounds) {  // every token row of this (b, h) inside [B, T, H, N]
+        const int64_t lim = static_cast<int64_t>(gridDim.x) * Tlen * kN, r0 = (b * Tlen * H + h) * kN;
+        if (!__syncthreads_and(in_bounds(status, r0, kN, lim) && in_bounds(status, r0 + (Tlen - 1) * H * kN, kN, lim)))
+            return;
+    }
     const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
     const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
@@ -217,7 +223,8 @@ wkv6_bwd_forward_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const 
         const RowStage<U, R> &st = stg[c & 1];
         for (int tt = 0; tt < nt; ++tt) {
             const int64_t t = t0 + tt;
-            if (t % kBlock == 0) {  // checkpoint: the state before this token
+            if (t % kBlock == 0 &&  // checkpoint: the state before this token
+                in_bounds(status, (n * nblk + t / kBlock) * (kN * kN) + i * kN, kN, gridDim.x * nblk * kN * kN)) {
                 float *cp = ckpt + (n * nblk + t / kBlock) * (kN * kN) + i * kN;
 #pragma unroll
                 for (int m = 0; m < E / 4; ++m)
@@ -256,7 +263,7 @@ __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
                      const T *__restrict__ dy, const float *__restrict__ dsT, const float *__restrict__ ckpt,
-                     float *__restrict__ dk, float *__restrict__ dw, int omega, const int *only)
+                     float *__restrict__ dk, float *__restrict__ dw, int omega, const int *only, int *status)
 {
     using U = typename Store<T>::type;
     constexpr int R = kThreads / TPR, E = kN / TPR, G = E / 4;
@@ -265,6 +272,11 @@ wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     float4(*stash)[G][kThreads] = reinterpret_cast<float4(*)[G][kThreads]>(smem + 2 * sizeof(RowStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
     if (only && !only[n]) return;
+    if (kDebugBounds) {  // every token row of this (b, h) inside [B, T, H, N]
+        const int64_t lim = static_cast<int64_t>(gridDim.x) * Tlen * kN, r0 = (b * Tlen * H + h) * kN;
+        if (!__syncthreads_and(in_bounds(status, r0, kN, lim) && in_bounds(status, r0 + (Tlen - 1) * H * kN, kN, lim)))
+            return;
+    }
     const int rg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, il = tid / TPR;
     const int i = R * rg + il;
     const int64_t nblk = (Tlen + kBlock - 1) / kBlock;
@@ -280,6 +292,7 @@ wkv6_bwd_rows_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     // this thread's part of a block's checkpoint, loaded one block ahead
     float4 nx[G];
     auto ck = [&](int64_t cb) {
+        if (!in_bounds(status, (n * nblk + cb) * (kN * kN) + i * kN, kN, gridDim.x * nblk * kN * kN)) return;
         const float *cp = ckpt + (n * nblk + cb) * (kN * kN) + i * kN;
 #pragma unroll
         for (int m = 0; m < G; ++m) nx[m] = *reinterpret_cast<const float4 *>(cp + ent<TPR>(p, 4 * m));
@@ -373,7 +386,7 @@ __global__ void __launch_bounds__(kThreads)
 wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                      const T *__restrict__ w, const float *__restrict__ u, const T *__restrict__ dy,
                      const float *__restrict__ dsT, float *__restrict__ dv, float *__restrict__ ds0, int omega,
-                     const int *only)
+                     const int *only, int *status)
 {
     using U = typename Store<T>::type;
     constexpr int S = kThreads / TPR, R = S * CPT, E = kN / TPR;
@@ -382,6 +395,11 @@ wkv6_bwd_cols_kernel(int64_t Tlen, int64_t H, const T *__restrict__ r, const T *
     ColWork<R> &wk = *reinterpret_cast<ColWork<R> *>(smem + sizeof(ColStage<U, R>));
     const int64_t n = blockIdx.x, b = n / H, h = n % H;
     if (only && !only[n]) return;
+    if (kDebugBounds) {  // every token row of this (b, h) inside [B, T, H, N]
+        const int64_t lim = static_cast<int64_t>(gridDim.x) * Tlen * kN, r0 = (b * Tlen * H + h) * kN;
+        if (!__syncthreads_and(in_bounds(status, r0, kN, lim) && in_bounds(status, r0 + (Tlen - 1) * H * kN, kN, lim)))
+            return;
+    }
     const int cg = blockIdx.y, tid = threadIdx.x, p = tid % TPR, jl = tid / TPR;
     const int warp = tid / 32, lane = tid % 32;
     const int64_t nchunks = (Tlen + kChunk - 1) / kChunk;
@@ -545,16 +563,16 @@ cudaError_t launch_all(const Wkv6BwdArgs &a, const BwdLayout &L, const int *only
     const T *dy = static_cast<const T *>(a.dy);
     // grid: (b, h) x the row (column) groups of a head
     wkv6_bwd_forward_kernel<T, kFwdTPR><<<dim3(nbh, kFwdTPR / 2), kThreads, fwd_smem<T>(), s>>>(
-        a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om, only);
+        a.T, a.H, r, k, v, w, a.u, a.s0, dy, a.dr, ckpt, du_part, om, only, a.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_rows_kernel<T, kRowsTPR><<<dim3(nbh, kRowsTPR / 2), kThreads, rows_smem<T>(), s>>>(
-        a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om, only);
+        a.T, a.H, r, k, v, w, a.u, dy, a.dsT, ckpt, a.dk, a.dw, om, only, a.status);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     wkv6_bwd_cols_kernel<T, kColsTPR, kColsCPT><<<dim3(nbh, kN / (kThreads / kColsTPR * kColsCPT)), kThreads,
                                                    cols_smem<T>(), s>>>(
-        a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om, only);
+        a.T, a.H, r, k, w, a.u, dy, a.dsT, a.dv, a.ds0, om, only, a.status);
     return cudaGetLastError();
 }
 

@@ -200,6 +200,12 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
         const int cc = REV ? nch - 1 - n : n;
         const int s = n % kSStages;
         const uint32_t dst = smem_u32(sm + s * L::stage), bar = bar_full0 + 8 * s;
+        // debug build: the chunk starts inside T; the next forward state inside the
+        // checkpoints (a copy that fails is not issued; its wait then runs out)
+        if (!tma_coord_ok(p.status, 0, 2, kN, static_cast<int64_t>(cc) * kC, p.T)) return;
+        if (REV && !in_bounds(p.status, (bh * (nch + 1) + cc + 1) * kC, kC,
+                              static_cast<int64_t>(gridDim.x) * (nch + 1) * kC))
+            return;
         bar_expect_tx(bar, L::stage);
         tma_load_4d(dst, &map_x, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
         tma_load_4d(dst + kTile, &map_y, 0, static_cast<int>(h), cc * kC, static_cast<int>(b), bar);
@@ -284,9 +290,14 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
         const int q = warp - 4, lr = lane & 15, hi = lane >> 4, row = 16 * q + lr, colh = 32 * hi;
         const uint32_t tl = tbase + (static_cast<uint32_t>(32 * q) << 16);
         const bool issuer_mma = tid == 128;
+        const int64_t nbh = gridDim.x;
+        // debug build: this thread's entries of the checkpoints, row dots and states
+        const bool ck_ok = in_bounds(p.status, ((bh * nck + nck - 1) * kN + row) * kN + colh, 32, nbh * nck * kN * kN) &&
+                           in_bounds(p.status, (bh * nch + nch - 1) * kN + row, 1, nbh * nch * kN);
+        const bool st_ok = in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nbh * kN * kN);
         {
             float v[32];
-            if (p.init) {
+            if (p.init && st_ok) {
                 const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -320,7 +331,7 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
             if (issuer_tma && n > 0 && issued < nch) issue(issued++);
             float v[32];
             tmem_ld32(tl, v);
-            st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, v);
+            if (ck_ok) st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, v);
             if (REV) {  // rowdot(dS_end, S_end): S_end = the forward state after chunk cc
                 float part = 0.f;
 #pragma unroll
@@ -331,7 +342,7 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
                     for (int e = 0; e < 8; ++e) part = fmaf(v[8 * i + e], x[e], part);
                 }
                 part += __shfl_xor_sync(0xffffffffu, part, 16);
-                if (hi == 0) p.rowdot[(bh * nch + cc) * kN + row] = part;
+                if (hi == 0 && ck_ok) p.rowdot[(bh * nch + cc) * kN + row] = part;
             }
             const float d = Dv[s * 64 + row];
 #pragma unroll
@@ -359,9 +370,9 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
                 fence_after();
                 float v[32];
                 tmem_ld32(tl, v);
-                if (!REV)
+                if (!REV && ck_ok)
                     st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, v);
-                else if (p.fin)
+                else if (REV && p.fin && st_ok)
                     st_f32x32(p.fin + (bh * kN + row) * kN + colh, v);
             }
         }
@@ -531,6 +542,15 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
         const int64_t t0 = static_cast<int64_t>(cc) * kC;
         const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
         waited = 0;
+        if (kDebugBounds) {  // the chunk inside T, its checkpoint rows, u, row dots and du shares
+            const int64_t nbh = nitems / nch;
+            const bool ok =
+                tma_coord_ok(p.status, 0, 2, kN, t0, p.T) && in_bounds(p.status, bh, 1, nbh) &&
+                in_bounds(p.status, (bh * (nch + 1) + cc) * kC, kC, nbh * (nch + 1) * kC) &&
+                in_bounds(p.status, (bh * nch + cc) * kC, kC, nbh * nch * kC) &&
+                in_bounds(p.status, h * kN, kN, p.H * kN) && in_bounds(p.status, (bh * nch + cc) * kN, kN, nitems * kN);
+            if (!__syncthreads_and(ok)) continue;
+        }
         if (tid == 0) {
             bulk_wait_read<0>();  // the previous item's gradient stores have read their slots
             bar_expect_tx(bar_full, 7 * kTile);

@@ -86,6 +86,7 @@ struct ChunkedParams {
     int state_only;        // 1: only the segment's local end state (from zero) and decay
     float *seg;            // [B*H][segments-1][N*N + N]: local end state, then decay product
     int nseg;              // segments per sequence
+    int64_t seg_cap;       // floats of scratch behind seg (index checks of the debug build)
     // in-place state update of a split sequence (sT == s0): the state-only pass copies s0
     // here (segment 0's CTAs) and the full pass reads the copy, so no CTA can read s0 after
     // the last segment has overwritten it
@@ -100,9 +101,13 @@ constexpr int kSegStride = kN * kN + kN;
 // TMA of chunk c (r, k, v, w tiles of one head) into its stage, one thread.
 __device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full0, const CUtensorMap *mr,
                                             const CUtensorMap *mk, const CUtensorMap *mv,
-                                            const CUtensorMap *mw, int c, int cabs, int h, int b, bool with_r)
+                                            const CUtensorMap *mw, int c, int cabs, int h, int b, bool with_r,
+                                            int *status, int64_t T)
 {
     const int s = c % kStages;  // c counts chunks within this CTA's segment
+    // debug build: a tile starting past T is not issued (its wait then runs out)
+    if (!tma_coord_ok(status, 0, 2, kN, static_cast<int64_t>(cabs) * kC, T)) return;
+    if (!in_bounds(status, OFF_STAGE + s * kStageBytes, kStageBytes, OFF_SB)) return;
     const uint32_t dst = smem_u32(sm + OFF_STAGE + s * kStageBytes);
     const uint32_t bar = bar_full0 + 8 * s;
     bar_expect_tx(bar, with_r ? kStageBytes : kStageBytes - kTile);
@@ -163,6 +168,10 @@ template <bool GATED>
 __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[32], int64_t tok, int64_t b,
                                             int64_t h, int colh, bool valid, const float *lns)
 {
+    // debug build: the row must be a token of the sequence and lie inside y (and g)
+    valid = valid && in_bounds(p.status, tok, 1, p.T) &&
+            in_bounds(p.status, ((b * p.T + tok) * p.H + h) * kN + colh, 32,
+                      static_cast<int64_t>(gridDim.x) * p.T * kN);
     if (GATED) {
         float s = 0.f;
 #pragma unroll
@@ -288,7 +297,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         int n0 = 0;
         for (; n0 < kStages - 1 && n0 < nchunks; ++n0)
             issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, n0, cb + n0, static_cast<int>(h),
-                        static_cast<int>(b), !so);
+                        static_cast<int>(b), !so, p.status, T);
         misc[8] = n0;
     }
 
@@ -304,7 +313,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         const int a = warp, hf = lane >> 4, cq = lane & 15;
         const int t0h = 16 * a + 8 * hf;
         const uint32_t cbyte = 8 * cq;
-        const Q4 u4 = ld_q4(p.u + h * kN + 4 * cq);
+        const Q4 u4 = in_bounds(p.status, h * kN + 4 * cq, 4, p.H * kN) ? ld_q4(p.u + h * kN + 4 * cq) : one4();
         for (int c = 0; c < nchunks && !abort; ++c) {
             const int s = c % kStages;
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
@@ -484,7 +493,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         int issued = misc[8];
         if (GATED && !so) {  // the head's LayerNorm scale and shift (read after the loop's first barrier)
             const int t = tid - kPrepThreads;
-            lns[t] = t < kN ? p.ln_w[h * kN + t] : p.ln_b[h * kN + t - kN];
+            if (in_bounds(p.status, h * kN + (t & (kN - 1)), 1, p.H * kN))
+                lns[t] = t < kN ? p.ln_w[h * kN + t] : p.ln_b[h * kN + t - kN];
         }
 
         // scores of chunk c into TMEM (issuer only)
@@ -513,7 +523,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 
         int ok = 1;
         if (iss_a && !abort && !so) ok = issue_scores(0);
-        if (so && p.s0copy && g == 0) {  // in-place split: keep s0 for the full pass
+        const int64_t nstate = static_cast<int64_t>(gridDim.x) * kN * kN;  // floats of s0 / sT
+        // debug build: TMEM columns of this thread inside the allocation
+        in_bounds(p.status, COL_O + colh, 32, kTmemCols);
+        if (so && p.s0copy && g == 0 && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
+            // in-place split: keep s0 for the full pass
             const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
             float4 *dst = reinterpret_cast<float4 *>(p.s0copy + (bh * kN + row) * kN + colh);
 #pragma unroll
@@ -522,7 +536,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         {   // initial state into TMEM: s0 advanced over the earlier segments (zero for a
             // state-only pass, which wants the segment's local contribution)
             float v[32];
-            if (p.s0 && !so) {
+            if (p.s0 && !so && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
                 const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -538,6 +552,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             }
             if (!so) {
                 for (int gp = 0; gp < g; ++gp) {  // S <- diag(D_g') S + S_g'
+                    if (!in_bounds(p.status, (bh * (p.nseg - 1) + gp) * kSegStride, kSegStride, p.seg_cap)) break;
                     const float *sg = p.seg + (bh * (p.nseg - 1) + gp) * kSegStride;
                     const float d = sg[kN * kN + row];
                     const float4 *src = reinterpret_cast<const float4 *>(sg + row * kN + colh);
@@ -575,7 +590,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 if (issuer) {
                     while (issued < nchunks && issued <= c + kStages - 1) {
                         issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
-                                    static_cast<int>(h), static_cast<int>(b), false);
+                                    static_cast<int>(h), static_cast<int>(b), false, p.status, T);
                         ++issued;
                     }
                     misc[8] = issued;
@@ -610,12 +625,14 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     fence_after();
                     float sv[32];
                     tmem_ld32(tlane + COL_S, sv);
-                    float *sg = p.seg + (bh * (p.nseg - 1) + g) * kSegStride;
-                    float4 *dst = reinterpret_cast<float4 *>(sg + row * kN + colh);
+                    if (in_bounds(p.status, (bh * (p.nseg - 1) + g) * kSegStride, kSegStride, p.seg_cap)) {
+                        float *sg = p.seg + (bh * (p.nseg - 1) + g) * kSegStride;
+                        float4 *dst = reinterpret_cast<float4 *>(sg + row * kN + colh);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i)
-                        dst[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
-                    if (hi == 0) sg[kN * kN + row] = dprod;
+                        for (int i = 0; i < 8; ++i)
+                            dst[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
+                        if (hi == 0) sg[kN * kN + row] = dprod;
+                    }
                 }
             }
         } else {
@@ -652,7 +669,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     const int user = issued - 2;  // chunk that would use this stage as scratch
                     if (user >= c && misc[2 + user % kStages]) break;
                     issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
-                                static_cast<int>(h), static_cast<int>(b), true);
+                                static_cast<int>(h), static_cast<int>(b), true, p.status, T);
                     ++issued;
                 }
                 misc[8] = issued;
@@ -772,7 +789,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 const int64_t t0 = static_cast<int64_t>(cb + nchunks - 1) * kC;
                 const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
                 store_y_row<GATED>(p, ov, t0 + row, b, h, colh, row < tv, lns);
-                if (p.sT && g == p.nseg - 1) {
+                if (p.sT && g == p.nseg - 1 && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
                     float sv[32];
                     tmem_ld32(tlane + COL_S, sv);
                     float4 *sd = reinterpret_cast<float4 *>(p.sT + (bh * kN + row) * kN + colh);
@@ -964,6 +981,7 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
                       static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G),
+                      static_cast<int64_t>(bh) * (G - 1) * kSegStride,
                       nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     float *seg = nullptr;
     if (G > 1) {
@@ -1079,6 +1097,7 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
                       static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G),
+                      (G - 1) * per_segment / static_cast<int64_t>(sizeof(float)),
                       nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     if (G > 1) {
         // the state-only pass writes every scratch entry the full pass reads (the s0 copy of

@@ -50,7 +50,7 @@ template <typename T>
 __global__ void __launch_bounds__(kN)
 wkv6_serial_kernel(int64_t T_len, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
-                   const float *s0, T *__restrict__ y, float *sT, int omega)
+                   const float *s0, T *__restrict__ y, float *sT, int omega, int *status)
 {
     __shared__ __align__(16) float sr[2][kN], sk[2][kN], sw[2][kN];
     __shared__ __align__(16) float su[kN];
@@ -58,6 +58,13 @@ wkv6_serial_kernel(int64_t T_len, int64_t H, const T *__restrict__ r, const T *_
     const int64_t n = blockIdx.x;  // b * H + h
     const int64_t b = n / H, h = n % H;
     const int j = threadIdx.x;
+    if (kDebugBounds) {  // every token row of this (b, h) inside [B, T, H, N]; u of the head
+        const int64_t lim = static_cast<int64_t>(gridDim.x) * T_len * kN;
+        const int64_t b0 = (b * T_len * H + h) * kN + j;
+        const bool ok = in_bounds(status, b0, 1, lim) && in_bounds(status, b0 + (T_len - 1) * H * kN, 1, lim) &&
+                        in_bounds(status, h * kN + j, 1, H * kN);
+        if (!__syncthreads_and(ok)) return;
+    }
 
     float S[kN];
     const float *s0p = s0 ? s0 + n * kN * kN : nullptr;
@@ -142,7 +149,7 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
                    const T *__restrict__ v, const T *__restrict__ w,
                    const float *__restrict__ u, const float *s0, T *__restrict__ y, float *sT,
                    const T *__restrict__ g, const float *__restrict__ ln_w, const float *__restrict__ ln_b,
-                   float eps, int omega)
+                   float eps, int omega, int *status)
 {
     __shared__ __align__(16) float red[16][kN];
     __shared__ float bred[16];
@@ -152,6 +159,14 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
     const int64_t h = n % H;
     const int tid = threadIdx.x, ig = tid >> 4, j4 = tid & 15;
     const int64_t vbase = n * kN;
+    if (kDebugBounds) {  // the token row, the state block and u of this thread
+        const int64_t nall = gridDim.x;
+        const bool ok = in_bounds(status, vbase + 4 * ig, 4, nall * kN) &&
+                        in_bounds(status, vbase + 4 * j4, 4, nall * kN) &&
+                        in_bounds(status, n * kN * kN + (4 * ig + 3) * kN + 4 * j4, 4, nall * kN * kN) &&
+                        in_bounds(status, h * kN + 4 * ig, 4, H * kN);
+        if (!__syncthreads_and(ok)) return;
+    }
 
     const float4 rr = ld4(r + vbase + 4 * ig);
     const float4 kk = ld4(k + vbase + 4 * ig);
@@ -233,12 +248,12 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s)
         wkv6_serial_kernel<T><<<static_cast<unsigned>(blocks), kN, 0, s>>>(
             a.T, a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k),
             static_cast<const T *>(a.v), static_cast<const T *>(a.w), a.u, a.s0,
-            static_cast<T *>(a.y), a.sT, a.omega ? 1 : 0);
+            static_cast<T *>(a.y), a.sT, a.omega ? 1 : 0, a.status);
     } else {
         wkv6_serial_kernel<float><<<static_cast<unsigned>(blocks), kN, 0, s>>>(
             a.T, a.H, static_cast<const float *>(a.r), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), static_cast<const float *>(a.w), a.u, a.s0,
-            static_cast<float *>(a.y), a.sT, a.omega ? 1 : 0);
+            static_cast<float *>(a.y), a.sT, a.omega ? 1 : 0, a.status);
     }
     return cudaGetLastError();
 }
@@ -254,12 +269,13 @@ cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s)
         wkv6_decode_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k),
             static_cast<const T *>(a.v), static_cast<const T *>(a.w), a.u, a.s0,
-            static_cast<T *>(a.y), a.sT, static_cast<const T *>(a.g), a.ln_w, a.ln_b, a.eps, a.omega ? 1 : 0);
+            static_cast<T *>(a.y), a.sT, static_cast<const T *>(a.g), a.ln_w, a.ln_b, a.eps, a.omega ? 1 : 0,
+            a.status);
     } else {
         wkv6_decode_kernel<float><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
             a.H, static_cast<const float *>(a.r), static_cast<const float *>(a.k),
             static_cast<const float *>(a.v), static_cast<const float *>(a.w), a.u, a.s0,
-            static_cast<float *>(a.y), a.sT, nullptr, nullptr, nullptr, 0.f, a.omega ? 1 : 0);
+            static_cast<float *>(a.y), a.sT, nullptr, nullptr, nullptr, 0.f, a.omega ? 1 : 0, a.status);
     }
     return cudaGetLastError();
 }

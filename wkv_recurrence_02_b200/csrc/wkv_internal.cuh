@@ -12,11 +12,38 @@ namespace wkv {
 
 // Status codes written by kernels into the device status word (same values as rwkv_status).
 constexpr int kStatusTimeout = -6;
+constexpr int kStatusBounds = -9;
 
 // Record the first device-side error; later errors keep the first one.
 __device__ __forceinline__ void record_status(int *status, int code)
 {
     if (status) atomicCAS(status, 0, code);
+}
+
+// Index checks of the debug build.  Compiled with WKV_DEBUG_BOUNDS, in_bounds() checks that the
+// n elements from index i lie inside [0, limit), records RWKV_ERR_BOUNDS in the device status
+// word when they do not, and returns the answer, so that the caller skips the access (nothing
+// traps).  In ordinary builds it is the constant true and the checks compile away.
+#ifdef WKV_DEBUG_BOUNDS
+constexpr bool kDebugBounds = true;
+#else
+constexpr bool kDebugBounds = false;
+#endif
+__device__ __forceinline__ bool in_bounds(int *status, int64_t i, int64_t n, int64_t limit)
+{
+    if (!kDebugBounds) return true;
+    const bool ok = i >= 0 && n >= 0 && i + n <= limit;
+    if (!ok) record_status(status, kStatusBounds);
+    return ok;
+}
+// A TMA tile coordinate pair for an innermost coordinate x of element size es: x must start on
+// a 16-byte boundary and inside the tensor, and the outer coordinate inside its extent.
+__device__ __forceinline__ bool tma_coord_ok(int *status, int64_t x, int es, int64_t xdim, int64_t y, int64_t ydim)
+{
+    if (!kDebugBounds) return true;
+    const bool ok = x >= 0 && x < xdim && (x * es) % 16 == 0 && y >= 0 && y < ydim;
+    if (!ok) record_status(status, kStatusBounds);
+    return ok;
 }
 
 struct Wkv4Args {

@@ -9,6 +9,7 @@ Functions mirror the C entry points:
   wkv6_forward(r, k, v, w, u, s0=None, want_state=True) -> (y, sT)      | y
 The calls are asynchronous on torch's current CUDA stream.
 """
+import contextlib
 import ctypes
 import os
 import re
@@ -22,7 +23,7 @@ HEADER = os.path.join(os.path.dirname(_HERE), "include", "rwkv_wkv.h")
 RWKV_OK = 0
 STATUS_NAMES = {0: "RWKV_OK", -1: "RWKV_ERR_NULL", -2: "RWKV_ERR_SHAPE", -3: "RWKV_ERR_UNSUPPORTED",
                 -4: "RWKV_ERR_ALIAS", -5: "RWKV_ERR_CUDA", -6: "RWKV_ERR_TIMEOUT",
-                -7: "RWKV_ERR_ALIGN", -8: "RWKV_ERR_ARG"}
+                -7: "RWKV_ERR_ALIGN", -8: "RWKV_ERR_ARG", -9: "RWKV_ERR_BOUNDS"}
 ALGOS = {"auto": 0, "serial": 1, "chunked": 2}
 
 _i64 = ctypes.c_int64
@@ -95,8 +96,23 @@ def load(path: str = LIB_PATH):
     lib.rwkv_last_error.restype = ctypes.c_char_p
     lib.rwkv_abi_version.argtypes = []
     lib.rwkv_abi_version.restype = ctypes.c_int
+    lib.rwkv_debug_bounds.argtypes = []
+    lib.rwkv_debug_bounds.restype = ctypes.c_int
     _lib = lib
     return lib
+
+
+@contextlib.contextmanager
+def using_library(path: str):
+    """Route the calls of this module to another build of the library (e.g. the bounds-checked
+    debug build, libwkv_debug.so) inside the block; the default library is restored after."""
+    global _lib
+    prev = _lib
+    _lib = None
+    try:
+        yield load(path)
+    finally:
+        _lib = prev
 
 
 def _check(rc):
