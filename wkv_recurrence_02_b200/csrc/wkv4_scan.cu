@@ -658,16 +658,24 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     unsigned char *sbase = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                              ~static_cast<uintptr_t>(127));
     const uint32_t bar0 = smem_u32(sbase + NB * 2 * L * BLK);  // + 8 * buffer
+    // [warp][unit][(a, b, p) x NC channels, segment count]: each warp's scan total
+    float *wtot = reinterpret_cast<float *>(sbase + NB * 2 * L * BLK + 8 * NB);
 
     const int64_t C = p.C, T_len = p.T;
     const int64_t cblocks = (C + kCh - 1) / kCh;
     const int b = static_cast<int>(blockIdx.x / cblocks);
     const int c0 = static_cast<int>((blockIdx.x % cblocks) * kCh);
+    // Lanes: a row of block i (token i of all 32 segments, 16 channels each) is 32 x RB bytes;
+    // thread x reads its 8 bytes at 8 x, so each warp reads 256 contiguous bytes (no bank
+    // conflicts).  That makes lane l of warp h the unit q = l % U (NC channels) of segment
+    // h * SPW + l / U, with U units per row and SPW segments per warp.
+    constexpr int U = kCh / NC, SPW = kSegs / U;
     const int h = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int cb = c0 + NC * h;  // first channel of this lane
+    const int q = lane % U, seg_l = h * SPW + lane / U;  // this lane's unit and segment
+    const int cb = c0 + NC * q;                          // first channel of this lane
     if (kDebugBounds) {  // the batch row; this lane's state entries; its units inside a buffer
         const bool ok = in_bounds(p.status, b, 1, p.B) &&
-                        in_bounds(p.status, lane * RB + NC * static_cast<int>(sizeof(T)) * h + (L - 1) * BLK,
+                        in_bounds(p.status, 8 * static_cast<int>(threadIdx.x) + (L - 1) * BLK,
                                   NC * static_cast<int>(sizeof(T)), L * BLK) &&
                         (cb >= C || in_bounds(p.status, static_cast<int64_t>(b) * 3 * C + 2 * C + cb, 1, p.B * 3 * C));
         if (!__syncthreads_and(ok)) return;
@@ -733,9 +741,9 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         abort = __syncthreads_or(!mbar_wait(bar0 + 8 * (tile % NB), (tile / NB) & 1, p.spin_limit));
         if (abort) break;
         // this lane's unit in row 0 of its segment; row i is BLK bytes further
-        unsigned char *uk = sk + lane * RB + NC * static_cast<int>(sizeof(T)) * h;
-        const unsigned char *uv = sv + lane * RB + NC * static_cast<int>(sizeof(T)) * h;
-        const int nv = seg0 + lane < nsegs ? L : 0;
+        unsigned char *uk = sk + 8 * threadIdx.x;
+        const unsigned char *uv = sv + 8 * threadIdx.x;
+        const int nv = seg0 + seg_l < nsegs ? L : 0;
 
         // pass 1: local summaries against the segment's last key; key range
         St la[NC];
@@ -788,11 +796,13 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
         }
 
-        // inclusive scan over lanes (segment order) with segment lengths, then the
-        // exclusive prefix with the carry from earlier tiles folded in
+        // inclusive scan over this warp's segments (lanes U apart share a unit) with segment
+        // lengths; the warps' totals then meet in shared memory, and each lane folds the
+        // carry from earlier tiles, the earlier warps' totals and its warp's exclusive
+        // prefix, in segment order
         float n_inc = static_cast<float>(nv);
 #pragma unroll
-        for (int off = 1; off < kSegs; off <<= 1) {
+        for (int off = U; off < 32; off <<= 1) {
             const float on = __shfl_up_sync(0xffffffffu, n_inc, off);
 #pragma unroll
             for (int n = 0; n < NC; ++n) {
@@ -801,16 +811,34 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             }
             if (lane >= off) n_inc += on;
         }
-        float n_exc = __shfl_up_sync(0xffffffffu, n_inc, 1);
-        if (lane == 0) n_exc = 0.f;
-        const float n_tot = __shfl_sync(0xffffffffu, n_inc, kSegs - 1);
+        float n_exc = __shfl_up_sync(0xffffffffu, n_inc, U);
+        if (lane < U) n_exc = 0.f;
+        if (lane >= 32 - U) {  // the warp's total for unit q
+            float *tw = wtot + (h * U + q) * (3 * NC + 1);
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                tw[3 * n] = la[n].a;
+                tw[3 * n + 1] = la[n].b;
+                tw[3 * n + 2] = la[n].p;
+            }
+            tw[3 * NC] = n_inc;
+        }
+        __syncthreads();
         St pa[NC];
 #pragma unroll
         for (int n = 0; n < NC; ++n) {
-            St e = shfl_up(la[n], 1);
-            if (lane == 0) e = empty;
-            pa[n] = combine(carry[n], e, n_exc * w2[n]);
-            carry[n] = combine(carry[n], shfl_idx(la[n], kSegs - 1), n_tot * w2[n]);
+            St before = carry[n], all = carry[n];
+            for (int hw = 0; hw < kCh / NC; ++hw) {
+                const float *tw = wtot + (hw * U + q) * (3 * NC + 1);
+                const St t{tw[3 * n], tw[3 * n + 1], tw[3 * n + 2]};
+                const float nw = tw[3 * NC] * w2[n];
+                if (hw < h) before = combine(before, t, nw);
+                all = combine(all, t, nw);
+            }
+            St e = shfl_up(la[n], U);
+            if (lane < U) e = empty;
+            pa[n] = combine(before, e, n_exc * w2[n]);
+            carry[n] = all;
         }
 
         // pass 2: outputs from the exact incoming state; y replaces k in place
@@ -881,7 +909,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         return;
     }
 
-    if (p.sT && lane == 0) {
+    if (p.sT && h == 0 && lane < U) {  // every lane of a unit holds the same carry
         float *sp = p.sT + static_cast<int64_t>(b) * 3 * C;
 #pragma unroll
         for (int n = 0; n < NC; ++n) {
@@ -903,7 +931,9 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
     constexpr int RB = kCh * sizeof(T);
     constexpr int BLK = kSegs * RB;
     constexpr int kThr = 32 * (kCh / NC);
-    const size_t smem = NB * 2ull * L * BLK + 128 + 16;  // buffers of k and v blocks, slack, mbarriers
+    constexpr int U = kCh / NC;
+    // buffers of k and v blocks, alignment slack, mbarriers, the warps' scan totals
+    const size_t smem = NB * 2ull * L * BLK + 128 + 8 * NB + sizeof(float) * (kCh / NC) * U * (3 * NC + 1);
     auto enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     // 4-D view (channel, token within segment, segment, batch row) of [B, T, C]; L divides T
