@@ -10,6 +10,10 @@ One step is one pass of the whole hot path over synthetic inputs resident in HBM
   * WKV-6 decode: one T=1 step at B=256, H=64 with a random fp32 state, updated in place.
 The metric counts B*T tokens of every call (each WKV-4 layer call counts its own B*T).
 Inputs per step (~2.4 GB) exceed the 126 MB L2, so no L2 flush is needed between steps.
+The K timed steps are captured as one CUDA graph (22 kernel launches per step, the calls
+exactly as a user makes them) and replayed once between CUDA events, so host launch
+overhead is not timed; each call's own duration is then measured by replaying a graph of
+that call, and the end-to-end figure runs the same step eagerly through the public API.
 
 Under torchrun each rank runs the same step on its own GPU (the path shards over
 independent sequences/heads with no exchange step: weak scaling, no collective on the
@@ -185,7 +189,8 @@ def step_config(world):
     """The `config` object of the JSON line (the same for both arms)."""
     return {"workload": WORKLOAD, "tokens_per_step_per_gpu": STEP_TOKENS,
             "l2": "inputs larger than L2 (~2.4 GB per step per GPU); no flush",
-            "parallelism": f"replicas x{world} (independent sequences, no collective)"}
+            "parallelism": f"replicas x{world} (independent sequences, no collective)",
+            "launch": "the K steps captured as one CUDA graph, replayed once"}
 
 
 def max_over_ranks(values, dist, device=None):
@@ -215,28 +220,27 @@ def run_ours(args, rank, world, dist):
     dev = torch.device("cuda", local)
     ops.load()
     wl = Workload(torch, inputs, dev)
-    stream = torch.cuda.current_stream(dev)
+    stream = torch.cuda.Stream(dev)  # graphs are captured on a stream of their own
+    torch.cuda.set_stream(stream)
 
     def barrier():
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize(dev)
 
-    # warm-up
+    # warm-up (eager: sets up the library's per-device state, pools and kernel attributes)
     for _ in range(args.warmup):
         wl.step(ops)
     barrier()
 
-    # timed: whole steps, plus per-launch events for the per-kernel roofline
-    events = []
-
-    def rec(name, fn):
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fn()
-        b.record(stream)
-        events.append((name, a, b))
+    # timed: the K steps captured as one CUDA graph (22 launches per step, no host work
+    # between them), replayed once between a barrier and events on the launching stream
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for _ in range(args.steps):
+            wl.step(ops)
+    graph.replay()  # untimed: the first replay uploads the graph
+    barrier()
 
     sampler = ClockSampler(local)
     sampler.start()
@@ -246,16 +250,17 @@ def run_ours(args, rank, world, dist):
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(args.steps):
-        wl.step(ops, rec)
+    graph.replay()
     e1.record(stream)
     barrier()
     t_wall1 = time.time()
     sampler.stop()
     ms = e0.elapsed_time(e1)
-    per = {}
-    for name, a, b in events:
-        per.setdefault(name, []).append(a.elapsed_time(b))
+    del graph
+
+    # each call of the step on its own, for the per-kernel roofline: a CUDA graph of the call
+    # replayed back to back between events (the same launches, inputs and outputs as the step)
+    per = measure_calls(torch, ops, wl, stream, reps=20)
 
     # end to end through the public API with host buffers: H2D of every input, D2H of results
     e2e_ms, h2d, d2h = run_e2e(torch, ops, wl, stream, dev, max(3, min(args.steps, 10)), barrier)
@@ -327,6 +332,30 @@ def dominant_roofline(kern, fam, per, hbm, peak_kind):
             "achieved": round(achieved, 1), "peak": hbm, "peak_kind": peak_kind, "unit": "GB/s",
             "frac": round(achieved / hbm, 4), "frac_8TBps": round(achieved / NOMINAL_HBM_GBS, 4),
             "traffic": traffic, "traffic_note": note, "calls": calls}
+
+
+def measure_calls(torch, ops, wl, stream, reps):
+    """Per-call durations (ms) of the step's launches, keyed like Workload.step's names: each
+    call captured as a CUDA graph and replayed `reps` times between CUDA events."""
+    calls = []
+    wl.step(ops, lambda name, fn: calls.append((name, fn)))
+    torch.cuda.synchronize()
+    per = {}
+    for name, fn in calls:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        g.replay()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(reps):
+            g.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        per.setdefault(name, []).append(a.elapsed_time(b) / reps)
+        del g
+    return per
 
 
 def _time_us(torch, stream, dev, fn, reps):
