@@ -359,15 +359,23 @@ def measure_calls(torch, ops, wl, stream, reps):
 
 
 def _time_us(torch, stream, dev, fn, reps):
+    """Average duration (us) of fn's launches: fn captured as a CUDA graph (after three eager
+    calls) and the graph replayed `reps` times between CUDA events."""
     for _ in range(3):
         fn()
+    torch.cuda.synchronize(dev)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    g.replay()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
     a.record(stream)
     for _ in range(reps):
-        fn()
+        g.replay()
     b.record(stream)
     torch.cuda.synchronize(dev)
+    del g
     return a.elapsed_time(b) * 1e3 / reps
 
 
@@ -448,16 +456,8 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
     st[:, 0] = torch.randn(B, C, device=dev)
     st[:, 1] = 1.0 + torch.rand(B, C, device=dev)
     y = torch.empty_like(k)
-    for _ in range(3):
-        ops.wkv4_forward(w, u, k, v, s0=st, sT=st, y=y, want_state=True)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        ops.wkv4_forward(w, u, k, v, s0=st, sT=st, y=y, want_state=True)
-    b.record(stream)
-    torch.cuda.synchronize(dev)
-    us = a.elapsed_time(b) * 1e3 / reps
+    us = _time_us(torch, stream, dev, lambda: ops.wkv4_forward(w, u, k, v, s0=st, sT=st, y=y, want_state=True),
+                  reps)
     nbytes = B * C * (2 * 2 + 2 + 2 * 3 * 4) + 2 * C * 4  # k, v, y bf16; state in and out; w, u
     gbs = nbytes / (us * 1e-6) / 1e9
     rows["wkv4_decode_B2048_C4096"] = {"avg_us": round(us, 2), "algorithmic_bytes": nbytes,

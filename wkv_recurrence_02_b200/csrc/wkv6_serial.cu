@@ -20,9 +20,14 @@
 //    stores, so the 2 x 16 KB state stream per head is fully coalesced.  Partial
 //    outputs are reduced over the 16 row groups through shared memory.  With a gate g the
 //    64 outputs of the head go through the fused LayerNorm + SiLU gate before the store.
+//    It serves T == 1 calls with the fused output stage or without an initial state.
+//  * wkv6_decode_stream_kernel -- T == 1 with an initial state: the same update by
+//    persistent CTAs that stream the heads' states through a ring of bulk copies.
 // Both kernels can take the decay as its logit omega_t and form w_t = exp(-exp(omega_t)) as
 // they load it.
-#include "wkv_internal.cuh"
+#include "tc_common.cuh"
+
+#include <algorithm>
 
 namespace wkv {
 namespace {
@@ -236,6 +241,140 @@ wkv6_decode_kernel(int64_t H, const T *__restrict__ r, const T *__restrict__ k,
     }
 }
 
+// ------------------------------------------------------------ streaming decode (T == 1)
+// Persistent CTAs of 256 threads, four per SM, each walking heads n = blockIdx.x + i gridDim.x
+// through a 3-stage ring: the head's 16 KB state and its r, k, w, v vectors arrive by bulk
+// copies (mbarrier), the update is made in shared memory by the same 4 x 4 blocks as the
+// kernel above, and the new state leaves by a bulk store.  Two heads' copies stay in flight
+// while one is updated (about 130 KB per SM), so the state stream does not stall between
+// heads.  The stage of head i - 1 is refilled with head i + 2 once head i - 1's store has read
+// it.  Used for every T == 1 call with an initial state and no fused output stage.
+constexpr int kDStages = 3;
+constexpr int kDThreads = 256;
+template <typename T> constexpr int dstage_bytes() { return kN * kN * 4 + 4 * kN * static_cast<int>(sizeof(T)); }
+template <typename T> constexpr int decode_stream_smem()
+{
+    return kDStages * dstage_bytes<T>() + 16 * kN * 4 + 16 * 4 + 8 * kDStages + 128;
+}
+
+// Plain load of an element held in shared memory (ld() above is for global memory: its fp32
+// form is a read-only global load, which must not be given a shared-memory address).
+template <typename T> __device__ __forceinline__ float sld(const T *p);
+template <> __device__ __forceinline__ float sld<float>(const float *p) { return *p; }
+template <> __device__ __forceinline__ float sld<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+
+template <typename T>
+__global__ void __launch_bounds__(kDThreads)
+wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const T *__restrict__ k,
+                          const T *__restrict__ v, const T *__restrict__ w, const float *__restrict__ u,
+                          const float *s0, T *__restrict__ y, float *sT, int omega, int *status, uint32_t limit)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                                          ~static_cast<uintptr_t>(127));
+    constexpr int SB = dstage_bytes<T>();
+    float(*red)[kN] = reinterpret_cast<float(*)[kN]>(sm + kDStages * SB);
+    float *bred = reinterpret_cast<float *>(sm + kDStages * SB + 16 * kN * 4);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kDStages * SB + 16 * kN * 4 + 16 * 4);
+    const uint32_t bar0 = tc::smem_u32(&bars[0]);
+    const int tid = threadIdx.x, ig = tid >> 4, j4 = tid & 15;
+    const int64_t count = (BH - blockIdx.x + gridDim.x - 1) / gridDim.x;  // heads of this CTA
+
+    if (tid == 0) {
+        for (int s = 0; s < kDStages; ++s) tc::bar_init(bar0 + 8 * s, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    auto issue = [&](int64_t i) {  // one thread: the copies of this CTA's i-th head
+        const int64_t n = blockIdx.x + i * gridDim.x;
+        const int s = static_cast<int>(i % kDStages);
+        unsigned char *stg = sm + s * SB;
+        const uint32_t bar = bar0 + 8 * s;
+        if (!in_bounds(status, n * kN * kN, kN * kN, BH * kN * kN) || !in_bounds(status, n * kN, kN, BH * kN)) return;
+        tc::bar_expect_tx(bar, SB);
+        constexpr uint32_t VB = kN * sizeof(T);
+        tc::bulk_load(tc::smem_u32(stg), s0 + n * kN * kN, kN * kN * 4, bar);
+        tc::bulk_load(tc::smem_u32(stg + kN * kN * 4), r + n * kN, VB, bar);
+        tc::bulk_load(tc::smem_u32(stg + kN * kN * 4 + VB), k + n * kN, VB, bar);
+        tc::bulk_load(tc::smem_u32(stg + kN * kN * 4 + 2 * VB), w + n * kN, VB, bar);
+        tc::bulk_load(tc::smem_u32(stg + kN * kN * 4 + 3 * VB), v + n * kN, VB, bar);
+    };
+    if (tid == 0)
+        for (int64_t i = 0; i < kDStages && i < count; ++i) issue(i);
+
+    int abort = 0;
+    for (int64_t i = 0; i < count; ++i) {
+        const int64_t n = blockIdx.x + i * gridDim.x, h = n % H;
+        const int s = static_cast<int>(i % kDStages);
+        unsigned char *stg = sm + s * SB;
+        float *S = reinterpret_cast<float *>(stg);
+        const T *vr = reinterpret_cast<const T *>(stg + kN * kN * 4);
+        const T *vk = vr + kN, *vw = vr + 2 * kN, *vv = vr + 3 * kN;
+        const int ok = tc::bar_wait(bar0 + 8 * s, static_cast<uint32_t>((i / kDStages) & 1), limit);
+        if (__syncthreads_or(!ok)) {
+            abort = 1;
+            break;
+        }
+        float rr[4], kk[4], ww[4], uu[4], vj[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            rr[m] = sld(vr + 4 * ig + m);
+            kk[m] = sld(vk + 4 * ig + m);
+            const float wm = sld(vw + 4 * ig + m);
+            ww[m] = omega ? decay_of_logit(wm) : wm;
+            uu[m] = __ldg(u + h * kN + 4 * ig + m);  // global
+            vj[m] = sld(vv + 4 * j4 + m);
+        }
+        float o[4] = {0.f, 0.f, 0.f, 0.f};
+        float bonus = 0.f;
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+            float4 *row = reinterpret_cast<float4 *>(S + (4 * ig + m) * kN + 4 * j4);
+            float4 x = *row;
+            o[0] = fmaf(rr[m], x.x, o[0]);
+            o[1] = fmaf(rr[m], x.y, o[1]);
+            o[2] = fmaf(rr[m], x.z, o[2]);
+            o[3] = fmaf(rr[m], x.w, o[3]);
+            bonus = fmaf(rr[m] * uu[m], kk[m], bonus);
+            x.x = fmaf(ww[m], x.x, kk[m] * vj[0]);
+            x.y = fmaf(ww[m], x.y, kk[m] * vj[1]);
+            x.z = fmaf(ww[m], x.z, kk[m] * vj[2]);
+            x.w = fmaf(ww[m], x.w, kk[m] * vj[3]);
+            *row = x;
+        }
+        *reinterpret_cast<float4 *>(&red[ig][4 * j4]) = make_float4(o[0], o[1], o[2], o[3]);
+        if (j4 == 0) bred[ig] = bonus;
+        tc::fence_async_smem();  // the new state is read by the bulk store (async proxy)
+        __syncthreads();
+        if (tid == 0 && sT) {
+            if (in_bounds(status, n * kN * kN, kN * kN, BH * kN * kN)) tc::bulk_store(sT + n * kN * kN, tc::smem_u32(stg), kN * kN * 4);
+            tc::bulk_commit();
+        }
+        if (tid < kN) {
+            float acc = 0.f, bsum = 0.f;
+#pragma unroll
+            for (int rg = 0; rg < 16; ++rg) {
+                acc += red[rg][tid];
+                bsum += bred[rg];
+            }
+            st<T>(y + n * kN + tid, fmaf(bsum, sld(vv + tid), acc));
+        }
+        // the stage of head i - 1 takes head i + 2 once that head's store has read it
+        if (tid == 0 && i >= 1 && i + 2 < count) {
+            if (sT) tc::bulk_wait_read<1>();
+            issue(i + 2);
+        }
+        __syncthreads();  // red, bred and this stage are reused
+    }
+    if (abort) {
+        record_status(status, kStatusTimeout);
+        if (tid == 0)  // bounded: the copies in flight land before the CTA exits
+            for (int64_t i = 0; i < count && i < kDStages + 2; ++i)
+                tc::bar_wait(bar0 + 8 * static_cast<int>(i % kDStages), static_cast<uint32_t>((i / kDStages) & 1), limit);
+    }
+    if (tid == 0) tc::bulk_wait_all();
+}
+
 }  // namespace
 
 cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s)
@@ -258,12 +397,43 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s)
     return cudaGetLastError();
 }
 
+namespace {
+template <typename T> cudaError_t launch_decode_stream(const Wkv6Args &a, cudaStream_t s)
+{
+    static bool done[64] = {};
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!done[dev]) {  // racing first calls set the same attribute: harmless
+        e = cudaFuncSetAttribute(wkv6_decode_stream_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 decode_stream_smem<T>());
+        if (e != cudaSuccess) return e;
+        done[dev] = true;
+    }
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    int per_sm = 0;  // resident CTAs per SM (shared memory bound): the grid stays one wave
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, wkv6_decode_stream_kernel<T>, kDThreads,
+                                                      decode_stream_smem<T>());
+    if (e != cudaSuccess) return e;
+    const int64_t bh = a.B * a.H;
+    const unsigned grid = static_cast<unsigned>(std::min<int64_t>(bh, static_cast<int64_t>(std::max(per_sm, 1)) * sms));
+    wkv6_decode_stream_kernel<T><<<grid, kDThreads, decode_stream_smem<T>(), s>>>(
+        bh, a.H, static_cast<const T *>(a.r), static_cast<const T *>(a.k), static_cast<const T *>(a.v),
+        static_cast<const T *>(a.w), a.u, a.s0, static_cast<T *>(a.y), a.sT, a.omega ? 1 : 0, a.status, 100000u);
+    return cudaGetLastError();
+}
+}  // namespace
+
 cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s)
 {
     if (a.T != 1) return wkv6_serial_launch(a, s);
     const int64_t blocks = a.B * a.H;
     if (blocks == 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    // the streaming kernel: an initial state to stream, no fused output stage
+    if (a.s0 && !a.g)
+        return a.bf16 ? launch_decode_stream<__nv_bfloat16>(a, s) : launch_decode_stream<float>(a, s);
     if (a.bf16) {
         using T = __nv_bfloat16;
         wkv6_decode_kernel<T><<<static_cast<unsigned>(blocks), 256, 0, s>>>(
