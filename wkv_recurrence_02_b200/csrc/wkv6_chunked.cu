@@ -137,13 +137,19 @@ __device__ __forceinline__ float half_sum8(const float (&part)[8], int lane)
 
 // Chunk-end path operand rows of one 8-token half sub-block, four channels per thread:
 // Qx -> R slot, Kh -> K slot, and the bonus partials.  FULL: all 8 tokens valid.
+// 1 / prod_{j>=t} w_j is formed as (1/D) prod_{j<t} w_j: a forward running product from
+// `pre` = (1/D) times the product of w before this half, one reciprocal per channel and
+// chunk instead of one per element (on this path D >= 2^-100, so pre stays below 2^100).
 template <bool FULL>
 __device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t cbyte, int tv, const Q4 (&w)[8],
-                                          Q4 after, Q4 u, float (&part)[8])
+                                          Q4 after, Q4 pre, Q4 u, float (&part)[8])
 {
-    Q4 run = after;  // product of w over the tokens after the current one, to the chunk end
+    Q4 suf[8];  // product of w over the tokens after token m of this half, to the chunk end
+    suf[7] = after;
 #pragma unroll
-    for (int m = 7; m >= 0; --m) {
+    for (int m = 7; m >= 1; --m) suf[m - 1] = mul4(suf[m], w[m]);
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
         const int t = t0h + m;
         const uint32_t off = swz(t, cbyte);
         uint2 rr = make_uint2(0u, 0u), kk = rr;
@@ -152,11 +158,10 @@ __device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t c
             kk = ld_u2(st + SLOT_K, off);
         }
         const Q4 r = unpack4(rr), k = unpack4(kk);
-        const Q4 sin = mul4(run, w[m]);
-        st_u2(st + SLOT_R, off, pack4({mul2(r.a, rcp2(sin.a)), mul2(r.b, rcp2(sin.b))}));
-        st_u2(st + SLOT_K, off, pack4(mul4(k, run)));
+        st_u2(st + SLOT_R, off, pack4(mul4(r, pre)));
+        st_u2(st + SLOT_K, off, pack4(mul4(k, suf[m])));
         part[m] = bonus4(r, u, k);
-        run = sin;
+        pre = mul4(pre, w[m]);
     }
 }
 
@@ -319,14 +324,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
             const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
             const int tv = static_cast<int>(T - t0 < kC ? T - t0 : kC);
-            // one thread waits for the stage; the others park on the group barrier
-            int ok = tid == 0 ? bar_wait_spin(bar_full0 + 8 * s, (c / kStages) & 1, spin_limit) : 1;
-            if (named_sync_or(1, 128, !ok || misc[1])) {
-                abort = 1;
-                misc[1] = 1;
-                break;
-            }
-            bar_try(bar_full0 + 8 * s, (c / kStages) & 1);
+            // every thread waits for the stage itself (a group barrier here would hold all four
+            // warps until the slowest has seen the data); a timeout is voted on at the barrier
+            // below, where the whole group meets anyway
+            int ok = bar_wait_spin(bar_full0 + 8 * s, (c / kStages) & 1, spin_limit);
             // w of this half (1.0 past the end) and its product; the other half's product
             Q4 w[8];
             Q4 Gh = one4();
@@ -343,7 +344,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             }
             const Q4 Go = shfl_xor4(Gh, 16);
             if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
-            named_sync_or(1, 128, 0);
+            if (named_sync_or(1, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
+            }
             // sub-block products from shared memory (read by index there: a register array
             // indexed by the warp's sub-block would be placed in local memory)
             Q4 D = one4(), before = one4(), aft = one4();
@@ -377,8 +382,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     part[m] = 0.f;
                 }
             } else if (!safe) {
-                if (tv == kC) prep_fast<true>(st, t0h, cbyte, tv, w, after, u4, part);
-                else prep_fast<false>(st, t0h, cbyte, tv, w, after, u4, part);
+                const Q4 pre = mul4({rcp2(D.a), rcp2(D.b)}, mul4(before, lead));
+                if (tv == kC) prep_fast<true>(st, t0h, cbyte, tv, w, after, pre, u4, part);
+                else prep_fast<false>(st, t0h, cbyte, tv, w, after, pre, u4, part);
             } else {
                 // sub-block path; scratch = the stage two chunks ahead, free once chunk c-1 is done
                 unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
