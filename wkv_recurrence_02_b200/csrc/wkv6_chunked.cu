@@ -59,13 +59,17 @@ constexpr int OFF_STAGE = 0;                          // stage s: R | K | V | W
 constexpr int SLOT_R = 0, SLOT_K = kTile, SLOT_V = 2 * kTile, SLOT_W = 3 * kTile;
 // A chunk on the sub-block path borrows the stage two chunks ahead as scratch:
 constexpr int SCR_KB = 0, SCR_QI = kTile, SCR_QO = 2 * kTile;  // Qo_b at SCR_QO + 4096 b
-constexpr int OFF_SB = kStages * kStageBytes;         // bf16 (D S_prev) operand, chunk-end path
+// bf16 (D S_prev) operand of a chunk-end-path chunk.  A sub-block-path chunk keeps its state
+// operand in its own stage instead and uses this tile for its [4][16][16] fp32 exact diagonal
+// blocks (written once the previous chunk's products, the tile's last readers, are done).
+constexpr int OFF_SB = kStages * kStageBytes;
 constexpr int OFF_SMALL = OFF_SB + kTile;             // fp32 bookkeeping below
-constexpr int OFF_H = OFF_SMALL;                      // [4][64] 16-token sub-block products
-constexpr int OFF_D = OFF_H + 4 * 64 * 4;             // [stage][64] chunk decay
+// [chunk parity][4][64] 16-token sub-block products: two buffers, so a prep warp that has
+// moved on to the next chunk never overwrites products another warp is still reading
+constexpr int OFF_H = OFF_SMALL;
+constexpr int OFF_D = OFF_H + 2 * 4 * 64 * 4;         // [stage][64] chunk decay
 constexpr int OFF_UB = OFF_D + kStages * 64 * 4;      // [stage][64] bonus diagonal
-constexpr int OFF_DD = OFF_UB + kStages * 64 * 4;     // [4][16][16] exact diagonal blocks
-constexpr int OFF_BAR = OFF_DD + 4 * 16 * 16 * 4;     // mbarriers (8 bytes each)
+constexpr int OFF_BAR = OFF_UB + kStages * 64 * 4;    // mbarriers (8 bytes each)
 constexpr int OFF_MISC = OFF_BAR + 16 * 8;            // tmem base, flags
 constexpr int OFF_LN = OFF_MISC + 64;                 // [2][64] LayerNorm scale, shift of the head
 constexpr int kSmemBytes = OFF_LN + 2 * 64 * 4 + 1024; // + alignment slack
@@ -243,10 +247,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-    float *Hs = reinterpret_cast<float *>(sm + OFF_H);   // [4 sub-blocks][64 channels]
+    float *Hs2 = reinterpret_cast<float *>(sm + OFF_H);  // [parity][4 sub-blocks][64 channels]
     float *Dv = reinterpret_cast<float *>(sm + OFF_D);   // [stage][64]
     float *UB = reinterpret_cast<float *>(sm + OFF_UB);  // [stage][64]
-    float *DD = reinterpret_cast<float *>(sm + OFF_DD);
     float *lns = reinterpret_cast<float *>(sm + OFF_LN);  // gated output: [scale, shift][64]
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC);
@@ -328,6 +331,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             // warps until the slowest has seen the data); a timeout is voted on at the barrier
             // below, where the whole group meets anyway
             int ok = bar_wait_spin(bar_full0 + 8 * s, (c / kStages) & 1, spin_limit);
+            float *Hs = Hs2 + (c & 1) * 4 * 64;
             // w of this half (1.0 past the end) and its product; the other half's product
             Q4 w[8];
             Q4 Gh = one4();
@@ -431,7 +435,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                                 acc += rt.x * ki.x * f.x + rt.y * ki.y * f.y;
                             }
                         }
-                        DD[(ab * 16 + tt) * 16 + ii] = acc;
+                        reinterpret_cast<float *>(sm + OFF_SB)[(ab * 16 + tt) * 16 + ii] = acc;
                     }
                     named_sync_or(1, 128, 0);
                 }
@@ -691,6 +695,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 float va[32];
                 tmem_ld32(tlane + COL_AD, va);
                 if (safe) {
+                    const float *DD = reinterpret_cast<const float *>(sm + OFF_SB);
                     float vo[32];
                     tmem_ld32(tlane + COL_AO, vo);
 #pragma unroll
