@@ -85,16 +85,15 @@ struct ChunkedParams {
     int *status;
     uint32_t spin_limit;
     int inject_timeout;
-    // sequence split: CTA (bh, g) covers chunks [g * seg_chunks, (g + 1) * seg_chunks)
+    // sequence split: CTA (bh, g) covers chunks [g * seg_chunks, (g + 1) * seg_chunks) and
+    // starts from s0 carried over the pieces before it: `pieces` entries per segment of
+    // (end state from zero, decay product) in seg, written by the first pass
     int seg_chunks;        // chunks per segment (>= number of chunks when not split)
-    int state_only;        // 1: only the segment's local end state (from zero) and decay
-    float *seg;            // [B*H][segments-1][N*N + N]: local end state, then decay product
+    float *seg;            // [B*H][nsub][N*N + N]
     int nseg;              // segments per sequence
+    int pieces;            // first-pass pieces per segment
+    int nsub;              // first-pass pieces per sequence, (nseg - 1) * pieces
     int64_t seg_cap;       // floats of scratch behind seg (index checks of the debug build)
-    // in-place state update of a split sequence (sT == s0): the state-only pass copies s0
-    // here (segment 0's CTAs) and the full pass reads the copy, so no CTA can read s0 after
-    // the last segment has overwritten it
-    float *s0copy;         // [B*H][N*N] or null
     // fused output stage (null gate: plain y): y = SiLU(g) (ln_w (o - mean) rstd + ln_b)
     const __nv_bfloat16 *gate;
     const float *ln_w, *ln_b;
@@ -105,7 +104,7 @@ constexpr int kSegStride = kN * kN + kN;
 // TMA of chunk c (r, k, v, w tiles of one head) into its stage, one thread.
 __device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full0, const CUtensorMap *mr,
                                             const CUtensorMap *mk, const CUtensorMap *mv,
-                                            const CUtensorMap *mw, int c, int cabs, int h, int b, bool with_r,
+                                            const CUtensorMap *mw, int c, int cabs, int h, int b,
                                             int *status, int64_t T)
 {
     const int s = c % kStages;  // c counts chunks within this CTA's segment
@@ -114,9 +113,9 @@ __device__ __forceinline__ void issue_chunk(unsigned char *sm, uint32_t bar_full
     if (!in_bounds(status, OFF_STAGE + s * kStageBytes, kStageBytes, OFF_SB)) return;
     const uint32_t dst = smem_u32(sm + OFF_STAGE + s * kStageBytes);
     const uint32_t bar = bar_full0 + 8 * s;
-    bar_expect_tx(bar, with_r ? kStageBytes : kStageBytes - kTile);
+    bar_expect_tx(bar, kStageBytes);
     const int t0 = cabs * kC;
-    if (with_r) tma_load_4d(dst + SLOT_R, mr, 0, h, t0, b, bar);
+    tma_load_4d(dst + SLOT_R, mr, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_K, mk, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_V, mv, 0, h, t0, b, bar);
     tma_load_4d(dst + SLOT_W, mw, 0, h, t0, b, bar);
@@ -272,7 +271,6 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     const int g = blockIdx.y;                      // segment of the sequence
     const int cb = g * p.seg_chunks;               // its first chunk
     const int nchunks = min(p.seg_chunks, nchunks_all - cb);  // chunks in this segment
-    const bool so = p.state_only != 0;
     const uint32_t limit = p.spin_limit;
     const uint32_t spin_limit = p.spin_limit * 64u;
 
@@ -305,7 +303,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         int n0 = 0;
         for (; n0 < kStages - 1 && n0 < nchunks; ++n0)
             issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, n0, cb + n0, static_cast<int>(h),
-                        static_cast<int>(b), !so, p.status, T);
+                        static_cast<int>(b), p.status, T);
         misc[8] = n0;
     }
 
@@ -370,22 +368,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             // single chunk-end reference unless a chunk decay product is below 2^-100.  Every
             // warp's 32 lanes cover all 16 channel quads, so a warp vote is the chunk's vote
             // (the same in all four warps): no group barrier.
-            const int safe = so ? 0 : __any_sync(0xffffffffu, any_below(D, kFastMin));
+            const int safe = __any_sync(0xffffffffu, any_below(D, kFastMin));
             int hazard = 0;
             float part[8];
-            if (so) {
-                // local end state only: Kh[i] = k_i prod_{j>i} w_j (every factor <= 1)
-                Q4 run = after;
-#pragma unroll
-                for (int m = 7; m >= 0; --m) {
-                    const int t = t0h + m;
-                    const uint32_t off = swz(t, cbyte);
-                    const uint2 kk = t < tv ? ld_u2(st + SLOT_K, off) : make_uint2(0u, 0u);
-                    st_u2(st + SLOT_K, off, pack4(mul4(unpack4(kk), run)));
-                    run = mul4(run, w[m]);
-                    part[m] = 0.f;
-                }
-            } else if (!safe) {
+            if (!safe) {
                 const Q4 pre = mul4({rcp2(D.a), rcp2(D.b)}, mul4(before, lead));
                 if (tv == kC) prep_fast<true>(st, t0h, cbyte, tv, w, after, pre, u4, part);
                 else prep_fast<false>(st, t0h, cbyte, tv, w, after, pre, u4, part);
@@ -501,7 +487,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         const bool iss_o = issuer, iss_s = tid == kPrepThreads + 32, iss_a = tid == kPrepThreads + 64;
         const bool iss_t = tid == kPrepThreads + 96;
         int issued = misc[8];
-        if (GATED && !so) {  // the head's LayerNorm scale and shift (read after the loop's first barrier)
+        if (GATED) {  // the head's LayerNorm scale and shift (read after the loop's first barrier)
             const int t = tid - kPrepThreads;
             if (in_bounds(p.status, h * kN + (t & (kN - 1)), 1, p.H * kN))
                 lns[t] = t < kN ? p.ln_w[h * kN + t] : p.ln_b[h * kN + t - kN];
@@ -532,21 +518,13 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
         };
 
         int ok = 1;
-        if (iss_a && !abort && !so) ok = issue_scores(0);
+        if (iss_a && !abort) ok = issue_scores(0);
         const int64_t nstate = static_cast<int64_t>(gridDim.x) * kN * kN;  // floats of s0 / sT
         // debug build: TMEM columns of this thread inside the allocation
         in_bounds(p.status, COL_O + colh, 32, kTmemCols);
-        if (so && p.s0copy && g == 0 && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
-            // in-place split: keep s0 for the full pass
-            const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
-            float4 *dst = reinterpret_cast<float4 *>(p.s0copy + (bh * kN + row) * kN + colh);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[i] = src[i];
-        }
-        {   // initial state into TMEM: s0 advanced over the earlier segments (zero for a
-            // state-only pass, which wants the segment's local contribution)
+        {   // initial state into TMEM: s0 carried over the pieces before this segment
             float v[32];
-            if (p.s0 && !so && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
+            if (p.s0 && in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nstate)) {
                 const float4 *src = reinterpret_cast<const float4 *>(p.s0 + (bh * kN + row) * kN + colh);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -560,92 +538,22 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
 #pragma unroll
                 for (int i = 0; i < 32; ++i) v[i] = 0.f;
             }
-            if (!so) {
-                for (int gp = 0; gp < g; ++gp) {  // S <- diag(D_g') S + S_g'
-                    if (!in_bounds(p.status, (bh * (p.nseg - 1) + gp) * kSegStride, kSegStride, p.seg_cap)) break;
-                    const float *sg = p.seg + (bh * (p.nseg - 1) + gp) * kSegStride;
-                    const float d = sg[kN * kN + row];
-                    const float4 *src = reinterpret_cast<const float4 *>(sg + row * kN + colh);
+            for (int gp = 0; gp < g * p.pieces; ++gp) {  // S <- diag(D_piece) S + S_piece
+                if (!in_bounds(p.status, (bh * p.nsub + gp) * kSegStride, kSegStride, p.seg_cap)) break;
+                const float *sg = p.seg + (bh * p.nsub + gp) * kSegStride;
+                const float d = sg[kN * kN + row];
+                const float4 *src = reinterpret_cast<const float4 *>(sg + row * kN + colh);
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) {
-                        const float4 x = src[i];
-                        v[4 * i] = fmaf(d, v[4 * i], x.x);
-                        v[4 * i + 1] = fmaf(d, v[4 * i + 1], x.y);
-                        v[4 * i + 2] = fmaf(d, v[4 * i + 2], x.z);
-                        v[4 * i + 3] = fmaf(d, v[4 * i + 3], x.w);
-                    }
+                for (int i = 0; i < 8; ++i) {
+                    const float4 x = src[i];
+                    v[4 * i] = fmaf(d, v[4 * i], x.x);
+                    v[4 * i + 1] = fmaf(d, v[4 * i + 1], x.y);
+                    v[4 * i + 2] = fmaf(d, v[4 * i + 2], x.z);
+                    v[4 * i + 3] = fmaf(d, v[4 * i + 3], x.w);
                 }
             }
             tmem_st32(tlane + COL_S, v);
         }
-
-        if (so) {
-            // ---- state-only pass: S = diag(D) S + Kh^T V per chunk; then S and prod(D) out
-            float dprod = 1.f;
-            for (int c = 0; c < nchunks && !abort; ++c) {
-                const int s = c % kStages;
-                unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
-                if (issuer && ok) {
-                    ok = bar_wait_spin(bar_prep0 + 8 * s, (c / kStages) & 1, spin_limit);
-                    if (ok && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
-                }
-                if (named_sync_or(2, 128, !ok || misc[1])) {
-                    abort = 1;
-                    misc[1] = 1;
-                    break;
-                }
-                bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);
-                if (c > 0) bar_try(bar_O, (c - 1) & 1);
-                fence_after();
-                if (issuer) {
-                    while (issued < nchunks && issued <= c + kStages - 1) {
-                        issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
-                                    static_cast<int>(h), static_cast<int>(b), false, p.status, T);
-                        ++issued;
-                    }
-                    misc[8] = issued;
-                }
-                {
-                    float sv[32];
-                    tmem_ld32(tlane + COL_S, sv);
-                    const float d = Dv[s * 64 + row];
-                    dprod *= d;
-#pragma unroll
-                    for (int n = 0; n < 32; ++n) sv[n] *= d;
-                    tmem_st32(tlane + COL_S, sv);
-                }
-                fence_before();
-                named_sync_or(2, 128, 0);
-                fence_after();
-                if (issuer) {
-                    const uint32_t aV = smem_u32(st + SLOT_V), aKh = smem_u32(st + SLOT_K);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma(tbase + COL_S, desc_mn(aKh + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), 1);
-                    mma_commit(bar_O);
-                }
-            }
-            if (!abort) {
-                if (issuer) ok = bar_wait_spin(bar_O, (nchunks - 1) & 1, spin_limit);
-                if (named_sync_or(2, 128, !ok || misc[1])) {
-                    abort = 1;
-                    misc[1] = 1;
-                } else {
-                    bar_try(bar_O, (nchunks - 1) & 1);
-                    fence_after();
-                    float sv[32];
-                    tmem_ld32(tlane + COL_S, sv);
-                    if (in_bounds(p.status, (bh * (p.nseg - 1) + g) * kSegStride, kSegStride, p.seg_cap)) {
-                        float *sg = p.seg + (bh * (p.nseg - 1) + g) * kSegStride;
-                        float4 *dst = reinterpret_cast<float4 *>(sg + row * kN + colh);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            dst[i] = make_float4(sv[4 * i], sv[4 * i + 1], sv[4 * i + 2], sv[4 * i + 3]);
-                        if (hi == 0) sg[kN * kN + row] = dprod;
-                    }
-                }
-            }
-        } else {
 
         for (int c = 0; c < nchunks && !abort; ++c) {
             const int s = c % kStages;
@@ -679,7 +587,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     const int user = issued - 2;  // chunk that would use this stage as scratch
                     if (user >= c && misc[2 + user % kStages]) break;
                     issue_chunk(sm, bar_full0, &map_r, &map_k, &map_v, &map_w, issued, cb + issued,
-                                static_cast<int>(h), static_cast<int>(b), true, p.status, T);
+                                static_cast<int>(h), static_cast<int>(b), p.status, T);
                     ++issued;
                 }
                 misc[8] = issued;
@@ -810,7 +718,6 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 }
             }
         }
-        }  // full pass
     }
 
     // ---- drain after an abort, then release tensor memory
@@ -899,6 +806,18 @@ int sm_count()
 // A split call that updates its state in place (sT == s0) needs a copy of s0 in scratch.
 bool split_state_copy(const Wkv6Args &a) { return a.s0 != nullptr && a.sT == a.s0; }
 
+// Pieces per segment of the first pass: segments are halved (and halved again) while the
+// pieces keep >= 4 chunks and every (b, h, piece) CTA of the first pass fits on the GPU at
+// once, so that pass takes the time of a shorter piece.
+int64_t pieces_per_segment(int64_t bh, int64_t G, int64_t seg_chunks)
+{
+    if (G <= 1) return 1;
+    const int64_t slots = static_cast<int64_t>(wkv6_chunk_state_ctas_per_sm()) * sm_count();
+    int64_t m = 1;
+    while (seg_chunks % (2 * m) == 0 && seg_chunks / (2 * m) >= 4 && bh * (G - 1) * 2 * m <= slots) m *= 2;
+    return m;
+}
+
 // Kernel attributes (shared memory size, carveout), set once per device.
 cudaError_t configure_kernel()
 {
@@ -968,8 +887,8 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     const int64_t nchunks = (a.T + kC - 1) / kC;
 
     // Sequence split: with fewer (b, h) sequences than two per SM, cut each sequence into
-    // segments of >= 4 chunks that run side by side; a state-only pass first gives every
-    // segment its exact incoming state.
+    // segments of >= 4 chunks that run side by side; a first pass over pieces of the
+    // segments gives every segment its exact incoming state.
     int64_t G = 1;
     if (a.segments == 0) {
         const int64_t slots = 2LL * sm_count();
@@ -989,33 +908,29 @@ cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s)
     cudaError_t e = configure_kernel();
     if (e != cudaSuccess) return e;
 
+    const int64_t m = pieces_per_segment(bh, G, seg_chunks);
+    const int64_t nsub = (G - 1) * m;
+    const int64_t seg_floats = bh * nsub * kSegStride;
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
-                      static_cast<int>(seg_chunks), 0, nullptr, static_cast<int>(G),
-                      static_cast<int64_t>(bh) * (G - 1) * kSegStride,
-                      nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
+                      static_cast<int>(seg_chunks), nullptr, static_cast<int>(G), static_cast<int>(m),
+                      static_cast<int>(nsub), seg_floats,
+                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     float *seg = nullptr;
     if (G > 1) {
-        const size_t seg_floats = static_cast<size_t>(bh) * (G - 1) * kSegStride;
-        const size_t copy_floats = split_state_copy(a) ? static_cast<size_t>(bh) * kN * kN : 0;
+        const int64_t copy_floats = split_state_copy(a) ? bh * kN * kN : 0;
         cudaMemPool_t pool = nullptr;
         e = scratch_pool(&pool);
         if (e != cudaSuccess) return e;
-        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&seg), (seg_floats + copy_floats) * sizeof(float),
-                                    pool, s);
+        e = cudaMallocFromPoolAsync(reinterpret_cast<void **>(&seg),
+                                    static_cast<size_t>(seg_floats + copy_floats) * sizeof(float), pool, s);
         if (e != cudaSuccess) return e;
-        ChunkedParams pa = prm;
-        pa.state_only = 1;
-        pa.seg = seg;
-        if (copy_floats) {
-            pa.s0copy = seg + seg_floats;
-            prm.s0 = pa.s0copy;
-        }
-        auto kso = a.omega ? wkv6_chunked_kernel<false, true> : wkv6_chunked_kernel<false, false>;
-        kso<<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)), kThreads, kSmemBytes, s>>>(mr, mk, mv,
-                                                                                                      mw, pa);
-        e = cudaGetLastError();
+        float *s0copy = copy_floats ? seg + seg_floats : nullptr;
+        const ChunkStateArgs sa{a.T, a.H, bh, static_cast<int>(seg_chunks / m), static_cast<int>(nsub), seg,
+                                seg_floats, a.s0, s0copy, a.status, g_chunked_inject_timeout, a.omega};
+        e = wkv6_chunk_state_launch(mk, mv, mw, sa, s);
         prm.seg = seg;
+        if (s0copy) prm.s0 = s0copy;
     }
     if (e == cudaSuccess) {
         auto kern = prm.gate ? (a.omega ? wkv6_chunked_kernel<true, true> : wkv6_chunked_kernel<true, false>)
@@ -1091,7 +1006,11 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
     const int64_t seg_chunks = (nchunks + G - 1) / G;
     G = (nchunks + seg_chunks - 1) / seg_chunks;
     if (G > 65535) return cudaErrorInvalidConfiguration;
-    *scratch_needed = G > 1 ? static_cast<size_t>((G - 1) * per_segment + copy_bytes) : 0;
+    // first-pass pieces per segment, fewer if their entries do not fit in the array
+    int64_t m = pieces_per_segment(bh, G, seg_chunks);
+    while (m > 1 && (G - 1) * m * per_segment + copy_bytes > cap) m /= 2;
+    const int64_t nsub = (G - 1) * m;
+    *scratch_needed = G > 1 ? static_cast<size_t>(nsub * per_segment + copy_bytes) : 0;
     if (*scratch_needed > kNoAllocScratchBytes) return cudaErrorInvalidValue;
 
     float *seg = nullptr;
@@ -1105,25 +1024,22 @@ cudaError_t wkv6_chunked_launch_noalloc(const Wkv6Args &a, int segments, size_t 
         return cudaErrorInvalidValue;
     cudaError_t e = configure_kernel();
     if (e != cudaSuccess) return e;
+    const int64_t seg_floats = nsub * per_segment / static_cast<int64_t>(sizeof(float));
     ChunkedParams prm{a.T, a.H, a.u, a.s0, static_cast<__nv_bfloat16 *>(a.y), a.sT, a.status,
                       g_chunked_inject_timeout ? 100u : 100000u, g_chunked_inject_timeout,
-                      static_cast<int>(seg_chunks), 0, seg, static_cast<int>(G),
-                      (G - 1) * per_segment / static_cast<int64_t>(sizeof(float)),
-                      nullptr, static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
+                      static_cast<int>(seg_chunks), seg, static_cast<int>(G), static_cast<int>(m),
+                      static_cast<int>(nsub), seg_floats,
+                      static_cast<const __nv_bfloat16 *>(a.g), a.ln_w, a.ln_b, a.eps};
     if (G > 1) {
-        // the state-only pass writes every scratch entry the full pass reads (the s0 copy of
-        // an in-place call included): nothing in the array has to start at zero, and what an
+        // the first pass writes every scratch entry the full pass reads (the s0 copy of an
+        // in-place call included): nothing in the array has to start at zero, and what an
         // earlier call left there is never read
-        ChunkedParams pa = prm;
-        pa.state_only = 1;
-        if (copy_bytes) {
-            pa.s0copy = seg + (G - 1) * per_segment / static_cast<int64_t>(sizeof(float));
-            prm.s0 = pa.s0copy;
-        }
-        wkv6_chunked_kernel<false, false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G - 1)),
-                                            kThreads, kSmemBytes, s>>>(mr, mk, mv, mw, pa);
-        e = cudaGetLastError();
+        float *s0copy = copy_bytes ? seg + seg_floats : nullptr;
+        const ChunkStateArgs sa{a.T, a.H, bh, static_cast<int>(seg_chunks / m), static_cast<int>(nsub), seg,
+                                seg_floats, a.s0, s0copy, a.status, g_chunked_inject_timeout, false};
+        e = wkv6_chunk_state_launch(mk, mv, mw, sa, s);
         if (e != cudaSuccess) return e;
+        if (s0copy) prm.s0 = s0copy;
     }
     wkv6_chunked_kernel<false, false><<<dim3(static_cast<unsigned>(bh), static_cast<unsigned>(G)), kThreads,
                                         kSmemBytes, s>>>(

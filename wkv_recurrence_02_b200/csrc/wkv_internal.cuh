@@ -129,6 +129,28 @@ cudaError_t wkv6_serial_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_decode_launch(const Wkv6Args &a, cudaStream_t s);
 cudaError_t wkv6_chunked_launch(const Wkv6Args &a, cudaStream_t s);
 
+// First pass of a split chunked prefill: for every (b, h) and every piece of sub_chunks
+// 64-token chunks (pieces 0 .. nsub-1 of the sequence), the state the piece ends in when it
+// starts from zero and the product of its decays, written to seg[bh][piece] as 64 x 64
+// floats then 64 floats.  With s0copy set, the CTAs of piece 0 also copy s0 there (an
+// in-place split call reads its initial state from the copy).  Maps as from make_map over k,
+// v and w (w holding omega_t when omega is set).
+struct ChunkStateArgs {
+    int64_t T, H, bh;
+    int sub_chunks, nsub;
+    float *seg;
+    int64_t seg_cap;          // floats behind seg
+    const float *s0;
+    float *s0copy;
+    int *status;
+    int inject_timeout;
+    bool omega;
+};
+cudaError_t wkv6_chunk_state_launch(const CUtensorMap &mk, const CUtensorMap &mv, const CUtensorMap &mw,
+                                    const ChunkStateArgs &a, cudaStream_t s);
+// CTAs of the first-pass kernel that fit on one SM.
+int wkv6_chunk_state_ctas_per_sm();
+
 // The chunked kernel with its sequence-split scratch in a fixed device array (no
 // allocation).  Returns cudaErrorInvalidValue with *scratch_needed > capacity when the
 // requested split does not fit.
