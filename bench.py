@@ -180,7 +180,7 @@ class Workload:
                                                     s0=d["s0"], y=d["y"], sT=d["s0"]))
 
     # 12 WKV-4 layers, the Finch prefill, 4 long-context calls of two launches each (the
-    # state-only and full passes of the sequence split at 64 heads), the decode step; the
+    # first pass and the chunked pass of the sequence split at 64 heads), the decode step; the
     # ncu launch list of this step counts the same
     launches_per_step = 12 + 1 + 4 * 2 + 1
 

@@ -240,10 +240,12 @@ int rwkv_get_wkv6_algo(void);
 /* Sequence split of the chunked WKV-6 kernel on the calling thread.  Each (b, h) sequence
  * is walked by one CTA; when there are fewer sequences than two per SM the library cuts
  * every sequence into G segments (of at least four 64-token chunks) that run side by
- * side: a first state-only pass gives each segment's local end state and decay product,
- * and each segment then starts from its exact incoming state.  The result equals the
- * unsplit evaluation up to fp32 rounding order.  The split needs B*H*(G-1)*(N*N+N)*4 bytes
- * of scratch, plus B*H*N*N*4 bytes for a copy of s0 when the state is updated in place
+ * side: a first pass gives the end state (from zero) and decay product of P pieces of each
+ * segment but the last (P = 1, 2, 4 ...: halves while the pieces keep at least four chunks
+ * and the first pass fits on the GPU at once), and each segment then starts from its exact
+ * incoming state.  The result equals the unsplit evaluation up to fp32 rounding order.  The
+ * split needs B*H*(G-1)*P*(N*N+N)*4 bytes of scratch, plus B*H*N*N*4 bytes for a copy of s0
+ * when the state is updated in place
  * (sT == s0: the copy is taken before any segment runs, so no segment can read an s0 that
  * the last segment has already overwritten).  The scratch is taken stream-ordered (on the
  * calling thread's stream, within the call) from a memory pool the library keeps per
@@ -262,8 +264,10 @@ int rwkv_get_wkv6_segments(void);
  * fixed array inside the library (RWKV_NOALLOC_SCRATCH_BYTES per GPU, held by every GPU
  * that loads the library until the process exits) and never allocates or frees memory.
  *   segments: 0 = choose the split as rwkv_wkv6_forward_bf16 does, capped to what the
- *             array holds; n >= 1 = split into at most n segments.  A split needing more
- *             than RWKV_NOALLOC_SCRATCH_BYTES (B*H*(G-1)*(N*N+N)*4 bytes for G segments,
+ *             array holds; n >= 1 = split into at most n segments.  The first pass uses
+ *             P pieces per segment as the default entry point does, fewer (down to 1) when
+ *             their entries would not fit.  A split needing more than
+ *             RWKV_NOALLOC_SCRATCH_BYTES (B*H*(G-1)*P*(N*N+N)*4 bytes for G segments,
  *             plus B*H*N*N*4 bytes for the copy of s0 when sT == s0) is rejected with
  *             RWKV_ERR_SHAPE before any launch; rwkv_last_error() says why.
  * Arguments, layouts and the result are otherwise those of rwkv_wkv6_forward_bf16 (always

@@ -150,8 +150,9 @@ def test_wkv6_fast_decay_channels(wval):
 
 @pytest.mark.parametrize("segments", [1, 2, 3, 5])
 def test_wkv6_sequence_split(segments):
-    """The chunked kernel cut into segments (state-only pass, then every segment from its
-    exact incoming state) matches the oracle, with a ragged last chunk and random s0."""
+    """The chunked kernel cut into segments (a first pass gives the end states of pieces of
+    the segments, then every segment runs from its exact incoming state) matches the oracle,
+    with a ragged last chunk and random s0."""
     x = _inputs(2, 1000, 2, "bf16", 17, s0_std=0.1)
     y, sT = _gpu(x, s0=x["s0"], algo="chunked", segments=segments)
     torch.cuda.synchronize()

@@ -53,7 +53,7 @@ def test_gated_decode_matches_oracle():
 
 
 def test_gated_sequence_split_matches_oracle():
-    """B1 H8 T2048: the launcher splits each sequence (state-only pass, then the gated pass)."""
+    """B1 H8 T2048: the launcher splits each sequence (first pass, then the gated pass)."""
     y, sT, ry, rs = _run(1, 2048, 8, seed=8, segments=4)
     tol = TOL[torch.bfloat16]
     assert rel_inf(f64(y), ry) <= tol

@@ -68,7 +68,7 @@ def test_omega_serial_kernel_matches_oracle():
 
 
 def test_omega_sequence_split_matches_oracle():
-    """B1 H8 T2048 split into 4 segments: the state-only pass also forms w from omega."""
+    """B1 H8 T2048 split into 4 segments: the first pass also forms w from omega."""
     _check(_inputs(1, 2048, 8, seed=23), segments=4)
 
 

@@ -8,8 +8,8 @@ Every case first makes one untimed call (so a profiler can skip it with ``-s``),
   wkv4          RWKV-4 scan, B8 T1024 C768 bf16: one layer of the 169M model's shape
   finch         WKV-6 chunked prefill, B8 T1024 H32 N64 bf16 with s0 (256 CTAs, 16 chunks
                 each: the Finch-1.6B prefill shape at a quarter of its length)
-  long          WKV-6 chunked prefill with sequence split, B1 T4096 H64 (state-only pass
-                then full pass)
+  long          WKV-6 chunked prefill with sequence split, B1 T4096 H64 (first pass over
+                half-segment pieces, then the chunked pass)
   decode        WKV-6 T=1 decode, B256 H64 with the state updated in place (268 MB of state)
   wkv4_decode   RWKV-4 T=1 decode, B2048 C4096 bf16, (a, b, p) state updated in place
   finch_gated   the finch case through rwkv_wkv6_forward_gated_bf16 (head LayerNorm and
