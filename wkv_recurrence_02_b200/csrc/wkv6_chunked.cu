@@ -593,6 +593,14 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 misc[8] = issued;
             }
 
+            if (GATED) {  // the gate row of this thread's y row of chunk c (stored next iteration) into L2
+                const int64_t tok = t0 + row;
+                if (tok < T && in_bounds(p.status, ((b * T + tok) * p.H + h) * kN + colh, 32,
+                                         static_cast<int64_t>(gridDim.x) * T * kN)) {
+                    const __nv_bfloat16 *gp = p.gate + ((b * T + tok) * p.H + h) * kN + colh;
+                    asm volatile("prefetch.global.L2 [%0];" ::"l"(gp));
+                }
+            }
             // ---- y of chunk c-1, and P of chunk c (causal scores, bonus diagonal, bf16)
             {
                 if (c > 0) {
