@@ -467,7 +467,12 @@ def measure_next_rows(torch, inputs, ops, dev, stream, wl, reps=50):
 
 
 def run_e2e(torch, ops, wl, stream, dev, steps, barrier):
-    """Same step through the public API with inputs/outputs in pinned host memory."""
+    """Same step through the public API with inputs/outputs in pinned host memory.  Each call's
+    inputs go up on an upload stream and its outputs come back on a download stream, so the
+    copies of one call overlap the compute of others and the two directions overlap each
+    other; events order every reuse of a buffer (a call's inputs are not overwritten before
+    the previous step's compute and download of that call are done, its outputs not before
+    their previous download).  The timed region holds every copy of every timed step."""
     h_y4 = [torch.empty(8, 1024, 768, dtype=torch.bfloat16).pin_memory() for _ in range(12)]
     h_yf = torch.empty_like(wl.h_finch["r"]).pin_memory()
     h_sf = torch.empty_like(wl.h_finch["s0"]).pin_memory()
@@ -475,57 +480,70 @@ def run_e2e(torch, ops, wl, stream, dev, steps, barrier):
     h_sl = torch.empty(1, 64, 64, 64).pin_memory()
     h_yd = torch.empty_like(wl.h_dec["r"]).pin_memory()
     h_sd = torch.empty_like(wl.h_dec["s0"]).pin_memory()
-    h2d = d2h = 0
+    up_s = torch.cuda.Stream(device=dev)
+    down_s = torch.cuda.Stream(device=dev)
 
-    def one():
-        nonlocal h2d, d2h
-        h2d = d2h = 0
+    calls = []  # (inputs [(device, host)], compute, outputs [(host, device)])
+    for i, L in enumerate(wl.w4):
+        calls.append(([(L["k"], wl.h_kv[0]), (L["v"], wl.h_kv[1])],
+                      lambda L=L: ops.wkv4_forward(L["w"], L["u"], L["k"], L["v"], y=L["y"]),
+                      [(h_y4[i], L["y"])]))
+    f, hf = wl.finch, wl.h_finch
+    calls.append(([(f[n], hf[n]) for n in ("r", "k", "v", "w", "s0")],
+                  lambda: ops.wkv6_forward(f["r"], f["k"], f["v"], f["w"], f["u"], s0=f["s0"], y=f["y"],
+                                           sT=f["sT"]),
+                  [(h_yf, f["y"]), (h_sf, f["sT"])]))
+    g, hg = wl.long, wl.h_long
 
-        def up(dst, src):
-            nonlocal h2d
-            dst.copy_(src, non_blocking=True)
-            h2d += src.numel() * src.element_size()
-
-        def down(dst, src):
-            nonlocal d2h
-            dst.copy_(src, non_blocking=True)
-            d2h += src.numel() * src.element_size()
-
-        for i, L in enumerate(wl.w4):
-            up(L["k"], wl.h_kv[0])
-            up(L["v"], wl.h_kv[1])
-            ops.wkv4_forward(L["w"], L["u"], L["k"], L["v"], y=L["y"])
-            down(h_y4[i], L["y"])
-        f, hf = wl.finch, wl.h_finch
-        for n in ("r", "k", "v", "w", "s0"):
-            up(f[n], hf[n])
-        ops.wkv6_forward(f["r"], f["k"], f["v"], f["w"], f["u"], s0=f["s0"], y=f["y"], sT=f["sT"])
-        down(h_yf, f["y"])
-        down(h_sf, f["sT"])
-        g, hg = wl.long, wl.h_long
-        for n in ("r", "k", "v", "w"):
-            up(g[n], hg[n])
+    def long_calls():
         for c in range(4):
             sl = slice(c * 4096, (c + 1) * 4096)
             ops.wkv6_forward(g["r"][:, sl], g["k"][:, sl], g["v"][:, sl], g["w"][:, sl], g["u"],
-                             s0=None if c == 0 else g["s"][(c - 1) % 2], y=g["y"][:, sl],
-                             sT=g["s"][c % 2])
-        down(h_yl, g["y"])
-        down(h_sl, g["s"][1])
-        d, hd = wl.dec, wl.h_dec
-        for n in ("r", "k", "v", "w", "s0"):
-            up(d[n], hd[n])
-        ops.wkv6_forward(d["r"], d["k"], d["v"], d["w"], d["u"], s0=d["s0"], y=d["y"], sT=d["s0"])
-        down(h_yd, d["y"])
-        down(h_sd, d["s0"])
+                             s0=None if c == 0 else g["s"][(c - 1) % 2], y=g["y"][:, sl], sT=g["s"][c % 2])
+    calls.append(([(g[n], hg[n]) for n in ("r", "k", "v", "w")], long_calls,
+                  [(h_yl, g["y"]), (h_sl, g["s"][1])]))
+    d, hd = wl.dec, wl.h_dec
+    calls.append(([(d[n], hd[n]) for n in ("r", "k", "v", "w", "s0")],
+                  lambda: ops.wkv6_forward(d["r"], d["k"], d["v"], d["w"], d["u"], s0=d["s0"], y=d["y"],
+                                           sT=d["s0"]),
+                  [(h_yd, d["y"]), (h_sd, d["s0"])]))
+    h2d = sum(h.numel() * h.element_size() for ins, _, _ in calls for _, h in ins)
+    d2h = sum(dv.numel() * dv.element_size() for _, _, outs in calls for _, dv in outs)
+    done = [None] * len(calls)  # download-done event of each call in the previous step
+
+    def one():
+        for i, (ins, fn, outs) in enumerate(calls):
+            if done[i] is not None:
+                up_s.wait_event(done[i])
+            with torch.cuda.stream(up_s):
+                for dst, src in ins:
+                    dst.copy_(src, non_blocking=True)
+            ev_up = torch.cuda.Event()
+            ev_up.record(up_s)
+            stream.wait_event(ev_up)
+            with torch.cuda.stream(stream):
+                fn()
+            ev_c = torch.cuda.Event()
+            ev_c.record(stream)
+            down_s.wait_event(ev_c)
+            with torch.cuda.stream(down_s):
+                for dst, src in outs:
+                    dst.copy_(src, non_blocking=True)
+            done[i] = torch.cuda.Event()
+            done[i].record(down_s)
 
     one()
+    torch.cuda.synchronize(dev)
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
+    up_s.wait_event(e0)
+    down_s.wait_event(e0)
     for _ in range(steps):
         one()
+    stream.wait_stream(up_s)
+    stream.wait_stream(down_s)
     e1.record(stream)
     barrier()
     return e0.elapsed_time(e1) / steps, h2d, d2h
