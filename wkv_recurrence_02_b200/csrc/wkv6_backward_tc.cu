@@ -129,8 +129,8 @@ constexpr int kSStages = 3;
 template <bool REV> struct StateLayout {
     static constexpr int tiles = REV ? 4 : 3;                    // X | Y | W (| S_end)
     static constexpr int stage = tiles * kTile;
-    static constexpr int hs = kSStages * stage;                  // [4][64] sub-block decay products
-    static constexpr int dv = hs + 4 * 64 * 4;                   // [stage][64] chunk decay
+    static constexpr int hs = kSStages * stage;                  // [parity][4][64] sub-block decay products
+    static constexpr int dv = hs + 2 * 4 * 64 * 4;               // [stage][64] chunk decay
     static constexpr int bar = dv + kSStages * 64 * 4;           // full[3], prep[3], mma
     static constexpr int misc = bar + 64;                        // TMEM base, abort flag
     static constexpr int smem = misc + 64 + 1024;
@@ -162,7 +162,7 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
     using L = StateLayout<REV>;
     extern __shared__ unsigned char smem_raw[];
     unsigned char *sm = align1024(smem_raw);
-    float *Hs = reinterpret_cast<float *>(sm + L::hs);
+    float *Hs2 = reinterpret_cast<float *>(sm + L::hs);
     float *Dv = reinterpret_cast<float *>(sm + L::dv);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + L::misc);
@@ -229,13 +229,12 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
             unsigned char *st = sm + s * L::stage;
             const int64_t t0 = static_cast<int64_t>(cc) * kC;
             const int tv = static_cast<int>(p.T - t0 < kC ? p.T - t0 : kC);
-            const int ok = tid == 0 ? bar_wait_spin(bar_full0 + 8 * s, (n / kSStages) & 1, spin) : 1;
-            if (named_sync_or(1, 128, !ok || misc[1])) {
-                abort = 1;
-                misc[1] = 1;
-                break;
-            }
-            bar_try(bar_full0 + 8 * s, (n / kSStages) & 1);
+            // every thread waits for the stage itself; a timeout is voted on at the group barrier
+            // below.  The sub-block products are double-buffered by chunk parity: without a
+            // barrier at the start of each chunk, a warp that has moved on could otherwise
+            // overwrite products another warp still reads.
+            const int ok = bar_wait_spin(bar_full0 + 8 * s, (n / kSStages) & 1, spin);
+            float *Hs = Hs2 + (n & 1) * 4 * 64;
             Q4 w[8];
             Q4 Gh = one4();
 #pragma unroll
@@ -252,7 +251,11 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
             }
             const Q4 Go = shfl_xor4(Gh, 16);
             if (hf == 0) st_q4(Hs + a * 64 + 4 * cq, mul4(Gh, Go));
-            named_sync_or(1, 128, 0);
+            if (named_sync_or(1, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
+            }
             Q4 D = one4(), before = one4(), aft = one4();
 #pragma unroll
             for (int be = 0; be < 4; ++be) {
@@ -280,8 +283,6 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
                 }
             }
             if (warp == 0 && hf == 0) st_q4(Dv + s * 64 + 4 * cq, D);
-            // the sub-block products are read again for the next chunk only after every warp
-            // of the group has passed this chunk's first barrier
             fence_async_smem();
             bar_arrive(bar_prep0 + 8 * s);
         }
