@@ -258,6 +258,23 @@ def run_ours(args, rank, world, dist):
     ms = e0.elapsed_time(e1)
     del graph
 
+    # the spread of single steps: one step captured as a graph, each of 100 replays between
+    # its own events; the median is reported beside the K-step figure
+    g1 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g1, stream=stream):
+        wl.step(ops)
+    g1.replay()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(100)]
+    for a, b in ev:
+        a.record(stream)
+        g1.replay()
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    single = sorted(a.elapsed_time(b) for a, b in ev)
+    step_stats = {"median_ms": round(statistics.median(single), 4), "min_ms": round(single[0], 4),
+                  "p90_ms": round(single[89], 4), "reps": len(single)}
+    del g1
+
     # each call of the step on its own, for the per-kernel roofline: a CUDA graph of the call
     # replayed back to back between events (the same launches, inputs and outputs as the step)
     per = measure_calls(torch, ops, wl, stream, reps=20)
@@ -298,6 +315,7 @@ def run_ours(args, rank, world, dist):
         "ms_per_step": ms_max / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded torch CPU generator)",
         "config": step_config(world),
+        "single_step_replays": step_stats,
         "roofline": roofline,
         "parts": parts,
         "cpu_baseline": cpu,
