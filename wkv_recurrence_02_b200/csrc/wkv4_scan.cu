@@ -113,6 +113,13 @@ __device__ __forceinline__ P2 add2(P2 a, P2 b)
 }
 __device__ __forceinline__ P2 ex2_2(P2 x) { return pk(ex2(lo(x)), ex2(hi(x))); }
 __device__ __forceinline__ P2 rcp2(P2 x) { return pk(rcp(lo(x)), rcp(hi(x))); }
+// Both reciprocals from one: 1/x = y / (x y) and 1/y = x / (x y).  For 2^-60 <= x, y <= 2^60
+// the product stays a normal float; the result carries two more roundings than rcp2.
+__device__ __forceinline__ P2 rcp2_shared(P2 x)
+{
+    const float r = rcp(lo(x) * hi(x));
+    return mul2(pk(hi(x), lo(x)), pk(r, r));
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p)
 {
@@ -873,7 +880,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     for (int q = 0; q < NP; ++q) {
                         const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
                         const P2 bE = mul2(ub[q], E);
-                        o[q] = mul2(fma2(bE, vv[q], A[q]), rcp2(add2(Bs[q], bE)));
+                        o[q] = mul2(fma2(bE, vv[q], A[q]), rcp2_shared(add2(Bs[q], bE)));
                         A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
                         Bs[q] = fma2(dd[q], Bs[q], E);
                     }
