@@ -84,7 +84,8 @@ __device__ __forceinline__ void issue_stage(unsigned char *sm, uint32_t bar_full
 //              of the sub-block, channel quad cq), after exchanging sub-block decay products;
 //   warps 4-7  state: thread (q, lr, hi) holds row 16q + lr (a key channel) of the running
 //              state, value columns 32 hi .. 32 hi + 31, in registers.  Lane 0 of warp 4 also
-//              issues the TMA copies and the products KV = Kh^T V.
+//              issues the first TMA copies and the products KV = Kh^T V; lane 0 of warp 5
+//              refills a stage with chunk c + 3 once every state thread is done with chunk c.
 // Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> product), KV full
 // (tcgen05.commit -> state) and KV free (state -> product, and stage refill).
 template <bool OMEGA>
@@ -115,7 +116,8 @@ wkv6_chunk_state_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_
     const int nchunks = max(0, min(p.sub_chunks, nchunks_all - cb));
     const uint32_t limit = p.spin_limit;
     const uint32_t spin_limit = p.spin_limit * 64u;
-    const bool issuer = tid == 128;
+    const bool issuer = tid == 128;    // the products
+    const bool refiller = tid == 160;  // the TMA refills after the first kStages chunks
 
     if (tid == 0) {
         for (int s = 0; s < kStages; ++s) {
@@ -150,6 +152,7 @@ wkv6_chunk_state_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_
                         static_cast<int>(b), p.status, T);
         misc[2] = issued;
     }
+    if (refiller) issued = kStages < nchunks ? kStages : nchunks;
     int abort = 0;
     if (p.inject_timeout && tid == 0) abort = !bar_wait(bar_never, 0, limit);
     abort = __syncthreads_or(abort);
@@ -245,16 +248,6 @@ wkv6_chunk_state_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_
                         mma(tbase + 64 * bf, desc_mn(aK + 2048 * ks), desc_mn(aV + 2048 * ks), idesc(64, 1, 1), ks > 0);
                     mma_commit(bar_kvfull0 + 8 * bf);
                 }
-                // refill the stage of chunk c - 1 once that chunk has been consumed
-                if (ok && c >= 1 && issued < nchunks) {
-                    ok = bar_wait_spin(bar_kvfree0 + 8 * ((c - 1) & 1), ((c - 1) >> 1) & 1, spin_limit);
-                    if (ok) {
-                        issue_stage(sm, bar_full0, &map_k, &map_v, &map_w, issued, cb + issued, static_cast<int>(h),
-                                    static_cast<int>(b), p.status, T);
-                        ++issued;
-                        misc[2] = issued;
-                    }
-                }
             }
             if (ok) ok = bar_wait_spin(bar_kvfull0 + 8 * bf, (c >> 1) & 1, spin_limit);
             // the warp decides together (its lanes meet here, then read TMEM warp-wide)
@@ -276,6 +269,19 @@ wkv6_chunk_state_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_
             fence_before();
             bar_arrive(bar_kvfree0 + 8 * bf);
             dprod *= d;
+            // refill the stage of chunk c with chunk c + 3 as soon as every state thread has
+            // read its D (the product of chunk c is then complete too); a thread other than the
+            // issuer does it, so the next product is not held up
+            if (refiller && issued < nchunks) {
+                if (bar_wait_spin(bar_kvfree0 + 8 * bf, (c >> 1) & 1, spin_limit)) {
+                    issue_stage(sm, bar_full0, &map_k, &map_v, &map_w, issued, cb + issued, static_cast<int>(h),
+                                static_cast<int>(b), p.status, T);
+                    ++issued;
+                    misc[2] = issued;
+                } else {
+                    misc[1] = 1;  // the next vote of this warp ends the loop
+                }
+            }
         }
         if (!abort && in_bounds(p.status, (bh * p.nsub + g) * kSegStride, kSegStride, p.seg_cap)) {
             float *sg = p.seg + (bh * p.nsub + g) * kSegStride;
