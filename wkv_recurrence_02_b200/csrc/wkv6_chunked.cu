@@ -268,7 +268,9 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
     const int64_t b = bh / p.H, h = bh % p.H;
     const int64_t T = p.T;
     const int nchunks_all = static_cast<int>((T + kC - 1) / kC);
-    const int g = blockIdx.y;                      // segment of the sequence
+    // segment of the sequence; the last segments, which first combine the most pieces into
+    // their incoming state, are dispatched first
+    const int g = static_cast<int>(gridDim.y) - 1 - static_cast<int>(blockIdx.y);
     const int cb = g * p.seg_chunks;               // its first chunk
     const int nchunks = min(p.seg_chunks, nchunks_all - cb);  // chunks in this segment
     const uint32_t limit = p.spin_limit;
