@@ -28,6 +28,8 @@
 //
 // The products are tcgen05.mma kind::f16 (bf16 operands from 128-byte-swizzled shared
 // memory, fp32 accumulators in TMEM); S_prev is read from TMEM into a bf16 operand tile.
+// On the chunk-end path P is written back into tensor memory as bf16 pairs and the P V
+// product takes its A operand from there.
 // r, k, v, w tiles arrive by TMA (4-D tensor maps over [B, T, H, N], 128-byte swizzle,
 // zero fill past T) into a 3-stage ring.
 //
@@ -506,6 +508,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             for (int ks = 0; ks < 4; ++ks)
                 mma(tbase + COL_AD, desc_k(aR + 32 * ks), desc_k(aK + 32 * ks), idesc(64, 0, 0), ks > 0);
             if (misc[2 + s]) {
+                // these columns hold the previous chunk's P when that chunk took the chunk-end
+                // path: its O product must have read them first
+                if (c > 0 && !misc[2 + (c - 1) % kStages] && !bar_wait_spin(bar_O, (c - 1) & 1, spin_limit))
+                    return 0;
                 unsigned char *scr = sm + OFF_STAGE + ((c + 2) % kStages) * kStageBytes;
                 const uint32_t aKB = smem_u32(scr + SCR_KB), aQO = smem_u32(scr + SCR_QO);
 #pragma unroll
@@ -625,10 +631,32 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                 }
                 // causal mask per 16-column block kb of this row: kb < q kept, kb == q the
                 // diagonal block (columns before the row kept, the diagonal itself is the bonus
-                // term, written last), kb > q zero
-                unsigned char *pt = st + (safe ? SLOT_K : SLOT_W);
+                // term), kb > q zero.  Chunk-end path: P goes to tensor memory, bf16 pairs in the
+                // columns the sub-block path's scores use, and the O product reads it from there.
+                if (!safe) {
+                    const float ub = UB[s * 64 + row];
+                    uint32_t pw[16];
 #pragma unroll
-                for (int j = 0; j < 2; ++j) {
+                    for (int j = 0; j < 2; ++j) {
+                        const int kb = 2 * hi + j;
+#pragma unroll
+                        for (int n = 0; n < 16; n += 2) {
+                            float x0 = va[16 * j + n], x1 = va[16 * j + n + 1];
+                            if (kb > q) {
+                                x0 = 0.f;
+                                x1 = 0.f;
+                            } else if (kb == q) {
+                                x0 = n < lr ? x0 : (n == lr ? ub : 0.f);
+                                x1 = n + 1 < lr ? x1 : (n + 1 == lr ? ub : 0.f);
+                            }
+                            pw[8 * j + n / 2] = pack_bf16(x0, x1);
+                        }
+                    }
+                    tmem_st16w(tlane + COL_AO, pw);
+                }
+                unsigned char *pt = st + SLOT_K;
+#pragma unroll
+                for (int j = 0; j < 2 && safe; ++j) {
                     const int kb = 2 * hi + j;
                     float(&vb)[16] = *reinterpret_cast<float(*)[16]>(&va[16 * j]);
                     if (kb > q) {
@@ -643,7 +671,7 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                         st_row16_bf16(pt, row, 32 * kb, vb);
                     }
                 }
-                if (hi == (q >> 1))  // the thread that holds the diagonal block
+                if (safe && hi == (q >> 1))  // the thread that holds the diagonal block
                     *reinterpret_cast<__nv_bfloat16 *>(pt + swz(row, 2 * row)) = __float2bfloat16_rn(UB[s * 64 + row]);
             }
             // ---- state: S *= D in TMEM; operand = bf16(D S_prev) (chunk-end path) or bf16(S_prev)
@@ -671,9 +699,8 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             const uint32_t aV = smem_u32(st + SLOT_V);
             if (iss_o) {
                 // ---- O = P V + Q S_op
-                uint32_t aP, aQ, aSop;
+                uint32_t aP = 0, aQ, aSop;
                 if (!safe) {
-                    aP = smem_u32(st + SLOT_W);
                     aQ = smem_u32(st + SLOT_R);     // Qx
                     aSop = smem_u32(sm + OFF_SB);   // bf16(D S_prev)
                 } else {
@@ -682,9 +709,15 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     aQ = smem_u32(scr + SCR_QI);    // Qi
                     aSop = smem_u32(st + SLOT_R);   // bf16(S_prev)
                 }
+                if (!safe) {  // P from tensor memory: 16 K elements are 8 columns
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma(tbase + COL_O, desc_k(aP + 32 * ks), desc_mn(aV + 2048 * ks), idesc(64, 0, 1), ks > 0);
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_ts(tbase + COL_O, tbase + COL_AO + 8 * ks, desc_mn(aV + 2048 * ks), idesc(64, 0, 1), ks > 0);
+                } else {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma(tbase + COL_O, desc_k(aP + 32 * ks), desc_mn(aV + 2048 * ks), idesc(64, 0, 1), ks > 0);
+                }
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
                     mma(tbase + COL_O, desc_k(aQ + 32 * ks), desc_mn(aSop + 2048 * ks), idesc(64, 0, 1), 1);
