@@ -148,6 +148,21 @@ def test_wkv6_fast_decay_channels(wval):
     _check(x, s0=x["s0"], algo="chunked")
 
 
+def test_wkv6_paths_alternate_between_chunks():
+    """Chunks 2, 3 and 6 hold channels with w = 0.1 (chunk decay below 2^-100: the sub-block
+    path), chunk 8 a few tokens of w = 1e-30 (the exact diagonal blocks), every other chunk the
+    chunk-end path.  A sub-block chunk right after a chunk-end chunk reuses the tensor-memory
+    columns that held the previous chunk's P; every switch between the paths must match the
+    oracle."""
+    x = _inputs(2, 640, 2, "bf16", 21, s0_std=0.1)
+    w = x["w"].float()
+    w[:, 128:256, :, 24:32] = 0.1
+    w[:, 384:448, :, 24:32] = 0.1
+    w[:, 530:534, :, 40:44] = 1e-30
+    x["w"] = w.to(torch.bfloat16)
+    _check(x, s0=x["s0"], algo="chunked")
+
+
 @pytest.mark.parametrize("segments", [1, 2, 3, 5])
 def test_wkv6_sequence_split(segments):
     """The chunked kernel cut into segments (a first pass gives the end states of pieces of
