@@ -117,13 +117,16 @@ __device__ __forceinline__ void st_bf16x32(__nv_bfloat16 *dst, const float (&v)[
 // 256 threads = 8 warps in two groups.
 //   prep group (warps 0-3): warp a builds the operand rows of 16-token sub-block a (lane:
 //     8-token half hf, channel quad cq) and the chunk decay D, running ahead of the state;
-//   state group (warps 4-7): warp 4 + q serves TMEM lanes 32q.. of the state (rows 16q .. +
-//     15, two 32-column halves): per chunk it writes the checkpoint, scales the state by D
-//     and has one elected thread issue the four MMAs of the update; another elected thread
-//     of the group issues the TMA copies of later chunks (a 3-stage ring of X | Y | W tiles,
-//     and for the backward pass the forward checkpoint after the chunk, for the row dots).
-// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> state group), update
-// done (MMA commit -> state group; it also frees the stage of that chunk).
+//   state group (warps 4-7): thread (q, lr, hi) holds row 16q + lr of the state (value
+//     columns 32 hi .. 32 hi + 31) in fp32 registers.  Per chunk it writes the checkpoint,
+//     then takes S <- diag(D) S + X^T Y with X^T Y read from one of two TMEM buffers, so the
+//     tensor core never waits for the state: one elected thread issues each chunk's four
+//     MMAs as soon as its operands are formed and its buffer is free.  Another elected thread
+//     refills a stage (a 3-stage ring of X | Y | W tiles, and for the backward pass the
+//     forward checkpoint after the chunk, for the row dots) once every state thread is done
+//     with its chunk.
+// Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> product), product
+// full (MMA commit -> state group) and product free (state group -> product, stage refill).
 constexpr int kSThreads = 256;
 constexpr int kSStages = 3;
 template <bool REV> struct StateLayout {
@@ -131,8 +134,8 @@ template <bool REV> struct StateLayout {
     static constexpr int stage = tiles * kTile;
     static constexpr int hs = kSStages * stage;                  // [parity][4][64] sub-block decay products
     static constexpr int dv = hs + 2 * 4 * 64 * 4;               // [stage][64] chunk decay
-    static constexpr int bar = dv + kSStages * 64 * 4;           // full[3], prep[3], mma
-    static constexpr int misc = bar + 64;                        // TMEM base, abort flag
+    static constexpr int bar = dv + kSStages * 64 * 4;           // full[3], prep[3], kvfull[2], kvfree[2]
+    static constexpr int misc = bar + 128;                       // TMEM base, abort flag
     static constexpr int smem = misc + 64 + 1024;
 };
 
@@ -167,7 +170,8 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + L::bar);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + L::misc);
     const uint32_t bar_full0 = smem_u32(&bars[0]), bar_prep0 = smem_u32(&bars[kSStages]);
-    const uint32_t bar_mma = smem_u32(&bars[2 * kSStages]);
+    const uint32_t bar_kvfull0 = smem_u32(&bars[2 * kSStages]);      // + 8 * buffer
+    const uint32_t bar_kvfree0 = smem_u32(&bars[2 * kSStages + 2]);  // + 8 * buffer
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t bh = blockIdx.x, b = bh / p.H, h = bh % p.H;
@@ -181,14 +185,17 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
             bar_init(bar_full0 + 8 * s, 1);
             bar_init(bar_prep0 + 8 * s, 128);
         }
-        bar_init(bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            bar_init(bar_kvfull0 + 8 * i, 1);
+            bar_init(bar_kvfree0 + 8 * i, 128);
+        }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         misc[1] = 0;
     }
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_u32(const_cast<uint32_t *>(misc))),
-                     "r"(64));
+                     "r"(128));
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
     }
     fence_before();
@@ -296,43 +303,50 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
         const bool ck_ok = in_bounds(p.status, ((bh * nck + nck - 1) * kN + row) * kN + colh, 32, nbh * nck * kN * kN) &&
                            in_bounds(p.status, (bh * nch + nch - 1) * kN + row, 1, nbh * nch * kN);
         const bool st_ok = in_bounds(p.status, (bh * kN + row) * kN + colh, 32, nbh * kN * kN);
-        {
-            float v[32];
-            if (p.init && st_ok) {
-                const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
+        float S[32];
+        if (p.init && st_ok) {
+            const float4 *src = reinterpret_cast<const float4 *>(p.init + (bh * kN + row) * kN + colh);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const float4 x = src[i];
-                    v[4 * i] = x.x, v[4 * i + 1] = x.y, v[4 * i + 2] = x.z, v[4 * i + 3] = x.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 32; ++i) v[i] = 0.f;
+            for (int i = 0; i < 8; ++i) {
+                const float4 x = src[i];
+                S[4 * i] = x.x, S[4 * i + 1] = x.y, S[4 * i + 2] = x.z, S[4 * i + 3] = x.w;
             }
-            tmem_st32(tl, v);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) S[i] = 0.f;
         }
         for (int n = 0; n < nch; ++n) {
             const int cc = REV ? nch - 1 - n : n;
-            const int s = n % kSStages;
+            const int s = n % kSStages, bf = n & 1;
             unsigned char *st = sm + s * L::stage;
             int ok = 1;
             if (issuer_mma) {
+                // X^T Y of step n into buffer bf, once its operands are formed and the buffer's
+                // previous step (n - 2) has been read
                 ok = bar_wait_spin(bar_prep0 + 8 * s, (n / kSStages) & 1, spin);
-                if (ok && n > 0) ok = bar_wait_spin(bar_mma, (n - 1) & 1, spin);
+                if (ok && n >= 2) ok = bar_wait_spin(bar_kvfree0 + 8 * bf, ((n - 2) >> 1) & 1, spin);
+                if (ok) {
+                    fence_after();
+                    const uint32_t aX = smem_u32(st), aY = smem_u32(st + kTile);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma(tbase + 64 * bf, desc_mn(aX + 2048 * ks), desc_mn(aY + 2048 * ks), idesc(64, 1, 1), ks > 0);
+                    mma_commit(bar_kvfull0 + 8 * bf);
+                    ++committed;
+                }
             }
-            if (named_sync_or(2, 128, !ok || misc[1])) {
+            // the state entering chunk cc (forward) or leaving it (backward); it does not wait
+            // for the product
+            if (ck_ok) st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, S);
+            if (ok) ok = bar_wait_spin(bar_kvfull0 + 8 * bf, (n >> 1) & 1, spin);
+            // the warp decides together (its lanes meet here, then read TMEM warp-wide)
+            if (__any_sync(0xffffffffu, !ok || misc[1])) {
                 abort = 1;
                 misc[1] = 1;
                 break;
             }
-            bar_try(bar_prep0 + 8 * s, (n / kSStages) & 1);
-            if (n > 0) bar_try(bar_mma, (n - 1) & 1);
+            bar_try(bar_prep0 + 8 * s, (n / kSStages) & 1);  // D and the stage's tiles are visible
             fence_after();
-            // the stage of step n - 1 is free once its update is done: refill it
-            if (issuer_tma && n > 0 && issued < nch) issue(issued++);
-            float v[32];
-            tmem_ld32(tl, v);
-            if (ck_ok) st_bf16x32(p.ck + ((bh * nck + cc) * kN + row) * kN + colh, v);
             if (REV) {  // rowdot(dS_end, S_end): S_end = the forward state after chunk cc
                 float part = 0.f;
 #pragma unroll
@@ -340,42 +354,32 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
                     float x[8];
                     ld_row8(st + 3 * kTile, row, 2 * colh + 16 * i, x);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) part = fmaf(v[8 * i + e], x[e], part);
+                    for (int e = 0; e < 8; ++e) part = fmaf(S[8 * i + e], x[e], part);
                 }
                 part += __shfl_xor_sync(0xffffffffu, part, 16);
                 if (hi == 0 && ck_ok) p.rowdot[(bh * nch + cc) * kN + row] = part;
             }
             const float d = Dv[s * 64 + row];
+            float kv[32];
+            tmem_ld32(tl + 64 * bf, kv);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] *= d;
-            tmem_st32(tl, v);
+            for (int i = 0; i < 32; ++i) S[i] = fmaf(d, S[i], kv[i]);
             fence_before();
-            named_sync_or(2, 128, 0);
-            fence_after();
-            if (issuer_mma) {
-                const uint32_t aX = smem_u32(st), aY = smem_u32(st + kTile);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma(tbase, desc_mn(aX + 2048 * ks), desc_mn(aY + 2048 * ks), idesc(64, 1, 1), 1);
-                mma_commit(bar_mma);
-                ++committed;
+            bar_arrive(bar_kvfree0 + 8 * bf);
+            // refill the stage of step n with step n + 3 once every state thread is done with it
+            // (its product has completed, its D and tiles have been read)
+            if (issuer_tma && issued < nch) {
+                if (bar_wait_spin(bar_kvfree0 + 8 * bf, (n >> 1) & 1, spin))
+                    issue(issued++);
+                else
+                    misc[1] = 1;  // the next vote of this warp ends the loop
             }
         }
         if (!abort) {
-            const int ok = issuer_mma ? bar_wait_spin(bar_mma, (nch - 1) & 1, spin) : 1;
-            if (named_sync_or(2, 128, !ok || misc[1])) {
-                abort = 1;
-                misc[1] = 1;
-            } else {
-                bar_try(bar_mma, (nch - 1) & 1);
-                fence_after();
-                float v[32];
-                tmem_ld32(tl, v);
-                if (!REV && ck_ok)
-                    st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, v);
-                else if (REV && p.fin && st_ok)
-                    st_f32x32(p.fin + (bh * kN + row) * kN + colh, v);
-            }
+            if (!REV && ck_ok)
+                st_bf16x32(p.ck + ((bh * nck + nch) * kN + row) * kN + colh, S);
+            else if (REV && p.fin && st_ok)
+                st_f32x32(p.fin + (bh * kN + row) * kN + colh, S);
         }
     }
     fence_before();
@@ -390,12 +394,13 @@ wkv6_bwd_state_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_co
         if (issuer_tma)
             for (int n = issued - kSStages < 0 ? 0 : issued - kSStages; n < issued; ++n)
                 bar_wait(bar_full0 + 8 * (n % kSStages), (n / kSStages) & 1, limit);
-        if (tid == 128 && committed > 0) bar_wait(bar_mma, (committed - 1) & 1, limit);
+        if (tid == 128 && committed > 0)  // the products complete in order: wait for the last
+            bar_wait(bar_kvfull0 + 8 * ((committed - 1) & 1), ((committed - 1) >> 1) & 1, limit);
     }
     fence_before();
     __syncthreads();
     fence_after();
-    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(64));
+    if (warp == 0) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tbase), "r"(128));
 }
 
 // ================================================================ per-chunk gradients (K2)
