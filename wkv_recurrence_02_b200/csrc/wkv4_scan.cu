@@ -1072,6 +1072,83 @@ wkv4_decode_kernel(int64_t B, int64_t C, const float *__restrict__ w, const floa
     }
 }
 
+// Four adjacent channels of one token row: k, v loads and the y store in one access each.
+template <typename T> struct Row4;
+template <> struct Row4<float> {
+    __device__ static void load(const float *p, float (&x)[4])
+    {
+        const float4 q = *reinterpret_cast<const float4 *>(p);
+        x[0] = q.x, x[1] = q.y, x[2] = q.z, x[3] = q.w;
+    }
+    __device__ static void store(float *p, const float (&x)[4])
+    {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+template <> struct Row4<__nv_bfloat16> {
+    __device__ static void load(const __nv_bfloat16 *p, float (&x)[4])
+    {
+        const uint2 q = *reinterpret_cast<const uint2 *>(p);
+        x[0] = __uint_as_float(q.x << 16), x[1] = __uint_as_float(q.x & 0xFFFF0000u);
+        x[2] = __uint_as_float(q.y << 16), x[3] = __uint_as_float(q.y & 0xFFFF0000u);
+    }
+    __device__ static void store(__nv_bfloat16 *p, const float (&x)[4])
+    {
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(x[0], x[1]), hi = __floats2bfloat162_rn(x[2], x[3]);
+        *reinterpret_cast<uint2 *>(p) =
+            make_uint2(*reinterpret_cast<const uint32_t *>(&lo), *reinterpret_cast<const uint32_t *>(&hi));
+    }
+};
+
+// The decode step of wkv4_decode_kernel for C a multiple of 4: each thread owns 4 adjacent
+// channels, so every state row (a, b, p), w, u, k, v and y moves in one 16- or 8-byte access
+// (the launcher's pointers are 16-byte aligned and C % 4 == 0, so every offset is aligned).
+template <typename T>
+__global__ void __launch_bounds__(256)
+wkv4_decode4_kernel(int64_t B, int64_t C, const float *__restrict__ w, const float *__restrict__ u,
+                    const T *__restrict__ k, const T *__restrict__ v, const float *s0, T *__restrict__ y, float *sT,
+                    int *status)
+{
+    const int64_t c0 = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 4;
+    if (c0 >= C) return;
+    if (!in_bounds(status, c0, 4, C)) return;  // debug build: this thread's channels inside C
+    const float4 wq = *reinterpret_cast<const float4 *>(w + c0), uq = *reinterpret_cast<const float4 *>(u + c0);
+    const float w2[4] = {wq.x * kLog2e, wq.y * kLog2e, wq.z * kLog2e, wq.w * kLog2e};
+    const float u2[4] = {uq.x * kLog2e, uq.y * kLog2e, uq.z * kLog2e, uq.w * kLog2e};
+    for (int64_t b = blockIdx.y; b < B; b += gridDim.y) {
+        const int64_t i = b * C + c0;
+        float kk[4], vv[4];
+        Row4<T>::load(k + i, kk);
+        Row4<T>::load(v + i, vv);
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f}, sq[4] = {0.f, 0.f, 0.f, 0.f};
+        if (s0) {
+            const float *sp = s0 + b * 3 * C;
+            Row4<float>::load(sp + c0, sa);
+            Row4<float>::load(sp + C + c0, sb);
+            Row4<float>::load(sp + 2 * C + c0, sq);
+        }
+        float yo[4], na[4], nb[4], np[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float k2 = kk[j] * kLog2e;
+            St st{0.f, 0.f, kPEmpty};
+            if (sb[j] != 0.f) st = {sa[j], sb[j], fmaxf(sq[j] * kLog2e, kPEmpty)};
+            yo[j] = output(st, k2, vv[j], u2[j]);
+            update(st, k2, vv[j], w2[j]);
+            na[j] = st.a;
+            nb[j] = st.b;
+            np[j] = st.b == 0.f ? kPEmpty : st.p * kLn2;
+        }
+        Row4<T>::store(y + i, yo);
+        if (sT) {
+            float *tp = sT + b * 3 * C;
+            Row4<float>::store(tp + c0, na);
+            Row4<float>::store(tp + C + c0, nb);
+            Row4<float>::store(tp + 2 * C + c0, np);
+        }
+    }
+}
+
 template <typename T, int NV>
 cudaError_t launch_decode_v(const Wkv4Args &a, cudaStream_t s)
 {
@@ -1079,9 +1156,14 @@ cudaError_t launch_decode_v(const Wkv4Args &a, cudaStream_t s)
     const int64_t bx = (groups + 255) / 256;
     if (bx > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const unsigned by = static_cast<unsigned>(a.B < 65535 ? a.B : 65535);
-    wkv4_decode_kernel<T, NV><<<dim3(static_cast<unsigned>(bx), by), 256, 0, s>>>(
-        a.B, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
-        static_cast<T *>(a.y), a.sT, a.status);
+    if (NV == 4)
+        wkv4_decode4_kernel<T><<<dim3(static_cast<unsigned>(bx), by), 256, 0, s>>>(
+            a.B, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
+            static_cast<T *>(a.y), a.sT, a.status);
+    else
+        wkv4_decode_kernel<T, NV><<<dim3(static_cast<unsigned>(bx), by), 256, 0, s>>>(
+            a.B, a.C, a.w, a.u, static_cast<const T *>(a.k), static_cast<const T *>(a.v), a.s0,
+            static_cast<T *>(a.y), a.sT, a.status);
     return cudaGetLastError();
 }
 
@@ -1089,6 +1171,7 @@ template <typename T>
 cudaError_t launch_decode(const Wkv4Args &a, cudaStream_t s)
 {
     if (a.B == 0 || a.C == 0) return cudaSuccess;
+    if (a.C % 4 == 0) return launch_decode_v<T, 4>(a, s);
     return a.C % 2 == 0 ? launch_decode_v<T, 2>(a, s) : launch_decode_v<T, 1>(a, s);
 }
 
