@@ -359,12 +359,14 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
             }
             st<T>(y + n * kN + tid, fmaf(bsum, sld(vv + tid), acc));
         }
-        // the stage of head i - 1 takes head i + 2 once that head's store has read it
+        // the stage of head i - 1 takes head i + 2 once that head's store has read it (every
+        // thread is past head i - 1: the barrier above)
         if (tid == 0 && i >= 1 && i + 2 < count) {
             if (sT) tc::bulk_wait_read<1>();
             issue(i + 2);
         }
-        __syncthreads();  // red, bred and this stage are reused
+        // red and bred are written again only after the next head's first barrier, which every
+        // reader of this head's sums reaches after reading them
     }
     if (abort) {
         record_status(status, kStatusTimeout);
