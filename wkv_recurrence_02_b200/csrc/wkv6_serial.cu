@@ -262,6 +262,19 @@ template <typename T> constexpr int decode_stream_smem()
 template <typename T> __device__ __forceinline__ float sld(const T *p);
 template <> __device__ __forceinline__ float sld<float>(const float *p) { return *p; }
 template <> __device__ __forceinline__ float sld<__nv_bfloat16>(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+// four consecutive values from shared memory in one access (p aligned to 4 elements)
+template <typename T> __device__ __forceinline__ void sld4(const T *p, float (&x)[4]);
+template <> __device__ __forceinline__ void sld4<float>(const float *p, float (&x)[4])
+{
+    const float4 q = *reinterpret_cast<const float4 *>(p);
+    x[0] = q.x, x[1] = q.y, x[2] = q.z, x[3] = q.w;
+}
+template <> __device__ __forceinline__ void sld4<__nv_bfloat16>(const __nv_bfloat16 *p, float (&x)[4])
+{
+    const uint2 q = *reinterpret_cast<const uint2 *>(p);
+    x[0] = __uint_as_float(q.x << 16), x[1] = __uint_as_float(q.x & 0xFFFF0000u);
+    x[2] = __uint_as_float(q.y << 16), x[3] = __uint_as_float(q.y & 0xFFFF0000u);
+}
 
 template <typename T>
 __global__ void __launch_bounds__(kDThreads)
@@ -316,14 +329,17 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
             break;
         }
         float rr[4], kk[4], ww[4], uu[4], vj[4];
+        sld4(vr + 4 * ig, rr);
+        sld4(vk + 4 * ig, kk);
+        sld4(vw + 4 * ig, ww);
+        sld4(vv + 4 * j4, vj);
+        {
+            const float4 u4 = __ldg(reinterpret_cast<const float4 *>(u + h * kN + 4 * ig));  // global
+            uu[0] = u4.x, uu[1] = u4.y, uu[2] = u4.z, uu[3] = u4.w;
+        }
+        if (omega) {
 #pragma unroll
-        for (int m = 0; m < 4; ++m) {
-            rr[m] = sld(vr + 4 * ig + m);
-            kk[m] = sld(vk + 4 * ig + m);
-            const float wm = sld(vw + 4 * ig + m);
-            ww[m] = omega ? decay_of_logit(wm) : wm;
-            uu[m] = __ldg(u + h * kN + 4 * ig + m);  // global
-            vj[m] = sld(vv + 4 * j4 + m);
+            for (int m = 0; m < 4; ++m) ww[m] = decay_of_logit(ww[m]);
         }
         float o[4] = {0.f, 0.f, 0.f, 0.f};
         float bonus = 0.f;
