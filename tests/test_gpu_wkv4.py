@@ -156,10 +156,11 @@ def test_wkv4_state_chaining_full_tiles(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
-@pytest.mark.parametrize("C", [96, 37])
+@pytest.mark.parametrize("C", [96, 98, 37])
 def test_wkv4_decode_chained_in_place_matches_the_oracle(dtype, C):
     """40 single-token calls (the T = 1 decode kernel), the state updated in place, equal
-    the oracle over all 40 tokens: every y and the final (a, b, p) state."""
+    the oracle over all 40 tokens: every y and the final (a, b, p) state.  C = 96, 98 and 37
+    take the kernel's 4-, 2- and 1-channel-per-thread forms."""
     B, T = 4, 40
     x = inputs.wkv4_inputs(B, T, C, dtype, seed=21)
     w, u, k, v = dev(x["w"]), dev(x["u"]), dev(x["k"]), dev(x["v"])
