@@ -33,8 +33,8 @@
 //   wkv4_tma_kernel (the default, used when the row pitch is a multiple of 16 bytes, the
 //     segment length L divides T and T/L >= 32): the k and v tiles arrive by TMA as
 //     token-index-major blocks (block i = token i of all 32 segments); each warp holds one
-//     8-byte half of a 16-byte unit of channels; y replaces k in place and leaves by TMA
-//     store.
+//     8-byte half of a 16-byte unit of channels; pass 2 writes each lane's y rows straight
+//     to global memory as it produces them.
 //   wkv4_scan_kernel (every other shape: odd C, unaligned pointers, L not dividing T):
 //     warp = channel pair (2 channels per lane); k and v tiles are copied with cp.async
 //     into a [pair][segment][L+1] layout (the +1 pad and a 4-word skew per pair make both
@@ -630,22 +630,11 @@ __device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap *map
                  "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
                  : "memory");
 }
-__device__ __forceinline__ void tma_store_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3, uint32_t src)
-{
-    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(src)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-}
-__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-
 struct TmaParams {
     int64_t T, C, B;
     const float *w, *u, *s0;
     float *sT;
+    void *y;  // [B, T, C] of the kernel's element type
     int *status;
     uint32_t spin_limit;
 };
@@ -653,7 +642,7 @@ struct TmaParams {
 template <typename T, int L, int NB>
 __global__ void __launch_bounds__(32 * (kCh / Lane<T>::NC), 3)
 wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant__ CUtensorMap map_v,
-                const __grid_constant__ CUtensorMap map_y, const TmaParams p)
+                const TmaParams p)
 {
     constexpr int NC = Lane<T>::NC;              // channels per lane
     constexpr int NP = NC / 2;                   // f32x2 pairs per lane
@@ -738,8 +727,8 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     for (; tile < ntiles; ++tile) {
         const int seg0 = kSegs * tile;
         if (NB > 1 && tile + 1 < ntiles && h == 0) {
-            // the next tile goes to the other buffer, whose last tile's store must have read it
-            if (lane < L) bulk_wait_read();
+            // the next tile goes to the other buffer, which every thread has finished reading
+            // (the barrier at the end of the previous tile)
             issue(tile + 1);
             ++issued;
         }
@@ -848,7 +837,15 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             carry[n] = all;
         }
 
-        // pass 2: outputs from the exact incoming state; y replaces k in place
+        // pass 2: outputs from the exact incoming state; each lane writes its y rows to global
+        // memory as it goes (8 bytes per row: with every lane of a warp, 32 contiguous bytes of
+        // each of 8 segments), so the stores overlap the scan
+        T *yrow = static_cast<T *>(p.y) + (static_cast<int64_t>(b) * T_len + static_cast<int64_t>(seg0 + seg_l) * L) * C + cb;
+        const bool ystore = nv > 0 && cb < C &&  // debug build: the segment's rows inside y
+                            in_bounds(p.status, (static_cast<int64_t>(b) * T_len + static_cast<int64_t>(seg0 + seg_l) * L) * C + cb,
+                                      NC, p.B * T_len * C) &&
+                            in_bounds(p.status, (static_cast<int64_t>(b) * T_len + static_cast<int64_t>(seg0 + seg_l) * L + L - 1) * C + cb,
+                                      NC, p.B * T_len * C);
         bool fixed = true;
         float F[NC];
 #pragma unroll
@@ -870,8 +867,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
 #pragma unroll
             for (int i = 0; i < L; ++i) {
                 if (i < nv) {
-                    unsigned char *ui = uk + i * BLK;
-                    const uint2 ku = Lane<T>::load(ui);
+                    const uint2 ku = Lane<T>::load(uk + i * BLK);
                     const uint2 vu = Lane<T>::load(uv + i * BLK);
                     P2 kk[NP], vv[NP], o[NP];
                     Lane<T>::unpack(ku, kk);
@@ -884,12 +880,11 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
                         Bs[q] = fma2(dd[q], Bs[q], E);
                     }
-                    Lane<T>::store(ui, Lane<T>::pack(o));
+                    if (ystore) *reinterpret_cast<uint2 *>(yrow + static_cast<int64_t>(i) * C) = Lane<T>::pack(o);
                 }
             }
         } else {
-            // running-maximum steps, exact for any inputs; channel by channel (y_n replaces
-            // k_n only after k_n has been read)
+            // running-maximum steps, exact for any inputs; channel by channel
 #pragma unroll
             for (int n = 0; n < NC; ++n) {
                 St s = pa[n];
@@ -897,17 +892,14 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                     const float k2 = Unit<T>::get(uk + i * BLK, n) * kLog2e, vx = Unit<T>::get(uv + i * BLK, n);
                     const float o = output(s, k2, vx, u2[n]);
                     update(s, k2, vx, w2[n]);
-                    Unit<T>::put(uk + i * BLK, n, o);
+                    if (ystore) Elem<T>::put(yrow + static_cast<int64_t>(i) * C + n, o);
                 }
             }
         }
 
-        // y of this tile: one TMA store per segment (clipped at T and C)
-        fence_async_smem();
+        // every thread is done reading this tile's buffer before it is refilled
         __syncthreads();
-        if (h == 0 && lane < L) tma_store_4d(&map_y, c0, lane, seg0, b, smem_u32(sk + lane * BLK));
     }
-    if (h == 0) bulk_wait_all();
     if (abort) {
         record_status(p.status, kStatusTimeout);
         if (threadIdx.x == 0)  // bounded: let the copies in flight land before the CTA exits
@@ -951,10 +943,10 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
                                    static_cast<cuuint64_t>(a.T * a.C * sizeof(T))};
     const cuuint32_t box[4] = {static_cast<cuuint32_t>(kCh), 1, static_cast<cuuint32_t>(kSegs), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
-    CUtensorMap mk, mv, my;
-    const void *ptrs[3] = {a.k, a.v, a.y};
-    CUtensorMap *maps[3] = {&mk, &mv, &my};
-    for (int i = 0; i < 3; ++i)
+    CUtensorMap mk, mv;
+    const void *ptrs[2] = {a.k, a.v};
+    CUtensorMap *maps[2] = {&mk, &mv};
+    for (int i = 0; i < 2; ++i)
         if (enc(maps[i], Unit<T>::kMapType, 4, const_cast<void *>(ptrs[i]), dims, strides, box, estr,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
@@ -978,8 +970,8 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
         }
     }
     const int64_t blocks = a.B * ((a.C + kCh - 1) / kCh);
-    const TmaParams prm{a.T, a.C, a.B, a.w, a.u, a.s0, a.sT, a.status, 1u << 22};
-    kern<<<static_cast<unsigned>(blocks), kThr, smem, s>>>(mk, mv, my, prm);
+    const TmaParams prm{a.T, a.C, a.B, a.w, a.u, a.s0, a.sT, a.y, a.status, 1u << 22};
+    kern<<<static_cast<unsigned>(blocks), kThr, smem, s>>>(mk, mv, prm);
     return cudaGetLastError();
 }
 
