@@ -286,8 +286,11 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
     unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                           ~static_cast<uintptr_t>(127));
     constexpr int SB = dstage_bytes<T>();
-    float(*red)[kN] = reinterpret_cast<float(*)[kN]>(sm + kDStages * SB);
-    float *bred = reinterpret_cast<float *>(sm + kDStages * SB + 16 * kN * 4);
+    // per-warp partial sums of y and of the bonus, double-buffered by head parity:
+    // [parity][warp][64] and [parity][warp] (the same 16 x 64 + 16 floats as one buffer of
+    // per-row-group sums)
+    float(*red)[8][kN] = reinterpret_cast<float(*)[8][kN]>(sm + kDStages * SB);
+    float(*bred)[8] = reinterpret_cast<float(*)[8]>(sm + kDStages * SB + 16 * kN * 4);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + kDStages * SB + 16 * kN * 4 + 16 * 4);
     const uint32_t bar0 = tc::smem_u32(&bars[0]);
     const int tid = threadIdx.x, ig = tid >> 4, j4 = tid & 15;
@@ -323,11 +326,8 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
         float *S = reinterpret_cast<float *>(stg);
         const T *vr = reinterpret_cast<const T *>(stg + kN * kN * 4);
         const T *vk = vr + kN, *vw = vr + 2 * kN, *vv = vr + 3 * kN;
+        // each thread waits for the stage itself; the expiry vote is taken at the barrier below
         const int ok = tc::bar_wait(bar0 + 8 * s, static_cast<uint32_t>((i / kDStages) & 1), limit);
-        if (__syncthreads_or(!ok)) {
-            abort = 1;
-            break;
-        }
         float rr[4], kk[4], ww[4], uu[4], vj[4];
         sld4(vr + 4 * ig, rr);
         sld4(vk + 4 * ig, kk);
@@ -358,10 +358,18 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
             x.w = fmaf(ww[m], x.w, kk[m] * vj[3]);
             *row = x;
         }
-        *reinterpret_cast<float4 *>(&red[ig][4 * j4]) = make_float4(o[0], o[1], o[2], o[3]);
-        if (j4 == 0) bred[ig] = bonus;
+        // the warp's two row groups (lanes l and l ^ 16) summed first
+#pragma unroll
+        for (int q = 0; q < 4; ++q) o[q] += __shfl_xor_sync(0xffffffffu, o[q], 16);
+        bonus += __shfl_xor_sync(0xffffffffu, bonus, 16);
+        const int pb = static_cast<int>(i & 1), wp = tid >> 5;
+        if ((tid & 31) < 16) *reinterpret_cast<float4 *>(&red[pb][wp][4 * j4]) = make_float4(o[0], o[1], o[2], o[3]);
+        if ((tid & 31) == 0) bred[pb][wp] = bonus;
         tc::fence_async_smem();  // the new state is read by the bulk store (async proxy)
-        __syncthreads();
+        if (__syncthreads_or(!ok)) {  // the one barrier of a head; a stage wait that ran out ends here
+            abort = 1;
+            break;
+        }
         if (tid == 0 && sT) {
             if (in_bounds(status, n * kN * kN, kN * kN, BH * kN * kN)) tc::bulk_store(sT + n * kN * kN, tc::smem_u32(stg), kN * kN * 4);
             tc::bulk_commit();
@@ -369,9 +377,9 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
         if (tid < kN) {
             float acc = 0.f, bsum = 0.f;
 #pragma unroll
-            for (int rg = 0; rg < 16; ++rg) {
-                acc += red[rg][tid];
-                bsum += bred[rg];
+            for (int wq = 0; wq < 8; ++wq) {
+                acc += red[pb][wq][tid];
+                bsum += bred[pb][wq];
             }
             st<T>(y + n * kN + tid, fmaf(bsum, sld(vv + tid), acc));
         }
@@ -381,8 +389,8 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
             if (sT) tc::bulk_wait_read<1>();
             issue(i + 2);
         }
-        // red and bred are written again only after the next head's first barrier, which every
-        // reader of this head's sums reaches after reading them
+        // this head's partial sums are written again two heads on, after the next head's
+        // barrier, which every reader of them reaches after reading them
     }
     if (abort) {
         record_status(status, kStatusTimeout);
