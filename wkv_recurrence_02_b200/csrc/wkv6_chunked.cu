@@ -568,23 +568,13 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             unsigned char *st = sm + OFF_STAGE + s * kStageBytes;
             const int64_t t0 = static_cast<int64_t>(cb + c) * kC;
 
-            // scores of c and all MMAs of c-1 complete (three waiters side by side)
-            if (ok) {
-                if (iss_a) ok = bar_wait_spin(bar_A, c & 1, spin_limit);
-                else if (iss_o && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
-                else if (iss_s && c > 0) ok = bar_wait_spin(bar_S, (c - 1) & 1, spin_limit);
-            }
-            if (named_sync_or(2, 128, !ok || misc[1])) {
-                abort = 1;
-                misc[1] = 1;
-                break;
-            }
-            bar_try(bar_A, c & 1);
-            bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);
-            if (c > 0) {
-                bar_try(bar_O, (c - 1) & 1);
-                bar_try(bar_S, (c - 1) & 1);
-            }
+            // scores of c and all MMAs of c-1 complete: every thread waits itself, so each warp
+            // starts its pass as soon as they are; an expiry is voted on at the group barrier
+            // after the pass (the warps must not leave the loop on their own)
+            if (ok) ok = bar_wait_spin(bar_A, c & 1, spin_limit);
+            if (ok && c > 0) ok = bar_wait_spin(bar_O, (c - 1) & 1, spin_limit);
+            if (ok && c > 0) ok = bar_wait_spin(bar_S, (c - 1) & 1, spin_limit);
+            bar_try(bar_prep0 + 8 * s, (c / kStages) & 1);  // the prep group's writes are visible
             fence_after();
             const int safe = misc[2 + s], hazard = misc[5 + s];
 
@@ -693,7 +683,11 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
             }
             fence_async_smem();
             fence_before();
-            named_sync_or(2, 128, 0);
+            if (named_sync_or(2, 128, !ok || misc[1])) {
+                abort = 1;
+                misc[1] = 1;
+                break;
+            }
             fence_after();
 
             const uint32_t aV = smem_u32(st + SLOT_V);
