@@ -587,16 +587,16 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
             U[tid] = p.u[h * kN + tid];
             RD[tid] = p.rowdot[(bh * nch + cc) * kN + tid];
         }
+        // every thread waits for the tiles itself; an expiry is voted on at the group barrier
+        // of the prep below
         int ok = bar_wait(bar_full, ph, limit);
-        abort = __syncthreads_or(!ok);
-        if (abort) break;
-        waited = 1;
+        if (ok) waited = 1;
         {
             // ------------------------------------------------------------ operand rows
             // warp w: tokens 8w .. 8w + 7; lane: half hf (tokens 8w + 4hf .. + 3), channel quad cq
             const int hf = lane >> 4, cq = lane & 15, t0h = 8 * warp + 4 * hf;
             const uint32_t cbyte = 8 * cq;
-            const Q4 u4 = ld_q4(U + 4 * cq);
+            const Q4 u4 = ld_q4(p.u + h * kN + 4 * cq);  // U (staged above) is visible only after the barrier
             Q4 w[4];
             Q4 Gh = one4();
 #pragma unroll
@@ -612,7 +612,10 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
             }
             const Q4 Go = shfl_xor4(Gh, 16);
             if (hf == 0) st_q4(Hs + warp * 64 + 4 * cq, mul4(Gh, Go));
-            __syncthreads();
+            if (__syncthreads_or(!ok)) {
+                abort = 1;
+                break;
+            }
             Q4 D = one4(), before = one4(), aft = one4();
 #pragma unroll
             for (int g = 0; g < 8; ++g) {
@@ -726,10 +729,9 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
                 }
             }
         }
+        // each thread waits for the first products itself; the vote is at the next barrier
         ok = bar_wait(bar_m1, ph, limit);
-        abort = __syncthreads_or(!ok);
-        if (abort) break;
-        waited = 2;
+        if (ok) waited = 2;
         fence_after();
         {
             // ------------------------------------------------------------ Am and dAm
@@ -749,7 +751,10 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
         }
         fence_async_smem();
         fence_before();
-        __syncthreads();
+        if (__syncthreads_or(!ok)) {
+            abort = 1;
+            break;
+        }
         fence_after();
         if (iss && warp != 1) {
             const uint32_t aQ = smem_u32(TQX), aK = smem_u32(TKH), aG = smem_u32(TG), aDS = smem_u32(TDS);
@@ -772,10 +777,9 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
             }
             mma_commit(bar_m2);
         }
+        // each thread waits for the second products itself; the vote is at the next barrier
         ok = bar_wait(bar_m2, ph, limit);
-        abort = __syncthreads_or(!ok);
-        if (abort) break;
-        waited = 3;
+        if (ok) waited = 3;
         fence_after();
         {
             // ------------------------------------------------------------ gradients of row t
@@ -846,7 +850,10 @@ wkv6_bwd_chunk_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_co
 #pragma unroll
                 for (int n = 0; n < 16; ++n) Hs[sub * 64 + col0 + n] = rdr[n];
             fence_async_smem();
-            __syncthreads();
+            if (__syncthreads_or(!ok)) {
+                abort = 1;
+                break;
+            }
             if (tid == 0) {  // dv, dr, dk of this chunk
                 const int hh = static_cast<int>(h), bb = static_cast<int>(b), tt = static_cast<int>(t0);
                 tma_store_4d(&om.dv, 0, hh, tt, bb, smem_u32(TV));
