@@ -237,8 +237,10 @@ __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[
 //              (an MMA issue holds its thread for tens of cycles, so three issuers run side
 //              by side), and of warp 7 the TMA copies of later chunks.
 // Hand-offs are mbarriers: stage full (TMA -> prep), prep done (prep -> MMA issue), scores
-// done, O done, state done and stage empty (tcgen05.commit).  Per-chunk bookkeeping (bonus
-// diagonal, decay, path flags) lives beside the chunk's stage.
+// done, O done, state done and stage empty (tcgen05.commit).  Every TMEM thread waits on the
+// scores, O and state barriers itself, and the TMEM group meets once per chunk, after its
+// pass, before the products are issued.  Per-chunk bookkeeping (bonus diagonal, decay, path
+// flags) lives beside the chunk's stage.
 template <bool GATED, bool OMEGA>
 __global__ void __launch_bounds__(kThreads, 2)
 wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_constant__ CUtensorMap map_k,
