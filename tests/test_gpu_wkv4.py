@@ -156,6 +156,29 @@ def test_wkv4_state_chaining_full_tiles(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_wkv4_carried_state_of_any_weight(dtype):
+    """A carried state whose exponent p runs, channel by channel, from far below the new keys'
+    to far above them (-60 to 160 in natural-log units): where the state dominates, the
+    segments leave the fixed frame for the running-maximum steps (reading the keys from
+    global memory when pass 1 kept fp16 weights in their place); where it is comparable, the
+    stored weights are brought to its reference; where it is negligible it drops out."""
+    B, T, C = 2, 1024, 48
+    x = inputs.wkv4_inputs(B, T, C, dtype, seed=21)
+    rng = np.random.default_rng(22)
+    b = rng.uniform(0.5, 2.0, (B, C))
+    s0 = np.stack([rng.standard_normal((B, C)) * b, b, np.tile(np.linspace(-60.0, 160.0, C), (B, 1))], 1)
+    y, sT = ops.wkv4_forward(dev(x["w"]), dev(x["u"]), dev(x["k"]), dev(x["v"]),
+                             s0=torch.from_numpy(s0).float().cuda(), want_state=True)
+    torch.cuda.synchronize()
+    ref_y, ref_s = oracle.wkv4(f64(x["w"]), f64(x["u"]), f64(x["k"]), f64(x["v"]),
+                               s0=s0.astype(np.float32).astype(np.float64), want_state=True)
+    assert rel_inf(f64(y), ref_y) <= TOL[y.dtype]
+    ga, gb = wkv4_state_views(f64(sT))
+    ra, rb = wkv4_state_views(ref_s)
+    assert rel_inf(ga, ra) <= 1e-4 and np.max(np.abs(gb - rb)) <= 1e-3
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 @pytest.mark.parametrize("C", [96, 98, 37])
 def test_wkv4_decode_chained_in_place_matches_the_oracle(dtype, C):
     """40 single-token calls (the T = 1 decode kernel), the state updated in place, equal

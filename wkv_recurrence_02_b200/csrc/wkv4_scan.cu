@@ -17,14 +17,16 @@
 //           apart) the lane redoes its segment with the running-maximum step.  The
 //           segment's largest and smallest key are noted on the way, and the summary is
 //           renormalised (the denominator's binary exponent moved into the reference) so
-//           that the scan compares states by their true magnitude;
+//           that the scan compares states by their true magnitude.  (The TMA kernel's
+//           bf16 path instead takes the segment's largest exponent, less 15, as reference
+//           and keeps every weight as fp16 in its k slot for pass 2; see that kernel.);
 //   scan    a 5-step warp shuffle scan combines segment summaries across lanes, and the
 //           carry from earlier tiles (or s0) is folded in;
 //   pass 2  each lane re-walks its segment from its exact incoming state.  When every
 //           term lies within 2^60 of the segment's largest exponent (the normal case)
-//           the walk uses that fixed reference: one ex2 per key weight and one
-//           reciprocal per output; otherwise it repeats the running-maximum step, which
-//           is exact for any inputs.
+//           the walk uses that fixed reference: one ex2 per key weight (none where pass
+//           1's stored weight is read back) and one reciprocal per output; otherwise it
+//           repeats the running-maximum step, which is exact for any inputs.
 // Both channels of a lane are carried in 64-bit register pairs and advanced with packed
 // f32x2 arithmetic.
 //
@@ -33,8 +35,9 @@
 //   wkv4_tma_kernel (the default, used when the row pitch is a multiple of 16 bytes, the
 //     segment length L divides T and T/L >= 32): the k and v tiles arrive by TMA as
 //     token-index-major blocks (block i = token i of all 32 segments); each warp holds one
-//     8-byte half of a 16-byte unit of channels; pass 2 writes each lane's y rows straight
-//     to global memory as it produces them.
+//     8-byte half of a 16-byte unit of channels; warp 0 issues the first tile's copies
+//     before the CTA reads its parameters; pass 2 writes each lane's y rows straight to
+//     global memory as it produces them.
 //   wkv4_scan_kernel (every other shape: odd C, unaligned pointers, L not dividing T):
 //     warp = channel pair (2 channels per lane); k and v tiles are copied with cp.async
 //     into a [pair][segment][L+1] layout (the +1 pad and a 4-word skew per pair make both
@@ -637,7 +640,32 @@ struct TmaParams {
     void *y;  // [B, T, C] of the kernel's element type
     int *status;
     uint32_t spin_limit;
+    const void *k;  // [B, T, C]: the exact paths' keys once the tile's slots hold weights
 };
+
+// Four fp32 weights as fp16 in a lane's 8-byte k slot, and back.
+template <int N>
+__device__ __forceinline__ uint2 pack_h4(const P2 (&e)[N])
+{
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int q = 0; q < N; ++q)
+        asm("{\n\t.reg .f32 l, h;\n\tmov.b64 {l, h}, %1;\n\tcvt.rn.f16x2.f32 %0, h, l;\n\t}" : "=r"(w[q]) : "l"(e[q].r));
+    return make_uint2(w[0], w[1]);
+}
+template <int N>
+__device__ __forceinline__ void unpack_h4(uint2 u, P2 (&e)[N])
+{
+    const uint32_t w[2] = {u.x, u.y};
+#pragma unroll
+    for (int q = 0; q < N; ++q)
+        asm("{\n\t.reg .f16 a, b;\n\t.reg .f32 l, h;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 l, a;\n\t"
+            "cvt.f32.f16 h, b;\n\tmov.b64 %0, {l, h};\n\t}"
+            : "=l"(e[q].r)
+            : "r"(w[q]));
+}
+constexpr float kHalfShift = 15.f;  // stored weights are 2^{k - Rf} with Rf 15 below the largest exponent
+constexpr float kHalfSpan = 13.f;   // ... and stay fp16 normals (>= 2^-14) while k - Rf >= -13
 
 template <typename T, int L, int NB>
 __global__ void __launch_bounds__(32 * (kCh / Lane<T>::NC), 3)
@@ -676,6 +704,32 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         (cb >= C || in_bounds(p.status, static_cast<int64_t>(b) * 3 * C + 2 * C + cb, 1, p.B * 3 * C));
         if (!__syncthreads_and(ok)) return;
     }
+    const int nsegs = static_cast<int>(T_len / L);  // L divides T
+    const int ntiles = (nsegs + kSegs - 1) / kSegs;
+    // warp 0: lane i brings block i of k and v of tile tl into its buffer
+    auto issue = [&](int tl) {
+        unsigned char *bk = sbase + (tl % NB) * 2 * L * BLK;
+        const uint32_t bar = bar0 + 8 * (tl % NB);
+        if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
+        __syncwarp();
+        // debug build: channel block on a 16-byte boundary inside C, the tile's first segment
+        // inside T / L (a copy that fails is not issued; its wait then runs out)
+        if (lane < L && tma_coord_ok(p.status, c0, static_cast<int>(sizeof(T)), C, static_cast<int64_t>(kSegs) * tl,
+                                     T_len / L)) {
+            tma_load_4d(smem_u32(bk + lane * BLK), &map_k, c0, lane, kSegs * tl, b, bar);
+            tma_load_4d(smem_u32(bk + L * BLK + lane * BLK), &map_v, c0, lane, kSegs * tl, b, bar);
+        }
+    };
+    // the first tile's copies leave before anything else: the parameter loads below then
+    // overlap them instead of delaying them
+    if (h == 0) {
+        if (lane == 0) {
+            for (int i = 0; i < NB; ++i) mbar_init(bar0 + 8 * i, 1);
+            asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        }
+        __syncwarp();
+        if (ntiles > 0) issue(0);
+    }
 
     const St empty{0.f, 0.f, kPEmpty};
     float w2[NC], u2[NC];
@@ -699,30 +753,7 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         ub[q] = pk(ex2(u2[2 * q]), ex2(u2[2 * q + 1]));    // bonus factors
     }
     const P2 l2e = pk(kLog2e, kLog2e), nl2e = pk(-kLog2e, -kLog2e);
-
-    if (threadIdx.x == 0) {
-        for (int i = 0; i < NB; ++i) mbar_init(bar0 + 8 * i, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
     __syncthreads();
-
-    const int nsegs = static_cast<int>(T_len / L);  // L divides T
-    const int ntiles = (nsegs + kSegs - 1) / kSegs;
-    // warp 0: lane i brings block i of k and v of tile tl into its buffer
-    auto issue = [&](int tl) {
-        unsigned char *bk = sbase + (tl % NB) * 2 * L * BLK;
-        const uint32_t bar = bar0 + 8 * (tl % NB);
-        if (lane == 0) mbar_expect_tx(bar, 2u * L * BLK);
-        __syncwarp();
-        // debug build: channel block on a 16-byte boundary inside C, the tile's first segment
-        // inside T / L (a copy that fails is not issued; its wait then runs out)
-        if (lane < L && tma_coord_ok(p.status, c0, static_cast<int>(sizeof(T)), C, static_cast<int64_t>(kSegs) * tl,
-                                     T_len / L)) {
-            tma_load_4d(smem_u32(bk + lane * BLK), &map_k, c0, lane, kSegs * tl, b, bar);
-            tma_load_4d(smem_u32(bk + L * BLK + lane * BLK), &map_v, c0, lane, kSegs * tl, b, bar);
-        }
-    };
-    if (h == 0 && ntiles > 0) issue(0);
     int abort = 0, tile = 0, issued = ntiles > 0 ? 1 : 0;
     for (; tile < ntiles; ++tile) {
         const int seg0 = kSegs * tile;
@@ -741,15 +772,50 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
         const unsigned char *uv = sv + 8 * threadIdx.x;
         const int nv = seg0 + seg_l < nsegs ? L : 0;
 
-        // pass 1: local summaries against the segment's last key; key range
+        // pass 1: local summaries and the key range.  bf16 tiles take the segment's largest
+        // exponent (largest key, plus u when u > 0) less kHalfShift as the reference Rf, so
+        // that every weight 2^{k - Rf} lies in [2^-13, 2^15] when the keys' spread allows
+        // (f16ok); each weight then goes back into its k slot as fp16 and pass 2 reads it
+        // instead of forming it again.  fp32 tiles take the segment's last key.
         St la[NC];
         LaneRange<T> kr;
         kr.init();
 #pragma unroll
         for (int n = 0; n < NC; ++n) la[n] = empty;
+        constexpr bool kReuse = sizeof(T) == 2;
+        bool f16ok = kReuse;
+        float Rf[NC] = {};
+        // this lane's keys in global memory: the exact paths read them there once the tile's
+        // k slots may hold weights
+        const int64_t krow = (static_cast<int64_t>(b) * T_len + static_cast<int64_t>(seg0 + seg_l) * L) * C + cb;
+        auto key = [&](int i, int n) -> float {  // key n of the segment's row i, exact paths
+            if constexpr (kReuse) {
+                const int64_t at = krow + static_cast<int64_t>(i) * C + n;
+                return cb < C && in_bounds(p.status, at, 1, p.B * T_len * C)
+                           ? Elem<T>::get(static_cast<const T *>(p.k) + at)
+                           : 0.f;
+            } else {
+                return Unit<T>::get(uk + i * BLK, n);
+            }
+        };
         if (nv > 0) {
             P2 nF[NP], A[NP], Bs[NP];
-            {
+            if constexpr (kReuse) {
+#pragma unroll
+                for (int i = 0; i < L; ++i)
+                    if (i < nv) kr.add(Lane<T>::load(uk + i * BLK));
+#pragma unroll
+                for (int n = 0; n < NC; ++n) {
+                    Rf[n] = kr.max(n) * kLog2e + fmaxf(u2[n], 0.f) - kHalfShift;
+                    f16ok = f16ok && Rf[n] - kr.min(n) * kLog2e <= kHalfSpan;
+                }
+#pragma unroll
+                for (int q = 0; q < NP; ++q) {
+                    nF[q] = pk(-Rf[2 * q], -Rf[2 * q + 1]);
+                    A[q] = pk(0.f, 0.f);
+                    Bs[q] = A[q];
+                }
+            } else {
                 P2 kl[NP];
                 Lane<T>::unpack(Lane<T>::load(uk + (nv - 1) * BLK), kl);
 #pragma unroll
@@ -764,8 +830,8 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 if (i < nv) {
                     const uint2 ku = Lane<T>::load(uk + i * BLK);
                     const uint2 vu = Lane<T>::load(uv + i * BLK);
-                    kr.add(ku);
-                    P2 kk[NP], vv[NP];
+                    if constexpr (!kReuse) kr.add(ku);
+                    P2 kk[NP], vv[NP], Ek[NP];
                     Lane<T>::unpack(ku, kk);
                     Lane<T>::unpack(vu, vv);
 #pragma unroll
@@ -773,6 +839,10 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                         const P2 E = ex2_2(fma2(kk[q], l2e, nF[q]));
                         A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
                         Bs[q] = fma2(dd[q], Bs[q], E);
+                        Ek[q] = E;
+                    }
+                    if constexpr (kReuse) {
+                        if (f16ok) Lane<T>::store(uk + i * BLK, pack_h4(Ek));
                     }
                 }
             }
@@ -781,17 +851,15 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
                 const P2 a2 = A[n >> 1], b2 = Bs[n >> 1], f2 = nF[n >> 1];
                 const float an = n & 1 ? hi(a2) : lo(a2), bn = n & 1 ? hi(b2) : lo(b2);
                 const float fn = n & 1 ? hi(f2) : lo(f2);
-                if (w2[n] >= 0.f && bn <= 3.0e38f && fabsf(an) <= 3.0e38f) {
+                if (w2[n] >= 0.f && bn <= 3.0e38f && fabsf(an) <= 3.0e38f && (!kReuse || bn >= 0x1p-100f)) {
                     la[n] = normalized(an, bn, -fn);
-                } else {  // a weight overflowed (or negative decay): running-maximum steps
+                } else {  // a weight overflowed or underflowed (or negative decay): running-maximum steps
                     St s = empty;
-                    for (int i = 0; i < nv; ++i)
-                        update(s, Unit<T>::get(uk + i * BLK, n) * kLog2e, Unit<T>::get(uv + i * BLK, n), w2[n]);
+                    for (int i = 0; i < nv; ++i) update(s, key(i, n) * kLog2e, Unit<T>::get(uv + i * BLK, n), w2[n]);
                     la[n] = s;
                 }
             }
         }
-
         // inclusive scan over this warp's segments (lanes U apart share a unit) with segment
         // lengths; the warps' totals then meet in shared memory, and each lane folds the
         // carry from earlier tiles, the earlier warps' totals and its warp's exclusive
@@ -820,23 +888,38 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             tw[3 * NC] = n_inc;
         }
         __syncthreads();
+        // the state entering this lane's segment (carry, earlier warps, earlier lanes); the
+        // state after the whole tile only where a later tile or sT needs it
         St pa[NC];
+        const bool need_all = tile + 1 < ntiles || p.sT != nullptr;
+        St before[NC];
+#pragma unroll
+        for (int n = 0; n < NC; ++n) before[n] = carry[n];
+        for (int hw = 0; hw < h; ++hw) {
+            const float *tw = wtot + (hw * U + q) * (3 * NC + 1);
+#pragma unroll
+            for (int n = 0; n < NC; ++n)
+                before[n] = combine(before[n], St{tw[3 * n], tw[3 * n + 1], tw[3 * n + 2]}, tw[3 * NC] * w2[n]);
+        }
 #pragma unroll
         for (int n = 0; n < NC; ++n) {
-            St before = carry[n], all = carry[n];
-            for (int hw = 0; hw < kCh / NC; ++hw) {
-                const float *tw = wtot + (hw * U + q) * (3 * NC + 1);
-                const St t{tw[3 * n], tw[3 * n + 1], tw[3 * n + 2]};
-                const float nw = tw[3 * NC] * w2[n];
-                if (hw < h) before = combine(before, t, nw);
-                all = combine(all, t, nw);
-            }
             St e = shfl_up(la[n], U);
             if (lane < U) e = empty;
-            pa[n] = combine(before, e, n_exc * w2[n]);
-            carry[n] = all;
+            pa[n] = combine(before[n], e, n_exc * w2[n]);
         }
-
+        if (need_all) {
+#pragma unroll
+            for (int n = 0; n < NC; ++n) {
+                St all = carry[n];
+#pragma unroll
+                for (int hw = 0; hw < kCh / NC; ++hw) {
+                    const float *tw = wtot + (hw * U + q) * (3 * NC + 1);
+                    const St t{tw[3 * n], tw[3 * n + 1], tw[3 * n + 2]};
+                    all = combine(all, t, tw[3 * NC] * w2[n]);
+                }
+                carry[n] = all;
+            }
+        }
         // pass 2: outputs from the exact incoming state; each lane writes its y rows to global
         // memory as it goes (8 bytes per row: with every lane of a warp, 32 contiguous bytes of
         // each of 8 segments), so the stores overlap the scan
@@ -854,7 +937,37 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             fixed = fixed && w2[n] >= 0.f && fabsf(u2[n]) <= kFrame &&
                     F[n] - (u2[n] + kr.min(n) * kLog2e) <= kFrame;
         }
-        if (fixed) {
+        if (kReuse && fixed && f16ok) {
+            // pass 1's weights 2^{k - Rf}, read back from the k slots and brought to F
+            P2 A[NP], Bs[NP], sc[NP], ubs[NP];
+#pragma unroll
+            for (int q = 0; q < NP; ++q) {
+                const float s_lo = ex2(pa[2 * q].p - F[2 * q]), s_hi = ex2(pa[2 * q + 1].p - F[2 * q + 1]);
+                A[q] = pk(pa[2 * q].a * s_lo, pa[2 * q + 1].a * s_hi);
+                Bs[q] = pk(pa[2 * q].b * s_lo, pa[2 * q + 1].b * s_hi);
+                sc[q] = pk(ex2(Rf[2 * q] - F[2 * q]), ex2(Rf[2 * q + 1] - F[2 * q + 1]));
+                ubs[q] = mul2(ub[q], sc[q]);
+            }
+#pragma unroll
+            for (int i = 0; i < L; ++i) {
+                if (i < nv) {
+                    const uint2 eu = Lane<T>::load(uk + i * BLK);
+                    const uint2 vu = Lane<T>::load(uv + i * BLK);
+                    P2 e0[NP], vv[NP], o[NP];
+                    unpack_h4(eu, e0);
+                    Lane<T>::unpack(vu, vv);
+#pragma unroll
+                    for (int q = 0; q < NP; ++q) {
+                        const P2 E = mul2(e0[q], sc[q]);
+                        const P2 bE = mul2(ubs[q], e0[q]);
+                        o[q] = mul2(fma2(bE, vv[q], A[q]), rcp2_shared(add2(Bs[q], bE)));
+                        A[q] = fma2(dd[q], A[q], mul2(E, vv[q]));
+                        Bs[q] = fma2(dd[q], Bs[q], E);
+                    }
+                    if (ystore) *reinterpret_cast<uint2 *>(yrow + static_cast<int64_t>(i) * C) = Lane<T>::pack(o);
+                }
+            }
+        } else if (fixed) {
             // every weight is 2^{x - F} <= 1 and the bonus term keeps the denominator >= 2^-60
             P2 A[NP], Bs[NP], nF[NP];
 #pragma unroll
@@ -889,15 +1002,15 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
             for (int n = 0; n < NC; ++n) {
                 St s = pa[n];
                 for (int i = 0; i < nv; ++i) {
-                    const float k2 = Unit<T>::get(uk + i * BLK, n) * kLog2e, vx = Unit<T>::get(uv + i * BLK, n);
+                    const float k2 = key(i, n) * kLog2e, vx = Unit<T>::get(uv + i * BLK, n);
                     const float o = output(s, k2, vx, u2[n]);
                     update(s, k2, vx, w2[n]);
                     if (ystore) Elem<T>::put(yrow + static_cast<int64_t>(i) * C + n, o);
                 }
             }
         }
-
         // every thread is done reading this tile's buffer before it is refilled
+        if (kReuse && NB > 1) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
         __syncthreads();
     }
     if (abort) {
@@ -970,7 +1083,7 @@ cudaError_t launch_tma_L(const Wkv4Args &a, cudaStream_t s)
         }
     }
     const int64_t blocks = a.B * ((a.C + kCh - 1) / kCh);
-    const TmaParams prm{a.T, a.C, a.B, a.w, a.u, a.s0, a.sT, a.y, a.status, 1u << 22};
+    const TmaParams prm{a.T, a.C, a.B, a.w, a.u, a.s0, a.sT, a.y, a.status, 1u << 22, a.k};
     kern<<<static_cast<unsigned>(blocks), kThr, smem, s>>>(mk, mv, prm);
     return cudaGetLastError();
 }
