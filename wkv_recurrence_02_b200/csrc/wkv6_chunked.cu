@@ -183,6 +183,12 @@ __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[
             in_bounds(p.status, ((b * p.T + tok) * p.H + h) * kN + colh, 32,
                       static_cast<int64_t>(gridDim.x) * p.T * kN);
     if (GATED) {
+        uint4 gw[4] = {};  // the gate row, loaded first so that its latency overlaps the statistics
+        if (valid) {
+            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + ((b * p.T + tok) * p.H + h) * kN + colh);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) gw[v4] = gp[v4];
+        }
         float s = 0.f;
 #pragma unroll
         for (int n = 0; n < 32; ++n) s += ov[n];
@@ -197,18 +203,21 @@ __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[
         q += __shfl_xor_sync(0xffffffffu, q, 16);
         const float rstd = rsqrtf(q * (1.f / kN) + p.eps);
         if (valid) {
-            const uint4 *gp = reinterpret_cast<const uint4 *>(p.gate + ((b * p.T + tok) * p.H + h) * kN + colh);
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
-                const uint4 gw = gp[v4];
-                const uint32_t wd[4] = {gw.x, gw.y, gw.z, gw.w};
+                const uint32_t wd[4] = {gw[v4].x, gw[v4].y, gw[v4].z, gw[v4].w};
+                float sc[8], sh[8];  // LayerNorm scale and shift of these 8 channels, 16-byte loads
+                *reinterpret_cast<float4 *>(sc) = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4);
+                *reinterpret_cast<float4 *>(sc + 4) = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4 + 4);
+                *reinterpret_cast<float4 *>(sh) = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4);
+                *reinterpret_cast<float4 *>(sh + 4) = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4 + 4);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int n = 8 * v4 + e;
                     const float gv = __uint_as_float(e & 1 ? (wd[e >> 1] & 0xFFFF0000u) : (wd[e >> 1] << 16));
-                    // SiLU(g) = g / (1 + 2^(-g log2 e)), approximate exponential and reciprocal
-                    const float gate = gv * rcp_approx(1.f + ex2_approx(-gv * 1.4426950408889634f));
-                    ov[n] = gate * fmaf(lns[colh + n] * (ov[n] - mean), rstd, lns[kN + colh + n]);
+                    // SiLU(g) = g sigma(g) with sigma(g) = 1/2 + tanh(g/2)/2: one approximate tanh
+                    const float gate = gv * fmaf(0.5f, tanh_approx(0.5f * gv), 0.5f);
+                    ov[n] = gate * fmaf(sc[e] * (ov[n] - mean), rstd, sh[e]);
                 }
             }
         }
