@@ -358,6 +358,12 @@ __device__ __forceinline__ P2 fma2(P2 a, P2 b, P2 c)
     asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.r) : "l"(a.r), "l"(b.r), "l"(c.r));
     return d;
 }
+__device__ __forceinline__ P2 add2(P2 a, P2 b)
+{
+    P2 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.r) : "l"(a.r), "l"(b.r));
+    return d;
+}
 __device__ __forceinline__ P2 one2() { return pk(1.f, 1.f); }
 
 // bf16 pair (low half = first channel) -> exact fp32 pair

@@ -172,7 +172,7 @@ __device__ __forceinline__ void prep_fast(unsigned char *st, int t0h, uint32_t c
 
 // y row of token tok, head h: this thread's 32 of the 64 channels, the other 32 in lane
 // ^ 16.  With a gate, the head's LayerNorm (statistics over both halves) and the SiLU gate
-// are applied first.  Every lane of the warp calls this (the statistics pair lanes); only
+// are applied first, in f32x2 pairs, and the gated branch stores the row itself.  Every lane of the warp calls this (the statistics pair lanes); only
 // `valid` rows read g and store.
 template <bool GATED>
 __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[32], int64_t tok, int64_t b,
@@ -189,38 +189,64 @@ __device__ __forceinline__ void store_y_row(const ChunkedParams &p, float (&ov)[
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) gw[v4] = gp[v4];
         }
-        float s = 0.f;
+        // channel pairs in f32x2 registers: the statistics and the output stage take one
+        // instruction per two channels
+        P2 o2[16];
 #pragma unroll
-        for (int n = 0; n < 32; ++n) s += ov[n];
+        for (int i = 0; i < 16; ++i) o2[i] = pk(ov[2 * i], ov[2 * i + 1]);
+        P2 sa = o2[0], sb = o2[1];
+#pragma unroll
+        for (int i = 2; i < 16; i += 2) {
+            sa = add2(sa, o2[i]);
+            sb = add2(sb, o2[i + 1]);
+        }
+        sa = add2(sa, sb);
+        float s = lo(sa) + hi(sa);
         s += __shfl_xor_sync(0xffffffffu, s, 16);
         const float mean = s * (1.f / kN);
-        float q = 0.f;
+        const P2 nm = pk(-mean, -mean);
+        P2 qa = pk(0.f, 0.f), qb = qa;
 #pragma unroll
-        for (int n = 0; n < 32; ++n) {
-            const float d = ov[n] - mean;
-            q = fmaf(d, d, q);
+        for (int i = 0; i < 16; i += 2) {  // o2 now holds o - mean
+            o2[i] = add2(o2[i], nm);
+            o2[i + 1] = add2(o2[i + 1], nm);
+            qa = fma2(o2[i], o2[i], qa);
+            qb = fma2(o2[i + 1], o2[i + 1], qb);
         }
+        qa = add2(qa, qb);
+        float q = lo(qa) + hi(qa);
         q += __shfl_xor_sync(0xffffffffu, q, 16);
         const float rstd = rsqrtf(q * (1.f / kN) + p.eps);
         if (valid) {
+            const P2 rs2 = pk(rstd, rstd), half2 = pk(0.5f, 0.5f);
+            uint32_t yw[16];
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
                 const uint32_t wd[4] = {gw[v4].x, gw[v4].y, gw[v4].z, gw[v4].w};
-                float sc[8], sh[8];  // LayerNorm scale and shift of these 8 channels, 16-byte loads
-                *reinterpret_cast<float4 *>(sc) = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4);
-                *reinterpret_cast<float4 *>(sc + 4) = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4 + 4);
-                *reinterpret_cast<float4 *>(sh) = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4);
-                *reinterpret_cast<float4 *>(sh + 4) = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4 + 4);
+                // LayerNorm scale and shift of these 8 channels, 16-byte loads
+                const float4 ca = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4);
+                const float4 cb = *reinterpret_cast<const float4 *>(lns + colh + 8 * v4 + 4);
+                const float4 ha = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4);
+                const float4 hb = *reinterpret_cast<const float4 *>(lns + kN + colh + 8 * v4 + 4);
+                const P2 sc2[4] = {pk(ca.x, ca.y), pk(ca.z, ca.w), pk(cb.x, cb.y), pk(cb.z, cb.w)};
+                const P2 sh2[4] = {pk(ha.x, ha.y), pk(ha.z, ha.w), pk(hb.x, hb.y), pk(hb.z, hb.w)};
 #pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int n = 8 * v4 + e;
-                    const float gv = __uint_as_float(e & 1 ? (wd[e >> 1] & 0xFFFF0000u) : (wd[e >> 1] << 16));
-                    // SiLU(g) = g sigma(g) with sigma(g) = 1/2 + tanh(g/2)/2: one approximate tanh
-                    const float gate = gv * fmaf(0.5f, tanh_approx(0.5f * gv), 0.5f);
-                    ov[n] = gate * fmaf(sc[e] * (ov[n] - mean), rstd, sh[e]);
+                for (int e = 0; e < 4; ++e) {
+                    const P2 hg = mul2(unpack2(wd[e]), half2);  // g / 2
+                    const P2 t = fma2(mul2(sc2[e], o2[4 * v4 + e]), rs2, sh2[e]);
+                    // SiLU(g) t = g sigma(g) t with sigma(g) = (1 + tanh(g/2)) / 2, i.e.
+                    // (g t / 2)(1 + tanh(g / 2)): one approximate tanh per channel
+                    const P2 x2 = mul2(hg, t);
+                    yw[4 * v4 + e] = pack2(fma2(pk(tanh_approx(lo(hg)), tanh_approx(hi(hg))), x2, x2));
                 }
             }
+            // the stores last: a global store between them would hold back the shared loads of
+            // the scale and shift, which the compiler cannot prove it does not alias
+            uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * p.T + tok) * p.H + h) * kN + colh);
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) dst[v4] = make_uint4(yw[4 * v4], yw[4 * v4 + 1], yw[4 * v4 + 2], yw[4 * v4 + 3]);
         }
+        return;
     }
     if (valid) {
         uint4 *dst = reinterpret_cast<uint4 *>(p.y + ((b * p.T + tok) * p.H + h) * kN + colh);
