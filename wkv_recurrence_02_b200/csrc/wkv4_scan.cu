@@ -679,8 +679,10 @@ wkv4_tma_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_constant
     // NB buffers (tile tau in buffer tau % NB), each k blocks then v blocks; NB mbarriers.
     // With one buffer the launcher guarantees a single tile.
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sbase = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                                             ~static_cast<uintptr_t>(127));
+    // aligned by an offset on the __shared__ array itself (not through an integer), so the
+    // compiler keeps the shared state space: its accesses are shared loads and stores, which it
+    // may reorder freely around global ones
+    unsigned char *sbase = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
     const uint32_t bar0 = smem_u32(sbase + NB * 2 * L * BLK);  // + 8 * buffer
     // [warp][unit][(a, b, p) x NC channels, segment count]: each warp's scan total
     float *wtot = reinterpret_cast<float *>(sbase + NB * 2 * L * BLK + 8 * NB);

@@ -51,9 +51,11 @@ constexpr int kN = 64;                                // head size
 constexpr float kFastMin = 7.888609052210118e-31f;    // 2^-100: chunk-end reference guard
 constexpr float kWMin = 0.03125f;                     // 2^-5: smallest w the w-input path divides by
 
+// The first 1024-byte boundary at or after p (a __shared__ array), reached by an offset on p
+// itself rather than through an integer, so that the compiler keeps the shared state space.
 __device__ __forceinline__ unsigned char *align1024(unsigned char *p)
 {
-    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~static_cast<uintptr_t>(1023));
+    return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
 }
 
 // sum over the four channels of a * b

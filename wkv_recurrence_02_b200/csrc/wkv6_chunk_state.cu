@@ -94,8 +94,10 @@ wkv6_chunk_state_kernel(const __grid_constant__ CUtensorMap map_k, const __grid_
                         const __grid_constant__ CUtensorMap map_w, const Params p)
 {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // aligned by an offset on the __shared__ array itself (not through an integer), so the
+    // compiler keeps the shared state space: its accesses are shared loads and stores, which it
+    // may reorder freely around global ones
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
     volatile uint32_t *misc = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC);
     // misc: [0] TMEM base, [1] abort, [2] chunks whose TMA has been issued

@@ -283,8 +283,10 @@ wkv6_chunked_kernel(const __grid_constant__ CUtensorMap map_r, const __grid_cons
                     const ChunkedParams p)
 {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>(
-        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    // aligned by an offset on the __shared__ array itself (not through an integer), so the
+    // compiler keeps the shared state space: its accesses are shared loads and stores, which it
+    // may reorder freely around global ones
+    unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     float *Hs2 = reinterpret_cast<float *>(sm + OFF_H);  // [parity][4 sub-blocks][64 channels]
     float *Dv = reinterpret_cast<float *>(sm + OFF_D);   // [stage][64]
     float *UB = reinterpret_cast<float *>(sm + OFF_UB);  // [stage][64]

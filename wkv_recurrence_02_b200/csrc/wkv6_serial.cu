@@ -283,8 +283,10 @@ wkv6_decode_stream_kernel(int64_t BH, int64_t H, const T *__restrict__ r, const 
                           const float *s0, T *__restrict__ y, float *sT, int omega, int *status, uint32_t limit)
 {
     extern __shared__ unsigned char smem_raw[];
-    unsigned char *sm = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
-                                                          ~static_cast<uintptr_t>(127));
+    // aligned by an offset on the __shared__ array itself (not through an integer), so the
+    // compiler keeps the shared state space: its accesses are shared loads and stores, which it
+    // may reorder freely around global ones
+    unsigned char *sm = smem_raw + ((128u - (tc::smem_u32(smem_raw) & 127u)) & 127u);
     constexpr int SB = dstage_bytes<T>();
     // per-warp partial sums of y and of the bonus, double-buffered by head parity:
     // [parity][warp][64] and [parity][warp] (the same 16 x 64 + 16 floats as one buffer of
