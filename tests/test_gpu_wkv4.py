@@ -156,6 +156,26 @@ def test_wkv4_state_chaining_full_tiles(dtype):
 
 
 @pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+def test_wkv4_key_spreads_straddle_the_fp16_weight_range(dtype):
+    """Per-channel key scales from 1 to 8 (with u up to 3 where positive): a segment's key spread
+    runs from well inside to well beyond the 28 log2 units within which bf16 tiles keep pass 1's
+    weights as fp16 for pass 2, so lanes of one CTA take both forms side by side, over four
+    16-token-segment tiles."""
+    B, T, C = 2, 2048, 64
+    x = inputs.wkv4_inputs(B, T, C, dtype, seed=31)
+    scale = torch.linspace(1.0, 8.0, C)
+    k = (x["k"].float() * scale).to(x["k"].dtype)
+    u = x["u"] * 3.0
+    y, sT = ops.wkv4_forward(dev(x["w"]), dev(u), dev(k), dev(x["v"]), want_state=True)
+    torch.cuda.synchronize()
+    ref_y, ref_s = oracle.wkv4(f64(x["w"]), f64(u), f64(k), f64(x["v"]), want_state=True)
+    assert rel_inf(f64(y), ref_y) <= TOL[y.dtype]
+    ga, gb = wkv4_state_views(f64(sT))
+    ra, rb = wkv4_state_views(ref_s)
+    assert rel_inf(ga, ra) <= 1e-4 and np.max(np.abs(gb - rb)) <= 1e-3
+
+
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
 def test_wkv4_carried_state_of_any_weight(dtype):
     """A carried state whose exponent p runs, channel by channel, from far below the new keys'
     to far above them (-60 to 160 in natural-log units): where the state dominates, the
