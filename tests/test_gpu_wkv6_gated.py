@@ -107,3 +107,23 @@ def test_gate_closed_forms():
     assert torch.count_nonzero(y0) == 0
     gf = f64(g)
     assert rel_inf(f64(ys), gf / (1.0 + np.exp(-gf))) <= 1e-2
+
+
+def test_gate_silu_elementwise_on_a_grid():
+    """ln_w = 0, ln_b = 1 gives y = SiLU(g); on a grid of g from -8 to 8 every element is within
+    1 % of g / (1 + e^-g) (bf16 rounding of y alone is up to 0.39 %), through the chunked
+    kernel and the decode kernel."""
+    H = 2
+    g = torch.linspace(-8.0, 8.0, 4096 * H * 64).to(torch.bfloat16)
+    one, zero = torch.ones(H, 64, device="cuda"), torch.zeros(H, 64, device="cuda")
+    for B, T in [(1, 4096), (4096, 1)]:
+        x = inputs.wkv6_inputs(B, T, H, 64, "bf16", seed=14, s0_std=0.1)
+        xd = {n: dev(t) for n, t in x.items()}
+        gg = g.reshape(B, T, H, 64)
+        y = ops.wkv6_forward_gated(xd["r"], xd["k"], xd["v"], xd["w"], xd["u"], dev(gg), zero, one,
+                                   s0=xd["s0"], want_state=False)
+        torch.cuda.synchronize()
+        gf = f64(gg)
+        ref = gf / (1.0 + np.exp(-gf))
+        rel = np.abs(f64(y) - ref) / np.abs(ref)
+        assert np.max(rel[np.abs(gf) > 0]) <= 1e-2, (B, T, np.max(rel[np.abs(gf) > 0]))
